@@ -1,0 +1,178 @@
+"""CPU oracle for weight-only block-quantized matmul.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by the smoke check and by the
+CPU-baseline leg of ``bench.py``, never by the library's product path.  The
+arithmetic lives in ``bq_oracle.c`` (plain C, float64 accumulation, no FMA
+contraction); this module only marshals numpy arrays into it.
+
+Parity status of each function (what pins it, see ``tests/test_oracle_pins.py``):
+  f32/f16/bf16 conversions  -- numpy / torch conversions, exhaustive or 1M+ values
+  q4_0_quantize             -- closed forms: exact round trip, all-zero block,
+                               max-abs element -> q = 0, q range, error bound
+  q4_0_dequantize           -- hand-worked golden block, round trip
+  affine_quantize           -- closed forms: exact round trip, constant group,
+                               min -> 0 / max -> L, error bound
+  affine_dequantize         -- hand-worked golden groups (4 and 8 bit), round trip
+  matmul_ref                -- exact rational (fractions.Fraction) brute force
+                               on tiny non-square shapes, one-hot identities
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        from . import build as _build
+        _build.build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    I = ctypes.c_int
+    lib.oracle_f32_to_bf16_array.argtypes = [P, P, I64]
+    lib.oracle_bf16_to_f32_array.argtypes = [P, P, I64]
+    lib.oracle_f32_to_f16_array.argtypes = [P, P, I64]
+    lib.oracle_f16_to_f32_array.argtypes = [P, P, I64]
+    lib.oracle_q4_0_quantize.argtypes = [P, I64, I64, P, P]
+    lib.oracle_q4_0_dequantize.argtypes = [P, P, I64, I64, P]
+    lib.oracle_affine_quantize.argtypes = [P, I64, I64, I, I, P, P, P]
+    lib.oracle_affine_dequantize.argtypes = [P, P, P, I64, I64, I, I, P]
+    lib.oracle_matmul_ref.argtypes = [P, P, I64, I64, I64, P, I64, P, P, I]
+    lib.oracle_matmul_ref.restype = I
+    for name in ("oracle_f32_to_bf16_array", "oracle_bf16_to_f32_array", "oracle_f32_to_f16_array",
+                 "oracle_f16_to_f32_array", "oracle_q4_0_quantize", "oracle_q4_0_dequantize",
+                 "oracle_affine_quantize", "oracle_affine_dequantize"):
+        getattr(lib, name).restype = None
+    _lib = lib
+    return lib
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _ptr(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+# ---------------------------------------------------------------- conversions
+def f32_to_bf16(a) -> np.ndarray:
+    a = _c(a, np.float32)
+    out = np.empty(a.shape, np.uint16)
+    _load().oracle_f32_to_bf16_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def bf16_to_f32(a) -> np.ndarray:
+    a = _c(a, np.uint16)
+    out = np.empty(a.shape, np.float32)
+    _load().oracle_bf16_to_f32_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def f32_to_f16(a) -> np.ndarray:
+    a = _c(a, np.float32)
+    out = np.empty(a.shape, np.uint16)
+    _load().oracle_f32_to_f16_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def f16_to_f32(a) -> np.ndarray:
+    a = _c(a, np.uint16)
+    out = np.empty(a.shape, np.float32)
+    _load().oracle_f16_to_f32_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+# ---------------------------------------------------------------------- Q4_0
+def q4_0_quantize(w) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 w[N][K] -> (wq u8 [N][K/2], d fp16 bits u16 [N][K/32])."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    assert K % 32 == 0
+    wq = np.empty((N, K // 2), np.uint8)
+    d = np.empty((N, K // 32), np.uint16)
+    _load().oracle_q4_0_quantize(_ptr(w), N, K, _ptr(wq), _ptr(d))
+    return wq, d
+
+
+def q4_0_dequantize(wq, d) -> np.ndarray:
+    """(wq u8 [N][K/2], d fp16 bits [N][K/32]) -> bf16 bits u16 [N][K]."""
+    wq = _c(wq, np.uint8)
+    d = _c(d, np.uint16)
+    N, K = wq.shape[0], wq.shape[1] * 2
+    assert d.shape == (N, K // 32)
+    out = np.empty((N, K), np.uint16)
+    _load().oracle_q4_0_dequantize(_ptr(wq), _ptr(d), N, K, _ptr(out))
+    return out
+
+
+# -------------------------------------------------------------------- affine
+def affine_quantize(w, group_size: int = 64, bits: int = 4):
+    """fp32 w[N][K] -> (wq u32 [N][K*bits/32], scales bf16 bits, biases bf16 bits [N][K/group])."""
+    assert bits in (4, 8)
+    w = _c(w, np.float32)
+    N, K = w.shape
+    assert K % group_size == 0 and (K * bits) % 32 == 0
+    wq = np.empty((N, K * bits // 32), np.uint32)
+    s = np.empty((N, K // group_size), np.uint16)
+    b = np.empty((N, K // group_size), np.uint16)
+    _load().oracle_affine_quantize(_ptr(w), N, K, group_size, bits, _ptr(wq), _ptr(s), _ptr(b))
+    return wq, s, b
+
+
+def affine_dequantize(wq, scales, biases, group_size: int = 64, bits: int = 4) -> np.ndarray:
+    assert bits in (4, 8)
+    wq = _c(wq, np.uint32)
+    scales = _c(scales, np.uint16)
+    biases = _c(biases, np.uint16)
+    N = wq.shape[0]
+    K = wq.shape[1] * 32 // bits
+    assert scales.shape == (N, K // group_size) and biases.shape == scales.shape
+    out = np.empty((N, K), np.uint16)
+    _load().oracle_affine_dequantize(_ptr(wq), _ptr(scales), _ptr(biases), N, K, group_size, bits,
+                                     _ptr(out))
+    return out
+
+
+# -------------------------------------------------------------------- matmul
+def matmul_ref(x_bf16, w_bf16, rows=None, nthreads: int | None = None):
+    """float64 y[r][n] = sum_k x[rows[r]][k] * w[n][k] and a[r][n] = sum_k |x w|.
+
+    x_bf16: u16 [M][K]; w_bf16: u16 [N][K]; rows: optional 1-D int array of
+    selected rows of x.  Returns (y, a, threads_used).
+    """
+    x = _c(x_bf16, np.uint16)
+    w = _c(w_bf16, np.uint16)
+    M, K = x.shape
+    N, K2 = w.shape
+    assert K == K2
+    if rows is None:
+        r = None
+        R = M
+    else:
+        r = _c(rows, np.int64)
+        assert r.ndim == 1 and (r.size == 0 or (r.min() >= 0 and r.max() < M))
+        R = r.size
+    y = np.empty((R, N), np.float64)
+    a = np.empty((R, N), np.float64)
+    nt = nthreads or os.cpu_count() or 1
+    used = _load().oracle_matmul_ref(_ptr(x), _ptr(w), M, N, K,
+                                     _ptr(r) if r is not None else None, R,
+                                     _ptr(y), _ptr(a), nt)
+    return y, a, used
+
+
+def tolerance(a: np.ndarray) -> np.ndarray:
+    """Allowed |y_gpu - y_ref| for outputs with absolute-product sums ``a``."""
+    return 2e-3 * a + 1e-5

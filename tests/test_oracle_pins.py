@@ -1,0 +1,405 @@
+"""Pins for the CPU oracle: checks against facts fixed by the format definitions,
+by IEEE-754 and by exact arithmetic -- never against the oracle itself.
+
+The pages print no worked example, so each pin is a closed form (values that
+are exact by construction), an invariant of the quantizers, a reduction to a
+library routine (numpy / torch float conversions), or exact rational brute
+force (fractions.Fraction).  The last test plants mistakes in the oracle's
+outputs and checks that the pins notice them.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_quantized_gemm_quant_b200 import inputs
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+# --------------------------------------------------------------------------
+# helpers written from the layout statements (independent of the oracle)
+# --------------------------------------------------------------------------
+def pack_q4_0(q: np.ndarray) -> np.ndarray:
+    """q[N][K] codes in [0,15] -> bytes: byte j of a 32-block holds element j
+    (low nibble) and element j+16 (high nibble)."""
+    N, K = q.shape
+    qb = q.reshape(N, K // 32, 32).astype(np.uint8)
+    return (qb[:, :, :16] | (qb[:, :, 16:] << 4)).reshape(N, K // 2)
+
+
+def pack_affine(q: np.ndarray, bits: int) -> np.ndarray:
+    """q[N][K] -> u32 words, 32/bits codes per word, lowest bits first."""
+    N, K = q.shape
+    per = 32 // bits
+    qw = q.reshape(N, K // per, per).astype(np.uint64)
+    shifts = (np.arange(per, dtype=np.uint64) * bits)
+    return (qw << shifts).sum(axis=2).astype(np.uint32)
+
+
+def f32_from_bf16_bits(h: np.ndarray) -> np.ndarray:
+    return (h.astype(np.uint32) << 16).view(np.float32)
+
+
+def torch_bf16_bits(v32: np.ndarray) -> np.ndarray:
+    """Library rounding fp32 -> bf16 (round to nearest even)."""
+    return torch.from_numpy(np.ascontiguousarray(v32, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def np_f16_bits(v32: np.ndarray) -> np.ndarray:
+    return np.ascontiguousarray(v32, np.float32).astype(np.float16).view(np.uint16)
+
+
+# --------------------------------------------------------------------------
+# conversions: reduce to numpy / torch
+# --------------------------------------------------------------------------
+def test_f16_to_f32_exhaustive_vs_numpy():
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = oracle.f16_to_f32(h)
+    ref = h.view(np.float16).astype(np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def _interesting_f32_bits(n, seed):
+    rng = np.random.default_rng(seed)
+    u = rng.integers(0, 1 << 32, n, dtype=np.uint64).astype(np.uint32)
+    # concentrate on the fp16 range and on exact ties
+    e = rng.integers(90, 145, n // 2).astype(np.uint32)
+    m = rng.integers(0, 1 << 23, n // 2).astype(np.uint32)
+    s = rng.integers(0, 2, n // 2).astype(np.uint32)
+    near = (s << 31) | (e << 23) | m
+    tie16 = (near & ~np.uint32(0x1FFF)) | np.uint32(0x1000)      # fp16-normal ties
+    tie_bf = (near & ~np.uint32(0xFFFF)) | np.uint32(0x8000)     # bf16 ties
+    specials = np.array([0x00000000, 0x80000000, 0x7F800000, 0xFF800000, 0x477FE000, 0x477FF000,
+                         0x477FEFFF, 0x477FF001, 0x33800000, 0x33000000, 0x33000001, 0x33C00000,
+                         0x38800000, 0x387FFFFF, 0x00000001, 0x807FFFFF, 0x3F800000, 0x7F7FFFFF,
+                         0x7F7F8000, 0x7F7F7FFF], dtype=np.uint32)
+    return np.concatenate([u, near, tie16, tie_bf, specials])
+
+
+def test_f32_to_f16_vs_numpy():
+    bits = _interesting_f32_bits(400_000, 1)
+    v = bits.view(np.float32)
+    finite = np.isfinite(v) | np.isinf(v)
+    v = v[finite]
+    got = oracle.f32_to_f16(v)
+    ref = np_f16_bits(v)
+    assert np.array_equal(got, ref)
+
+
+def test_f32_to_bf16_vs_torch():
+    bits = _interesting_f32_bits(400_000, 2)
+    v = bits.view(np.float32)
+    v = v[~np.isnan(v)]
+    assert np.array_equal(oracle.f32_to_bf16(v), torch_bf16_bits(v))
+
+
+def test_bf16_to_f32_exhaustive_vs_torch():
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = oracle.bf16_to_f32(h)
+    ref = torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).to(torch.float32).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+# --------------------------------------------------------------------------
+# Q4_0
+# --------------------------------------------------------------------------
+def test_q4_0_dequant_closed_form_layout():
+    """Scales with few significant bits make every d*(q-8) exact in bf16, so the
+    expected values need no rounding; the bytes are packed from the layout
+    statement by hand, which pins nibble order, the -8 offset and the scale."""
+    rng = np.random.default_rng(3)
+    N, K = 5, 96
+    q = rng.integers(0, 16, (N, K))
+    d_vals = rng.choice([0.5, -1.5, 0.125, 3.0, -0.25, 1.0], size=(N, K // 32))
+    wq = pack_q4_0(q)
+    d16 = np_f16_bits(d_vals.astype(np.float32))
+    got = f32_from_bf16_bits(oracle.q4_0_dequantize(wq, d16))
+    expect = np.repeat(d_vals, 32, axis=1) * (q - 8)
+    assert np.array_equal(got.astype(np.float64), expect)
+
+
+def test_q4_0_dequant_specific_block():
+    # byte j = j | (15 - j) << 4: elements 0..15 are q = 0..15, elements 16..31 are q = 15..0
+    wq = np.array([[j | ((15 - j) << 4) for j in range(16)]], np.uint8)
+    d16 = np.array([[0x3800]], np.uint16)                   # 0.5
+    got = f32_from_bf16_bits(oracle.q4_0_dequantize(wq, d16))[0]
+    assert list(got[:16]) == [0.5 * (j - 8) for j in range(16)]
+    assert list(got[16:]) == [0.5 * (7 - j) for j in range(16)]
+
+
+def test_q4_0_dequant_rounding_reduces_to_library():
+    """Arbitrary finite fp16 scales (subnormals, signs) and codes: the fp32 product
+    d*(q-8) is exact (11-bit x 4-bit), so the result is the library's bf16
+    rounding of it, sign of zero included."""
+    g = inputs.generator(4)
+    N, K = 64, 256
+    wq = inputs.random_bytes((N, K // 2), g).numpy()
+    d16 = inputs.random_f16_bits((N, K // 32), g).numpy().view(np.uint16)
+    got = oracle.q4_0_dequantize(wq, d16)
+    d = np.repeat(d16.view(np.float16).astype(np.float32), 32, axis=1)
+    qb = wq.reshape(N, K // 32, 16)
+    q = np.concatenate([qb & 15, qb >> 4], axis=2).reshape(N, K).astype(np.float32)
+    exact = d * (q - np.float32(8))          # exact in fp32
+    assert np.array_equal(got, torch_bf16_bits(exact))
+
+
+def _exact_q4_0_blocks(rng, N, K):
+    """Blocks w = d*(q-8) with fp16 d whose products are exact in bf16, and at
+    least one q = 0 in every block (so the max-abs element is -8d)."""
+    q = rng.integers(1, 16, (N, K))
+    q.reshape(N, K // 32, 32)[:, :, 0] = 0
+    perm = rng.permuted(np.tile(np.arange(32), (N * K // 32, 1)), axis=1)
+    q = np.take_along_axis(q.reshape(-1, 32), perm, axis=1).reshape(N, K)
+    mant = rng.integers(0, 16, (N, K // 32))                 # 5-bit significands
+    expo = rng.integers(-12, 4, (N, K // 32))
+    sign = rng.choice([-1.0, 1.0], (N, K // 32))
+    d = sign * (1 + mant / 16.0) * np.exp2(expo)
+    w = np.repeat(d, 32, axis=1) * (q - 8)
+    return q, d, w.astype(np.float32)
+
+
+def test_q4_0_round_trip_exact():
+    rng = np.random.default_rng(5)
+    N, K = 16, 256
+    q, d, w = _exact_q4_0_blocks(rng, N, K)
+    wq, d16 = oracle.q4_0_quantize(w)
+    assert np.array_equal(d16, np_f16_bits(d.astype(np.float32)))
+    assert np.array_equal(wq, pack_q4_0(q))
+    back = f32_from_bf16_bits(oracle.q4_0_dequantize(wq, d16))
+    assert np.array_equal(back, w)
+
+
+def test_q4_0_all_zero_block():
+    w = np.zeros((2, 64), np.float32)
+    wq, d16 = oracle.q4_0_quantize(w)
+    assert np.all(wq == 0x88)
+    assert np.all((d16 & 0x7FFF) == 0)
+    out = oracle.q4_0_dequantize(wq, d16)
+    assert np.all((out & 0x7FFF) == 0)
+
+
+def test_q4_0_invariants_random():
+    g = inputs.generator(6)
+    w = inputs.weights_fp32(64, 1024, g).numpy()
+    wq, d16 = oracle.q4_0_quantize(w)
+    N, K = w.shape
+    blk = w.reshape(N, K // 32, 32)
+    qb = wq.reshape(N, K // 32, 16)
+    q = np.concatenate([qb & 15, qb >> 4], axis=2)            # element order 0..31
+    # the max-abs element (first on ties) maps to q = 0 and d = max / -8
+    idx = np.abs(blk).argmax(axis=2)
+    assert np.all(np.take_along_axis(q, idx[..., None], axis=2) == 0)
+    mx = np.take_along_axis(blk, idx[..., None], axis=2)[..., 0]
+    assert np.array_equal(d16, np_f16_bits(mx / np.float32(-8)))
+    # error bound: nearest code (half |d|) plus fp16 scale and bf16 output rounding;
+    # only an element equal to -max may clamp (error up to |d|)
+    d = d16.view(np.float16).astype(np.float64)[..., None]
+    deq = f32_from_bf16_bits(oracle.q4_0_dequantize(wq, d16)).reshape(N, K // 32, 32).astype(np.float64)
+    err = np.abs(blk - deq)
+    clamped = (q == 15) & (blk / (mx[..., None] / -8.0) > 7.5)
+    bound = np.where(clamped, 1.0, 0.5) * np.abs(d) + 8 * np.abs(d) * 2.0 ** -11 + np.abs(deq) * 2.0 ** -8
+    assert np.all(err <= bound * (1 + 1e-6))
+
+
+# --------------------------------------------------------------------------
+# affine
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("bits", [4, 8])
+def test_affine_dequant_closed_form_layout(bits):
+    rng = np.random.default_rng(7 + bits)
+    N, K, G = 3, 256, 64
+    L = (1 << bits) - 1
+    q = rng.integers(0, L + 1, (N, K))
+    s = rng.choice([0.25, 0.5, 0.0625], size=(N, K // G))      # b/s integer, q + b/s in [-48, 255]
+    b = rng.choice([-1.0, 0.0, -3.0, -0.5], size=(N, K // G))
+    wq = pack_affine(q, bits)
+    got = f32_from_bf16_bits(oracle.affine_dequantize(wq, torch_bf16_bits(s.astype(np.float32)),
+                                                      torch_bf16_bits(b.astype(np.float32)), G, bits))
+    expect = np.repeat(s, G, axis=1) * q + np.repeat(b, G, axis=1)
+    assert np.array_equal(got.astype(np.float64), expect)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_affine_dequant_rounding_reduces_to_library(bits):
+    """Random bf16 scale/bias with exponents close enough that scale*q + bias is
+    exact in fp32; the result is then the library's bf16 rounding of it."""
+    g = inputs.generator(8 + bits)
+    N, K, G = 32, 512, 64
+    L = (1 << bits) - 1
+    s16 = inputs.random_bf16_bits((N, K // G), g, 112, 116).numpy().view(np.uint16) & 0x7FFF
+    b16 = inputs.random_bf16_bits((N, K // G), g, 112, 120).numpy().view(np.uint16)
+    q = torch.randint(0, L + 1, (N, K), generator=g).numpy()
+    got = oracle.affine_dequantize(pack_affine(q, bits), s16, b16, G, bits)
+    s = np.repeat(f32_from_bf16_bits(s16), G, axis=1).astype(np.float64)
+    b = np.repeat(f32_from_bf16_bits(b16), G, axis=1).astype(np.float64)
+    exact = s * q + b
+    assert np.array_equal(exact.astype(np.float32).astype(np.float64), exact)   # exact in fp32
+    assert np.array_equal(got, torch_bf16_bits(exact.astype(np.float32)))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_affine_round_trip_exact(bits):
+    rng = np.random.default_rng(9 + bits)
+    N, K, G = 8, 256, 64
+    L = (1 << bits) - 1
+    q = rng.integers(0, L + 1, (N, K))
+    qg = q.reshape(N, K // G, G)
+    qg[:, :, 0] = 0
+    qg[:, :, 1] = L
+    e = rng.integers(-9, -3, (N, K // G)).astype(np.float64)
+    s = np.exp2(e)
+    b = -16.0 * s * rng.integers(0, 4, (N, K // G))
+    w = (np.repeat(s, G, axis=1) * q + np.repeat(b, G, axis=1)).astype(np.float32)
+    assert np.array_equal(torch_bf16_bits(w), np.ascontiguousarray(w).view(np.uint32) >> 16)  # bf16-valued
+    wq, s16, b16 = oracle.affine_quantize(w, G, bits)
+    assert np.array_equal(f32_from_bf16_bits(s16).astype(np.float64), s)
+    assert np.array_equal(f32_from_bf16_bits(b16).astype(np.float64), b)
+    assert np.array_equal(wq, pack_affine(q, bits))
+    back = f32_from_bf16_bits(oracle.affine_dequantize(wq, s16, b16, G, bits))
+    assert np.array_equal(back, w)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_affine_constant_group(bits):
+    w = np.full((2, 128), -0.375, np.float32)
+    w[1, 64:] = 0.0
+    wq, s16, b16 = oracle.affine_quantize(w, 64, bits)
+    assert np.all(s16 == 0) and np.all(wq == 0)
+    assert np.array_equal(f32_from_bf16_bits(b16), np.array([[-0.375, -0.375], [-0.375, 0.0]], np.float32))
+    back = f32_from_bf16_bits(oracle.affine_dequantize(wq, s16, b16, 64, bits))
+    assert np.array_equal(back, w)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_affine_invariants_random(bits):
+    g = inputs.generator(10 + bits)
+    N, K, G = 48, 1024, 64
+    L = (1 << bits) - 1
+    w = inputs.weights_bf16_valued(N, K, g).numpy()
+    wq, s16, b16 = oracle.affine_quantize(w, G, bits)
+    per = 32 // bits
+    q = ((wq[:, :, None] >> (np.arange(per, dtype=np.uint32) * bits)) & L).reshape(N, K)
+    wg = w.reshape(N, K // G, G)
+    qg = q.reshape(N, K // G, G)
+    # min maps to 0, max to L; scale = (max-min)/L and bias = min
+    assert np.all(np.take_along_axis(qg, wg.argmin(axis=2)[..., None], axis=2) == 0)
+    assert np.array_equal(b16, torch_bf16_bits(wg.min(axis=2)))
+    s_exact = (wg.max(axis=2) - wg.min(axis=2)) / np.float32(L)
+    assert np.array_equal(s16, torch_bf16_bits(s_exact))
+    # the max maps to L, except that a bf16 scale rounded above (max-min)/L may
+    # bring it down by one code (possible only when L is large next to 2^8)
+    q_max = np.take_along_axis(qg, wg.argmax(axis=2)[..., None], axis=2)[..., 0]
+    s_stored = f32_from_bf16_bits(s16)
+    assert np.all(q_max[s_stored <= s_exact] == L)
+    assert np.all(q_max >= L - 1)
+    if bits == 4:
+        assert np.all(q_max == L)
+    s = f32_from_bf16_bits(s16).astype(np.float64)[..., None]
+    deq = f32_from_bf16_bits(oracle.affine_dequantize(wq, s16, b16, G, bits)).reshape(N, K // G, G)
+    err = np.abs(wg.astype(np.float64) - deq)
+    bound = s * (0.5 + L * 2.0 ** -8) + np.abs(deq) * 2.0 ** -8
+    assert np.all(err <= bound * (1 + 1e-6))
+
+
+# --------------------------------------------------------------------------
+# matmul: exact rational brute force
+# --------------------------------------------------------------------------
+def _bf16_frac(h):
+    return Fraction(float(f32_from_bf16_bits(np.array([h], np.uint16))[0]))
+
+
+def test_matmul_ref_fraction_bruteforce():
+    g = inputs.generator(11)
+    M, N, K = 3, 5, 40
+    x = inputs.activations_bf16(M, K, g).view(torch.int16).numpy().view(np.uint16)
+    w = inputs.activations_bf16(N, K, g).view(torch.int16).numpy().view(np.uint16)
+    y, a, _ = oracle.matmul_ref(x, w, nthreads=2)
+    for m in range(M):
+        for n in range(N):
+            prods = [_bf16_frac(x[m, k]) * _bf16_frac(w[n, k]) for k in range(K)]
+            exact = sum(prods, Fraction(0))
+            exact_abs = sum((abs(p) for p in prods), Fraction(0))
+            assert abs(Fraction(y[m, n]) - exact) <= exact_abs * K * Fraction(1, 2 ** 52)
+            assert abs(Fraction(a[m, n]) - exact_abs) <= exact_abs * K * Fraction(1, 2 ** 52)
+
+
+def test_matmul_ref_one_hot_and_rows():
+    g = inputs.generator(12)
+    N, K = 7, 64
+    w = inputs.activations_bf16(N, K, g).view(torch.int16).numpy().view(np.uint16)
+    x = np.zeros((K, K), np.uint16)
+    x[np.arange(K), np.arange(K)] = 0x3F80                        # bf16 1.0
+    y, a, _ = oracle.matmul_ref(x, w)
+    assert np.array_equal(y, f32_from_bf16_bits(w).T.astype(np.float64))
+    assert np.array_equal(a, np.abs(y))
+    rows = np.array([5, 0, 63])
+    y2, _, _ = oracle.matmul_ref(x, w, rows=rows, nthreads=3)
+    assert np.array_equal(y2, y[rows])
+
+
+def test_quantized_chain_fraction_bruteforce():
+    """x . dequant(W)^T for a Q4_0 and an affine-8 weight, exact rationals."""
+    rng = np.random.default_rng(13)
+    M, N, K = 2, 3, 64
+    q = rng.integers(0, 16, (N, K))
+    d = np.array([[0.5, -0.25], [1.0, 0.125], [-2.0, 0.75]])
+    wq = pack_q4_0(q)
+    x = torch.randn(M, K, generator=inputs.generator(13)).to(torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    wb = oracle.q4_0_dequantize(wq, np_f16_bits(d.astype(np.float32)))
+    y, _, _ = oracle.matmul_ref(xb, wb)
+    for m in range(M):
+        for n in range(N):
+            exact = sum((Fraction(float(x[m, k])) * Fraction(d[n, k // 32]) * (int(q[n, k]) - 8)
+                         for k in range(K)), Fraction(0))
+            assert abs(Fraction(y[m, n]) - exact) <= Fraction(1, 2 ** 40)
+    q8 = rng.integers(0, 256, (N, K))
+    s = np.array([[0.0078125], [0.25], [2.0 ** -10]])
+    b = np.array([[-1.0], [0.5], [-0.125]])
+    w8 = oracle.affine_dequantize(pack_affine(q8, 8), torch_bf16_bits(s.astype(np.float32)),
+                                  torch_bf16_bits(b.astype(np.float32)), 64, 8)
+    y8, _, _ = oracle.matmul_ref(xb, w8)
+    for m in range(M):
+        for n in range(N):
+            exact = sum((Fraction(float(x[m, k])) * (Fraction(s[n, 0]) * int(q8[n, k]) + Fraction(b[n, 0]))
+                         for k in range(K)), Fraction(0))
+            assert abs(Fraction(y8[m, n]) - exact) <= Fraction(1, 2 ** 36)
+
+
+# --------------------------------------------------------------------------
+# planted mistakes: the pins above must notice each of these
+# --------------------------------------------------------------------------
+def test_pins_catch_planted_mistakes():
+    rng = np.random.default_rng(14)
+    N, K = 4, 64
+    q = rng.integers(0, 16, (N, K))
+    d = np.full((N, K // 32), 0.5)
+    wq = pack_q4_0(q)
+    d16 = np_f16_bits(d.astype(np.float32))
+    expect = np.repeat(d, 32, axis=1) * (q - 8)
+
+    def ok(deq_fn):
+        return np.array_equal(f32_from_bf16_bits(deq_fn(wq, d16)).astype(np.float64), expect)
+
+    assert ok(oracle.q4_0_dequantize)
+    swapped = lambda a, s: oracle.q4_0_dequantize(((a & 15) << 4) | (a >> 4), s)            # nibble order
+    plus8 = lambda a, s: oracle.f32_to_bf16(-f32_from_bf16_bits(oracle.q4_0_dequantize(a, s)))  # sign of offset
+    interleaved = lambda a, s: oracle.q4_0_dequantize(a, s).reshape(N, -1, 2, 16).transpose(0, 1, 3, 2).reshape(N, K)
+    for bad in (swapped, plus8, interleaved):
+        assert not ok(bad)
+    # matmul transposed operand / dropped term
+    g = inputs.generator(15)
+    x = inputs.activations_bf16(3, 32, g).view(torch.int16).numpy().view(np.uint16)
+    w = inputs.activations_bf16(3, 32, g).view(torch.int16).numpy().view(np.uint16)
+    y, _, _ = oracle.matmul_ref(x, w)
+    yt, _, _ = oracle.matmul_ref(w, x)
+    assert not np.allclose(y, yt)
+    ydrop, _, _ = oracle.matmul_ref(x[:, :31], w[:, :31])
+    assert not np.allclose(y, ydrop)
