@@ -1,0 +1,197 @@
+"""Thin Python binding of libbqgemm (include/bqgemm.h): argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; PyTorch
+provides device memory and the current stream.  There is no CPU fallback: the
+first call raises if libbqgemm.so is missing or the device is not sm_100.
+
+Names follow the C ABI: q4_0_dequantize, affine_dequantize, quant_matmul,
+quant_matmul_ex, bf16_matmul, q4_0_quantize, affine_quantize,
+quant_matmul_select_path, quant_matmul_workspace_size, bq_device_status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbqgemm.so")
+
+BQ_OK = 0
+STATUS = {0: "BQ_OK", 1: "BQ_ERR_NULL", 2: "BQ_ERR_SHAPE", 3: "BQ_ERR_UNSUPPORTED", 4: "BQ_ERR_ALIGN",
+          5: "BQ_ERR_CUDA", 6: "BQ_ERR_TIMEOUT", 7: "BQ_ERR_WORKSPACE", 8: "BQ_ERR_DEVICE"}
+PATH_AUTO, PATH_GEMV, PATH_TC_FUSED, PATH_DEQUANT_GEMM = 0, 1, 2, 3
+PATHS = {"auto": PATH_AUTO, "gemv": PATH_GEMV, "tc_fused": PATH_TC_FUSED, "dequant_gemm": PATH_DEQUANT_GEMM}
+
+_lib = None
+
+
+class BqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libbqgemm.so (loaded on first use; raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libbqgemm.so not found at {LIB_PATH}; build it with "
+                           "`python -c 'import __graft_entry__ as g; g.build()'` (no CPU fallback exists)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    sigs = {
+        "q4_0_dequantize": [P, P, P, I64, I64, P],
+        "affine_dequantize": [P, P, P, P, I64, I64, I, I, P],
+        "quant_matmul": [P, P, P, P, P, I64, I64, I64, I, I, I, P],
+        "quant_matmul_ex": [P, P, P, P, P, I64, I64, I64, I, I, I, I, P, SZ, P],
+        "quant_matmul_workspace_size": [I64, I64, I64, I, I, I],
+        "quant_matmul_select_path": [I64, I64, I64, I, I],
+        "bf16_matmul": [P, P, P, I64, I64, I64, P],
+        "q4_0_quantize": [P, P, P, I64, I64, P],
+        "affine_quantize": [P, P, P, P, I64, I64, I, I, P],
+        "bq_device_status": [],
+        "bq_status_string": [I],
+        "bq_version": [],
+    }
+    for name, args in sigs.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = I
+    L.quant_matmul_workspace_size.restype = SZ
+    L.bq_status_string.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def _check(status: int, where: str) -> None:
+    if status != BQ_OK:
+        raise BqError(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _bits16(t: torch.Tensor) -> torch.Tensor:
+    """bf16 / fp16 / int16 tensors are passed by their 16-bit patterns."""
+    if t.dtype not in (torch.bfloat16, torch.float16, torch.int16, torch.uint16):
+        raise TypeError(f"expected a 16-bit tensor, got {t.dtype}")
+    return t
+
+
+# ----------------------------------------------------------------- dequantize
+def q4_0_dequantize(wq: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    """wq u8 [N][K/2], scales fp16 [N][K/32] -> bf16 [N][K]."""
+    N, K = wq.shape[0], wq.shape[1] * 2
+    if out is None:
+        out = torch.empty(N, K, dtype=torch.bfloat16, device=wq.device)
+    _check(lib().q4_0_dequantize(_ptr(wq), _ptr(_bits16(scales)), _ptr(out), N, K, _stream(stream)),
+           "q4_0_dequantize")
+    return out
+
+
+def affine_dequantize(wq: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor, group_size: int = 64,
+                      bits: int = 4, out: torch.Tensor | None = None, stream=None):
+    """wq u32 (int32) [N][K*bits/32], scales/biases bf16 [N][K/group_size] -> bf16 [N][K]."""
+    N, K = wq.shape[0], wq.shape[1] * 32 // bits
+    if out is None:
+        out = torch.empty(N, K, dtype=torch.bfloat16, device=wq.device)
+    _check(lib().affine_dequantize(_ptr(wq), _ptr(_bits16(scales)), _ptr(_bits16(biases)), _ptr(out), N, K,
+                                   group_size, bits, _stream(stream)), "affine_dequantize")
+    return out
+
+
+# --------------------------------------------------------------------- matmul
+def _k_of(wq: torch.Tensor, biases, bits: int) -> int:
+    if biases is None:
+        return wq.shape[1] * 2
+    return wq.shape[1] * 32 // bits
+
+
+def quant_matmul(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor | None = None,
+                 group_size: int = 32, bits: int = 4, transpose: bool = True, out: torch.Tensor | None = None,
+                 stream=None):
+    """y[M][N] = x[M][K] . dequant(W)[N][K]^T (biases None: Q4_0)."""
+    return quant_matmul_ex(x, wq, scales, biases, group_size, bits, transpose, "auto", out=out, stream=stream)
+
+
+def quant_matmul_ex(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor | None = None,
+                    group_size: int = 32, bits: int = 4, transpose: bool = True, path="auto",
+                    workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None):
+    M, K = x.shape
+    N = wq.shape[0]
+    if K != _k_of(wq, biases, bits):
+        raise ValueError(f"K mismatch: x has {K}, weights hold {_k_of(wq, biases, bits)}")
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    p = PATHS[path] if isinstance(path, str) else int(path)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    fn = lib().quant_matmul_ex if (p != PATH_AUTO or workspace is not None) else None
+    if fn is None:
+        st = lib().quant_matmul(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(out), M, N, K, group_size, bits,
+                                1 if transpose else 0, _stream(stream))
+    else:
+        st = fn(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(out), M, N, K, group_size, bits,
+                1 if transpose else 0, p, _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "quant_matmul")
+    return out
+
+
+def quant_matmul_select_path(M: int, N: int, K: int, group_size: int, bits: int) -> int:
+    return lib().quant_matmul_select_path(M, N, K, group_size, bits)
+
+
+def quant_matmul_workspace_size(M: int, N: int, K: int, group_size: int, bits: int, path="auto") -> int:
+    p = PATHS[path] if isinstance(path, str) else int(path)
+    return lib().quant_matmul_workspace_size(M, N, K, group_size, bits, p)
+
+
+def bf16_matmul(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    """y[M][N] = x[M][K] . w[N][K]^T, bf16 in/out, fp32 accumulation (tcgen05)."""
+    M, K = x.shape
+    N = w.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _check(lib().bf16_matmul(_ptr(x), _ptr(w), _ptr(out), M, N, K, _stream(stream)), "bf16_matmul")
+    return out
+
+
+# ------------------------------------------------------------------- quantize
+def q4_0_quantize(w: torch.Tensor, stream=None):
+    """fp32 w [N][K] -> (wq u8 [N][K/2], scales fp16 [N][K/32])."""
+    N, K = w.shape
+    wq = torch.empty(N, K // 2, dtype=torch.uint8, device=w.device)
+    d = torch.empty(N, K // 32, dtype=torch.float16, device=w.device)
+    _check(lib().q4_0_quantize(_ptr(w), _ptr(wq), _ptr(d), N, K, _stream(stream)), "q4_0_quantize")
+    return wq, d
+
+
+def affine_quantize(w: torch.Tensor, group_size: int = 64, bits: int = 4, stream=None):
+    """fp32 w [N][K] -> (wq int32 [N][K*bits/32], scales bf16, biases bf16 [N][K/group_size])."""
+    N, K = w.shape
+    wq = torch.empty(N, K * bits // 32, dtype=torch.int32, device=w.device)
+    s = torch.empty(N, K // group_size, dtype=torch.bfloat16, device=w.device)
+    b = torch.empty(N, K // group_size, dtype=torch.bfloat16, device=w.device)
+    _check(lib().affine_quantize(_ptr(w), _ptr(wq), _ptr(s), _ptr(b), N, K, group_size, bits, _stream(stream)),
+           "affine_quantize")
+    return wq, s, b
+
+
+def bq_device_status() -> int:
+    """Synchronize the device and return (and clear) the library's device error status."""
+    return lib().bq_device_status()

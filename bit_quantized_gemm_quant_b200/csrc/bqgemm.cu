@@ -1,0 +1,507 @@
+// bqgemm.cu -- host side of libbqgemm: argument checks, the M-threshold
+// dispatcher, TMA descriptor creation, kernel launches and the C ABI declared
+// in include/bqgemm.h.  Built as one translation unit with the kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "bqgemm.h"
+#include "common.cuh"
+#include "dequant.cuh"
+#include "gemv.cuh"
+#include "tc_gemm.cuh"
+
+namespace bq {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kGemvMaxM = 32;
+
+// ------------------------------------------------------------------ device info
+struct DeviceInfo {
+    bool ok = false;
+    int num_sms = 0;
+    int max_smem_optin = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+bool g_dev_init[kMaxDevices] = {};
+
+bq_status current_device(int* dev_out, DeviceInfo* info_out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_dev_init[dev]) {
+        DeviceInfo di;
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return BQ_ERR_CUDA;
+        di.ok = (major == 10 && minor == 0);
+        g_dev[dev] = di;
+        g_dev_init[dev] = true;
+    }
+    if (!g_dev[dev].ok) return BQ_ERR_DEVICE;
+    *dev_out = dev;
+    *info_out = g_dev[dev];
+    return BQ_OK;
+}
+
+// ------------------------------------------------------------------ checks
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+enum class WFmt { Q4_0, AFF4, AFF8 };
+
+// Format and shape checks shared by quant_matmul and its helpers (host only).
+bq_status check_format(const void* biases, int64_t N, int64_t K, int group_size, int bits, WFmt* fmt)
+{
+    if (N < 0 || K < 0) return BQ_ERR_SHAPE;
+    if (biases == nullptr) {
+        if (bits != 4 || group_size != 32) return BQ_ERR_UNSUPPORTED;
+        if (K % 32 != 0) return BQ_ERR_SHAPE;
+        *fmt = WFmt::Q4_0;
+    } else {
+        if (bits != 4 && bits != 8) return BQ_ERR_UNSUPPORTED;
+        if (group_size != 64) return BQ_ERR_UNSUPPORTED;
+        if (K % group_size != 0) return BQ_ERR_SHAPE;
+        *fmt = bits == 4 ? WFmt::AFF4 : WFmt::AFF8;
+    }
+    return BQ_OK;
+}
+
+// check_format selects the format from the biases pointer; these stand in for
+// it where only the format matters (no dereference).
+const void* const kAffineTag = reinterpret_cast<const void*>(uintptr_t(16));
+
+// Without a biases pointer the format is inferred: group_size 32 with 4 bits is
+// Q4_0, anything else is affine.
+const void* format_tag(int group_size, int bits)
+{
+    return (group_size == 32 && bits == 4) ? nullptr : kAffineTag;
+}
+
+bq_status launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+int grid_for(int64_t items, int threads, const DeviceInfo& di)
+{
+    int64_t g = (items + threads - 1) / threads;
+    g = std::min<int64_t>(g, (int64_t)di.num_sms * 16);
+    return (int)std::max<int64_t>(g, 1);
+}
+
+// ------------------------------------------------------------------ env config
+struct DispatchCfg {
+    int tc_min_m = kGemvMaxM + 1;
+    int64_t pair_min_m = 0;   // 0: never
+};
+
+const DispatchCfg& dispatch_cfg()
+{
+    static DispatchCfg cfg = [] {
+        DispatchCfg c;
+        if (const char* v = std::getenv("BQ_TC_MIN_M")) {
+            long t = std::strtol(v, nullptr, 10);
+            c.tc_min_m = (int)std::min<long>(std::max<long>(t, 1), kGemvMaxM + 1);
+        }
+        if (const char* v = std::getenv("BQ_PAIR_MIN_M")) {
+            long long t = std::strtoll(v, nullptr, 10);
+            c.pair_min_m = t > 0 ? t : 0;
+        }
+        return c;
+    }();
+    return cfg;
+}
+
+int select_path(int64_t M, int64_t K, WFmt)
+{
+    const DispatchCfg& c = dispatch_cfg();
+    if (M < c.tc_min_m) return BQ_PATH_GEMV;
+    if (c.pair_min_m > 0 && M >= c.pair_min_m) return BQ_PATH_DEQUANT_GEMM;
+    return (K % 64 == 0) ? BQ_PATH_TC_FUSED : BQ_PATH_DEQUANT_GEMM;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// Row-major 2-D [rows][cols] tensor, tile box [box_rows][box_cols].
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* ptr, int64_t rows, int64_t cols,
+              int box_rows, int box_cols, CUtensorMapSwizzle sw)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t gstride[1] = {(cuuint64_t)(cols * elem_bytes)};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estride[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(ptr), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ tensor-core GEMM
+// Token tile bn (MMA N): minimise waves * (bn + per-tile overhead) over the SMs.
+int choose_bn(int64_t M, int64_t N, int num_sms)
+{
+    const int64_t ntiles = (N + 127) / 128;
+    int best_bn = 16;
+    int64_t best_cost = INT64_MAX;
+    for (int bn = 16; bn <= 256; bn += 16) {
+        const int64_t tiles = ((M + bn - 1) / bn) * ntiles;
+        const int64_t waves = (tiles + num_sms - 1) / num_sms;
+        const int64_t cost = waves * (bn + 32);
+        if (cost < best_cost || (cost == best_cost && bn > best_bn)) {
+            best_cost = cost;
+            best_bn = bn;
+        }
+        if (bn >= M) break;   // larger tiles only add padding
+    }
+    return best_bn;
+}
+
+template <int MODE>
+bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void* a_src, const uint16_t* scales,
+                    const uint16_t* biases, uint16_t* y, int64_t M, int64_t N, int64_t K, cudaStream_t st)
+{
+    using C = TcCfg<MODE>;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return BQ_ERR_SHAPE;
+    const int bn = choose_bn(M, N, di.num_sms);
+    const uint32_t stage = tc_stage_bytes(MODE, bn);
+    const int budget = di.max_smem_optin - 1024 - 256;
+    const int stages = std::min<int>(8, budget / (int)stage);
+    if (stages < 2) return BQ_ERR_UNSUPPORTED;
+    const size_t smem = 1024 + (size_t)stages * stage + 256;
+
+    CUtensorMap tm_x, tm_a;
+    if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, M, K, bn, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BQ_ERR_CUDA;
+    bool ok;
+    if (MODE == kModeBF16)
+        ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a_src, N, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a_src, N, K * (MODE == kModeAff8 ? 1 : 2) / 2, 128,
+                      C::kCodeBytesPerRow, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return BQ_ERR_CUDA;
+
+    static bool attr_done[kMaxDevices] = {};
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 di.max_smem_optin) != cudaSuccess)
+            return BQ_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    TcParams p;
+    p.scales = scales;
+    p.biases = biases;
+    p.y = y;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.bn = bn;
+    p.stages = stages;
+    int cols = 32;
+    while (cols < bn) cols <<= 1;
+    p.tmem_cols = cols;
+    dim3 grid((unsigned)((M + bn - 1) / bn), (unsigned)((N + 127) / 128));
+    if (grid.y > 65535u) return BQ_ERR_SHAPE;
+    tc_gemm_kernel<MODE><<<grid, C::kThreads, smem, st>>>(tm_x, tm_a, p);
+    return launch_status();
+}
+
+// ------------------------------------------------------------------ GEMV
+template <Fmt F, int NT, int RT, int KS>
+bq_status launch_gemv_cfg(const uint16_t* x, const void* wq, const uint16_t* s, const uint16_t* b, uint16_t* y,
+                          int64_t M, int64_t N, int64_t K, int group_size, cudaStream_t st)
+{
+    const int64_t rows_per_cta = 16 * RT;
+    const int64_t grid = (N + rows_per_cta - 1) / rows_per_cta;
+    if (grid > INT32_MAX) return BQ_ERR_SHAPE;
+    gemv_kernel<F, NT, RT, KS><<<(unsigned)grid, 32 * KS, 0, st>>>(
+        x, reinterpret_cast<const uint8_t*>(wq), s, b, y, (int)M, (int)N, (int)K, group_size);
+    return launch_status();
+}
+
+template <Fmt F>
+bq_status launch_gemv(const uint16_t* x, const void* wq, const uint16_t* s, const uint16_t* b, uint16_t* y,
+                      int64_t M, int64_t N, int64_t K, int group_size, cudaStream_t st)
+{
+    if (N > INT32_MAX || K > INT32_MAX) return BQ_ERR_SHAPE;
+    if (M <= 8) return launch_gemv_cfg<F, 1, 1, 8>(x, wq, s, b, y, M, N, K, group_size, st);
+    if (M <= 16) return launch_gemv_cfg<F, 2, 1, 8>(x, wq, s, b, y, M, N, K, group_size, st);
+    return launch_gemv_cfg<F, 4, 2, 8>(x, wq, s, b, y, M, N, K, group_size, st);
+}
+
+// ------------------------------------------------------------------ library workspace
+struct Workspace {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+};
+Workspace g_ws[kMaxDevices];
+
+bq_status library_workspace(int dev, size_t need, void** out)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace& w = g_ws[dev];
+    if (w.bytes < need) {
+        if (w.ptr) cudaFree(w.ptr);
+        w.ptr = nullptr;
+        w.bytes = 0;
+        if (cudaMalloc(&w.ptr, need) != cudaSuccess) {
+            w.ptr = nullptr;
+            return BQ_ERR_CUDA;
+        }
+        w.bytes = need;
+    }
+    *out = w.ptr;
+    return BQ_OK;
+}
+
+size_t workspace_for(int path, int64_t N, int64_t K)
+{
+    return path == BQ_PATH_DEQUANT_GEMM ? (size_t)N * (size_t)K * 2u : 0u;
+}
+
+bq_status dequant_any(WFmt fmt, const void* wq, const void* scales, const void* biases, uint16_t* out, int64_t N,
+                      int64_t K, int group_size, const DeviceInfo& di, cudaStream_t st)
+{
+    if (fmt == WFmt::Q4_0) {
+        const int64_t nb = N * (K / 32);
+        q4_0_dequant_kernel<<<grid_for(nb, 256, di), 256, 0, st>>>(
+            reinterpret_cast<const uint8_t*>(wq), reinterpret_cast<const uint16_t*>(scales), out, nb);
+    } else if (fmt == WFmt::AFF4) {
+        const int64_t nc = N * (K / 32);
+        affine_dequant_kernel<4><<<grid_for(nc, 256, di), 256, 0, st>>>(
+            reinterpret_cast<const uint32_t*>(wq), reinterpret_cast<const uint16_t*>(scales),
+            reinterpret_cast<const uint16_t*>(biases), out, nc, K, group_size);
+    } else {
+        const int64_t nc = N * (K / 16);
+        affine_dequant_kernel<8><<<grid_for(nc, 256, di), 256, 0, st>>>(
+            reinterpret_cast<const uint32_t*>(wq), reinterpret_cast<const uint16_t*>(scales),
+            reinterpret_cast<const uint16_t*>(biases), out, nc, K, group_size);
+    }
+    return launch_status();
+}
+
+bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, const void* biases, uint16_t* y,
+                      int64_t M, int64_t N, int64_t K, int group_size, int bits, int transpose, int path,
+                      void* workspace, size_t workspace_bytes, cudaStream_t st)
+{
+    if (transpose != 1) return BQ_ERR_UNSUPPORTED;
+    if (path < BQ_PATH_AUTO || path > BQ_PATH_DEQUANT_GEMM) return BQ_ERR_UNSUPPORTED;
+    if (M < 0) return BQ_ERR_SHAPE;
+    WFmt fmt;
+    bq_status s = check_format(biases, N, K, group_size, bits, &fmt);
+    if (s != BQ_OK) return s;
+    if (!x || !wq || !scales || !y) return BQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(wq) || !aligned16(scales) || !aligned16(y) || (biases && !aligned16(biases)) ||
+        (workspace && !aligned16(workspace)))
+        return BQ_ERR_ALIGN;
+    if (path == BQ_PATH_AUTO) path = select_path(M, K, fmt);
+    if (path == BQ_PATH_GEMV && M > kGemvMaxM) return BQ_ERR_UNSUPPORTED;
+    if (path == BQ_PATH_TC_FUSED && K % 64 != 0) return BQ_ERR_UNSUPPORTED;
+    const size_t need = workspace_for(path, N, K);
+    if (workspace && workspace_bytes < need) return BQ_ERR_WORKSPACE;
+
+    int dev;
+    DeviceInfo di;
+    if ((s = current_device(&dev, &di)) != BQ_OK) return s;
+    if (M == 0 || N == 0) return BQ_OK;
+    if (K == 0) return cudaMemsetAsync(y, 0, (size_t)M * (size_t)N * 2u, st) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+
+    const uint16_t* sc = reinterpret_cast<const uint16_t*>(scales);
+    const uint16_t* bi = reinterpret_cast<const uint16_t*>(biases);
+    switch (path) {
+    case BQ_PATH_GEMV:
+        if (fmt == WFmt::Q4_0) return launch_gemv<Fmt::Q4_0>(x, wq, sc, bi, y, M, N, K, group_size, st);
+        if (fmt == WFmt::AFF4) return launch_gemv<Fmt::AFF4>(x, wq, sc, bi, y, M, N, K, group_size, st);
+        return launch_gemv<Fmt::AFF8>(x, wq, sc, bi, y, M, N, K, group_size, st);
+    case BQ_PATH_TC_FUSED:
+        if (fmt == WFmt::Q4_0) return launch_tc<kModeQ4_0>(di, dev, x, wq, sc, bi, y, M, N, K, st);
+        if (fmt == WFmt::AFF4) return launch_tc<kModeAff4>(di, dev, x, wq, sc, bi, y, M, N, K, st);
+        return launch_tc<kModeAff8>(di, dev, x, wq, sc, bi, y, M, N, K, st);
+    default: {
+        void* ws = workspace;
+        if (!ws && (s = library_workspace(dev, need, &ws)) != BQ_OK) return s;
+        uint16_t* wb = reinterpret_cast<uint16_t*>(ws);
+        if ((s = dequant_any(fmt, wq, scales, biases, wb, N, K, group_size, di, st)) != BQ_OK) return s;
+        return launch_tc<kModeBF16>(di, dev, x, wb, nullptr, nullptr, y, M, N, K, st);
+    }
+    }
+}
+
+}  // namespace
+}  // namespace bq
+
+using namespace bq;
+
+extern "C" {
+
+bq_status q4_0_dequantize(const uint8_t* wq, const uint16_t* scales_f16, uint16_t* out_bf16, int64_t N, int64_t K,
+                          bq_stream_t stream)
+{
+    if (N < 0 || K < 0 || K % 32 != 0) return BQ_ERR_SHAPE;
+    if (!wq || !scales_f16 || !out_bf16) return BQ_ERR_NULL;
+    if (!aligned16(wq) || !aligned16(scales_f16) || !aligned16(out_bf16)) return BQ_ERR_ALIGN;
+    int dev;
+    DeviceInfo di;
+    bq_status s = current_device(&dev, &di);
+    if (s != BQ_OK) return s;
+    if (N == 0 || K == 0) return BQ_OK;
+    return dequant_any(WFmt::Q4_0, wq, scales_f16, nullptr, out_bf16, N, K, 32, di, (cudaStream_t)stream);
+}
+
+bq_status affine_dequantize(const uint32_t* wq, const uint16_t* scales_bf16, const uint16_t* biases_bf16,
+                            uint16_t* out_bf16, int64_t N, int64_t K, int group_size, int bits, bq_stream_t stream)
+{
+    WFmt fmt;
+    bq_status s = check_format(kAffineTag, N, K, group_size, bits, &fmt);
+    if (s != BQ_OK) return s;
+    if (!wq || !scales_bf16 || !biases_bf16 || !out_bf16) return BQ_ERR_NULL;
+    if (!aligned16(wq) || !aligned16(scales_bf16) || !aligned16(biases_bf16) || !aligned16(out_bf16))
+        return BQ_ERR_ALIGN;
+    int dev;
+    DeviceInfo di;
+    if ((s = current_device(&dev, &di)) != BQ_OK) return s;
+    if (N == 0 || K == 0) return BQ_OK;
+    return dequant_any(fmt, wq, scales_bf16, biases_bf16, out_bf16, N, K, group_size, di, (cudaStream_t)stream);
+}
+
+bq_status quant_matmul(const uint16_t* x_bf16, const void* wq, const void* scales, const void* biases,
+                       uint16_t* y_bf16, int64_t M, int64_t N, int64_t K, int group_size, int bits, int transpose,
+                       bq_stream_t stream)
+{
+    return matmul_impl(x_bf16, wq, scales, biases, y_bf16, M, N, K, group_size, bits, transpose, BQ_PATH_AUTO,
+                       nullptr, 0, (cudaStream_t)stream);
+}
+
+bq_status quant_matmul_ex(const uint16_t* x_bf16, const void* wq, const void* scales, const void* biases,
+                          uint16_t* y_bf16, int64_t M, int64_t N, int64_t K, int group_size, int bits, int transpose,
+                          int path, void* workspace, size_t workspace_bytes, bq_stream_t stream)
+{
+    return matmul_impl(x_bf16, wq, scales, biases, y_bf16, M, N, K, group_size, bits, transpose, path, workspace,
+                       workspace_bytes, (cudaStream_t)stream);
+}
+
+size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int group_size, int bits, int path)
+{
+    WFmt fmt;
+    if (M < 0 || check_format(format_tag(group_size, bits), N, K, group_size, bits, &fmt) != BQ_OK) return 0;
+    if (path == BQ_PATH_AUTO) path = select_path(M, K, fmt);
+    return workspace_for(path, N, K);
+}
+
+int quant_matmul_select_path(int64_t M, int64_t N, int64_t K, int group_size, int bits)
+{
+    WFmt fmt;
+    if (M < 0 || check_format(format_tag(group_size, bits), N, K, group_size, bits, &fmt) != BQ_OK) return -1;
+    return select_path(M, K, fmt);
+}
+
+bq_status bf16_matmul(const uint16_t* x_bf16, const uint16_t* w_bf16, uint16_t* y_bf16, int64_t M, int64_t N,
+                      int64_t K, bq_stream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0 || K % 8 != 0) return BQ_ERR_SHAPE;
+    if (!x_bf16 || !w_bf16 || !y_bf16) return BQ_ERR_NULL;
+    if (!aligned16(x_bf16) || !aligned16(w_bf16) || !aligned16(y_bf16)) return BQ_ERR_ALIGN;
+    int dev;
+    DeviceInfo di;
+    bq_status s = current_device(&dev, &di);
+    if (s != BQ_OK) return s;
+    if (M == 0 || N == 0) return BQ_OK;
+    if (K == 0)
+        return cudaMemsetAsync(y_bf16, 0, (size_t)M * N * 2u, (cudaStream_t)stream) == cudaSuccess ? BQ_OK
+                                                                                                  : BQ_ERR_CUDA;
+    return launch_tc<kModeBF16>(di, dev, x_bf16, w_bf16, nullptr, nullptr, y_bf16, M, N, K, (cudaStream_t)stream);
+}
+
+bq_status q4_0_quantize(const float* w, uint8_t* wq, uint16_t* scales_f16, int64_t N, int64_t K, bq_stream_t stream)
+{
+    if (N < 0 || K < 0 || K % 32 != 0) return BQ_ERR_SHAPE;
+    if (!w || !wq || !scales_f16) return BQ_ERR_NULL;
+    if (!aligned16(w) || !aligned16(wq) || !aligned16(scales_f16)) return BQ_ERR_ALIGN;
+    int dev;
+    DeviceInfo di;
+    bq_status s = current_device(&dev, &di);
+    if (s != BQ_OK) return s;
+    const int64_t nb = N * (K / 32);
+    if (nb == 0) return BQ_OK;
+    q4_0_quant_kernel<<<grid_for(nb, 256, di), 256, 0, (cudaStream_t)stream>>>(w, wq, scales_f16, nb);
+    return launch_status();
+}
+
+bq_status affine_quantize(const float* w, uint32_t* wq, uint16_t* scales_bf16, uint16_t* biases_bf16, int64_t N,
+                          int64_t K, int group_size, int bits, bq_stream_t stream)
+{
+    WFmt fmt;
+    bq_status s = check_format(kAffineTag, N, K, group_size, bits, &fmt);
+    if (s != BQ_OK) return s;
+    if (!w || !wq || !scales_bf16 || !biases_bf16) return BQ_ERR_NULL;
+    if (!aligned16(w) || !aligned16(wq) || !aligned16(scales_bf16) || !aligned16(biases_bf16)) return BQ_ERR_ALIGN;
+    int dev;
+    DeviceInfo di;
+    if ((s = current_device(&dev, &di)) != BQ_OK) return s;
+    const int64_t ng = N * (K / group_size);
+    if (ng == 0) return BQ_OK;
+    if (bits == 4)
+        affine_quant_kernel<4><<<grid_for(ng, 256, di), 256, 0, (cudaStream_t)stream>>>(w, wq, scales_bf16,
+                                                                                         biases_bf16, ng, group_size);
+    else
+        affine_quant_kernel<8><<<grid_for(ng, 256, di), 256, 0, (cudaStream_t)stream>>>(w, wq, scales_bf16,
+                                                                                         biases_bf16, ng, group_size);
+    return launch_status();
+}
+
+bq_status bq_device_status(void)
+{
+    if (cudaDeviceSynchronize() != cudaSuccess) return BQ_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return BQ_ERR_CUDA;
+    if (v == 0) return BQ_OK;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return BQ_ERR_CUDA;
+    return BQ_ERR_TIMEOUT;
+}
+
+const char* bq_status_string(int status)
+{
+    switch (status) {
+    case BQ_OK: return "BQ_OK";
+    case BQ_ERR_NULL: return "BQ_ERR_NULL: a required pointer is NULL";
+    case BQ_ERR_SHAPE: return "BQ_ERR_SHAPE: invalid size or K not a multiple of the block/group";
+    case BQ_ERR_UNSUPPORTED: return "BQ_ERR_UNSUPPORTED: bits/group_size/transpose/path not supported";
+    case BQ_ERR_ALIGN: return "BQ_ERR_ALIGN: a device pointer is not 16-byte aligned";
+    case BQ_ERR_CUDA: return "BQ_ERR_CUDA: CUDA runtime or launch error";
+    case BQ_ERR_TIMEOUT: return "BQ_ERR_TIMEOUT: a device-side bounded wait ran out";
+    case BQ_ERR_WORKSPACE: return "BQ_ERR_WORKSPACE: workspace missing or too small";
+    case BQ_ERR_DEVICE: return "BQ_ERR_DEVICE: current device is not sm_100";
+    default: return "unknown bq_status";
+    }
+}
+
+int bq_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,174 @@
+// dequant.cuh -- Q4_0 / affine dequantize and quantize kernels (HBM-bound, bit-exact).
+//
+// Dequantize is the first half of the unfused pair the MLX issue page measures
+// ("quantized_matmul takes 14-41% longer than dequantize + bf16 matmul at
+// prefill sizes (> 512 tokens)", Repro: x @ mx.dequantize(...).T).  Quantize is
+// input preparation (mx.quantize on the same page); its integer codes are
+// decided in fp32 with explicitly rounded operations so they are reproducible.
+#pragma once
+
+#include "common.cuh"
+
+namespace bq {
+
+// ----------------------------------------------------------------------------
+// Q4_0 dequantize: one thread per 32-weight block (16 code bytes + one fp16 d).
+// out = bf16_rne(d * (q - 8)); the fp32 product is exact (11 x 4 significant
+// bits), so this matches the plain definition bit for bit.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+q4_0_dequant_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ d16,
+                    uint16_t* __restrict__ out, int64_t nblocks)
+{
+    for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < nblocks;
+         b += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 raw = ldg_stream(wq + b * 16);
+        const float d = f16_bits_to_f32(__ldg(d16 + b));
+        const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t lo[8], hi[8];   // lo: elements 0..15, hi: elements 16..31, packed in pairs
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const uint32_t b0 = (words[w] >> (16 * p)) & 0xFFu;
+                const uint32_t b1 = (words[w] >> (16 * p + 8)) & 0xFFu;
+                const float l0 = __fmul_rn(d, (float)((int)(b0 & 15u) - 8));
+                const float l1 = __fmul_rn(d, (float)((int)(b1 & 15u) - 8));
+                const float h0 = __fmul_rn(d, (float)((int)(b0 >> 4) - 8));
+                const float h1 = __fmul_rn(d, (float)((int)(b1 >> 4) - 8));
+                lo[2 * w + p] = pack_bf16x2_rn(l0, l1);
+                hi[2 * w + p] = pack_bf16x2_rn(h0, h1);
+            }
+        }
+        uint4* o = reinterpret_cast<uint4*>(out + b * 32);
+        o[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        o[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+        o[2] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        o[3] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Affine dequantize: one thread per 16 packed bytes (32 codes at 4 bits, 16 at
+// 8 bits).  out = bf16_rne(fmaf(scale, q, bias)).
+// ----------------------------------------------------------------------------
+template <int BITS>
+__global__ void __launch_bounds__(256)
+affine_dequant_kernel(const uint32_t* __restrict__ wq, const uint16_t* __restrict__ scales,
+                      const uint16_t* __restrict__ biases, uint16_t* __restrict__ out,
+                      int64_t nchunks, int64_t K, int group_size)
+{
+    constexpr int kPer = 32 / BITS;          // codes per word
+    constexpr int kElems = 4 * kPer;         // codes per 16-byte chunk
+    constexpr uint32_t kMask = (1u << BITS) - 1u;
+    const int64_t chunks_per_row = K / kElems;
+    const int64_t groups_per_row = K / group_size;
+    for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < nchunks;
+         c += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = c / chunks_per_row;
+        const int64_t k0 = (c % chunks_per_row) * kElems;
+        const uint4 raw = ldg_stream(wq + c * 4);
+        const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
+        // A chunk never straddles a group: kElems (32 or 16) divides group_size.
+        const int64_t gi = n * groups_per_row + k0 / group_size;
+        const float s = bf16_bits_to_f32(__ldg(scales + gi));
+        const float bb = bf16_bits_to_f32(__ldg(biases + gi));
+        uint32_t packed[kElems / 2];
+#pragma unroll
+        for (int e = 0; e < kElems; e += 2) {
+            const uint32_t q0 = (words[e / kPer] >> (BITS * (e % kPer))) & kMask;
+            const uint32_t q1 = (words[(e + 1) / kPer] >> (BITS * ((e + 1) % kPer))) & kMask;
+            packed[e / 2] = pack_bf16x2_rn(__fmaf_rn(s, (float)q0, bb), __fmaf_rn(s, (float)q1, bb));
+        }
+        uint4* o = reinterpret_cast<uint4*>(out + n * K + k0);
+#pragma unroll
+        for (int v = 0; v < kElems / 8; ++v)
+            o[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Q4_0 quantize: one thread per block, same operation order as the definition.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+q4_0_quant_kernel(const float* __restrict__ w, uint8_t* __restrict__ wq, uint16_t* __restrict__ d16,
+                  int64_t nblocks)
+{
+    for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < nblocks;
+         b += (int64_t)gridDim.x * blockDim.x) {
+        const float* blk = w + b * 32;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            const float4 t = *reinterpret_cast<const float4*>(blk + j);
+            v[j] = t.x; v[j + 1] = t.y; v[j + 2] = t.z; v[j + 3] = t.w;
+        }
+        float amax = 0.0f, mx = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float a = fabsf(v[j]);
+            if (a > amax) { amax = a; mx = v[j]; }
+        }
+        const float d = __fdiv_rn(mx, -8.0f);
+        const float id = (d != 0.0f) ? __fdiv_rn(1.0f, d) : 0.0f;
+        d16[b] = __half_as_ushort(__float2half_rn(d));
+        uint32_t out[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            int q0 = (int)__fadd_rn(__fmul_rn(v[j], id), 8.5f);
+            int q1 = (int)__fadd_rn(__fmul_rn(v[j + 16], id), 8.5f);
+            q0 = min(15, max(0, q0));
+            q1 = min(15, max(0, q1));
+            out[j / 4] |= (uint32_t)(q0 | (q1 << 4)) << (8 * (j % 4));
+        }
+        *reinterpret_cast<uint4*>(wq + b * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Affine quantize: one thread per group.  scale = bf16((max - min) / L),
+// bias = bf16(min); q = clamp(rint((w - bias) / scale), 0, L) from the stored
+// bf16 values (q = 0 when scale == 0).
+// ----------------------------------------------------------------------------
+template <int BITS>
+__global__ void __launch_bounds__(256)
+affine_quant_kernel(const float* __restrict__ w, uint32_t* __restrict__ wq, uint16_t* __restrict__ scales,
+                    uint16_t* __restrict__ biases, int64_t ngroups, int group_size)
+{
+    constexpr int L = (1 << BITS) - 1;
+    constexpr int kPer = 32 / BITS;
+    for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < ngroups;
+         g += (int64_t)gridDim.x * blockDim.x) {
+        const float* grp = w + g * group_size;
+        float mn = grp[0], mx = grp[0];
+        for (int j = 1; j < group_size; ++j) {
+            const float v = grp[j];
+            if (v < mn) mn = v;
+            if (v > mx) mx = v;
+        }
+        const float scale_f = __fdiv_rn(__fsub_rn(mx, mn), (float)L);
+        const uint32_t s16 = f32_to_bf16_bits(scale_f);
+        const uint32_t b16 = f32_to_bf16_bits(mn);
+        scales[g] = (uint16_t)s16;
+        biases[g] = (uint16_t)b16;
+        const float s = bf16_bits_to_f32(s16);
+        const float bb = bf16_bits_to_f32(b16);
+        uint32_t* out = wq + g * (group_size / kPer);
+        for (int j0 = 0; j0 < group_size; j0 += kPer) {
+            uint32_t word = 0u;
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) {
+                int q = 0;
+                if (s != 0.0f) {
+                    float r = rintf(__fdiv_rn(__fsub_rn(grp[j0 + e], bb), s));
+                    r = fminf(fmaxf(r, 0.0f), (float)L);
+                    q = (int)r;
+                }
+                word |= (uint32_t)q << (BITS * e);
+            }
+            out[j0 / kPer] = word;
+        }
+    }
+}
+
+}  // namespace bq

@@ -1,0 +1,214 @@
+/*
+ * bqgemm.h -- C ABI of the B200 (sm_100a) weight-only block-quantized matmul
+ * library, libbqgemm.so.
+ *
+ * The library computes y[M,N] = x[M,K] . dequant(Wq)[N,K]^T with bf16
+ * activations x, bf16 output y and fp32 accumulation, for two weight formats:
+ *
+ *  - Q4_0, the llama.cpp format of "et-backend: Q4_0 matrix-engine GEMM
+ *    rewrite for prefill" (Overview) and of the SYCL "reordered" MMVQ path of
+ *    "2026-05-06 Q4 sync-after focused repro" (Important source touch points).
+ *    Blocks of 32 weights along K share one fp16 scale d; w = d * (q - 8),
+ *    q in [0, 15].  Layout (the "reordered" two-plane form):
+ *      wq     u8   [N][K/2]   byte j of block b of row n at n*K/2 + 16*b + j,
+ *                             low nibble = element 32b + j,
+ *                             high nibble = element 32b + j + 16
+ *      scales fp16 [N][K/32]  (raw IEEE half bits)
+ *
+ *  - MLX-style affine, the format of mx.quantize / mx.dequantize /
+ *    mx.quantized_matmul on "quantized_matmul takes 14-41% longer than
+ *    dequantize + bf16 matmul at prefill sizes (> 512 tokens)" (Repro).
+ *    Groups of group_size (= 64) weights along K share a bf16 scale and a bf16
+ *    bias; w = scale * q + bias, q in [0, 2^bits - 1], bits in {4, 8}.
+ *      wq      u32  [N][K*bits/32]  element k at bits bits*(k % (32/bits)) of
+ *                                   word k / (32/bits) (lowest bits first)
+ *      scales  bf16 [N][K/group_size]
+ *      biases  bf16 [N][K/group_size]
+ *
+ * Tensors are row-major and contiguous: x bf16 [M][K], y bf16 [M][N],
+ * W (and its dequantized form) [N][K] -- the transpose=True convention of
+ * mx.quantized_matmul, one output feature per weight row.
+ *
+ * Conventions for every entry point below:
+ *  - Pointers marked "device" are device (HBM) addresses; the caller owns
+ *    every buffer and the library never frees caller memory.
+ *  - Device pointers must be 16-byte aligned (BQ_ERR_ALIGN otherwise).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) and the call returns without waiting for it.
+ *  - Arguments are checked on the host before anything is launched; a failed
+ *    check returns its error code and enqueues nothing.  A launch failure
+ *    returns BQ_ERR_CUDA.  Errors raised later on the device (a bounded wait
+ *    that ran out) are reported by bq_device_status().
+ *  - M == 0 or N == 0 is an empty problem and returns BQ_OK with no work.
+ *  - There is no CPU fallback: every call runs on the current CUDA device.
+ */
+#ifndef BQGEMM_H
+#define BQGEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define BQ_API __attribute__((visibility("default")))
+#else
+#define BQ_API
+#endif
+
+typedef struct CUstream_st* bq_stream_t;   /* same type as cudaStream_t */
+
+typedef enum {
+    BQ_OK = 0,
+    BQ_ERR_NULL = 1,          /* a required pointer is NULL */
+    BQ_ERR_SHAPE = 2,         /* negative size, or K not a multiple of the block / group */
+    BQ_ERR_UNSUPPORTED = 3,   /* bits / group_size / transpose / path not supported */
+    BQ_ERR_ALIGN = 4,         /* a device pointer is not 16-byte aligned */
+    BQ_ERR_CUDA = 5,          /* a CUDA runtime or launch error */
+    BQ_ERR_TIMEOUT = 6,       /* a device-side bounded wait ran out (see bq_device_status) */
+    BQ_ERR_WORKSPACE = 7,     /* the caller's workspace is missing or too small */
+    BQ_ERR_DEVICE = 8         /* the current device is not sm_100 */
+} bq_status;
+
+/* Kernel paths of quant_matmul_ex. */
+typedef enum {
+    BQ_PATH_AUTO = 0,          /* the M-threshold dispatcher chooses (quant_matmul_select_path) */
+    BQ_PATH_GEMV = 1,          /* decode path: in-register dequant feeding warp-level MMA, M <= 32 */
+    BQ_PATH_TC_FUSED = 2,      /* prefill path: on-chip dequant feeding a tcgen05/TMEM GEMM */
+    BQ_PATH_DEQUANT_GEMM = 3   /* the unfused pair: *_dequantize into a bf16 workspace, then bf16_matmul */
+} bq_path;
+
+/*
+ * q4_0_dequantize -- out[n][k] = bf16_rne(fp32(d[n][k/32]) * (q[n][k] - 8)).
+ * The fp32 product is exact, so the result is bit-exact with the plain
+ * definition (sign of zero included).  The dequantize half of the workaround
+ * on the MLX issue page (Repro: x @ mx.dequantize(...).T), for Q4_0.
+ *   wq         device u8   [N][K/2]   packed codes (layout above)
+ *   scales_f16 device u16  [N][K/32]  fp16 bits of d
+ *   out_bf16   device u16  [N][K]     bf16 bits, written
+ *   N, K       N >= 0, K >= 0, K % 32 == 0
+ */
+BQ_API bq_status q4_0_dequantize(const uint8_t* wq, const uint16_t* scales_f16, uint16_t* out_bf16,
+                          int64_t N, int64_t K, bq_stream_t stream);
+
+/*
+ * affine_dequantize -- out[n][k] = bf16_rne(fmaf(scale, q, bias)) for the group
+ * of k: one fp32 fused multiply-add, one rounding to bf16.  mx.dequantize on
+ * the MLX issue page (Repro).
+ *   wq          device u32 [N][K*bits/32]
+ *   scales_bf16 device u16 [N][K/group_size]
+ *   biases_bf16 device u16 [N][K/group_size]
+ *   out_bf16    device u16 [N][K], written
+ *   group_size  64;  bits  4 or 8;  K % group_size == 0
+ */
+BQ_API bq_status affine_dequantize(const uint32_t* wq, const uint16_t* scales_bf16, const uint16_t* biases_bf16,
+                            uint16_t* out_bf16, int64_t N, int64_t K, int group_size, int bits,
+                            bq_stream_t stream);
+
+/*
+ * quant_matmul -- y[M][N] = bf16_rne(sum_k x[m][k] * dequant(W)[n][k]), fp32
+ * accumulation.  mx.quantized_matmul(x, wq, scales, biases, transpose=True,
+ * group_size, bits) on the MLX issue page (Repro); its result equals
+ * x @ dequantize(...).T up to accumulation order.
+ *   x_bf16   device u16 [M][K]
+ *   wq       device: u8 [N][K/2] (Q4_0) or u32 [N][K*bits/32] (affine)
+ *   scales   device: fp16 [N][K/32] (Q4_0) or bf16 [N][K/group_size] (affine)
+ *   biases   device bf16 [N][K/group_size]; NULL selects Q4_0 (then bits must be
+ *            4 and group_size 32)
+ *   y_bf16   device u16 [M][N], written
+ *   transpose  must be 1 (W stored [N][K]); 0 returns BQ_ERR_UNSUPPORTED
+ * The path is chosen by quant_matmul_select_path.  A path that needs scratch
+ * memory (the unfused pair) uses a per-device buffer that the library
+ * allocates on first need, grows on demand and keeps until process exit; a
+ * first call that allocates must therefore not be made during stream capture.
+ */
+BQ_API bq_status quant_matmul(const uint16_t* x_bf16, const void* wq, const void* scales, const void* biases,
+                       uint16_t* y_bf16, int64_t M, int64_t N, int64_t K, int group_size, int bits,
+                       int transpose, bq_stream_t stream);
+
+/*
+ * quant_matmul_ex -- quant_matmul with an explicit path (bq_path) and an
+ * optional caller-owned device workspace.  With workspace == NULL the library's
+ * per-device buffer is used as in quant_matmul; otherwise workspace_bytes must
+ * be >= quant_matmul_workspace_size(...) (BQ_ERR_WORKSPACE if not).  Forcing
+ * BQ_PATH_GEMV with M > 32 returns BQ_ERR_UNSUPPORTED.
+ */
+BQ_API bq_status quant_matmul_ex(const uint16_t* x_bf16, const void* wq, const void* scales, const void* biases,
+                          uint16_t* y_bf16, int64_t M, int64_t N, int64_t K, int group_size, int bits,
+                          int transpose, int path, void* workspace, size_t workspace_bytes,
+                          bq_stream_t stream);
+
+/* Bytes of workspace quant_matmul_ex needs for this problem and path
+ * (path AUTO: the dispatcher's choice).  0 when the path needs none or the
+ * arguments are invalid.  Having no biases pointer, this call and
+ * quant_matmul_select_path take group_size 32 with bits 4 as Q4_0 and any
+ * other combination as affine. */
+BQ_API size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int group_size, int bits, int path);
+
+/*
+ * quant_matmul_select_path -- the M-threshold dispatcher (host only, no CUDA
+ * call).  After the size threshold asked for on the MLX issue page (Question:
+ * pick the dequantize path above some M) and the decode/prefill split of
+ * "et-backend: Q4_0 matrix-engine GEMM rewrite for prefill" (Overview: decode
+ * routes to the vector-dot kernel).  Returns a bq_path other than AUTO:
+ *   M <  tc_min_m                 -> BQ_PATH_GEMV        (tc_min_m default 33)
+ *   M >= pair_min_m               -> BQ_PATH_DEQUANT_GEMM (pair_min_m default: never)
+ *   otherwise                     -> BQ_PATH_TC_FUSED when K % 64 == 0,
+ *                                    else BQ_PATH_DEQUANT_GEMM
+ * Environment overrides, read once per process: BQ_TC_MIN_M (clamped to
+ * [1, 33]; the GEMV handles at most 32 tokens) and BQ_PAIR_MIN_M (0 or unset:
+ * never).  Returns -1 for arguments quant_matmul would reject.
+ */
+BQ_API int quant_matmul_select_path(int64_t M, int64_t N, int64_t K, int group_size, int bits);
+
+/*
+ * bf16_matmul -- y[M][N] = bf16_rne(sum_k x[m][k] * w[n][k]), fp32
+ * accumulation on the tcgen05 tensor cores: the plain bf16 matmul of the
+ * unfused pair (MLX issue page, Repro: "x @ dense.T").
+ *   x_bf16 device [M][K]; w_bf16 device [N][K]; y_bf16 device [M][N]; K % 8 == 0.
+ */
+BQ_API bq_status bf16_matmul(const uint16_t* x_bf16, const uint16_t* w_bf16, uint16_t* y_bf16,
+                      int64_t M, int64_t N, int64_t K, bq_stream_t stream);
+
+/*
+ * q4_0_quantize -- fp32 w[N][K] -> Q4_0 (input preparation, mx.quantize's
+ * counterpart).  Per block of 32: m = the element of largest |w| (first wins a
+ * tie), d = m / -8 (fp32), stored as fp16; q = min(15, trunc(w * (1/d) + 8.5))
+ * with 1/d taken as 0 when d == 0.
+ *   w device f32 [N][K]; wq device u8 [N][K/2]; scales_f16 device u16 [N][K/32].
+ */
+BQ_API bq_status q4_0_quantize(const float* w, uint8_t* wq, uint16_t* scales_f16, int64_t N, int64_t K,
+                        bq_stream_t stream);
+
+/*
+ * affine_quantize -- fp32 w[N][K] -> affine codes (mx.quantize on the MLX issue
+ * page, Repro).  Per group: scale = bf16((max - min) / (2^bits - 1)),
+ * bias = bf16(min), q = clamp(round_half_even((w - bias) / scale), 0, 2^bits - 1)
+ * from the stored bf16 scale and bias (q = 0 when scale == 0).
+ *   w device f32 [N][K]; wq device u32 [N][K*bits/32]; scales/biases device bf16 [N][K/group_size].
+ */
+BQ_API bq_status affine_quantize(const float* w, uint32_t* wq, uint16_t* scales_bf16, uint16_t* biases_bf16,
+                          int64_t N, int64_t K, int group_size, int bits, bq_stream_t stream);
+
+/*
+ * bq_device_status -- waits for the current device to finish its work, then
+ * reads and clears the library's device error word: BQ_OK, or BQ_ERR_TIMEOUT
+ * when a kernel's bounded wait on a shared-memory barrier ran out (the kernel
+ * then skipped its remaining work and exited cleanly; its output is not valid).
+ * BQ_ERR_CUDA if the device cannot be queried.
+ */
+BQ_API bq_status bq_device_status(void);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+BQ_API const char* bq_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+BQ_API int bq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BQGEMM_H */

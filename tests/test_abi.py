@@ -1,0 +1,132 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports every
+entry point the header declares, rejects bad arguments before launching
+anything, and the M-threshold dispatcher picks the expected path at the
+boundaries (after the host-predicate gates of the vllm.cpp issue page, Gates:
+T=1 / T=19 / T=64 checks of a token-count route)."""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bqgemm.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    import __graft_entry__
+    __graft_entry__.build()
+    import bit_quantized_gemm_quant_b200 as bq
+    return bq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^BQ_API\s+[\w\s\*]+?\b(\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for required in ("q4_0_dequantize", "affine_dequantize", "quant_matmul"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", L._name], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    assert set(declared_functions()) <= exported
+
+
+def test_status_strings_and_version(L):
+    for code in range(9):
+        assert L.bq_status_string(code)
+    assert L.bq_status_string(99) == b"unknown bq_status"
+    assert L.bq_version() >= 100
+
+
+P = ctypes.c_void_p
+ALIGNED = P(0x1000)
+MISALIGNED = P(0x1008)
+
+
+def qmm(L, x=ALIGNED, wq=ALIGNED, s=ALIGNED, b=None, y=ALIGNED, M=16, N=256, K=512, g=32, bits=4, tr=1, path=0,
+        ws=None, wsb=0):
+    return L.quant_matmul_ex(x, wq, s, b, y, M, N, K, g, bits, tr, path, ws, wsb, None)
+
+
+def test_quant_matmul_rejects_before_launch(L):
+    # every case fails validation on the host, so no CUDA call is ever made
+    assert qmm(L, tr=0) == 3                                  # transpose=0 unsupported
+    assert qmm(L, path=7) == 3
+    assert qmm(L, M=-1) == 2
+    assert qmm(L, N=-1) == 2
+    assert qmm(L, K=48) == 2                                  # Q4_0 needs K % 32 == 0
+    assert qmm(L, bits=8) == 3                                # Q4_0 is 4-bit only
+    assert qmm(L, g=64) == 3                                  # ... with group 32
+    assert qmm(L, b=ALIGNED, g=32, bits=4) == 3               # affine needs group 64
+    assert qmm(L, b=ALIGNED, g=64, bits=3) == 3               # bits in {4, 8}
+    assert qmm(L, b=ALIGNED, g=64, bits=4, K=96) == 2         # K % group
+    assert qmm(L, x=None) == 1
+    assert qmm(L, wq=None) == 1
+    assert qmm(L, s=None) == 1
+    assert qmm(L, y=None) == 1
+    assert qmm(L, x=MISALIGNED) == 4
+    assert qmm(L, y=MISALIGNED) == 4
+    assert qmm(L, b=MISALIGNED, g=64) == 4
+    assert qmm(L, M=64, path=1) == 3                          # GEMV is M <= 32 only
+    assert qmm(L, K=544, M=64, path=2) == 3                   # fused TC needs K % 64 == 0
+    assert qmm(L, M=64, path=3, ws=ALIGNED, wsb=16) == 7      # workspace too small
+    assert L.quant_matmul(ALIGNED, ALIGNED, ALIGNED, None, ALIGNED, 16, 256, 512, 32, 4, 0, None) == 3
+
+
+def test_other_entry_points_reject_before_launch(L):
+    assert L.q4_0_dequantize(ALIGNED, ALIGNED, ALIGNED, 4, 48, None) == 2
+    assert L.q4_0_dequantize(None, ALIGNED, ALIGNED, 4, 64, None) == 1
+    assert L.q4_0_dequantize(MISALIGNED, ALIGNED, ALIGNED, 4, 64, None) == 4
+    assert L.affine_dequantize(ALIGNED, ALIGNED, None, ALIGNED, 4, 64, 64, 4, None) == 1
+    assert L.affine_dequantize(ALIGNED, ALIGNED, ALIGNED, ALIGNED, 4, 64, 64, 5, None) == 3
+    assert L.affine_dequantize(ALIGNED, ALIGNED, ALIGNED, ALIGNED, 4, 96, 64, 4, None) == 2
+    assert L.bf16_matmul(ALIGNED, ALIGNED, ALIGNED, 4, 4, 12, None) == 2
+    assert L.bf16_matmul(None, ALIGNED, ALIGNED, 4, 4, 16, None) == 1
+    assert L.q4_0_quantize(ALIGNED, ALIGNED, MISALIGNED, 4, 64, None) == 4
+    assert L.affine_quantize(ALIGNED, ALIGNED, ALIGNED, ALIGNED, 4, 64, 32, 4, None) == 3
+
+
+BOUNDARY_M = [1, 2, 8, 19, 31, 32, 33, 63, 64, 65, 127, 128, 129, 511, 512, 513]
+
+
+def test_dispatcher_boundaries(L):
+    for M in BOUNDARY_M:
+        for g, bits in ((32, 4), (64, 4), (64, 8)):
+            p = L.quant_matmul_select_path(M, 12288, 4096, g, bits)
+            assert p == (1 if M <= 32 else 2), (M, g, bits, p)
+    # K % 64 != 0 (Q4_0 only): prefill goes through the unfused pair
+    assert L.quant_matmul_select_path(512, 256, 544, 32, 4) == 3
+    assert L.quant_matmul_select_path(8, 256, 544, 32, 4) == 1
+    assert L.quant_matmul_select_path(-1, 256, 512, 32, 4) == -1
+    assert L.quant_matmul_select_path(8, 256, 512, 64, 5) == -1
+    assert L.quant_matmul_workspace_size(512, 256, 544, 32, 4, 0) == 256 * 544 * 2
+    assert L.quant_matmul_workspace_size(512, 256, 512, 32, 4, 0) == 0
+    assert L.quant_matmul_workspace_size(512, 256, 512, 64, 8, 3) == 256 * 512 * 2
+
+
+def _select_in_subprocess(env_extra, Ms):
+    code = ("import sys; sys.path.insert(0, %r); import bit_quantized_gemm_quant_b200 as bq; "
+            "print([bq.quant_matmul_select_path(m, 4096, 4096, 64, 4) for m in %r])" % (ROOT, Ms))
+    env = dict(os.environ, **env_extra)
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, check=True)
+    return eval(out.stdout.strip())
+
+
+def test_dispatcher_env_overrides(L):
+    Ms = [1, 8, 19, 32, 33, 512, 4096]
+    assert _select_in_subprocess({}, Ms) == [1, 1, 1, 1, 2, 2, 2]
+    assert _select_in_subprocess({"BQ_TC_MIN_M": "8"}, Ms) == [1, 2, 2, 2, 2, 2, 2]
+    assert _select_in_subprocess({"BQ_TC_MIN_M": "1000"}, Ms) == [1, 1, 1, 1, 2, 2, 2]   # clamped to 33
+    assert _select_in_subprocess({"BQ_PAIR_MIN_M": "512"}, Ms) == [1, 1, 1, 1, 2, 3, 3]
+    assert _select_in_subprocess({"BQ_PAIR_MIN_M": "0"}, Ms) == [1, 1, 1, 1, 2, 2, 2]

@@ -1,0 +1,101 @@
+"""GPU dequantize and quantize kernels vs the CPU oracle: bit-exact (integer
+codes, fp16/bf16 scale bits and bf16 outputs compared as bit patterns, sign of
+zero included)."""
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_gemm_quant_b200 as bq
+import oracle
+from bit_quantized_gemm_quant_b200 import inputs
+from _helpers import Problem, u16
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 64), (3, 128), (250, 192), (256, 512), (64, 4096)]
+
+
+def _gpu_dequant(p: Problem):
+    wq, s, b = p.device()
+    if p.fmt == "q4_0":
+        out = bq.q4_0_dequantize(wq, s)
+    else:
+        out = bq.affine_dequantize(wq, s, b, p.group_size, p.bits)
+    torch.cuda.synchronize()
+    return u16(out)
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "affine4", "affine8"])
+@pytest.mark.parametrize("N,K", SHAPES)
+def test_dequant_bit_exact(fmt, N, K):
+    p = Problem(fmt, N, K, seed=N + K)
+    assert np.array_equal(_gpu_dequant(p), p.wb)
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "affine4", "affine8"])
+def test_dequant_bit_exact_full_size(fmt):
+    p = Problem(fmt, 12288, 4096)
+    assert np.array_equal(_gpu_dequant(p), p.wb)
+
+
+def test_q4_0_dequant_random_codes_and_scale_bits():
+    """Arbitrary bytes and arbitrary finite fp16 scales (subnormals, negatives, +-0)."""
+    g = inputs.generator(21)
+    N, K = 300, 1024
+    wq = inputs.random_bytes((N, K // 2), g).numpy()
+    d = inputs.random_f16_bits((N, K // 32), g).numpy().view(np.uint16)
+    ref = oracle.q4_0_dequantize(wq, d)
+    out = bq.q4_0_dequantize(torch.from_numpy(wq).cuda(), torch.from_numpy(d.view(np.int16)).cuda().view(torch.float16))
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(out), ref)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_affine_dequant_random_codes_and_scale_bits(bits):
+    g = inputs.generator(22 + bits)
+    N, K = 300, 1024
+    wq = inputs.random_u32((N, K * bits // 32), g).numpy()
+    s = inputs.random_bf16_bits((N, K // 64), g, 100, 140).numpy().view(np.uint16)
+    b = inputs.random_bf16_bits((N, K // 64), g, 100, 140).numpy().view(np.uint16)
+    ref = oracle.affine_dequantize(wq.view(np.uint32), s, b, 64, bits)
+    out = bq.affine_dequantize(torch.from_numpy(wq).cuda(), torch.from_numpy(s.view(np.int16)).cuda().view(torch.bfloat16),
+                               torch.from_numpy(b.view(np.int16)).cuda().view(torch.bfloat16), 64, bits)
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(out), ref)
+
+
+def test_dequant_empty():
+    wq = torch.zeros(0, 16, dtype=torch.uint8, device="cuda")
+    d = torch.zeros(0, 1, dtype=torch.float16, device="cuda")
+    out = bq.q4_0_dequantize(wq, d)
+    assert out.shape == (0, 32)
+
+
+# ------------------------------------------------------------------ quantize
+@pytest.mark.parametrize("N,K", [(3, 64), (250, 512), (12288, 4096)])
+def test_q4_0_quantize_bit_exact(N, K):
+    g = inputs.generator(N)
+    w = inputs.weights_fp32(N, K, g)
+    w[0, :32] = 0.0                      # all-zero block
+    w[min(1, N - 1), 32:64] = 0.01       # all-equal block (first index wins)
+    w[min(2, N - 1), 0] = -w[min(2, N - 1), 1].abs() - 0.1
+    w[min(2, N - 1), 1] = -w[min(2, N - 1), 0]   # max-abs tie with opposite signs
+    wq_ref, d_ref = oracle.q4_0_quantize(w.numpy())
+    wq, d = bq.q4_0_quantize(w.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(wq.cpu().numpy(), wq_ref)
+    assert np.array_equal(u16(d), d_ref)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("N,K", [(3, 64), (250, 512), (12288, 4096)])
+def test_affine_quantize_bit_exact(bits, N, K):
+    g = inputs.generator(N + bits)
+    w = inputs.weights_bf16_valued(N, K, g)
+    w[0, :64] = -0.375                   # constant group: scale 0
+    wq_ref, s_ref, b_ref = oracle.affine_quantize(w.numpy(), 64, bits)
+    wq, s, b = bq.affine_quantize(w.cuda(), 64, bits)
+    torch.cuda.synchronize()
+    assert np.array_equal(wq.cpu().numpy().view(np.uint32), wq_ref)
+    assert np.array_equal(u16(s), s_ref)
+    assert np.array_equal(u16(b), b_ref)

@@ -1,0 +1,177 @@
+"""quant_matmul on every kernel path vs the CPU oracle's float64 reference:
+|y_gpu - y_ref| <= 2e-3 * sum_k |x_k w_k| + 1e-5 for every checked output,
+where w is the oracle's bf16 dequantization (the equivalence
+quantized_matmul == x @ dequantize(...).T of the MLX issue page, Repro)."""
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_gemm_quant_b200 as bq
+import oracle
+from bit_quantized_gemm_quant_b200 import inputs
+from _helpers import Problem, assert_within_tolerance, reference, u16
+
+pytestmark = pytest.mark.gpu
+
+GEMV_M = [1, 2, 8, 9, 16, 19, 32]
+TC_M = [1, 16, 33, 100, 256, 300]
+
+
+def run(p: Problem, x: torch.Tensor, path: str):
+    wq, s, b = p.device()
+    y = bq.quant_matmul_ex(x.cuda(), wq, s, b, p.group_size, p.bits, True, path)
+    torch.cuda.synchronize()
+    return y
+
+
+def check(p: Problem, M: int, path: str, rows=None):
+    x = p.x(M)
+    y = run(p, x, path)
+    y_ref, a_ref = reference(x, p.wb, rows)
+    got = y if rows is None else y[torch.as_tensor(rows, device=y.device)]
+    assert_within_tolerance(got, y_ref, a_ref, f"{p.fmt} {path} M={M} N={p.N} K={p.K}")
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "affine4", "affine8"])
+@pytest.mark.parametrize("N,K", [(256, 512), (300, 1024)])
+def test_small_all_paths(fmt, N, K):
+    p = Problem(fmt, N, K, seed=N * 7 + K)
+    for M in GEMV_M:
+        check(p, M, "gemv")
+        check(p, M, "auto")
+    for M in TC_M:
+        check(p, M, "tc_fused")
+        check(p, M, "dequant_gemm")
+        check(p, M, "auto")
+
+
+def test_q4_0_ragged_k_uses_pair():
+    p = Problem("q4_0", 130, 544, seed=5)      # K % 64 == 32: no fused tile, the pair handles it
+    assert bq.quant_matmul_select_path(200, 130, 544, 32, 4) == bq.PATH_DEQUANT_GEMM
+    for M in (1, 7, 40, 200):
+        check(p, M, "auto")
+    for M in (3, 32):
+        check(p, M, "gemv")
+
+
+@pytest.mark.parametrize("M", [1, 8, 32])
+def test_q4_0_decode_config_full(M):
+    p = Problem("q4_0", 12288, 4096)
+    check(p, M, "auto")
+
+
+def _sample_rows(M, n=64, seed=0):
+    rng = np.random.default_rng(seed + M)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, size=min(n, M), replace=False)]))
+    return rows
+
+
+@pytest.mark.parametrize("M", [512, 2048, 8192])
+def test_affine4_prefill_config_sampled(M):
+    p = Problem("affine4", 12288, 4096)
+    rows = _sample_rows(M)
+    check(p, M, "auto", rows)
+    check(p, M, "dequant_gemm", rows)
+
+
+@pytest.mark.parametrize("M", [1, 32, 512, 2048, 8192])
+def test_affine8_sweep_config(M):
+    p = Problem("affine8", 12288, 4096)
+    rows = None if M <= 32 else _sample_rows(M)
+    check(p, M, "auto", rows)
+    if M >= 512:
+        check(p, M, "dequant_gemm", rows)
+
+
+@pytest.mark.parametrize("M", [1, 512])
+def test_llama_1b_layer_shapes(M):
+    for i, (N, K) in enumerate(((2048, 2048), (512, 2048), (8192, 2048), (2048, 8192))):
+        p = Problem("q4_0", N, K, seed=100 + i)
+        check(p, M, "auto", None if M == 1 else _sample_rows(M, 32))
+
+
+# ---------------------------------------------------------------- edge cases
+PATHS_FOR = {1: ["gemv", "tc_fused", "dequant_gemm"], 64: ["tc_fused", "dequant_gemm"]}
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "affine4", "affine8"])
+def test_one_hot_rows_are_exact(fmt):
+    """x = e_k gives y[:, n] = dequant(W)[n][k] exactly (one exact product, already bf16)."""
+    p = Problem(fmt, 200, 512, seed=9)
+    for M, paths in ((32, ["gemv", "tc_fused", "dequant_gemm"]), (64, ["tc_fused", "dequant_gemm"])):
+        ks = np.random.default_rng(M).choice(512, M, replace=False)
+        x = torch.zeros(M, 512, dtype=torch.bfloat16)
+        x[torch.arange(M), torch.as_tensor(ks)] = 1.0
+        for path in paths:
+            y = run(p, x, path)
+            assert np.array_equal(u16(y), p.wb[:, ks].T.copy()), (fmt, M, path)
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "affine4", "affine8"])
+def test_all_equal_weights_tight_tolerance(fmt):
+    """x = 1 and every dequantized weight equal: |y| = sum|x w|, so the output's
+    own bf16 rounding uses almost all of the tolerance."""
+    N, K = 130, 1024
+    if fmt == "q4_0":
+        w = np.full((N, K), -0.0123456, np.float32)     # every code 0, d = w / -8 with 11 significant bits
+    else:
+        w = np.full((N, K), 0.0123456, np.float32)
+        w = torch.from_numpy(w).to(torch.bfloat16).float().numpy()
+    p = Problem(fmt, N, K, w=w)
+    for M, paths in ((8, ["gemv", "tc_fused", "dequant_gemm"]), (100, ["tc_fused", "dequant_gemm"])):
+        x = torch.ones(M, K, dtype=torch.bfloat16)
+        y_ref, a_ref = reference(x, p.wb)
+        assert np.allclose(np.abs(y_ref), a_ref)
+        for path in paths:
+            assert_within_tolerance(run(p, x, path), y_ref, a_ref, f"{fmt} {path} M={M}")
+
+
+def test_zero_weights_give_zero():
+    p = Problem("q4_0", 64, 256, w=np.zeros((64, 256), np.float32))
+    for M, path in ((4, "gemv"), (4, "tc_fused"), (80, "tc_fused"), (80, "dequant_gemm")):
+        y = run(p, p.x(M), path)
+        assert torch.all(y.float() == 0), path
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "affine4", "affine8"])
+def test_deterministic(fmt):
+    p = Problem(fmt, 300, 1024, seed=3)
+    for M, path in ((5, "gemv"), (32, "gemv"), (100, "tc_fused"), (100, "dequant_gemm")):
+        x = p.x(M)
+        ys = [u16(run(p, x, path)) for _ in range(3)]
+        assert np.array_equal(ys[0], ys[1]) and np.array_equal(ys[0], ys[2]), (fmt, path)
+
+
+def test_empty_problems():
+    p = Problem("affine4", 64, 128)
+    wq, s, b = p.device()
+    x0 = torch.zeros(0, 128, dtype=torch.bfloat16, device="cuda")
+    assert bq.quant_matmul(x0, wq, s, b, 64, 4).shape == (0, 64)
+    x = p.x(4).cuda()
+    y = torch.full((4, 0), 1.0, dtype=torch.bfloat16, device="cuda")
+    wq0 = torch.zeros(0, 16, dtype=torch.int32, device="cuda")
+    s0 = torch.zeros(0, 2, dtype=torch.bfloat16, device="cuda")
+    assert bq.quant_matmul(x, wq0, s0, s0, 64, 4).shape == (4, 0)
+    # K == 0: an empty sum, y = 0
+    xk = torch.zeros(3, 0, dtype=torch.bfloat16, device="cuda")
+    wk = torch.zeros(5, 0, dtype=torch.uint8, device="cuda")
+    sk = torch.zeros(5, 0, dtype=torch.float16, device="cuda")
+    out = torch.full((3, 5), 7.0, dtype=torch.bfloat16, device="cuda")
+    bq.quant_matmul(xk, wk, sk, None, 32, 4, out=out)
+    torch.cuda.synchronize()
+    assert torch.all(out.float() == 0)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 64), (37, 200, 72), (300, 129, 640), (64, 256, 8)])
+def test_bf16_matmul(M, N, K):
+    g = inputs.generator(M + N + K)
+    x = inputs.activations_bf16(M, K, g)
+    w = inputs.activations_bf16(N, K, g)
+    y = bq.bf16_matmul(x.cuda(), w.cuda())
+    torch.cuda.synchronize()
+    y_ref, a_ref = reference(x, u16(w))
+    assert_within_tolerance(y, y_ref, a_ref, f"bf16_matmul {M}x{N}x{K}")
+
+
+def test_device_status_clean():
+    assert bq.bq_device_status() == 0
