@@ -72,9 +72,15 @@ def _check(status: int, where: str) -> None:
         raise BqError(status, where)
 
 
+_EMPTY_TAG = ctypes.c_void_p(16)   # non-NULL, 16-byte aligned, never dereferenced (empty tensor)
+
+
 def _ptr(t: torch.Tensor | None):
     if t is None:
         return None
+    if t.numel() == 0:
+        # an empty tensor has no storage; a NULL biases pointer would select Q4_0
+        return _EMPTY_TAG
     if not t.is_cuda:
         raise ValueError("tensors must live on a CUDA device")
     if not t.is_contiguous():

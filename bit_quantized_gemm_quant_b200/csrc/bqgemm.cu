@@ -203,8 +203,8 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     if (MODE == kModeBF16)
         ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a_src, N, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B);
     else
-        ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a_src, N, K * (MODE == kModeAff8 ? 1 : 2) / 2, 128,
-                      C::kCodeBytesPerRow, CU_TENSOR_MAP_SWIZZLE_NONE);
+        ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a_src, N, (MODE == kModeAff8) ? K : K / 2, 128,
+                      C::kCodeBytesPerRow, CU_TENSOR_MAP_SWIZZLE_NONE);   // packed code bytes per row
     if (!ok) return BQ_ERR_CUDA;
 
     static bool attr_done[kMaxDevices] = {};
@@ -233,14 +233,14 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
 }
 
 // ------------------------------------------------------------------ GEMV
-template <Fmt F, int NT, int RT, int KS>
+template <Fmt F, int NT, int RT, int KS, int PIPE, int MINB>
 bq_status launch_gemv_cfg(const uint16_t* x, const void* wq, const uint16_t* s, const uint16_t* b, uint16_t* y,
                           int64_t M, int64_t N, int64_t K, int group_size, cudaStream_t st)
 {
     const int64_t rows_per_cta = 16 * RT;
     const int64_t grid = (N + rows_per_cta - 1) / rows_per_cta;
     if (grid > INT32_MAX) return BQ_ERR_SHAPE;
-    gemv_kernel<F, NT, RT, KS><<<(unsigned)grid, 32 * KS, 0, st>>>(
+    gemv_kernel<F, NT, RT, KS, PIPE, MINB><<<(unsigned)grid, 32 * KS, 0, st>>>(
         x, reinterpret_cast<const uint8_t*>(wq), s, b, y, (int)M, (int)N, (int)K, group_size);
     return launch_status();
 }
@@ -250,9 +250,12 @@ bq_status launch_gemv(const uint16_t* x, const void* wq, const uint16_t* s, cons
                       int64_t M, int64_t N, int64_t K, int group_size, cudaStream_t st)
 {
     if (N > INT32_MAX || K > INT32_MAX) return BQ_ERR_SHAPE;
-    if (M <= 8) return launch_gemv_cfg<F, 1, 1, 8>(x, wq, s, b, y, M, N, K, group_size, st);
-    if (M <= 16) return launch_gemv_cfg<F, 2, 1, 8>(x, wq, s, b, y, M, N, K, group_size, st);
-    return launch_gemv_cfg<F, 4, 2, 8>(x, wq, s, b, y, M, N, K, group_size, st);
+    // Launch shapes measured on B200 at N = 12288, K = 4096: 32 weight rows per CTA,
+    // K split over 4 (8 at M > 16) warps, 2-deep load pipeline; MINB CTAs per SM
+    // keep the whole grid resident in one wave.
+    if (M <= 8) return launch_gemv_cfg<F, 1, 2, 4, 2, 3>(x, wq, s, b, y, M, N, K, group_size, st);
+    if (M <= 16) return launch_gemv_cfg<F, 2, 2, 4, 2, 2>(x, wq, s, b, y, M, N, K, group_size, st);
+    return launch_gemv_cfg<F, 4, 2, 8, 1, 1>(x, wq, s, b, y, M, N, K, group_size, st);
 }
 
 // ------------------------------------------------------------------ library workspace
@@ -312,10 +315,19 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
 {
     if (transpose != 1) return BQ_ERR_UNSUPPORTED;
     if (path < BQ_PATH_AUTO || path > BQ_PATH_DEQUANT_GEMM) return BQ_ERR_UNSUPPORTED;
-    if (M < 0) return BQ_ERR_SHAPE;
+    if (M < 0 || N < 0 || K < 0) return BQ_ERR_SHAPE;
+    if (M == 0 || N == 0) return BQ_OK;      // empty problem: nothing is read or written
     WFmt fmt;
     bq_status s = check_format(biases, N, K, group_size, bits, &fmt);
     if (s != BQ_OK) return s;
+    int dev;
+    DeviceInfo di;
+    if (K == 0) {                            // empty sum: y = 0
+        if (!y) return BQ_ERR_NULL;
+        if (!aligned16(y)) return BQ_ERR_ALIGN;
+        if ((s = current_device(&dev, &di)) != BQ_OK) return s;
+        return cudaMemsetAsync(y, 0, (size_t)M * (size_t)N * 2u, st) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+    }
     if (!x || !wq || !scales || !y) return BQ_ERR_NULL;
     if (!aligned16(x) || !aligned16(wq) || !aligned16(scales) || !aligned16(y) || (biases && !aligned16(biases)) ||
         (workspace && !aligned16(workspace)))
@@ -326,11 +338,7 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
     const size_t need = workspace_for(path, N, K);
     if (workspace && workspace_bytes < need) return BQ_ERR_WORKSPACE;
 
-    int dev;
-    DeviceInfo di;
     if ((s = current_device(&dev, &di)) != BQ_OK) return s;
-    if (M == 0 || N == 0) return BQ_OK;
-    if (K == 0) return cudaMemsetAsync(y, 0, (size_t)M * (size_t)N * 2u, st) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 
     const uint16_t* sc = reinterpret_cast<const uint16_t*>(scales);
     const uint16_t* bi = reinterpret_cast<const uint16_t*>(biases);
@@ -364,13 +372,13 @@ bq_status q4_0_dequantize(const uint8_t* wq, const uint16_t* scales_f16, uint16_
                           bq_stream_t stream)
 {
     if (N < 0 || K < 0 || K % 32 != 0) return BQ_ERR_SHAPE;
+    if (N == 0 || K == 0) return BQ_OK;
     if (!wq || !scales_f16 || !out_bf16) return BQ_ERR_NULL;
     if (!aligned16(wq) || !aligned16(scales_f16) || !aligned16(out_bf16)) return BQ_ERR_ALIGN;
     int dev;
     DeviceInfo di;
     bq_status s = current_device(&dev, &di);
     if (s != BQ_OK) return s;
-    if (N == 0 || K == 0) return BQ_OK;
     return dequant_any(WFmt::Q4_0, wq, scales_f16, nullptr, out_bf16, N, K, 32, di, (cudaStream_t)stream);
 }
 
@@ -380,13 +388,13 @@ bq_status affine_dequantize(const uint32_t* wq, const uint16_t* scales_bf16, con
     WFmt fmt;
     bq_status s = check_format(kAffineTag, N, K, group_size, bits, &fmt);
     if (s != BQ_OK) return s;
+    if (N == 0 || K == 0) return BQ_OK;
     if (!wq || !scales_bf16 || !biases_bf16 || !out_bf16) return BQ_ERR_NULL;
     if (!aligned16(wq) || !aligned16(scales_bf16) || !aligned16(biases_bf16) || !aligned16(out_bf16))
         return BQ_ERR_ALIGN;
     int dev;
     DeviceInfo di;
     if ((s = current_device(&dev, &di)) != BQ_OK) return s;
-    if (N == 0 || K == 0) return BQ_OK;
     return dequant_any(fmt, wq, scales_bf16, biases_bf16, out_bf16, N, K, group_size, di, (cudaStream_t)stream);
 }
 
@@ -425,30 +433,34 @@ bq_status bf16_matmul(const uint16_t* x_bf16, const uint16_t* w_bf16, uint16_t* 
                       int64_t K, bq_stream_t stream)
 {
     if (M < 0 || N < 0 || K < 0 || K % 8 != 0) return BQ_ERR_SHAPE;
-    if (!x_bf16 || !w_bf16 || !y_bf16) return BQ_ERR_NULL;
-    if (!aligned16(x_bf16) || !aligned16(w_bf16) || !aligned16(y_bf16)) return BQ_ERR_ALIGN;
+    if (M == 0 || N == 0) return BQ_OK;
+    if (!y_bf16) return BQ_ERR_NULL;
+    if (!aligned16(y_bf16)) return BQ_ERR_ALIGN;
     int dev;
     DeviceInfo di;
-    bq_status s = current_device(&dev, &di);
-    if (s != BQ_OK) return s;
-    if (M == 0 || N == 0) return BQ_OK;
-    if (K == 0)
+    bq_status s;
+    if (K == 0) {
+        if ((s = current_device(&dev, &di)) != BQ_OK) return s;
         return cudaMemsetAsync(y_bf16, 0, (size_t)M * N * 2u, (cudaStream_t)stream) == cudaSuccess ? BQ_OK
                                                                                                   : BQ_ERR_CUDA;
+    }
+    if (!x_bf16 || !w_bf16) return BQ_ERR_NULL;
+    if (!aligned16(x_bf16) || !aligned16(w_bf16)) return BQ_ERR_ALIGN;
+    if ((s = current_device(&dev, &di)) != BQ_OK) return s;
     return launch_tc<kModeBF16>(di, dev, x_bf16, w_bf16, nullptr, nullptr, y_bf16, M, N, K, (cudaStream_t)stream);
 }
 
 bq_status q4_0_quantize(const float* w, uint8_t* wq, uint16_t* scales_f16, int64_t N, int64_t K, bq_stream_t stream)
 {
     if (N < 0 || K < 0 || K % 32 != 0) return BQ_ERR_SHAPE;
+    const int64_t nb = N * (K / 32);
+    if (nb == 0) return BQ_OK;
     if (!w || !wq || !scales_f16) return BQ_ERR_NULL;
     if (!aligned16(w) || !aligned16(wq) || !aligned16(scales_f16)) return BQ_ERR_ALIGN;
     int dev;
     DeviceInfo di;
     bq_status s = current_device(&dev, &di);
     if (s != BQ_OK) return s;
-    const int64_t nb = N * (K / 32);
-    if (nb == 0) return BQ_OK;
     q4_0_quant_kernel<<<grid_for(nb, 256, di), 256, 0, (cudaStream_t)stream>>>(w, wq, scales_f16, nb);
     return launch_status();
 }
@@ -459,13 +471,13 @@ bq_status affine_quantize(const float* w, uint32_t* wq, uint16_t* scales_bf16, u
     WFmt fmt;
     bq_status s = check_format(kAffineTag, N, K, group_size, bits, &fmt);
     if (s != BQ_OK) return s;
+    const int64_t ng = N * (K / group_size);
+    if (ng == 0) return BQ_OK;
     if (!w || !wq || !scales_bf16 || !biases_bf16) return BQ_ERR_NULL;
     if (!aligned16(w) || !aligned16(wq) || !aligned16(scales_bf16) || !aligned16(biases_bf16)) return BQ_ERR_ALIGN;
     int dev;
     DeviceInfo di;
     if ((s = current_device(&dev, &di)) != BQ_OK) return s;
-    const int64_t ng = N * (K / group_size);
-    if (ng == 0) return BQ_OK;
     if (bits == 4)
         affine_quant_kernel<4><<<grid_for(ng, 256, di), 256, 0, (cudaStream_t)stream>>>(w, wq, scales_bf16,
                                                                                          biases_bf16, ng, group_size);

@@ -65,6 +65,24 @@ BQ_DEVINL uint32_t and_or(uint32_t a, uint32_t mask, uint32_t magic)
     return d;
 }
 
+// Immediate-operand forms: the constants stay in the instruction stream instead
+// of occupying registers (which the compiler would otherwise rematerialize).
+template <uint32_t MASK, uint32_t MAGIC>
+BQ_DEVINL uint32_t and_or_i(uint32_t a)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(MASK), "n"(MAGIC));
+    return d;
+}
+
+template <uint32_t C>
+BQ_DEVINL uint32_t hsub2_bf16_i(uint32_t a)
+{
+    uint32_t d;
+    asm("{\n\t.reg .b32 c;\n\tmov.b32 c, %2;\n\tsub.rn.bf16x2 %0, %1, c;\n\t}" : "=r"(d) : "r"(a), "n"(C));
+    return d;
+}
+
 // 16-byte global loads that bypass L1 allocation for streamed weights.
 BQ_DEVINL uint4 ldg_stream(const void* p)
 {

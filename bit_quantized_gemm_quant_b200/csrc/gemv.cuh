@@ -27,7 +27,14 @@
 
 namespace bq {
 
+
 enum class Fmt : int { Q4_0 = 0, AFF4 = 1, AFF8 = 2 };
+
+#ifndef BQ_Q4_ROUTE
+#define BQ_Q4_ROUTE 0
+#endif
+// Q4_0 dequant route of the decode kernel: 0 = packed-bf16 split-scale, 1 = fp32 FMA magic.
+constexpr int kQ4Route = BQ_Q4_ROUTE;
 
 template <Fmt F> struct FmtTraits;
 template <> struct FmtTraits<Fmt::Q4_0> { static constexpr int kChunkElems = 32; static constexpr int kBits = 4; };
@@ -44,105 +51,201 @@ BQ_DEVINL void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Per-chunk scale data of one row, already expanded for the conversion.
+// Per-chunk scale data of one row, expanded for the conversion.
+//  Q4_0: fp32 (d * 2^-s, -(2^(23-s) + 8) * d) for s = 8, 12, 16 (see dequant_word)
+//  AFF4: bf16x2 (scale, scale) and (bias, bias)
+//  AFF8: fp32 scale and bias
 struct ChunkScale {
-    uint32_t s0, s1;   // Q4_0: d_hi2, d_lo2 | AFF4: scale2, bias2 | AFF8: fp32 bits of scale, bias
+    float a[3], c[3];
+    uint32_t s2, b2;
 };
 
+// Raw 16-bit scale (and bias) bits of one row's chunk; zero for masked rows/chunks.
 template <Fmt F>
-BQ_DEVINL ChunkScale load_scale(const uint16_t* scales, const uint16_t* biases, int64_t idx, bool valid)
+BQ_DEVINL void load_scale_raw(const uint16_t* scales, const uint16_t* biases, int64_t idx, bool valid,
+                              uint32_t& s_raw, uint32_t& b_raw)
 {
-    ChunkScale cs{0u, 0u};
-    if (!valid) return cs;
-    if constexpr (F == Fmt::Q4_0) {
-        const float d = f16_bits_to_f32(__ldg(scales + idx));
-        const uint32_t hi = f32_to_bf16_bits(d);
-        const uint32_t lo = f32_to_bf16_bits(__fsub_rn(d, bf16_bits_to_f32(hi)));   // exact
-        cs.s0 = hi | (hi << 16);
-        cs.s1 = lo | (lo << 16);
+    s_raw = valid ? (uint32_t)__ldg(scales + idx) : 0u;
+    if constexpr (F != Fmt::Q4_0) b_raw = valid ? (uint32_t)__ldg(biases + idx) : 0u;
+    else b_raw = 0u;
+}
+
+// Expansion happens where the scale is used, so the load above stays asynchronous.
+template <Fmt F>
+BQ_DEVINL ChunkScale expand_scale(uint32_t s_raw, uint32_t b_raw)
+{
+    ChunkScale cs;
+    if constexpr (F == Fmt::Q4_0 && kQ4Route == 0) {
+        const float d = f16_bits_to_f32(s_raw);
+        cs.s2 = pack_bf16x2_rn(d, d);                                           // d_hi in both halves
+        const float lo = __fsub_rn(d, __uint_as_float(cs.s2 << 16));           // d - d_hi, exact
+        cs.b2 = pack_bf16x2_rn(lo, lo);                                         // exact in bf16
+    } else if constexpr (F == Fmt::Q4_0) {
+        const float d = f16_bits_to_f32(s_raw);
+        // (2^(23-s) + 8) has at most 13 significant bits and d at most 11, so
+        // every constant below is exact in fp32.
+        cs.a[0] = __fmul_rn(d, 0x1p-8f);  cs.c[0] = __fmul_rn(d, -32776.0f);
+        cs.a[1] = __fmul_rn(d, 0x1p-12f); cs.c[1] = __fmul_rn(d, -2056.0f);
+        cs.a[2] = __fmul_rn(d, 0x1p-16f); cs.c[2] = __fmul_rn(d, -136.0f);
     } else if constexpr (F == Fmt::AFF4) {
-        const uint32_t s = __ldg(scales + idx), b = __ldg(biases + idx);
-        cs.s0 = s | (s << 16);
-        cs.s1 = b | (b << 16);
+        cs.s2 = s_raw | (s_raw << 16);
+        cs.b2 = b_raw | (b_raw << 16);
     } else {
-        cs.s0 = __float_as_uint(bf16_bits_to_f32(__ldg(scales + idx)));
-        cs.s1 = __float_as_uint(bf16_bits_to_f32(__ldg(biases + idx)));
+        cs.a[0] = bf16_bits_to_f32(s_raw);
+        cs.c[0] = bf16_bits_to_f32(b_raw);
     }
     return cs;
 }
 
-// Dequantize one 32-bit word of codes into the two A pairs of MMA `j` of the
-// chunk: `first` for k-slots (2t, 2t+1), `second` for (2t+8, 2t+9).
+// Dequantize one 32-bit word of codes into the A pairs of the MMAs it feeds:
+// p[0], p[1] = (first, second) of the first MMA, p[2], p[3] of the second
+// (AFF8: one MMA, p[0], p[1]).  "first" fills k-slots (2t, 2t+1) and "second"
+// (2t+8, 2t+9) of the thread's quad position t.
+//
+// Q4_0, exact: a nibble q placed at bit s >= 8 of the fp32 magic 2^23 gives
+// f = 2^23 + q*2^s, and fma(f, d*2^-s, -(2^(23-s)+8)*d) = (q-8)*d exactly (the
+// addend is exact because s >= 8, the result has <= 14 significant bits), so
+// cvt.rn.bf16x2 rounds d*(q-8) once: bit-identical to the plain definition.
+// The word holds bytes 4i..4i+3 of the block: nibbles n0..n7 are elements
+// 4i, 4i+16, 4i+1, 4i+17, 4i+2, 4i+18, 4i+3, 4i+19; pairs are emitted in
+// natural element order so the activations need no permutation.
 template <Fmt F>
-BQ_DEVINL void dequant_pairs(uint32_t word, int sub, const ChunkScale& cs, uint32_t& first, uint32_t& second)
+BQ_DEVINL void dequant_word(uint32_t word, const ChunkScale& cs, uint32_t (&p)[4])
 {
-    if constexpr (F == Fmt::Q4_0) {
-        // sub 0: (e, e+2) from low nibbles of bytes 0,2 and (e+16, e+18) from high nibbles
-        // sub 1: (e+1, e+3) and (e+17, e+19)   [e = 4 * word index]
-        const uint32_t w = word >> (8 * sub);
-        const uint32_t r0 = and_or(w, 0x000F000Fu, 0x43004300u);        // 128 + q
-        const uint32_t r1 = and_or(w >> 4, 0x000F000Fu, 0x43004300u);
-        const uint32_t q0 = hsub2_bf16(r0, 0x43084308u);                 // q - 8, exact
-        const uint32_t q1 = hsub2_bf16(r1, 0x43084308u);
-        first = hfma2_bf16(q0, cs.s0, hmul2_bf16(q0, cs.s1));
-        second = hfma2_bf16(q1, cs.s0, hmul2_bf16(q1, cs.s1));
+    if constexpr (F == Fmt::Q4_0 && kQ4Route == 0) {
+        // bf16 route: d = d_hi + d_lo (d_hi = bf16(d), d_lo exact in bf16); with
+        // qm8 = q - 8 exact, fma(qm8, d_hi, qm8 * d_lo) rounds the exact qm8 * d once.
+        // Pairs: (4i, 4i+2), (4i+16, 4i+18), (4i+1, 4i+3), (4i+17, 4i+19).
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t qm8 = hsub2_bf16_i<0x43084308u>(and_or_i<0x000F000Fu, 0x43004300u>(word >> (4 * k)));
+            p[k] = hfma2_bf16(qm8, cs.s2, hmul2_bf16(qm8, cs.b2));
+        }
+    } else if constexpr (F == Fmt::Q4_0) {
+        constexpr uint32_t kMagic = 0x4B000000u;
+        const uint32_t lo = word << 8, hi = word >> 12;
+        const float w0 = __fmaf_rn(__uint_as_float(and_or_i<0x00F00u, kMagic>(lo)), cs.a[0], cs.c[0]);    // 4i
+        const float w1 = __fmaf_rn(__uint_as_float(and_or_i<0x0F000u, kMagic>(lo)), cs.a[1], cs.c[1]);    // 4i+16
+        const float w2 = __fmaf_rn(__uint_as_float(and_or_i<0x00F00u, kMagic>(word)), cs.a[0], cs.c[0]);  // 4i+1
+        const float w3 = __fmaf_rn(__uint_as_float(and_or_i<0x0F000u, kMagic>(word)), cs.a[1], cs.c[1]);  // 4i+17
+        const float w4 = __fmaf_rn(__uint_as_float(and_or_i<0xF0000u, kMagic>(word)), cs.a[2], cs.c[2]);  // 4i+2
+        const float w5 = __fmaf_rn(__uint_as_float(and_or_i<0x00F00u, kMagic>(hi)), cs.a[0], cs.c[0]);    // 4i+18
+        const float w6 = __fmaf_rn(__uint_as_float(and_or_i<0x0F000u, kMagic>(hi)), cs.a[1], cs.c[1]);    // 4i+3
+        const float w7 = __fmaf_rn(__uint_as_float(and_or_i<0xF0000u, kMagic>(hi)), cs.a[2], cs.c[2]);    // 4i+19
+        p[0] = pack_bf16x2_rn(w0, w2);   // (4i, 4i+1)
+        p[1] = pack_bf16x2_rn(w1, w3);   // (4i+16, 4i+17)
+        p[2] = pack_bf16x2_rn(w4, w6);   // (4i+2, 4i+3)
+        p[3] = pack_bf16x2_rn(w5, w7);   // (4i+18, 4i+19)
     } else if constexpr (F == Fmt::AFF4) {
-        // sub 0: (e, e+4), (e+1, e+5); sub 1: (e+2, e+6), (e+3, e+7)   [e = 8 * word index]
-        const uint32_t w = word >> (8 * sub);
-        const uint32_t r0 = and_or(w, 0x000F000Fu, 0x43004300u);
-        const uint32_t r1 = and_or(w >> 4, 0x000F000Fu, 0x43004300u);
-        const uint32_t q0 = hsub2_bf16(r0, 0x43004300u);                 // q, exact
-        const uint32_t q1 = hsub2_bf16(r1, 0x43004300u);
-        first = hfma2_bf16(q0, cs.s0, cs.s1);
-        second = hfma2_bf16(q1, cs.s0, cs.s1);
+        // nibble n = element 8i+n.  (word >> 4n) & 0x000F000F | 0x4300 -> bf16 (128+q_n, 128+q_{n+4});
+        // subtracting 128 is exact; one fma.rn.bf16x2 rounds scale*q + bias once.
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            const uint32_t r = and_or_i<0x000F000Fu, 0x43004300u>(word >> (4 * n));
+            p[n] = hfma2_bf16(hsub2_bf16_i<0x43004300u>(r), cs.s2, cs.b2);   // (8i+n, 8i+n+4)
+        }
     } else {
-        // one word per MMA: (e, e+1) and (e+2, e+3)   [e = 4 * word index]
-        const float s = __uint_as_float(cs.s0), b = __uint_as_float(cs.s1);
         float f[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            f[i] = __fsub_rn(__uint_as_float(prmt(word, 0x4B000000u, 0x7650u | i)), 8388608.0f);
-        first = pack_bf16x2_rn(__fmaf_rn(s, f[0], b), __fmaf_rn(s, f[1], b));
-        second = pack_bf16x2_rn(__fmaf_rn(s, f[2], b), __fmaf_rn(s, f[3], b));
+        for (int e = 0; e < 4; ++e)
+            f[e] = __fsub_rn(__uint_as_float(prmt(word, 0x4B000000u, 0x7650u | e)), 8388608.0f);   // byte e
+        p[0] = pack_bf16x2_rn(__fmaf_rn(cs.a[0], f[0], cs.c[0]), __fmaf_rn(cs.a[0], f[1], cs.c[0]));
+        p[1] = pack_bf16x2_rn(__fmaf_rn(cs.a[0], f[2], cs.c[0]), __fmaf_rn(cs.a[0], f[3], cs.c[0]));
+        p[2] = p[3] = 0u;
     }
 }
 
-// B pairs of MMA j (0..7 for 32-element chunks, 0..3 for 16) from the 32 (or
-// 16) activations of the chunk, held as 16 (or 8) u32 pairs (x[2i], x[2i+1]).
+// B pairs (activations) matching dequant_word's A pairs for word i of the
+// chunk; xw holds the chunk's activations as u32 pairs (x[2j], x[2j+1]).
 template <Fmt F>
-BQ_DEVINL void x_pairs(const uint32_t* xw, int j, uint32_t& first, uint32_t& second)
+BQ_DEVINL void x_word_pairs(const uint32_t* xw, int i, uint32_t (&b)[4])
 {
-    if constexpr (F == Fmt::Q4_0) {
-        const int w = j >> 1;
-        const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
-        first = prmt(xw[2 * w], xw[2 * w + 1], sel);
-        second = prmt(xw[8 + 2 * w], xw[8 + 2 * w + 1], sel);
+    if constexpr (F == Fmt::Q4_0 && kQ4Route == 0) {
+        // p[0] = (4i, 4i+2) / p[1] = (4i+16, 4i+18) feed the first MMA, p[2], p[3] the second
+        b[0] = prmt(xw[2 * i], xw[2 * i + 1], 0x5410u);            // x[4i], x[4i+2]
+        b[1] = prmt(xw[8 + 2 * i], xw[9 + 2 * i], 0x5410u);        // x[4i+16], x[4i+18]
+        b[2] = prmt(xw[2 * i], xw[2 * i + 1], 0x7632u);            // x[4i+1], x[4i+3]
+        b[3] = prmt(xw[8 + 2 * i], xw[9 + 2 * i], 0x7632u);        // x[4i+17], x[4i+19]
+    } else if constexpr (F == Fmt::Q4_0) {
+        b[0] = xw[2 * i];         // x[4i], x[4i+1]
+        b[1] = xw[8 + 2 * i];     // x[4i+16], x[4i+17]
+        b[2] = xw[2 * i + 1];     // x[4i+2], x[4i+3]
+        b[3] = xw[9 + 2 * i];     // x[4i+18], x[4i+19]
     } else if constexpr (F == Fmt::AFF4) {
-        const int w = j >> 1, o = j & 1;
-        first = prmt(xw[4 * w + o], xw[4 * w + o + 2], 0x5410u);
-        second = prmt(xw[4 * w + o], xw[4 * w + o + 2], 0x7632u);
+        b[0] = prmt(xw[4 * i], xw[4 * i + 2], 0x5410u);       // (8i, 8i+4)
+        b[1] = prmt(xw[4 * i], xw[4 * i + 2], 0x7632u);       // (8i+1, 8i+5)
+        b[2] = prmt(xw[4 * i + 1], xw[4 * i + 3], 0x5410u);   // (8i+2, 8i+6)
+        b[3] = prmt(xw[4 * i + 1], xw[4 * i + 3], 0x7632u);   // (8i+3, 8i+7)
     } else {
-        first = xw[2 * j];
-        second = xw[2 * j + 1];
+        b[0] = xw[2 * i];
+        b[1] = xw[2 * i + 1];
+        b[2] = b[3] = 0u;
     }
 }
 
 template <Fmt F, int RT>
 struct GemvStage {
-    uint4 w[RT][2];
-    ChunkScale s[RT][2];
+    uint4 w[RT][2];          // 16 code bytes of rows g and g+8 of each m16 tile
+    uint32_t s[RT][2];       // raw scale bits
+    uint32_t b[RT][2];       // raw bias bits (affine)
 };
 
-// One CTA: 16*RT weight rows x all K, KSPLIT warps splitting K; M <= 8*NT tokens.
-template <Fmt F, int NT, int RT, int KSPLIT>
-__global__ void __launch_bounds__(32 * KSPLIT)
+template <Fmt F, int NT>
+BQ_DEVINL void load_x_chunk(const uint16_t* __restrict__ x, int M, int K, int g, int c, bool cvalid,
+                            uint32_t (&xw)[NT][FmtTraits<F>::kChunkElems / 2])
+{
+    constexpr int kCE = FmtTraits<F>::kChunkElems;
+    constexpr int kXWords = kCE / 2;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const int m = 8 * n + g;
+        if (cvalid && m < M) {
+            const uint16_t* xp = x + (int64_t)m * K + (int64_t)c * kCE;
+#pragma unroll
+            for (int v = 0; v < kXWords / 4; ++v) {
+                const uint4 q = ldg_cached(xp + 8 * v);
+                xw[n][4 * v] = q.x; xw[n][4 * v + 1] = q.y; xw[n][4 * v + 2] = q.z; xw[n][4 * v + 3] = q.w;
+            }
+        } else {
+#pragma unroll
+            for (int v = 0; v < kXWords; ++v) xw[n][v] = 0u;
+        }
+    }
+}
+
+// Loads of one 4-chunk step (per thread: one 16-byte chunk of each of its rows).
+template <Fmt F, int RT>
+BQ_DEVINL void load_step(GemvStage<F, RT>& st, const uint8_t* __restrict__ wq, const uint16_t* __restrict__ scales,
+                         const uint16_t* __restrict__ biases, int row_base, int g, int N, int c, bool cvalid,
+                         int64_t row_bytes, int64_t scale_row, int chunks_per_group)
+{
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int row = row_base + 16 * r + 8 * h + g;
+            const bool v = cvalid && row < N;
+            st.w[r][h] = v ? ldg_stream(wq + row * row_bytes + 16 * (int64_t)c) : make_uint4(0, 0, 0, 0);
+            load_scale_raw<F>(scales, biases, row * scale_row + c / chunks_per_group, v, st.s[r][h], st.b[r][h]);
+        }
+}
+
+// One CTA: 16*RT weight rows x all K; KSPLIT warps split K into contiguous
+// ranges and reduce through shared memory; M <= 8*NT tokens.  Each warp runs a
+// software pipeline over its 4-chunk steps with PIPE register stages: the
+// weight loads of step s + PIPE are issued before step s is computed, so every
+// load has PIPE steps of other work to hide behind and no warp ever waits a
+// full memory round trip between batches.
+template <Fmt F, int NT, int RT, int KSPLIT, int PIPE, int MINB>
+__global__ void __launch_bounds__(32 * KSPLIT, MINB)
 gemv_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
             const uint16_t* __restrict__ scales, const uint16_t* __restrict__ biases,
             uint16_t* __restrict__ y, int M, int N, int K, int group_size)
 {
     using T = FmtTraits<F>;
     constexpr int kCE = T::kChunkElems;
-    constexpr int kMmaPerChunk = kCE / 4;     // each MMA takes 4 of a thread's chunk elements
+    constexpr int kWords = 4;                                   // 16-byte chunk
+    constexpr int kMmaPerWord = (F == Fmt::AFF8) ? 1 : 2;
     constexpr int kXWords = kCE / 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -152,77 +255,70 @@ gemv_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
     const int per_warp = (nchunks + KSPLIT - 1) / KSPLIT;
     const int c_begin = warp * per_warp;
     const int c_end = min(nchunks, c_begin + per_warp);
+    const int nsteps = (c_end - c_begin + 3) / 4;
     const int64_t scale_row = (F == Fmt::Q4_0) ? (K / 32) : (K / group_size);
     const int chunks_per_group = (F == Fmt::Q4_0) ? 1 : group_size / kCE;
 
-    float acc[RT][NT][4];
+    // Two accumulator sets (even / odd MMA of a word) halve the dependent MMA chain.
+    float acc[2][RT][NT][4];
 #pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[r][n][i] = 0.0f;
-
-    auto load_stage = [&](GemvStage<F, RT>& st, int c0) {
-        const int c = c0 + t;
-        const bool cvalid = c < c_end;
+    for (int e = 0; e < 2; ++e)
 #pragma unroll
         for (int r = 0; r < RT; ++r)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int row = row_base + 16 * r + 8 * h + g;
-                const bool v = cvalid && row < N;
-                st.w[r][h] = v ? ldg_stream(wq + row * row_bytes + 16 * (int64_t)c) : make_uint4(0, 0, 0, 0);
-                st.s[r][h] = load_scale<F>(scales, biases, row * scale_row + c / chunks_per_group, v);
-            }
-    };
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[e][r][n][i] = 0.0f;
 
-    GemvStage<F, RT> cur, nxt;
-    if (c_begin < c_end) load_stage(cur, c_begin);
-    for (int c0 = c_begin; c0 < c_end; c0 += 4) {
-        if (c0 + 4 < c_end) load_stage(nxt, c0 + 4);
-        const int c = c0 + t;
-        const bool cvalid = c < c_end;
-        // activations of this chunk for each token tile
-        uint32_t xw[NT][kXWords];
+    auto step_chunk = [&](int s) { return c_begin + 4 * s + t; };
+    GemvStage<F, RT> ring[PIPE];
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int m = 8 * n + g;
-            if (cvalid && m < M) {
-                const uint16_t* xp = x + (int64_t)m * K + (int64_t)c * kCE;
+    for (int d = 0; d < PIPE; ++d)
+        load_step<F, RT>(ring[d], wq, scales, biases, row_base, g, N, step_chunk(d), d < nsteps && step_chunk(d) < c_end,
+                         row_bytes, scale_row, chunks_per_group);
+
+    for (int s0 = 0; s0 < nsteps; s0 += PIPE) {
 #pragma unroll
-                for (int v = 0; v < kXWords / 4; ++v) {
-                    const uint4 q = ldg_cached(xp + 8 * v);
-                    xw[n][4 * v] = q.x; xw[n][4 * v + 1] = q.y; xw[n][4 * v + 2] = q.z; xw[n][4 * v + 3] = q.w;
+        for (int d = 0; d < PIPE; ++d) {
+            const int s = s0 + d;
+            if (s < nsteps) {
+                const int c = step_chunk(s);
+                uint32_t xw[NT][kXWords];
+                load_x_chunk<F, NT>(x, M, K, g, c, c < c_end, xw);
+                ChunkScale cs[RT][2];
+#pragma unroll
+                for (int r = 0; r < RT; ++r)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) cs[r][h] = expand_scale<F>(ring[d].s[r][h], ring[d].b[r][h]);
+#pragma unroll
+                for (int i = 0; i < kWords; ++i) {
+                    uint32_t b[NT][4];
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) x_word_pairs<F>(xw[n], i, b[n]);
+#pragma unroll
+                    for (int r = 0; r < RT; ++r) {
+                        uint32_t pa[2][4];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint4 wv = ring[d].w[r][h];
+                            const uint32_t word = i == 0 ? wv.x : i == 1 ? wv.y : i == 2 ? wv.z : wv.w;
+                            dequant_word<F>(word, cs[r][h], pa[h]);
+                        }
+#pragma unroll
+                        for (int mm = 0; mm < kMmaPerWord; ++mm)
+#pragma unroll
+                            for (int n = 0; n < NT; ++n)
+                                // A regs: row g first, row g+8 first, row g second, row g+8 second
+                                mma_bf16_16816(acc[mm][r][n], pa[0][2 * mm], pa[1][2 * mm], pa[0][2 * mm + 1],
+                                               pa[1][2 * mm + 1], b[n][2 * mm], b[n][2 * mm + 1]);
+                    }
                 }
-            } else {
-#pragma unroll
-                for (int v = 0; v < kXWords; ++v) xw[n][v] = 0u;
+                // refill this ring slot with step s + PIPE (PIPE - 1 steps of cover)
+                const int cn = step_chunk(s + PIPE);
+                load_step<F, RT>(ring[d], wq, scales, biases, row_base, g, N, cn, s + PIPE < nsteps && cn < c_end,
+                                 row_bytes, scale_row, chunks_per_group);
             }
         }
-#pragma unroll
-        for (int j = 0; j < kMmaPerChunk; ++j) {
-            uint32_t b0[NT], b1[NT];
-#pragma unroll
-            for (int n = 0; n < NT; ++n) x_pairs<F>(xw[n], j, b0[n], b1[n]);
-#pragma unroll
-            for (int r = 0; r < RT; ++r) {
-                uint32_t a[4];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint4 wv = cur.w[r][h];
-                    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
-                    uint32_t f, s;
-                    if constexpr (F == Fmt::AFF8) dequant_pairs<F>(words[j], 0, cur.s[r][h], f, s);
-                    else dequant_pairs<F>(words[j >> 1], j & 1, cur.s[r][h], f, s);
-                    a[h] = f;          // a0a1 (row g) / a2a3 (row g+8)
-                    a[2 + h] = s;      // a4a5 / a6a7
-                }
-#pragma unroll
-                for (int n = 0; n < NT; ++n) mma_bf16_16816(acc[r][n], a[0], a[1], a[2], a[3], b0[n], b1[n]);
-            }
-        }
-        cur = nxt;
     }
 
     // Reduce the KSPLIT partial tiles through shared memory.
@@ -231,10 +327,10 @@ gemv_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
     for (int r = 0; r < RT; ++r)
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
-            red[warp][16 * r + g][8 * n + 2 * t] = acc[r][n][0];
-            red[warp][16 * r + g][8 * n + 2 * t + 1] = acc[r][n][1];
-            red[warp][16 * r + g + 8][8 * n + 2 * t] = acc[r][n][2];
-            red[warp][16 * r + g + 8][8 * n + 2 * t + 1] = acc[r][n][3];
+            red[warp][16 * r + g][8 * n + 2 * t] = acc[0][r][n][0] + acc[1][r][n][0];
+            red[warp][16 * r + g][8 * n + 2 * t + 1] = acc[0][r][n][1] + acc[1][r][n][1];
+            red[warp][16 * r + g + 8][8 * n + 2 * t] = acc[0][r][n][2] + acc[1][r][n][2];
+            red[warp][16 * r + g + 8][8 * n + 2 * t + 1] = acc[0][r][n][3] + acc[1][r][n][3];
         }
     __syncthreads();
     for (int idx = threadIdx.x; idx < 16 * RT * 8 * NT; idx += 32 * KSPLIT) {

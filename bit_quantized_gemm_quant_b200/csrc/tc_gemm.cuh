@@ -66,13 +66,6 @@ BQ_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, u
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-BQ_DEVINL uint4 ld_shared_v4(uint32_t addr)
-{
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
-                 : "memory");
-    return v;
-}
 
 // --- dequantization of one thread's 32 weights (half a k-block of one row) ---
 
@@ -86,8 +79,8 @@ BQ_DEVINL void deq_q4_0_half(uint4 raw, uint32_t dhi2, uint32_t dlo2, uint32_t a
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
             const uint32_t t = prmt(words[w], 0u, p ? 0x4342u : 0x4140u);   // [b, 0, b', 0]
-            const uint32_t l = hsub2_bf16(and_or(t, 0x000F000Fu, 0x43004300u), 0x43084308u);
-            const uint32_t u = hsub2_bf16(and_or(t >> 4, 0x000F000Fu, 0x43004300u), 0x43084308u);
+            const uint32_t l = hsub2_bf16_i<0x43084308u>(and_or_i<0x000F000Fu, 0x43004300u>(t));
+            const uint32_t u = hsub2_bf16_i<0x43084308u>(and_or_i<0x000F000Fu, 0x43004300u>(t >> 4));
             lo[2 * w + p] = hfma2_bf16(l, dhi2, hmul2_bf16(l, dlo2));
             hi[2 * w + p] = hfma2_bf16(u, dhi2, hmul2_bf16(u, dlo2));
         }
@@ -108,7 +101,7 @@ BQ_DEVINL void deq_aff4_half(uint4 raw, uint32_t s2, uint32_t b2, uint32_t a_til
         uint32_t v[4];   // v[n] = (element n, element n+4) of the word
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
-            const uint32_t q = hsub2_bf16(and_or(words[i] >> (4 * n), 0x000F000Fu, 0x43004300u), 0x43004300u);
+            const uint32_t q = hsub2_bf16_i<0x43004300u>(and_or_i<0x000F000Fu, 0x43004300u>(words[i] >> (4 * n)));
             v[n] = hfma2_bf16(q, s2, b2);
         }
         st_shared_v4(a_tile + sw128_offset(r, 4 * h + i), prmt(v[0], v[1], 0x5410u), prmt(v[2], v[3], 0x5410u),

@@ -65,6 +65,21 @@ BQ_DEVINL bool mbar_wait(uint32_t bar, uint32_t parity)
     return true;
 }
 
+BQ_DEVINL uint4 ld_shared_v4(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+BQ_DEVINL uint32_t ld_shared_u16(uint32_t addr)
+{
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 // ------------------------------------------------------------------ TMA
 BQ_DEVINL void tma_prefetch_desc(const CUtensorMap* map)
 {
@@ -78,6 +93,14 @@ BQ_DEVINL void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];"
         ::"r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y) : "memory");
+}
+
+// 1-D bulk copy global -> this CTA's shared memory (no multicast); completes
+// `bytes` on `bar`.  Addresses and size must be multiples of 16 bytes.
+BQ_DEVINL void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05

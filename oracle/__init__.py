@@ -173,6 +173,21 @@ def matmul_ref(x_bf16, w_bf16, rows=None, nthreads: int | None = None):
     return y, a, used
 
 
-def tolerance(a: np.ndarray) -> np.ndarray:
-    """Allowed |y_gpu - y_ref| for outputs with absolute-product sums ``a``."""
-    return 2e-3 * a + 1e-5
+def bf16_half_ulp(y: np.ndarray) -> np.ndarray:
+    """Half a bf16 unit in the last place of |y| (float64): the largest error the
+    output's own round-to-nearest to bf16 (8 significant bits) can add."""
+    ay = np.abs(np.asarray(y, np.float64))
+    e = np.floor(np.log2(np.where(ay > 0, ay, 1.0)))
+    e = np.maximum(e, -126.0)                       # bf16 subnormal spacing below 2^-126
+    return np.where(ay > 0, np.exp2(e - 8.0), 0.0)
+
+
+def tolerance(a: np.ndarray, y_ref: np.ndarray | None = None) -> np.ndarray:
+    """Allowed |y_gpu - y_ref| for outputs with absolute-product sums ``a``:
+    2e-3 * a + 1e-5 for the accumulation, plus half a bf16 ulp of y_ref for the
+    rounding of the bf16 output itself (which alone can reach 2^-8 |y|, above
+    2e-3 * a whenever |y| is close to a)."""
+    tol = 2e-3 * a + 1e-5
+    if y_ref is not None:
+        tol = tol + bf16_half_ulp(y_ref)
+    return tol

@@ -55,7 +55,7 @@ def assert_within_tolerance(y_gpu: torch.Tensor, y_ref: np.ndarray, a_ref: np.nd
     assert got.shape == y_ref.shape, (got.shape, y_ref.shape)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     err = np.abs(got - y_ref)
-    tol = oracle.tolerance(a_ref)
+    tol = oracle.tolerance(a_ref, y_ref)
     bad = err > tol
     if bad.any():
         i = np.unravel_index(np.argmax(err - tol), err.shape)

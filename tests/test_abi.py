@@ -130,3 +130,14 @@ def test_dispatcher_env_overrides(L):
     assert _select_in_subprocess({"BQ_TC_MIN_M": "1000"}, Ms) == [1, 1, 1, 1, 2, 2, 2]   # clamped to 33
     assert _select_in_subprocess({"BQ_PAIR_MIN_M": "512"}, Ms) == [1, 1, 1, 1, 2, 3, 3]
     assert _select_in_subprocess({"BQ_PAIR_MIN_M": "0"}, Ms) == [1, 1, 1, 1, 2, 2, 2]
+
+
+def test_empty_problems_need_no_pointers(L):
+    # empty shapes return BQ_OK before any pointer is looked at (torch gives NULL for empty tensors)
+    assert qmm(L, x=None, wq=None, s=None, y=None, M=0) == 0
+    assert qmm(L, x=None, wq=None, s=None, y=None, N=0) == 0
+    assert qmm(L, y=None, K=0) == 1                   # K == 0 still writes y = 0
+    assert L.q4_0_dequantize(None, None, None, 0, 64, None) == 0
+    assert L.affine_dequantize(None, None, None, None, 4, 0, 64, 8, None) == 0
+    assert L.bf16_matmul(None, None, None, 0, 4, 16, None) == 0
+    assert L.q4_0_quantize(None, None, None, 0, 64, None) == 0
