@@ -194,7 +194,10 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     const int budget = di.max_smem_optin - 1024 - 256;
     const int stages = std::min<int>(8, budget / (int)stage);
     if (stages < 2) return BQ_ERR_UNSUPPORTED;
-    const size_t smem = 1024 + (size_t)stages * stage + 256;
+    size_t smem = 1024 + (size_t)stages * stage + 256;
+    // Fused modes allocate all 512 TMEM columns: keep them at one CTA per SM so
+    // no allocation ever waits for another CTA's release.
+    if (MODE != kModeBF16) smem = std::max<size_t>(smem, (size_t)di.max_smem_optin / 2 + 1024);
 
     CUtensorMap tm_x, tm_a;
     if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, M, K, bn, 64, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -223,9 +226,11 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     p.K = (int)K;
     p.bn = bn;
     p.stages = stages;
+    p.vec_scales = (K % 512 == 0) ? 1 : 0;
     int cols = 32;
     while (cols < bn) cols <<= 1;
-    p.tmem_cols = cols;
+    p.tmem_cols = (MODE == kModeBF16) ? cols : 512;   // fused: accumulator + staged A tiles (see tc_gemm.cuh)
+    if (MODE != kModeBF16 && 256 + 32 * stages > 512) return BQ_ERR_UNSUPPORTED;
     dim3 grid((unsigned)((M + bn - 1) / bn), (unsigned)((N + 127) / 128));
     if (grid.y > 65535u) return BQ_ERR_SHAPE;
     tc_gemm_kernel<MODE><<<grid, C::kThreads, smem, st>>>(tm_x, tm_a, p);

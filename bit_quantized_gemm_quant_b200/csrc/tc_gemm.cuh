@@ -38,7 +38,7 @@ template <int MODE> struct TcCfg {
     static constexpr int kMmaWarp = kTmaWarp + 1;
     static constexpr int kThreads = 32 * (kMmaWarp + 1);
     static constexpr int kCodeBytesPerRow = (MODE == kModeAff8) ? 64 : 32;   // per 64-element k-block
-    static constexpr uint32_t kABytes = 128 * 128;
+    static constexpr uint32_t kABytes = (MODE == kModeBF16) ? 128 * 128 : 0;   // fused: A lives in TMEM
     static constexpr uint32_t kCBytes = (MODE == kModeBF16) ? 0 : 128 * kCodeBytesPerRow;
 };
 
@@ -50,30 +50,25 @@ struct TcParams {
     int bn;                   // token tile = MMA N, multiple of 16 in [16, 256]
     int stages;
     int tmem_cols;            // power of two >= max(32, bn)
+    int vec_scales;           // scale rows are 16-byte aligned and hold whole 8-scale windows
 };
 
+// Shared memory per pipeline stage: the activation tile (bn x 64 bf16, 128B
+// swizzled) plus either the bf16 weight tile (128 x 64) or the packed codes.
+// Fused modes keep the dequantized weight tile in TMEM instead.
 __host__ __device__ constexpr uint32_t tc_stage_bytes(int mode, int bn)
 {
-    return 128u * 128u + (uint32_t)bn * 128u + (mode == kModeBF16 ? 0u : (mode == kModeAff8 ? 128u * 64u : 128u * 32u));
+    return (uint32_t)bn * 128u +
+           (mode == kModeBF16 ? 128u * 128u : (mode == kModeAff8 ? 128u * 64u : 128u * 32u));
 }
-
-// Byte offset of the 16-byte chunk `c` (K elements 8c..8c+7) of row `r` in a
-// 128B-swizzled K-major tile with 128-byte rows.
-BQ_DEVINL uint32_t sw128_offset(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
-
-BQ_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
-{
-    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
 
 // --- dequantization of one thread's 32 weights (half a k-block of one row) ---
+// Each returns 16 bf16x2 registers in natural K order: out[j] = (2j, 2j+1).
 
-// Q4_0: d = d_hi + d_lo split (see gemv.cuh); the 16 code bytes of one block.
-BQ_DEVINL void deq_q4_0_half(uint4 raw, uint32_t dhi2, uint32_t dlo2, uint32_t a_tile, int r, int h)
+// Q4_0: exact, d = d_hi + d_lo split (see gemv.cuh); the 16 code bytes of one block.
+BQ_DEVINL void deq_q4_0_half(uint4 raw, uint32_t dhi2, uint32_t dlo2, uint32_t (&out)[16])
 {
     const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
-    uint32_t lo[8], hi[8];   // natural-order pairs: lo = elements 0..15, hi = 16..31
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
 #pragma unroll
@@ -81,19 +76,14 @@ BQ_DEVINL void deq_q4_0_half(uint4 raw, uint32_t dhi2, uint32_t dlo2, uint32_t a
             const uint32_t t = prmt(words[w], 0u, p ? 0x4342u : 0x4140u);   // [b, 0, b', 0]
             const uint32_t l = hsub2_bf16_i<0x43084308u>(and_or_i<0x000F000Fu, 0x43004300u>(t));
             const uint32_t u = hsub2_bf16_i<0x43084308u>(and_or_i<0x000F000Fu, 0x43004300u>(t >> 4));
-            lo[2 * w + p] = hfma2_bf16(l, dhi2, hmul2_bf16(l, dlo2));
-            hi[2 * w + p] = hfma2_bf16(u, dhi2, hmul2_bf16(u, dlo2));
+            out[2 * w + p] = hfma2_bf16(l, dhi2, hmul2_bf16(l, dlo2));        // elements 4w+2p, +1
+            out[8 + 2 * w + p] = hfma2_bf16(u, dhi2, hmul2_bf16(u, dlo2));    // elements 16+4w+2p, +1
         }
     }
-    const int c0 = 4 * h;
-    st_shared_v4(a_tile + sw128_offset(r, c0 + 0), lo[0], lo[1], lo[2], lo[3]);
-    st_shared_v4(a_tile + sw128_offset(r, c0 + 1), lo[4], lo[5], lo[6], lo[7]);
-    st_shared_v4(a_tile + sw128_offset(r, c0 + 2), hi[0], hi[1], hi[2], hi[3]);
-    st_shared_v4(a_tile + sw128_offset(r, c0 + 3), hi[4], hi[5], hi[6], hi[7]);
 }
 
 // Affine 4-bit: 4 words of sequential nibbles; w = fma.rn.bf16x2(q, scale, bias).
-BQ_DEVINL void deq_aff4_half(uint4 raw, uint32_t s2, uint32_t b2, uint32_t a_tile, int r, int h)
+BQ_DEVINL void deq_aff4_half(uint4 raw, uint32_t s2, uint32_t b2, uint32_t (&out)[16])
 {
     const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
@@ -104,47 +94,86 @@ BQ_DEVINL void deq_aff4_half(uint4 raw, uint32_t s2, uint32_t b2, uint32_t a_til
             const uint32_t q = hsub2_bf16_i<0x43004300u>(and_or_i<0x000F000Fu, 0x43004300u>(words[i] >> (4 * n)));
             v[n] = hfma2_bf16(q, s2, b2);
         }
-        st_shared_v4(a_tile + sw128_offset(r, 4 * h + i), prmt(v[0], v[1], 0x5410u), prmt(v[2], v[3], 0x5410u),
-                     prmt(v[0], v[1], 0x7632u), prmt(v[2], v[3], 0x7632u));
+        out[4 * i + 0] = prmt(v[0], v[1], 0x5410u);
+        out[4 * i + 1] = prmt(v[2], v[3], 0x5410u);
+        out[4 * i + 2] = prmt(v[0], v[1], 0x7632u);
+        out[4 * i + 3] = prmt(v[2], v[3], 0x7632u);
     }
 }
 
 // Affine 8-bit: 8 words of bytes; w = bf16_rne(fmaf(scale, q, bias)).
-BQ_DEVINL void deq_aff8_half(uint4 raw0, uint4 raw1, float s, float b, uint32_t a_tile, int r, int h)
+BQ_DEVINL void deq_aff8_half(uint4 raw0, uint4 raw1, float s, float b, uint32_t (&out)[16])
 {
     const uint32_t words[8] = {raw0.x, raw0.y, raw0.z, raw0.w, raw1.x, raw1.y, raw1.z, raw1.w};
-    uint32_t o[16];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         float f[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
             f[e] = __fsub_rn(__uint_as_float(prmt(words[i], 0x4B000000u, 0x7650u | e)), 8388608.0f);
-        o[2 * i] = pack_bf16x2_rn(__fmaf_rn(s, f[0], b), __fmaf_rn(s, f[1], b));
-        o[2 * i + 1] = pack_bf16x2_rn(__fmaf_rn(s, f[2], b), __fmaf_rn(s, f[3], b));
+        out[2 * i] = pack_bf16x2_rn(__fmaf_rn(s, f[0], b), __fmaf_rn(s, f[1], b));
+        out[2 * i + 1] = pack_bf16x2_rn(__fmaf_rn(s, f[2], b), __fmaf_rn(s, f[3], b));
     }
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-        st_shared_v4(a_tile + sw128_offset(r, 4 * h + c), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
 }
 
 struct DeqScale { uint32_t a, b; };
 
+// Scales of one dequant thread's row, fetched a whole window of k-blocks ahead:
+// one 16-byte vector holds 8 consecutive 16-bit scales = 4 k-blocks of Q4_0
+// (two blocks per k-block) or 8 k-blocks of affine (one group per k-block).
 template <int MODE>
-BQ_DEVINL DeqScale deq_load_scale(const TcParams& p, int row, int it, int h)
+struct ScaleWindow {
+    static constexpr int kSpan = (MODE == kModeQ4_0) ? 4 : 8;   // k-blocks per window
+    uint4 s, b;
+};
+
+BQ_DEVINL uint32_t halfword(const uint4& v, int k)
 {
-    DeqScale r{0u, 0u};
-    if (row >= p.N) return r;
-    if constexpr (MODE == kModeQ4_0) {
-        const float d = f16_bits_to_f32(__ldg(p.scales + (int64_t)row * (p.K / 32) + 2 * it + h));
-        const uint32_t hi = f32_to_bf16_bits(d);
-        const uint32_t lo = f32_to_bf16_bits(__fsub_rn(d, bf16_bits_to_f32(hi)));
-        r.a = hi | (hi << 16);
-        r.b = lo | (lo << 16);
+    const uint32_t w = (k < 2) ? v.x : (k < 4) ? v.y : (k < 6) ? v.z : v.w;
+    return (w >> (16 * (k & 1))) & 0xFFFFu;
+}
+
+template <int MODE>
+BQ_DEVINL ScaleWindow<MODE> load_scale_window(const TcParams& p, int row, int win)
+{
+    ScaleWindow<MODE> w;
+    w.s = w.b = make_uint4(0, 0, 0, 0);
+    if (row >= p.N) return w;
+    const int per_row = (MODE == kModeQ4_0) ? p.K / 32 : p.K / 64;          // 16-bit scales per row
+    const int first = win * 8;
+    const uint16_t* srow = p.scales + (int64_t)row * per_row;
+    const uint16_t* brow = p.biases + (int64_t)row * per_row;
+    if (first >= per_row) return w;                                           // window past the row end
+    if (p.vec_scales) {                                                       // 16-byte aligned rows, whole windows
+        w.s = __ldg(reinterpret_cast<const uint4*>(srow + first));
+        if constexpr (MODE != kModeQ4_0) w.b = __ldg(reinterpret_cast<const uint4*>(brow + first));
     } else {
-        const int64_t gi = (int64_t)row * (p.K / 64) + it;
-        r.a = __ldg(p.scales + gi);
-        r.b = __ldg(p.biases + gi);
+        uint32_t sv[8], bv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const bool in = first + k < per_row;
+            sv[k] = in ? __ldg(srow + first + k) : 0u;
+            bv[k] = (MODE != kModeQ4_0 && in) ? __ldg(brow + first + k) : 0u;
+        }
+        w.s = make_uint4(sv[0] | sv[1] << 16, sv[2] | sv[3] << 16, sv[4] | sv[5] << 16, sv[6] | sv[7] << 16);
+        w.b = make_uint4(bv[0] | bv[1] << 16, bv[2] | bv[3] << 16, bv[4] | bv[5] << 16, bv[6] | bv[7] << 16);
+    }
+    return w;
+}
+
+// Expanded scale of k-block `it` (half `h` for Q4_0) from its window.
+template <int MODE>
+BQ_DEVINL DeqScale window_scale(const ScaleWindow<MODE>& w, int it, int h)
+{
+    DeqScale r;
+    if constexpr (MODE == kModeQ4_0) {
+        const float d = f16_bits_to_f32(halfword(w.s, 2 * (it % 4) + h));
+        r.a = pack_bf16x2_rn(d, d);                                            // d_hi
+        const float lo = __fsub_rn(d, __uint_as_float(r.a << 16));           // d - d_hi, exact
+        r.b = pack_bf16x2_rn(lo, lo);
+    } else {
+        r.a = halfword(w.s, it % 8);
+        r.b = halfword(w.b, it % 8);
     }
     return r;
 }
@@ -163,10 +192,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     const uint32_t b_bytes = (uint32_t)p.bn * 128u;
 
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    const uint32_t a_base = base;
-    const uint32_t b_base = a_base + (uint32_t)S * C::kABytes;
-    const uint32_t c_base = b_base + (uint32_t)S * b_bytes;
+    const uint32_t b_base = base;                                      // activation tiles (1024-aligned)
+    const uint32_t a_base = b_base + (uint32_t)S * b_bytes;            // bf16 weight tiles (kModeBF16)
+    const uint32_t c_base = a_base + (uint32_t)S * C::kABytes;         // packed code tiles (fused)
     const uint32_t bar_base = c_base + (uint32_t)S * C::kCBytes;
+    // TMEM columns: accumulator [0, bn); fused modes keep stage s of the
+    // dequantized weight tile (128 lanes x 64 bf16 = 32 columns) at 256 + 32 s.
+    auto a_tmem_col = [&](int s) { return 256u + 32u * (uint32_t)s; };
     auto full_bar = [&](int s) { return bar_base + 8u * (uint32_t)s; };
     auto afull_bar = [&](int s) { return bar_base + 8u * (uint32_t)(S + s); };
     auto empty_bar = [&](int s) { return bar_base + 8u * (uint32_t)(2 * S + s); };
@@ -226,12 +258,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     if (!mbar_wait(afull_bar(s), ph)) break;
                 }
                 tc_fence_after();
-                const uint32_t a_addr = a_base + (uint32_t)s * C::kABytes;
                 const uint32_t b_addr = b_base + (uint32_t)s * b_bytes;
+                if constexpr (MODE == kModeBF16) {
+                    const uint32_t a_addr = a_base + (uint32_t)s * C::kABytes;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16_ss(tmem_base, umma_desc_k_sw128(a_addr + 32u * kk), umma_desc_k_sw128(b_addr + 32u * kk),
-                                idesc, (it | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(tmem_base, umma_desc_k_sw128(a_addr + 32u * kk),
+                                    umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it | kk) != 0 ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)   // K = 16 per MMA = 8 TMEM columns of A
+                        umma_f16_ts(tmem_base, tmem_base + a_tmem_col(s) + 8u * kk,
+                                    umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it | kk) != 0 ? 1u : 0u);
+                }
                 umma_commit(empty_bar(s));
             }
             umma_commit(tmem_full_bar);   // also on an early exit: nothing stays in flight
@@ -242,25 +281,33 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int r = 32 * (warp & 3) + lane;   // weight row within the tile
         const int h = warp >> 2;                // which 32-element half of each k-block
         const int row = n0 + r;
-        DeqScale sc = deq_load_scale<MODE>(p, row, 0, h);
+        constexpr int kSpan = ScaleWindow<MODE>::kSpan;
+        ScaleWindow<MODE> win_cur = load_scale_window<MODE>(p, row, 0);
+        ScaleWindow<MODE> win_nxt = load_scale_window<MODE>(p, row, 1);
         for (int it = 0; it < nk; ++it) {
             const int s = it % S;
             const uint32_t ph = (uint32_t)(it / S) & 1u;
-            const DeqScale sc_next = (it + 1 < nk) ? deq_load_scale<MODE>(p, row, it + 1, h) : sc;
+            if (it > 0 && it % kSpan == 0) {                  // next window; fetch the one after it
+                win_cur = win_nxt;
+                win_nxt = load_scale_window<MODE>(p, row, it / kSpan + 1);
+            }
+            const DeqScale sc = window_scale<MODE>(win_cur, it, h);
             if (!mbar_wait(full_bar(s), ph)) break;
             const uint32_t codes = c_base + (uint32_t)s * C::kCBytes + (uint32_t)(r * C::kCodeBytesPerRow);
-            const uint32_t a_tile = a_base + (uint32_t)s * C::kABytes;
+            uint32_t wv[16];
             if constexpr (MODE == kModeQ4_0) {
-                deq_q4_0_half(ld_shared_v4(codes + 16u * h), sc.a, sc.b, a_tile, r, h);
+                deq_q4_0_half(ld_shared_v4(codes + 16u * h), sc.a, sc.b, wv);
             } else if constexpr (MODE == kModeAff4) {
-                deq_aff4_half(ld_shared_v4(codes + 16u * h), sc.a | (sc.a << 16), sc.b | (sc.b << 16), a_tile, r, h);
+                deq_aff4_half(ld_shared_v4(codes + 16u * h), sc.a | (sc.a << 16), sc.b | (sc.b << 16), wv);
             } else {
                 deq_aff8_half(ld_shared_v4(codes + 32u * h), ld_shared_v4(codes + 32u * h + 16u),
-                              bf16_bits_to_f32(sc.a), bf16_bits_to_f32(sc.b), a_tile, r, h);
+                              bf16_bits_to_f32(sc.a), bf16_bits_to_f32(sc.b), wv);
             }
-            fence_proxy_async_smem();
+            // row r = TMEM lane r; this thread's 32 weights = 16 columns of the stage's A tile
+            tmem_st_32x32b_x16(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + a_tmem_col(s) + 16u * h, wv);
+            tmem_wait_st();
+            tc_fence_before();
             mbar_arrive(afull_bar(s));
-            sc = sc_next;
         }
     }
 
