@@ -322,7 +322,10 @@ def run_prefill(args, world, device, peaks, fmt, Ms):
         y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
         flops = 2.0 * M * N * K
         reps = max(2, min(50, int(2e13 / flops)))
-        t_fused = kernel_seconds([lambda: bq.quant_matmul_ex(x, wq, s, b, gs, bits, True, "tc_fused", out=y)], reps)
+        fused_path = "tc_fused" if M > 32 else "gemv"
+        t_fused = kernel_seconds([lambda: bq.quant_matmul_ex(x, wq, s, b, gs, bits, True, fused_path, out=y)], reps)
+        t_auto = kernel_seconds([lambda: bq.quant_matmul_ex(x, wq, s, b, gs, bits, True, "auto", workspace=ws,
+                                                           out=y)], reps)
         t_pair = kernel_seconds([lambda: bq.quant_matmul_ex(x, wq, s, b, gs, bits, True, "dequant_gemm",
                                                            workspace=ws, out=y)], reps)
         wb = ws.view(N, K)
@@ -339,7 +342,9 @@ def run_prefill(args, world, device, peaks, fmt, Ms):
                        "pair_tflops": round(flops / t_pair / 1e12, 1),
                        "bf16_gemm_tflops": round(flops / t_gemm / 1e12, 1),
                        "cublas_bf16_tflops": round(flops / t_cublas / 1e12, 1),
-                       "fused_us": round(t_fused * 1e6, 2), "pair_us": round(t_pair * 1e6, 2)}
+                       "fused_us": round(t_fused * 1e6, 2), "pair_us": round(t_pair * 1e6, 2),
+                       "auto_path": bq.quant_matmul_select_path(M, N, K, gs, bits),
+                       "auto_tflops": round(flops / t_auto / 1e12, 1)}
         del x, y
     return res, total_flops / total_s / 1e12
 
@@ -380,7 +385,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["q4_0_decode", "affine4_prefill", "affine8_sweep"], default="q4_0_decode")
+    ap.add_argument("--workload", choices=["q4_0_decode", "affine4_prefill", "affine8_sweep", "q4_0_prefill"],
+                    default="q4_0_decode")
+    ap.add_argument("--ms", type=str, default=None, help="comma-separated M list for a prefill workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the secondary prefill measurement")
@@ -420,13 +427,17 @@ def main(argv=None):
             pre, _ = run_prefill(args, world, device, peaks, "affine4", (2048,))
             r["secondary"] = {"prefill_affine4_n12288_k4096_m2048": pre["2048"]}
     else:
-        fmt, Ms = ("affine4", (512, 2048, 8192)) if args.workload == "affine4_prefill" else \
-            ("affine8", (1, 32, 512, 2048, 8192))
+        fmt, Ms = {"affine4_prefill": ("affine4", (512, 2048, 8192)),
+                   "affine8_sweep": ("affine8", (1, 32, 512, 2048, 8192)),
+                   "q4_0_prefill": ("q4_0", (512, 2048, 8192))}[args.workload]
+        if args.ms:
+            Ms = tuple(int(v) for v in args.ms.split(","))
         with ClockSampler(local_rank) as clk:
             res, tflops = run_prefill(args, world, device, peaks, fmt, Ms)
         r = {"value": round(tflops, 1), "unit": "TFLOP/s", "ms_per_step": None, "higher_is_better": True,
              "dtype": f"{fmt} weights, bf16 activations, fp32 accumulate",
-             "config": {"workload": f"{fmt}_g64_n12288_k4096", "M": list(Ms)}, "per_m": res,
+             "config": {"workload": f"{fmt}_g{_fmt_args(fmt)[0]}_n12288_k4096", "M": list(Ms)}, "per_m": res,
+             "crossover_m": next((int(m) for m, v in res.items() if v["pair_us"] < v["fused_us"]), None),
              "roofline": {"bound": "tensor", "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                           "frac": round(tflops / peaks["bf16_tflops"], 4), "achieved": round(tflops, 1),
                           "traffic": None},
@@ -438,7 +449,7 @@ def main(argv=None):
             "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": r["dtype"], "data": "synthetic (seeded N(0, 0.02) weights, N(0, 1) bf16 activations)",
             "config": dict(r["config"], parallelism=f"replicas x{world}")}
-    for k in ("per_m", "roofline", "e2e", "gpu_launches", "clocks", "secondary"):
+    for k in ("per_m", "crossover_m", "roofline", "e2e", "gpu_launches", "clocks", "secondary"):
         if k in r:
             line[k] = r[k]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -164,16 +164,19 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void
 }
 
 // ------------------------------------------------------------------ tensor-core GEMM
-// Token tile bn (MMA N): minimise waves * (bn + per-tile overhead) over the SMs.
-int choose_bn(int64_t M, int64_t N, int num_sms)
+// Token tile bn (MMA N) for the persistent kernel: each CTA runs
+// ceil(tiles / grid) tiles, each costing about bn + overhead (token units; the
+// overhead stands for per-tile work independent of bn, e.g. dequantization).
+int choose_bn(int64_t M, int64_t N, int num_sms, int max_bn, int overhead)
 {
     const int64_t ntiles = (N + 127) / 128;
     int best_bn = 16;
     int64_t best_cost = INT64_MAX;
-    for (int bn = 16; bn <= 256; bn += 16) {
+    for (int bn = 16; bn <= max_bn; bn += 16) {
         const int64_t tiles = ((M + bn - 1) / bn) * ntiles;
-        const int64_t waves = (tiles + num_sms - 1) / num_sms;
-        const int64_t cost = waves * (bn + 32);
+        const int64_t grid = std::min<int64_t>(tiles, num_sms);
+        const int64_t rounds = (tiles + grid - 1) / grid;
+        const int64_t cost = rounds * (bn + overhead);
         if (cost < best_cost || (cost == best_cost && bn > best_bn)) {
             best_cost = cost;
             best_bn = bn;
@@ -189,15 +192,18 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
 {
     using C = TcCfg<MODE>;
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return BQ_ERR_SHAPE;
-    const int bn = choose_bn(M, N, di.num_sms);
+    constexpr bool kFused = MODE != kModeBF16;
+    // TMEM (512 columns): two accumulators acc_stride columns apart and, in fused
+    // modes, one 32-column dequantized weight tile per pipeline stage.
+    const int bn = kFused ? choose_bn(M, N, di.num_sms, 192, 64) : choose_bn(M, N, di.num_sms, 256, 32);
+    const int acc_stride = kFused ? (bn + 31) / 32 * 32 : 256;
     const uint32_t stage = tc_stage_bytes(MODE, bn);
-    const int budget = di.max_smem_optin - 1024 - 256;
-    const int stages = std::min<int>(8, budget / (int)stage);
-    if (stages < 2) return BQ_ERR_UNSUPPORTED;
-    size_t smem = 1024 + (size_t)stages * stage + 256;
-    // Fused modes allocate all 512 TMEM columns: keep them at one CTA per SM so
-    // no allocation ever waits for another CTA's release.
-    if (MODE != kModeBF16) smem = std::max<size_t>(smem, (size_t)di.max_smem_optin / 2 + 1024);
+    const int budget = di.max_smem_optin - 1024 - 512;
+    int stages = std::min<int>(8, budget / (int)stage);
+    if (kFused) stages = std::min(stages, (512 - 2 * acc_stride) / 32);
+    if (stages < 3) return BQ_ERR_UNSUPPORTED;
+    // one CTA per SM: the kernel allocates all 512 TMEM columns
+    const size_t smem = std::max<size_t>(1024 + (size_t)stages * stage + 512, (size_t)di.max_smem_optin / 2 + 1024);
 
     CUtensorMap tm_x, tm_a;
     if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, M, K, bn, 64, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -226,13 +232,13 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     p.K = (int)K;
     p.bn = bn;
     p.stages = stages;
+    p.m_tiles = (int)((M + bn - 1) / bn);
+    const int64_t tiles = (int64_t)p.m_tiles * ((N + 127) / 128);
+    if (tiles > INT32_MAX) return BQ_ERR_SHAPE;
+    p.tiles = (int)tiles;
+    p.acc_stride = acc_stride;
     p.vec_scales = (K % 512 == 0) ? 1 : 0;
-    int cols = 32;
-    while (cols < bn) cols <<= 1;
-    p.tmem_cols = (MODE == kModeBF16) ? cols : 512;   // fused: accumulator + staged A tiles (see tc_gemm.cuh)
-    if (MODE != kModeBF16 && 256 + 32 * stages > 512) return BQ_ERR_UNSUPPORTED;
-    dim3 grid((unsigned)((M + bn - 1) / bn), (unsigned)((N + 127) / 128));
-    if (grid.y > 65535u) return BQ_ERR_SHAPE;
+    const unsigned grid = (unsigned)std::min<int64_t>(tiles, di.num_sms);
     tc_gemm_kernel<MODE><<<grid, C::kThreads, smem, st>>>(tm_x, tm_a, p);
     return launch_status();
 }

@@ -19,9 +19,14 @@
 //                 "et-backend: Q4_0 matrix-engine GEMM rewrite for prefill"
 //                 (Overview), mapped to the B200 tensor cores.
 //
-// Warp roles: warps [0, kDeqWarps) dequantize (fused modes); warps 0..3 also
-// run the epilogue (TMEM -> registers -> bf16 -> global); one warp issues TMA,
-// one issues tcgen05.mma (one elected thread) and owns the TMEM allocation.
+// The kernel is persistent: one CTA per SM walks a static schedule of
+// (weight tile, token tile) pairs, token tiles fastest so that concurrently
+// running CTAs share weight tiles in L2.  Two TMEM accumulators let a separate
+// epilogue warpgroup drain tile i while the MMA warp already accumulates tile
+// i + 1, and the producer runs ahead across tile boundaries.
+// Warp roles: [0, kDeqWarps) dequantize (fused modes), four epilogue warps
+// (TMEM -> registers -> bf16 -> global), one TMA producer warp, one MMA warp
+// (one elected thread issues every tcgen05.mma and owns the TMEM allocation).
 // Every mbarrier wait is bounded (see mbar_wait); on a timeout each role skips
 // its remaining work, the MMA thread still commits, and TMEM is freed.
 #pragma once
@@ -34,11 +39,12 @@ enum : int { kModeBF16 = 0, kModeQ4_0 = 1, kModeAff4 = 2, kModeAff8 = 3 };
 
 template <int MODE> struct TcCfg {
     static constexpr int kDeqWarps = (MODE == kModeBF16) ? 0 : 8;
-    static constexpr int kTmaWarp = (MODE == kModeBF16) ? 4 : kDeqWarps;
+    static constexpr int kEpiWarp0 = kDeqWarps;          // 4 warps: lane quarter = warp % 4
+    static constexpr int kTmaWarp = kEpiWarp0 + 4;
     static constexpr int kMmaWarp = kTmaWarp + 1;
     static constexpr int kThreads = 32 * (kMmaWarp + 1);
     static constexpr int kCodeBytesPerRow = (MODE == kModeAff8) ? 64 : 32;   // per 64-element k-block
-    static constexpr uint32_t kABytes = (MODE == kModeBF16) ? 128 * 128 : 0;   // fused: A lives in TMEM
+    static constexpr uint32_t kABytes = (MODE == kModeBF16) ? 128 * 128 : 0;   // fused: weight tile in TMEM
     static constexpr uint32_t kCBytes = (MODE == kModeBF16) ? 0 : 128 * kCodeBytesPerRow;
 };
 
@@ -49,17 +55,28 @@ struct TcParams {
     int M, N, K;
     int bn;                   // token tile = MMA N, multiple of 16 in [16, 256]
     int stages;
-    int tmem_cols;            // power of two >= max(32, bn)
+    int m_tiles;              // token tiles per weight tile
+    int tiles;                // total tiles
+    int acc_stride;           // TMEM columns between the two accumulators
     int vec_scales;           // scale rows are 16-byte aligned and hold whole 8-scale windows
 };
 
 // Shared memory per pipeline stage: the activation tile (bn x 64 bf16, 128B
-// swizzled) plus either the bf16 weight tile (128 x 64) or the packed codes.
-// Fused modes keep the dequantized weight tile in TMEM instead.
+// swizzled K-major) plus the bf16 weight tile (kModeBF16, same layout) or the
+// packed codes (fused modes; their dequantized tile goes to TMEM).
 __host__ __device__ constexpr uint32_t tc_stage_bytes(int mode, int bn)
 {
-    return (uint32_t)bn * 128u +
-           (mode == kModeBF16 ? 128u * 128u : (mode == kModeAff8 ? 128u * 64u : 128u * 32u));
+    return (uint32_t)bn * 128u + (mode == kModeBF16 ? 128u * 128u : (mode == kModeAff8 ? 128u * 64u : 128u * 32u));
+}
+
+// Byte offset of the 16-byte chunk `c` (K elements 8c..8c+7) of row `r` in a
+// 128B-swizzled K-major tile with 128-byte rows (the layout TMA writes and the
+// UMMA descriptor describes): chunk c of row r sits at position c ^ (r mod 8).
+BQ_DEVINL uint32_t sw128_offset(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+BQ_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 // --- dequantization of one thread's 32 weights (half a k-block of one row) ---
@@ -185,8 +202,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     using C = TcCfg<MODE>;
     extern __shared__ uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * p.bn;
-    const int n0 = blockIdx.y * 128;
     const int nk = (p.K + 63) / 64;
     const int S = p.stages;
     const uint32_t b_bytes = (uint32_t)p.bn * 128u;
@@ -196,29 +211,39 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     const uint32_t a_base = b_base + (uint32_t)S * b_bytes;            // bf16 weight tiles (kModeBF16)
     const uint32_t c_base = a_base + (uint32_t)S * C::kABytes;         // packed code tiles (fused)
     const uint32_t bar_base = c_base + (uint32_t)S * C::kCBytes;
-    // TMEM columns: accumulator [0, bn); fused modes keep stage s of the
-    // dequantized weight tile (128 lanes x 64 bf16 = 32 columns) at 256 + 32 s.
-    auto a_tmem_col = [&](int s) { return 256u + 32u * (uint32_t)s; };
+    // barriers per stage: landed (TMA), weight tile written (fused), free (MMA done);
+    // per accumulator: ready, drained; and MMA done
     auto full_bar = [&](int s) { return bar_base + 8u * (uint32_t)s; };
-    auto afull_bar = [&](int s) { return bar_base + 8u * (uint32_t)(S + s); };
-    auto empty_bar = [&](int s) { return bar_base + 8u * (uint32_t)(2 * S + s); };
-    const uint32_t tmem_full_bar = bar_base + 8u * (uint32_t)(3 * S);
-    const uint32_t tmem_slot = tmem_full_bar + 8u;
+    auto empty_bar = [&](int s) { return bar_base + 8u * (uint32_t)(S + s); };
+    auto afull_bar = [&](int s) { return bar_base + 8u * (uint32_t)(2 * S + s); };
+    auto tfull_bar = [&](int b) { return bar_base + 8u * (uint32_t)(3 * S + b); };      // accumulator b ready
+    auto tempty_bar = [&](int b) { return bar_base + 8u * (uint32_t)(3 * S + 2 + b); };  // accumulator b drained
+    const uint32_t mma_done_bar = bar_base + 8u * (uint32_t)(3 * S + 4);
+    // TMEM columns: accumulators at 0 and acc_stride; fused modes keep stage s of
+    // the dequantized weight tile (128 lanes x 64 bf16 = 32 columns) after them.
+    auto a_tmem_col = [&](int s) { return 2u * (uint32_t)p.acc_stride + 32u * (uint32_t)s; };
+    const uint32_t tmem_slot = mma_done_bar + 8u;
     uint8_t* smem_gen = smem_raw + (base - smem_u32(smem_raw));
     volatile uint32_t* tmem_slot_ptr = reinterpret_cast<volatile uint32_t*>(smem_gen + (tmem_slot - base));
+    auto tile_n0 = [&](int t) { return (t / p.m_tiles) * 128; };
+    auto tile_m0 = [&](int t) { return (t % p.m_tiles) * p.bn; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
-            mbar_init(afull_bar(s), C::kDeqWarps * 32);
             mbar_init(empty_bar(s), 1);
+            mbar_init(afull_bar(s), C::kDeqWarps);
         }
-        mbar_init(tmem_full_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 128);
+        }
+        mbar_init(mma_done_bar, 1);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
     if (warp == C::kMmaWarp) {
-        tmem_alloc(tmem_slot, (uint32_t)p.tmem_cols);
+        tmem_alloc(tmem_slot, 512u);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -227,97 +252,80 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     const uint32_t tmem_base = *tmem_slot_ptr;
 
     if (warp == C::kTmaWarp) {
+        // ---------------- producer ----------------
         if (lane == 0) {
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_a);
-            int issued = 0;
-            for (int it = 0; it < nk; ++it) {
-                const int s = it % S;
-                const uint32_t ph = (uint32_t)(it / S) & 1u;
-                if (!mbar_wait(empty_bar(s), ph ^ 1u)) break;
-                mbar_arrive_expect_tx(full_bar(s), b_bytes + (MODE == kModeBF16 ? C::kABytes : C::kCBytes));
-                tma_load_2d(b_base + (uint32_t)s * b_bytes, &tm_x, full_bar(s), it * 64, m0);
-                if constexpr (MODE == kModeBF16)
-                    tma_load_2d(a_base + (uint32_t)s * C::kABytes, &tm_a, full_bar(s), it * 64, n0);
-                else
-                    tma_load_2d(c_base + (uint32_t)s * C::kCBytes, &tm_a, full_bar(s), it * C::kCodeBytesPerRow, n0);
-                ++issued;
+            int g = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
+                const int n0 = tile_n0(t), m0 = tile_m0(t);
+                for (int it = 0; it < nk; ++it, ++g) {
+                    const int s = g % S;
+                    if (!mbar_wait(empty_bar(s), ((uint32_t)(g / S) & 1u) ^ 1u)) { ok = false; break; }
+                    mbar_arrive_expect_tx(full_bar(s), b_bytes + (MODE == kModeBF16 ? C::kABytes : C::kCBytes));
+                    tma_load_2d(b_base + (uint32_t)s * b_bytes, &tm_x, full_bar(s), it * 64, m0);
+                    if constexpr (MODE == kModeBF16)
+                        tma_load_2d(a_base + (uint32_t)s * C::kABytes, &tm_a, full_bar(s), it * 64, n0);
+                    else
+                        tma_load_2d(c_base + (uint32_t)s * C::kCBytes, &tm_a, full_bar(s), it * C::kCodeBytesPerRow, n0);
+                }
             }
             // Drain: every issued copy has landed before this CTA may exit.
-            for (int it = (issued > S ? issued - S : 0); it < issued; ++it)
-                mbar_wait(full_bar(it % S), (uint32_t)(it / S) & 1u);
+            for (int q = (g > S ? g - S : 0); q < g; ++q)
+                mbar_wait(full_bar(q % S), (uint32_t)(q / S) & 1u);
         }
     } else if (warp == C::kMmaWarp) {
+        // ---------------- MMA issuer ----------------
         if (lane == 0) {
             const uint32_t idesc = umma_idesc_bf16_f32(128, p.bn);
-            for (int it = 0; it < nk; ++it) {
-                const int s = it % S;
-                const uint32_t ph = (uint32_t)(it / S) & 1u;
-                if (!mbar_wait(full_bar(s), ph)) break;
-                if constexpr (MODE != kModeBF16) {
-                    if (!mbar_wait(afull_bar(s), ph)) break;
-                }
+            int g = 0, lt = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++lt) {
+                const int acc = lt & 1;
+                if (!mbar_wait(tempty_bar(acc), ((uint32_t)(lt >> 1) & 1u) ^ 1u)) break;
                 tc_fence_after();
-                const uint32_t b_addr = b_base + (uint32_t)s * b_bytes;
-                if constexpr (MODE == kModeBF16) {
-                    const uint32_t a_addr = a_base + (uint32_t)s * C::kABytes;
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.acc_stride);
+                for (int it = 0; it < nk; ++it, ++g) {
+                    const int s = g % S;
+                    const uint32_t ph = (uint32_t)(g / S) & 1u;
+                    if (!mbar_wait(full_bar(s), ph)) { ok = false; break; }
+                    if constexpr (MODE != kModeBF16) {
+                        if (!mbar_wait(afull_bar(s), ph)) { ok = false; break; }
+                    }
+                    tc_fence_after();
+                    const uint32_t b_addr = b_base + (uint32_t)s * b_bytes;
+                    if constexpr (MODE == kModeBF16) {
+                        const uint32_t a_addr = a_base + (uint32_t)s * C::kABytes;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16_ss(tmem_base, umma_desc_k_sw128(a_addr + 32u * kk),
-                                    umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it | kk) != 0 ? 1u : 0u);
-                } else {
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_f16_ss(d_tmem, umma_desc_k_sw128(a_addr + 32u * kk),
+                                        umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it | kk) != 0 ? 1u : 0u);
+                    } else {
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)   // K = 16 per MMA = 8 TMEM columns of A
-                        umma_f16_ts(tmem_base, tmem_base + a_tmem_col(s) + 8u * kk,
-                                    umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)   // K = 16 per MMA = 8 TMEM columns of A
+                            umma_f16_ts(d_tmem, tmem_base + a_tmem_col(s) + 8u * kk,
+                                        umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(empty_bar(s));
                 }
-                umma_commit(empty_bar(s));
+                umma_commit(tfull_bar(acc));
             }
-            umma_commit(tmem_full_bar);   // also on an early exit: nothing stays in flight
-            mbar_wait(tmem_full_bar, 0);
+            umma_commit(mma_done_bar);   // nothing stays in flight past this point
+            mbar_wait(mma_done_bar, 0);
         }
         __syncwarp();
-    } else if (MODE != kModeBF16 && warp < C::kDeqWarps) {
-        const int r = 32 * (warp & 3) + lane;   // weight row within the tile
-        const int h = warp >> 2;                // which 32-element half of each k-block
-        const int row = n0 + r;
-        constexpr int kSpan = ScaleWindow<MODE>::kSpan;
-        ScaleWindow<MODE> win_cur = load_scale_window<MODE>(p, row, 0);
-        ScaleWindow<MODE> win_nxt = load_scale_window<MODE>(p, row, 1);
-        for (int it = 0; it < nk; ++it) {
-            const int s = it % S;
-            const uint32_t ph = (uint32_t)(it / S) & 1u;
-            if (it > 0 && it % kSpan == 0) {                  // next window; fetch the one after it
-                win_cur = win_nxt;
-                win_nxt = load_scale_window<MODE>(p, row, it / kSpan + 1);
-            }
-            const DeqScale sc = window_scale<MODE>(win_cur, it, h);
-            if (!mbar_wait(full_bar(s), ph)) break;
-            const uint32_t codes = c_base + (uint32_t)s * C::kCBytes + (uint32_t)(r * C::kCodeBytesPerRow);
-            uint32_t wv[16];
-            if constexpr (MODE == kModeQ4_0) {
-                deq_q4_0_half(ld_shared_v4(codes + 16u * h), sc.a, sc.b, wv);
-            } else if constexpr (MODE == kModeAff4) {
-                deq_aff4_half(ld_shared_v4(codes + 16u * h), sc.a | (sc.a << 16), sc.b | (sc.b << 16), wv);
-            } else {
-                deq_aff8_half(ld_shared_v4(codes + 32u * h), ld_shared_v4(codes + 32u * h + 16u),
-                              bf16_bits_to_f32(sc.a), bf16_bits_to_f32(sc.b), wv);
-            }
-            // row r = TMEM lane r; this thread's 32 weights = 16 columns of the stage's A tile
-            tmem_st_32x32b_x16(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + a_tmem_col(s) + 16u * h, wv);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(afull_bar(s));
-        }
-    }
-
-    // Epilogue: warps 0..3, TMEM lane quarter = warp.
-    if (warp < 4) {
-        const bool ok = mbar_wait(tmem_full_bar, 0);
-        tc_fence_after();
-        if (ok) {
-            const int row = n0 + 32 * warp + lane;
-            const uint32_t lane_addr = tmem_base + ((uint32_t)(32 * warp) << 16);
+    } else if (warp >= C::kEpiWarp0 && warp < C::kEpiWarp0 + 4) {
+        // ---------------- epilogue ----------------
+        const int q4 = warp & 3;                                       // TMEM lane quarter
+        int lt = 0;
+        for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++lt) {
+            const int acc = lt & 1;
+            if (!mbar_wait_warp(tfull_bar(acc), (uint32_t)(lt >> 1) & 1u)) break;
+            tc_fence_after();
+            const int row = tile_n0(t) + 32 * q4 + lane;
+            const int m0 = tile_m0(t);
+            const uint32_t lane_addr = tmem_base + ((uint32_t)(32 * q4) << 16) + (uint32_t)(acc * p.acc_stride);
             for (int c0 = 0; c0 < p.bn; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld_32x32b_x16(lane_addr + (uint32_t)c0, v);
@@ -330,12 +338,64 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(tempty_bar(acc));
+        }
+    } else if (MODE != kModeBF16 && warp < C::kDeqWarps) {
+        // ---------------- dequantization ----------------
+        const int r = 32 * (warp & 3) + lane;   // weight row within the tile = TMEM lane
+        const int h = warp >> 2;                // which 32-element half of each k-block
+        constexpr int kSpan = ScaleWindow<MODE>::kSpan;
+        const int nwin = (nk + kSpan - 1) / kSpan;
+        // Scale windows form one stream over this CTA's (tile, window) pairs, so
+        // the first window of the next tile is already in flight at a tile boundary.
+        auto load_q = [&](int q) {
+            const int t = blockIdx.x + (q / nwin) * gridDim.x;
+            const int row = t < p.tiles ? tile_n0(t) + r : p.N;
+            return load_scale_window<MODE>(p, row, q % nwin);
+        };
+        int q_cur = 0;
+        ScaleWindow<MODE> win_cur = load_q(0);
+        ScaleWindow<MODE> win_nxt = load_q(1);
+        int g = 0, ti = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++ti) {
+            for (int it = 0; it < nk; ++it, ++g) {
+                const int s = g % S;
+                const int q = ti * nwin + it / kSpan;
+                if (q_cur < q) {                                  // advance one window, fetch the one after
+                    win_cur = win_nxt;
+                    ++q_cur;
+                    win_nxt = load_q(q_cur + 1);
+                }
+                const DeqScale sc = window_scale<MODE>(win_cur, it, h);
+                if (!mbar_wait_warp(full_bar(s), (uint32_t)(g / S) & 1u)) { ok = false; break; }
+                const uint32_t codes = c_base + (uint32_t)s * C::kCBytes + (uint32_t)(r * C::kCodeBytesPerRow);
+                uint32_t wv[16];
+                if constexpr (MODE == kModeQ4_0) {
+                    deq_q4_0_half(ld_shared_v4(codes + 16u * h), sc.a, sc.b, wv);
+                } else if constexpr (MODE == kModeAff4) {
+                    deq_aff4_half(ld_shared_v4(codes + 16u * h), sc.a | (sc.a << 16), sc.b | (sc.b << 16), wv);
+                } else {
+                    deq_aff8_half(ld_shared_v4(codes + 32u * h), ld_shared_v4(codes + 32u * h + 16u),
+                                  bf16_bits_to_f32(sc.a), bf16_bits_to_f32(sc.b), wv);
+                }
+                // This thread's 32 weights = 16 TMEM columns of its lane (row r) in
+                // stage s.  The stage's previous tile was consumed by the MMA of
+                // k-block g - S: its smem stage was freed before this one was filled.
+                tmem_st_32x32b_x16(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + a_tmem_col(s) + 16u * h, wv);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(afull_bar(s));
+            }
         }
     }
+
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == C::kMmaWarp) tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
+    if (warp == C::kMmaWarp) tmem_dealloc(tmem_base, 512u);
 }
 
 }  // namespace bq

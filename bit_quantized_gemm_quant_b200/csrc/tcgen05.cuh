@@ -37,12 +37,15 @@ BQ_DEVINL void mbar_arrive(uint32_t bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// try_wait with a suspend-time hint: a warp whose phase is not complete sleeps in
+// hardware (up to the hint, 10 ms) and is woken when the phase completes, so
+// waiting warps do not take issue slots from working ones.
 BQ_DEVINL bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 10000000;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
@@ -63,6 +66,17 @@ BQ_DEVINL bool mbar_wait(uint32_t bar, uint32_t parity)
         }
     }
     return true;
+}
+
+// Warp-level wait: lane 0 polls the barrier, then __syncwarp orders every lane
+// of the warp after lane 0's acquire; 32 pollers per warp become one.
+BQ_DEVINL bool mbar_wait_warp(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity) ? 1u : 0u;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
 }
 
 BQ_DEVINL uint4 ld_shared_v4(uint32_t addr)
