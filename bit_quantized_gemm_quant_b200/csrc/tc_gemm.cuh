@@ -253,16 +253,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
     if (warp == C::kTmaWarp) {
         // ---------------- producer ----------------
-        if (lane == 0) {
+        // The whole warp walks the schedule (stage index and phase advance
+        // incrementally, no division); one elected lane issues the copies.
+        const bool leader = elect_one();
+        if (leader) {
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_a);
-            int g = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
-                const int n0 = tile_n0(t), m0 = tile_m0(t);
-                for (int it = 0; it < nk; ++it, ++g) {
-                    const int s = g % S;
-                    if (!mbar_wait(empty_bar(s), ((uint32_t)(g / S) & 1u) ^ 1u)) { ok = false; break; }
+        }
+        int s = 0, issued = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
+            const int n0 = tile_n0(t), m0 = tile_m0(t);
+            for (int it = 0; it < nk; ++it) {
+                if (!mbar_wait_warp(empty_bar(s), ph ^ 1u)) { ok = false; break; }
+                if (leader) {
                     mbar_arrive_expect_tx(full_bar(s), b_bytes + (MODE == kModeBF16 ? C::kABytes : C::kCBytes));
                     tma_load_2d(b_base + (uint32_t)s * b_bytes, &tm_x, full_bar(s), it * 64, m0);
                     if constexpr (MODE == kModeBF16)
@@ -270,30 +275,36 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     else
                         tma_load_2d(c_base + (uint32_t)s * C::kCBytes, &tm_a, full_bar(s), it * C::kCodeBytesPerRow, n0);
                 }
+                __syncwarp();
+                ++issued;
+                if (++s == S) { s = 0; ph ^= 1u; }
             }
-            // Drain: every issued copy has landed before this CTA may exit.
-            for (int q = (g > S ? g - S : 0); q < g; ++q)
-                mbar_wait(full_bar(q % S), (uint32_t)(q / S) & 1u);
+        }
+        // Drain: every issued copy has landed before this CTA may exit.  Walk the
+        // last min(issued, S) stages backwards from the next stage to be used.
+        for (int q = 0; q < S && q < issued; ++q) {
+            if (--s < 0) { s = S - 1; ph ^= 1u; }
+            mbar_wait_warp(full_bar(s), ph);
         }
     } else if (warp == C::kMmaWarp) {
         // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            const uint32_t idesc = umma_idesc_bf16_f32(128, p.bn);
-            int g = 0, lt = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++lt) {
-                const int acc = lt & 1;
-                if (!mbar_wait(tempty_bar(acc), ((uint32_t)(lt >> 1) & 1u) ^ 1u)) break;
+        const bool leader = elect_one();
+        const uint32_t idesc = umma_idesc_bf16_f32(128, p.bn);
+        int s = 0, lt = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++lt) {
+            const int acc = lt & 1;
+            if (!mbar_wait_warp(tempty_bar(acc), ((uint32_t)(lt >> 1) & 1u) ^ 1u)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.acc_stride);
+            for (int it = 0; it < nk; ++it) {
+                if (!mbar_wait_warp(full_bar(s), ph)) { ok = false; break; }
+                if constexpr (MODE != kModeBF16) {
+                    if (!mbar_wait_warp(afull_bar(s), ph)) { ok = false; break; }
+                }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.acc_stride);
-                for (int it = 0; it < nk; ++it, ++g) {
-                    const int s = g % S;
-                    const uint32_t ph = (uint32_t)(g / S) & 1u;
-                    if (!mbar_wait(full_bar(s), ph)) { ok = false; break; }
-                    if constexpr (MODE != kModeBF16) {
-                        if (!mbar_wait(afull_bar(s), ph)) { ok = false; break; }
-                    }
-                    tc_fence_after();
+                if (leader) {
                     const uint32_t b_addr = b_base + (uint32_t)s * b_bytes;
                     if constexpr (MODE == kModeBF16) {
                         const uint32_t a_addr = a_base + (uint32_t)s * C::kABytes;
@@ -309,12 +320,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     }
                     umma_commit(empty_bar(s));
                 }
-                umma_commit(tfull_bar(acc));
+                __syncwarp();
+                if (++s == S) { s = 0; ph ^= 1u; }
             }
-            umma_commit(mma_done_bar);   // nothing stays in flight past this point
-            mbar_wait(mma_done_bar, 0);
+            if (leader) umma_commit(tfull_bar(acc));
+            __syncwarp();
         }
+        if (leader) umma_commit(mma_done_bar);   // nothing stays in flight past this point
         __syncwarp();
+        mbar_wait_warp(mma_done_bar, 0);
     } else if (warp >= C::kEpiWarp0 && warp < C::kEpiWarp0 + 4) {
         // ---------------- epilogue ----------------
         const int q4 = warp & 3;                                       // TMEM lane quarter
@@ -357,11 +371,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         int q_cur = 0;
         ScaleWindow<MODE> win_cur = load_q(0);
         ScaleWindow<MODE> win_nxt = load_q(1);
-        int g = 0, ti = 0;
+        int s = 0, ti = 0;
+        uint32_t ph = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++ti) {
-            for (int it = 0; it < nk; ++it, ++g) {
-                const int s = g % S;
+            for (int it = 0; it < nk; ++it) {
                 const int q = ti * nwin + it / kSpan;
                 if (q_cur < q) {                                  // advance one window, fetch the one after
                     win_cur = win_nxt;
@@ -369,7 +383,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     win_nxt = load_q(q_cur + 1);
                 }
                 const DeqScale sc = window_scale<MODE>(win_cur, it, h);
-                if (!mbar_wait_warp(full_bar(s), (uint32_t)(g / S) & 1u)) { ok = false; break; }
+                if (!mbar_wait_warp(full_bar(s), ph)) { ok = false; break; }
                 const uint32_t codes = c_base + (uint32_t)s * C::kCBytes + (uint32_t)(r * C::kCodeBytesPerRow);
                 uint32_t wv[16];
                 if constexpr (MODE == kModeQ4_0) {
@@ -381,13 +395,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                                   bf16_bits_to_f32(sc.a), bf16_bits_to_f32(sc.b), wv);
                 }
                 // This thread's 32 weights = 16 TMEM columns of its lane (row r) in
-                // stage s.  The stage's previous tile was consumed by the MMA of
-                // k-block g - S: its smem stage was freed before this one was filled.
+                // stage s.  The stage's previous tile was consumed by the MMA S
+                // k-blocks back: its smem stage was freed before this one was filled.
                 tmem_st_32x32b_x16(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + a_tmem_col(s) + 16u * h, wv);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(afull_bar(s));
+                if (++s == S) { s = 0; ph ^= 1u; }
             }
         }
     }
