@@ -349,6 +349,51 @@ def run_prefill(args, world, device, peaks, fmt, Ms):
     return res, total_flops / total_s / 1e12
 
 
+def run_stack(args, world, device, peaks):
+    """Llama-3.2-1B-shaped projection stack, Q4_0: the 112 matmuls of 16 layers (q, k, v, o,
+    gate, up, down), each layer with its own weights (547 MB packed > L2), at M = 512 and
+    M = 1.  One CUDA graph holds the whole stack; tokens/s = M / stack time."""
+    import torch
+    import bit_quantized_gemm_quant_b200 as bq
+    from bit_quantized_gemm_quant_b200 import inputs, workloads
+    wl = workloads.LLAMA_1B_STACK
+    g = inputs.generator(wl.seed, str(device.type) if device.type == "cuda" else "cpu")
+    mats = []
+    for _layer in range(wl.layers):
+        for (N, K) in wl.shapes:
+            w = inputs.weights_fp32(N, K, g, device=device)
+            wq, d = bq.q4_0_quantize(w)
+            mats.append((N, K, wq, d))
+            del w
+    torch.cuda.synchronize()
+    packed = sum(workloads.packed_weight_bytes("q4_0", N, K, 32) for N, K, _, _ in mats)
+    params = sum(N * K for N, K, _, _ in mats)
+    gx = inputs.generator(wl.seed + 1)
+    per_m, launches = {}, 0
+    for M in wl.Ms:
+        xs = {K: inputs.activations_bf16(M, K, gx).to(device) for K in sorted({K for _, K, _, _ in mats})}
+        ys = [torch.empty(M, N, dtype=torch.bfloat16, device=device) for N, _, _, _ in mats]
+
+        def stack():
+            for (N, K, wq, d), y in zip(mats, ys):
+                bq.quant_matmul(xs[K], wq, d, None, 32, 4, out=y)
+        gt = GraphTimer(stack)
+        for _ in range(max(3, args.warmup // 50)):
+            gt.replay()
+        reps = max(3, min(200, args.steps // 100))
+        sec = max_over_ranks(time_graphs([gt], reps, world, device) / reps, world, device)
+        paths = sorted({bq.quant_matmul_select_path(M, N, K, 32, 4) for N, K, _, _ in mats})
+        launches += reps * len(mats)
+        per_m[str(M)] = {"us_per_stack": round(sec * 1e6, 2), "tokens_per_s": round(aggregate(M, world, sec), 1),
+                         "tflops": round(2.0 * M * params / sec / 1e12, 2),
+                         "frac_tensor": round(2.0 * M * params / sec / 1e12 / peaks["bf16_tflops"], 4),
+                         "gbs": round(packed / sec / 1e9, 1),
+                         "frac_hbm": round(packed / sec / 1e9 / peaks["hbm_gbs"], 4),
+                         "paths": [{v: k for k, v in bq.PATHS.items()}.get(p_, p_) for p_ in paths]}
+        del gt, xs, ys
+    return per_m, packed, params, launches
+
+
 # ----------------------------------------------------------------------------- CPU oracle (baseline / reference arm)
 def oracle_decode_sample(budget_s: float):
     """Time the CPU oracle on the decode workload: per step, dequantize W and take the
@@ -385,7 +430,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["q4_0_decode", "affine4_prefill", "affine8_sweep", "q4_0_prefill"],
+    ap.add_argument("--workload", choices=["q4_0_decode", "affine4_prefill", "affine8_sweep", "q4_0_prefill",
+                                           "llama1b_stack"],
                     default="q4_0_decode")
     ap.add_argument("--ms", type=str, default=None, help="comma-separated M list for a prefill workload")
     ap.add_argument("--no-e2e", action="store_true")
@@ -426,6 +472,19 @@ def main(argv=None):
         if not args.no_prefill:
             pre, _ = run_prefill(args, world, device, peaks, "affine4", (2048,))
             r["secondary"] = {"prefill_affine4_n12288_k4096_m2048": pre["2048"]}
+    elif args.workload == "llama1b_stack":
+        with ClockSampler(local_rank) as clk:
+            per_m, packed, params, launches = run_stack(args, world, device, peaks)
+        r = {"value": per_m["512"]["tokens_per_s"], "unit": "tokens/s", "ms_per_step": per_m["512"]["us_per_stack"] / 1e3,
+             "dtype": "q4_0 weights, bf16 activations, fp32 accumulate",
+             "config": {"workload": "llama3.2_1b_q4_0_projection_stack_16_layers", "M": [512, 1],
+                        "params": params, "packed_bytes": packed,
+                        "l2": f"{packed / 1e6:.0f} MB of distinct packed weights per stack (> 126 MB L2)"},
+             "per_m": per_m,
+             "roofline": {"bound": "tensor", "kernel": "whole stack at M=512", "achieved": per_m["512"]["tflops"],
+                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": per_m["512"]["frac_tensor"],
+                          "traffic": None},
+             "clocks": clk.summary(), "gpu_launches": launches, "e2e": None}
     else:
         fmt, Ms = {"affine4_prefill": ("affine4", (512, 2048, 8192)),
                    "affine8_sweep": ("affine8", (1, 32, 512, 2048, 8192)),

@@ -1,0 +1,63 @@
+"""Host logic of bench.py's multi-rank path, on CPU with the gloo backend (world size 2).
+
+Each rank of a multi-GPU run times its own replica; the reported time is the
+maximum over ranks and the value is the work of all ranks over that time.
+"""
+from __future__ import annotations
+
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, out):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update({"RANK": str(rank), "LOCAL_RANK": str(rank), "WORLD_SIZE": str(world),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        r, lr, w = bench.dist_env()
+        seconds = 0.5 + rank          # rank 1 is the slow one
+        slowest = bench.max_over_ranks(seconds, w, device="cpu")
+        value = bench.aggregate(100.0, w, slowest)
+        dist.barrier()
+        out.put((r, lr, w, slowest, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_aggregate_gloo():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0, f"rank exited with {p.exitcode}"
+    got = sorted(q.get(timeout=10) for _ in range(world))
+    for r, (rank, local_rank, w, slowest, value) in enumerate(got):
+        assert (rank, local_rank, w) == (r, r, world)
+        assert slowest == pytest.approx(1.5)          # the max, not the caller's own time
+        assert value == pytest.approx(200.0 / 1.5)    # both ranks' work over the slowest time
+
+
+def test_single_rank_helpers():
+    assert bench.max_over_ranks(3.25, 1) == 3.25
+    assert bench.aggregate(10.0, 1, 2.0) == 5.0
+    # every copy is used exactly once per cycle of n_copies launches
+    n, per = 12, 3
+    seen = [bench.rotation(n, per, step, j) for step in range(4) for j in range(per)]
+    assert sorted(seen) == list(range(n))
