@@ -48,6 +48,7 @@ def lib() -> ctypes.CDLL:
         "affine_dequantize": [P, P, P, P, I64, I64, I, I, P],
         "quant_matmul": [P, P, P, P, P, I64, I64, I64, I, I, I, P],
         "quant_matmul_ex": [P, P, P, P, P, I64, I64, I64, I, I, I, I, P, SZ, P],
+        "quant_matmul_noalloc": [P, P, P, P, P, I64, I64, I64, I, I, I, P],
         "quant_matmul_workspace_size": [I64, I64, I64, I, I, I],
         "quant_matmul_select_path": [I64, I64, I64, I, I],
         "bf16_matmul": [P, P, P, I64, I64, I64, P],
@@ -155,6 +156,27 @@ def quant_matmul_ex(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, bia
         st = fn(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(out), M, N, K, group_size, bits,
                 1 if transpose else 0, p, _ptr(workspace), ws_bytes, _stream(stream))
     _check(st, "quant_matmul")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def quant_matmul_noalloc(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor | None,
+                         out: torch.Tensor, group_size: int = 32, bits: int = 4, transpose: bool = True, stream=None):
+    """quant_matmul for callers that must not allocate: the library uses its fixed
+    32 MiB device scratch (N * K <= 16 Mi weights) and allocates nothing.  `out`
+    (bf16 [M][N]) is required, since creating it here would allocate."""
+    M, K = x.shape
+    N = wq.shape[0]
+    if K != _k_of(wq, biases, bits):
+        raise ValueError(f"K mismatch: x has {K}, weights hold {_k_of(wq, biases, bits)}")
+    if tuple(out.shape) != (M, N) or out.dtype != torch.bfloat16:
+        raise ValueError("out must be a bf16 tensor of shape [M][N]")
+    _check(lib().quant_matmul_noalloc(_ptr(x), _ptr(wq), _ptr(_bits16(scales)),
+                                      None if biases is None else _ptr(_bits16(biases)), _ptr(out), M, N, K,
+                                      group_size, bits, 1 if transpose else 0, _stream(stream)),
+           "quant_matmul_noalloc")
     return out
 
 

@@ -372,6 +372,29 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
     }
 }
 
+// ------------------------------------------------------------------ allocation-free scratch
+// Scratch of quant_matmul_noalloc: the bf16 copy of W that the unfused pair
+// stages between its two kernels, as a fixed array of the device image.  Host
+// code must not pass the name itself to a kernel (on the host it is a stand-in,
+// not a device address); noalloc_scratch looks the address up per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[BQ_NOALLOC_SCRATCH_BYTES];
+void* g_noalloc_ptr[kMaxDevices];
+
+bq_status noalloc_scratch(int dev, void** out)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_ptr[dev]) {                // once per device, with `dev` current
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return BQ_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return BQ_OK;
+}
+
 }  // namespace
 }  // namespace bq
 
@@ -423,6 +446,28 @@ bq_status quant_matmul_ex(const uint16_t* x_bf16, const void* wq, const void* sc
 {
     return matmul_impl(x_bf16, wq, scales, biases, y_bf16, M, N, K, group_size, bits, transpose, path, workspace,
                        workspace_bytes, (cudaStream_t)stream);
+}
+
+bq_status quant_matmul_noalloc(const uint16_t* x_bf16, const void* wq, const void* scales, const void* biases,
+                               uint16_t* y_bf16, int64_t M, int64_t N, int64_t K, int group_size, int bits,
+                               int transpose, bq_stream_t stream)
+{
+    if (transpose != 1) return BQ_ERR_UNSUPPORTED;
+    if (M < 0 || N < 0 || K < 0) return BQ_ERR_SHAPE;
+    WFmt fmt;
+    bq_status s = check_format(biases, N, K, group_size, bits, &fmt);
+    if (s != BQ_OK) return s;
+    if (M == 0 || N == 0 || K == 0)           // nothing to stage: no scratch involved
+        return matmul_impl(x_bf16, wq, scales, biases, y_bf16, M, N, K, group_size, bits, transpose,
+                           BQ_PATH_DEQUANT_GEMM, nullptr, 0, (cudaStream_t)stream);
+    if ((uint64_t)N > (uint64_t)(BQ_NOALLOC_SCRATCH_BYTES / 2u) / (uint64_t)K) return BQ_ERR_WORKSPACE;
+    int dev;
+    DeviceInfo di;
+    if ((s = current_device(&dev, &di)) != BQ_OK) return s;
+    void* ws = nullptr;
+    if ((s = noalloc_scratch(dev, &ws)) != BQ_OK) return s;
+    return matmul_impl(x_bf16, wq, scales, biases, y_bf16, M, N, K, group_size, bits, transpose,
+                       BQ_PATH_DEQUANT_GEMM, ws, BQ_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream);
 }
 
 size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int group_size, int bits, int path)

@@ -129,6 +129,36 @@ BQ_API bq_status quant_matmul(const uint16_t* x_bf16, const void* wq, const void
                        int transpose, bq_stream_t stream);
 
 /*
+ * quant_matmul_noalloc -- quant_matmul for callers that must not allocate.
+ * No page has a counterpart of this call; it exists for programs where the
+ * library may not call cudaMalloc: hosts that own all device memory through
+ * their own pool or that budget it once at start-up, and latency-critical
+ * callers that cannot afford an allocation's implicit synchronization on a
+ * first call.  It computes the same y as quant_matmul, always through the
+ * unfused pair (q4_0_dequantize / affine_dequantize into scratch, then the
+ * bf16 tensor-core GEMM), with the bf16 copy of W staged in a fixed 32 MiB
+ * array that is part of the library's device image.
+ *   Arguments, layouts, validation and errors are those of quant_matmul.
+ *   Limit: N * K * 2 bytes must fit in BQ_NOALLOC_SCRATCH_BYTES (N * K at most
+ *   16,777,216 weights, e.g. 4096 x 4096); larger problems return
+ *   BQ_ERR_WORKSPACE before anything is launched.
+ *   Memory: every device that loads the library holds the 32 MiB array until
+ *   the process exits.  The call itself makes no cudaMalloc / cudaFree and calls
+ *   no allocating library routine.
+ *   Set-up: the first call on each device, with that device current, looks up
+ *   the array's device address (cudaGetSymbolAddress) and caches it; make that
+ *   first call before any stream capture.
+ *   Sharing: all calls on a device use the same array and it keeps the last
+ *   call's contents (each call overwrites the part it uses before reading it).
+ *   Calls whose execution overlaps on the GPU -- on different streams without
+ *   ordering between them -- race on the array; order them on one stream.
+ */
+#define BQ_NOALLOC_SCRATCH_BYTES (32u << 20)
+BQ_API bq_status quant_matmul_noalloc(const uint16_t* x_bf16, const void* wq, const void* scales,
+                                      const void* biases, uint16_t* y_bf16, int64_t M, int64_t N, int64_t K,
+                                      int group_size, int bits, int transpose, bq_stream_t stream);
+
+/*
  * quant_matmul_ex -- quant_matmul with an explicit path (bq_path) and an
  * optional caller-owned device workspace.  With workspace == NULL the library's
  * per-device buffer is used as in quant_matmul; otherwise workspace_bytes must
