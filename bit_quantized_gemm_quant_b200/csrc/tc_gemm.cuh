@@ -24,7 +24,8 @@
 // running CTAs share weight tiles in L2.  Two TMEM accumulators let a separate
 // epilogue warpgroup drain tile i while the MMA warp already accumulates tile
 // i + 1, and the producer runs ahead across tile boundaries.
-// Warp roles: [0, kDeqWarps) dequantize (fused modes), four epilogue warps
+// Warp roles: [0, kDeqWarps) dequantize (fused modes: groups of eight that take
+// k-blocks in turn), four epilogue warps
 // (TMEM -> registers -> bf16 -> global), one TMA producer warp, one MMA warp
 // (one elected thread issues every tcgen05.mma and owns the TMEM allocation).
 // Every mbarrier wait is bounded (see mbar_wait); on a timeout each role skips
@@ -38,7 +39,9 @@ namespace bq {
 enum : int { kModeBF16 = 0, kModeQ4_0 = 1, kModeAff4 = 2, kModeAff8 = 3 };
 
 template <int MODE> struct TcCfg {
-    static constexpr int kDeqWarps = (MODE == kModeBF16) ? 0 : 8;
+    // Fused modes: kDeqGroups groups of eight dequant warps take k-blocks in turn.
+    static constexpr int kDeqGroups = 2;
+    static constexpr int kDeqWarps = (MODE == kModeBF16) ? 0 : 8 * kDeqGroups;
     static constexpr int kEpiWarp0 = kDeqWarps;          // 4 warps: lane quarter = warp % 4
     static constexpr int kTmaWarp = kEpiWarp0 + 4;
     static constexpr int kMmaWarp = kTmaWarp + 1;
@@ -232,7 +235,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
-            mbar_init(afull_bar(s), C::kDeqWarps);
+            mbar_init(afull_bar(s), 8);               // one group of dequant warps per k-block
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
@@ -253,58 +256,54 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
     if (warp == C::kTmaWarp) {
         // ---------------- producer ----------------
-        // The whole warp walks the schedule (stage index and phase advance
-        // incrementally, no division); one elected lane issues the copies.
-        const bool leader = elect_one();
-        if (leader) {
+        // One lane runs the whole schedule; the stage index and phase advance
+        // incrementally (no division in the loop).
+        if (lane == 0) {
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_a);
-        }
-        int s = 0, issued = 0;
-        uint32_t ph = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
-            const int n0 = tile_n0(t), m0 = tile_m0(t);
-            for (int it = 0; it < nk; ++it) {
-                if (!mbar_wait_warp(empty_bar(s), ph ^ 1u)) { ok = false; break; }
-                if (leader) {
+            int s = 0, issued = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
+                const int n0 = tile_n0(t), m0 = tile_m0(t);
+                for (int it = 0; it < nk; ++it) {
+                    if (!mbar_wait(empty_bar(s), ph ^ 1u)) { ok = false; break; }
                     mbar_arrive_expect_tx(full_bar(s), b_bytes + (MODE == kModeBF16 ? C::kABytes : C::kCBytes));
                     tma_load_2d(b_base + (uint32_t)s * b_bytes, &tm_x, full_bar(s), it * 64, m0);
                     if constexpr (MODE == kModeBF16)
                         tma_load_2d(a_base + (uint32_t)s * C::kABytes, &tm_a, full_bar(s), it * 64, n0);
                     else
                         tma_load_2d(c_base + (uint32_t)s * C::kCBytes, &tm_a, full_bar(s), it * C::kCodeBytesPerRow, n0);
+                    ++issued;
+                    if (++s == S) { s = 0; ph ^= 1u; }
                 }
-                __syncwarp();
-                ++issued;
-                if (++s == S) { s = 0; ph ^= 1u; }
+            }
+            // Drain: every issued copy has landed before this CTA may exit.  Walk the
+            // last min(issued, S) stages backwards from the next stage to be used.
+            for (int q = 0; q < S && q < issued; ++q) {
+                if (--s < 0) { s = S - 1; ph ^= 1u; }
+                mbar_wait(full_bar(s), ph);
             }
         }
-        // Drain: every issued copy has landed before this CTA may exit.  Walk the
-        // last min(issued, S) stages backwards from the next stage to be used.
-        for (int q = 0; q < S && q < issued; ++q) {
-            if (--s < 0) { s = S - 1; ph ^= 1u; }
-            mbar_wait_warp(full_bar(s), ph);
-        }
+        __syncwarp();
     } else if (warp == C::kMmaWarp) {
         // ---------------- MMA issuer ----------------
-        const bool leader = elect_one();
-        const uint32_t idesc = umma_idesc_bf16_f32(128, p.bn);
-        int s = 0, lt = 0;
-        uint32_t ph = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++lt) {
-            const int acc = lt & 1;
-            if (!mbar_wait_warp(tempty_bar(acc), ((uint32_t)(lt >> 1) & 1u) ^ 1u)) break;
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.acc_stride);
-            for (int it = 0; it < nk; ++it) {
-                if (!mbar_wait_warp(full_bar(s), ph)) { ok = false; break; }
-                if constexpr (MODE != kModeBF16) {
-                    if (!mbar_wait_warp(afull_bar(s), ph)) { ok = false; break; }
-                }
+        if (lane == 0) {
+            const uint32_t idesc = umma_idesc_bf16_f32(128, p.bn);
+            int s = 0, lt = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++lt) {
+                const int acc = lt & 1;
+                if (!mbar_wait(tempty_bar(acc), ((uint32_t)(lt >> 1) & 1u) ^ 1u)) break;
                 tc_fence_after();
-                if (leader) {
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.acc_stride);
+                for (int it = 0; it < nk; ++it) {
+                    if (!mbar_wait(full_bar(s), ph)) { ok = false; break; }
+                    if constexpr (MODE != kModeBF16) {
+                        if (!mbar_wait(afull_bar(s), ph)) { ok = false; break; }
+                    }
+                    tc_fence_after();
                     const uint32_t b_addr = b_base + (uint32_t)s * b_bytes;
                     if constexpr (MODE == kModeBF16) {
                         const uint32_t a_addr = a_base + (uint32_t)s * C::kABytes;
@@ -319,16 +318,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                                         umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it | kk) != 0 ? 1u : 0u);
                     }
                     umma_commit(empty_bar(s));
+                    if (++s == S) { s = 0; ph ^= 1u; }
                 }
-                __syncwarp();
-                if (++s == S) { s = 0; ph ^= 1u; }
+                umma_commit(tfull_bar(acc));
             }
-            if (leader) umma_commit(tfull_bar(acc));
-            __syncwarp();
+            umma_commit(mma_done_bar);   // nothing stays in flight past this point
+            mbar_wait(mma_done_bar, 0);
         }
-        if (leader) umma_commit(mma_done_bar);   // nothing stays in flight past this point
         __syncwarp();
-        mbar_wait_warp(mma_done_bar, 0);
     } else if (warp >= C::kEpiWarp0 && warp < C::kEpiWarp0 + 4) {
         // ---------------- epilogue ----------------
         const int q4 = warp & 3;                                       // TMEM lane quarter
@@ -358,7 +355,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     } else if (MODE != kModeBF16 && warp < C::kDeqWarps) {
         // ---------------- dequantization ----------------
         const int r = 32 * (warp & 3) + lane;   // weight row within the tile = TMEM lane
-        const int h = warp >> 2;                // which 32-element half of each k-block
+        const int h = (warp >> 2) & 1;          // which 32-element half of each k-block
+        const int grp = warp >> 3;              // this warp's group takes k-blocks kb with kb % groups == grp
         constexpr int kSpan = ScaleWindow<MODE>::kSpan;
         const int nwin = (nk + kSpan - 1) / kSpan;
         // Scale windows form one stream over this CTA's (tile, window) pairs, so
@@ -371,16 +369,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         int q_cur = 0;
         ScaleWindow<MODE> win_cur = load_q(0);
         ScaleWindow<MODE> win_nxt = load_q(1);
-        int s = 0, ti = 0;
+        int s = 0, ti = 0, kb = 0;
         uint32_t ph = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++ti) {
-            for (int it = 0; it < nk; ++it) {
+            for (int it = 0; it < nk; ++it, ++kb) {
                 const int q = ti * nwin + it / kSpan;
                 if (q_cur < q) {                                  // advance one window, fetch the one after
                     win_cur = win_nxt;
                     ++q_cur;
                     win_nxt = load_q(q_cur + 1);
+                }
+                if (C::kDeqGroups > 1 && kb % C::kDeqGroups != grp) {   // another group's k-block
+                    if (++s == S) { s = 0; ph ^= 1u; }
+                    continue;
                 }
                 const DeqScale sc = window_scale<MODE>(win_cur, it, h);
                 if (!mbar_wait_warp(full_bar(s), ph)) { ok = false; break; }

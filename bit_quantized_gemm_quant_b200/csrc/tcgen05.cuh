@@ -79,19 +79,6 @@ BQ_DEVINL bool mbar_wait_warp(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// One lane of a converged warp (the same lane on every call): the issuing lane
-// for TMA and tcgen05.mma, so that the rest of the loop stays warp-uniform.
-BQ_DEVINL bool elect_one()
-{
-    uint32_t pred;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\t"
-        "elect.sync r|p, 0xffffffff;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(pred));
-    return pred != 0;
-}
-
 BQ_DEVINL uint4 ld_shared_v4(uint32_t addr)
 {
     uint4 v;
