@@ -39,9 +39,12 @@ namespace bq {
 enum : int { kModeBF16 = 0, kModeQ4_0 = 1, kModeAff4 = 2, kModeAff8 = 3 };
 
 template <int MODE> struct TcCfg {
-    // Fused modes: kDeqGroups groups of eight dequant warps take k-blocks in turn.
+    // Fused modes: kDeqGroups groups of dequant warps take k-blocks in turn.  A
+    // group covers the 128 rows of a k-block: 4 warps (one per TMEM lane quarter)
+    // expanding 64 weights per thread, or 8 warps expanding 32.
     static constexpr int kDeqGroups = 2;
-    static constexpr int kDeqWarps = (MODE == kModeBF16) ? 0 : 8 * kDeqGroups;
+    static constexpr int kDeqWarpsPerGroup = 8;
+    static constexpr int kDeqWarps = (MODE == kModeBF16) ? 0 : kDeqWarpsPerGroup * kDeqGroups;
     static constexpr int kEpiWarp0 = kDeqWarps;          // 4 warps: lane quarter = warp % 4
     static constexpr int kTmaWarp = kEpiWarp0 + 4;
     static constexpr int kMmaWarp = kTmaWarp + 1;
@@ -235,7 +238,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
-            mbar_init(afull_bar(s), 8);               // one group of dequant warps per k-block
+            mbar_init(afull_bar(s), C::kDeqWarpsPerGroup);   // one group of dequant warps per k-block
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
@@ -355,8 +358,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     } else if (MODE != kModeBF16 && warp < C::kDeqWarps) {
         // ---------------- dequantization ----------------
         const int r = 32 * (warp & 3) + lane;   // weight row within the tile = TMEM lane
-        const int h = (warp >> 2) & 1;          // which 32-element half of each k-block
-        const int grp = warp >> 3;              // this warp's group takes k-blocks kb with kb % groups == grp
+        constexpr int kHalves = 8 / C::kDeqWarpsPerGroup;   // 32-element halves of a k-block per thread
+        const int h0 = (C::kDeqWarpsPerGroup == 8) ? ((warp >> 2) & 1) : 0;
+        const int grp = warp / C::kDeqWarpsPerGroup;   // takes k-blocks kb with kb % groups == grp
         constexpr int kSpan = ScaleWindow<MODE>::kSpan;
         const int nwin = (nk + kSpan - 1) / kSpan;
         // Scale windows form one stream over this CTA's (tile, window) pairs, so
@@ -384,22 +388,26 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     if (++s == S) { s = 0; ph ^= 1u; }
                     continue;
                 }
-                const DeqScale sc = window_scale<MODE>(win_cur, it, h);
                 if (!mbar_wait_warp(full_bar(s), ph)) { ok = false; break; }
                 const uint32_t codes = c_base + (uint32_t)s * C::kCBytes + (uint32_t)(r * C::kCodeBytesPerRow);
-                uint32_t wv[16];
-                if constexpr (MODE == kModeQ4_0) {
-                    deq_q4_0_half(ld_shared_v4(codes + 16u * h), sc.a, sc.b, wv);
-                } else if constexpr (MODE == kModeAff4) {
-                    deq_aff4_half(ld_shared_v4(codes + 16u * h), sc.a | (sc.a << 16), sc.b | (sc.b << 16), wv);
-                } else {
-                    deq_aff8_half(ld_shared_v4(codes + 32u * h), ld_shared_v4(codes + 32u * h + 16u),
-                                  bf16_bits_to_f32(sc.a), bf16_bits_to_f32(sc.b), wv);
+#pragma unroll
+                for (int hh = 0; hh < kHalves; ++hh) {
+                    const int h = h0 + hh;
+                    const DeqScale sc = window_scale<MODE>(win_cur, it, h);
+                    uint32_t wv[16];
+                    if constexpr (MODE == kModeQ4_0) {
+                        deq_q4_0_half(ld_shared_v4(codes + 16u * h), sc.a, sc.b, wv);
+                    } else if constexpr (MODE == kModeAff4) {
+                        deq_aff4_half(ld_shared_v4(codes + 16u * h), sc.a | (sc.a << 16), sc.b | (sc.b << 16), wv);
+                    } else {
+                        deq_aff8_half(ld_shared_v4(codes + 32u * h), ld_shared_v4(codes + 32u * h + 16u),
+                                      bf16_bits_to_f32(sc.a), bf16_bits_to_f32(sc.b), wv);
+                    }
+                    // These 32 weights = 16 TMEM columns of lane r in stage s.  The
+                    // stage's previous tile was consumed by the MMA S k-blocks back:
+                    // its smem stage was freed before this one was filled.
+                    tmem_st_32x32b_x16(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + a_tmem_col(s) + 16u * h, wv);
                 }
-                // This thread's 32 weights = 16 TMEM columns of its lane (row r) in
-                // stage s.  The stage's previous tile was consumed by the MMA S
-                // k-blocks back: its smem stage was freed before this one was filled.
-                tmem_st_32x32b_x16(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + a_tmem_col(s) + 16u * h, wv);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
