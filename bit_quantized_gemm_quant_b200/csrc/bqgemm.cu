@@ -194,13 +194,28 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return BQ_ERR_SHAPE;
     constexpr bool kFused = MODE != kModeBF16;
     // TMEM (512 columns): two accumulators acc_stride columns apart and, in fused
-    // modes, one 32-column dequantized weight tile per pipeline stage.
-    const int bn = kFused ? choose_bn(M, N, di.num_sms, 192, 64) : choose_bn(M, N, di.num_sms, 256, 32);
+    // modes, one 32-column dequantized weight tile per pipeline stage.  A fused
+    // tile wider than 192 tokens leaves room for one accumulator only; it is taken
+    // when it needs fewer rounds of tiles over the SMs than the best tile <= 192.
+    int bn = kFused ? choose_bn(M, N, di.num_sms, 192, 64) : choose_bn(M, N, di.num_sms, 256, 32);
+    int num_acc = 2;
+    if (kFused && M > 192) {
+        const int64_t wtiles = (N + 127) / 128;
+        auto rounds = [&](int b) {
+            const int64_t t = ((M + b - 1) / b) * wtiles;
+            return (t + di.num_sms - 1) / di.num_sms;
+        };
+        const int wide = (int)std::min<int64_t>(256, (M + 15) / 16 * 16);
+        if (wide > 192 && rounds(wide) < rounds(bn)) {
+            bn = wide;
+            num_acc = 1;
+        }
+    }
     const int acc_stride = kFused ? (bn + 31) / 32 * 32 : 256;
     const uint32_t stage = tc_stage_bytes(MODE, bn);
     const int budget = di.max_smem_optin - 1024 - 512;
     int stages = std::min<int>(8, budget / (int)stage);
-    if (kFused) stages = std::min(stages, (512 - 2 * acc_stride) / 32);
+    if (kFused) stages = std::min(stages, (512 - num_acc * acc_stride) / 32);
     if (stages < 3) return BQ_ERR_UNSUPPORTED;
     // one CTA per SM: the kernel allocates all 512 TMEM columns
     const size_t smem = std::max<size_t>(1024 + (size_t)stages * stage + 512, (size_t)di.max_smem_optin / 2 + 1024);
@@ -237,6 +252,7 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     if (tiles > INT32_MAX) return BQ_ERR_SHAPE;
     p.tiles = (int)tiles;
     p.acc_stride = acc_stride;
+    p.num_acc = num_acc;
     p.vec_scales = (K % 512 == 0) ? 1 : 0;
     const unsigned grid = (unsigned)std::min<int64_t>(tiles, di.num_sms);
     tc_gemm_kernel<MODE><<<grid, C::kThreads, smem, st>>>(tm_x, tm_a, p);

@@ -64,6 +64,7 @@ struct TcParams {
     int m_tiles;              // token tiles per weight tile
     int tiles;                // total tiles
     int acc_stride;           // TMEM columns between the two accumulators
+    int num_acc;              // 2: the epilogue drains one tile while the next accumulates; 1: bn up to 256
     int vec_scales;           // scale rows are 16-byte aligned and hold whole 8-scale windows
 };
 
@@ -225,9 +226,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     auto tfull_bar = [&](int b) { return bar_base + 8u * (uint32_t)(3 * S + b); };      // accumulator b ready
     auto tempty_bar = [&](int b) { return bar_base + 8u * (uint32_t)(3 * S + 2 + b); };  // accumulator b drained
     const uint32_t mma_done_bar = bar_base + 8u * (uint32_t)(3 * S + 4);
-    // TMEM columns: accumulators at 0 and acc_stride; fused modes keep stage s of
+    // TMEM columns: accumulators at 0 (and acc_stride); fused modes keep stage s of
     // the dequantized weight tile (128 lanes x 64 bf16 = 32 columns) after them.
-    auto a_tmem_col = [&](int s) { return 2u * (uint32_t)p.acc_stride + 32u * (uint32_t)s; };
+    auto a_tmem_col = [&](int s) { return (uint32_t)(p.num_acc * p.acc_stride) + 32u * (uint32_t)s; };
+    // Accumulator of the lt-th local tile and the parity of its use count.
+    auto acc_of = [&](int lt) { return p.num_acc == 2 ? (lt & 1) : 0; };
+    auto acc_phase = [&](int lt) { return (uint32_t)(p.num_acc == 2 ? (lt >> 1) : lt) & 1u; };
     const uint32_t tmem_slot = mma_done_bar + 8u;
     uint8_t* smem_gen = smem_raw + (base - smem_u32(smem_raw));
     volatile uint32_t* tmem_slot_ptr = reinterpret_cast<volatile uint32_t*>(smem_gen + (tmem_slot - base));
@@ -297,8 +301,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             uint32_t ph = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++lt) {
-                const int acc = lt & 1;
-                if (!mbar_wait(tempty_bar(acc), ((uint32_t)(lt >> 1) & 1u) ^ 1u)) break;
+                const int acc = acc_of(lt);
+                if (!mbar_wait(tempty_bar(acc), acc_phase(lt) ^ 1u)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.acc_stride);
                 for (int it = 0; it < nk; ++it) {
@@ -334,8 +338,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int q4 = warp & 3;                                       // TMEM lane quarter
         int lt = 0;
         for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++lt) {
-            const int acc = lt & 1;
-            if (!mbar_wait_warp(tfull_bar(acc), (uint32_t)(lt >> 1) & 1u)) break;
+            const int acc = acc_of(lt);
+            if (!mbar_wait_warp(tfull_bar(acc), acc_phase(lt))) break;
             tc_fence_after();
             const int row = tile_n0(t) + 32 * q4 + lane;
             const int m0 = tile_m0(t);
