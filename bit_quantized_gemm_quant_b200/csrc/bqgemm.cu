@@ -101,9 +101,14 @@ int grid_for(int64_t items, int threads, const DeviceInfo& di)
 }
 
 // ------------------------------------------------------------------ env config
+// Default fused/pair threshold, from B200 sweeps of the 12288 x 4096 projection
+// (affine 4/8-bit and Q4_0): the fused kernel is faster up to 768 tokens, the
+// unfused pair from about 1024 tokens (equal for affine4 there, 5% ahead for Q4_0).
+constexpr int64_t kDefaultPairMinM = 1024;
+
 struct DispatchCfg {
     int tc_min_m = kGemvMaxM + 1;
-    int64_t pair_min_m = 0;   // 0: never
+    int64_t pair_min_m = kDefaultPairMinM;   // 0: never
 };
 
 const DispatchCfg& dispatch_cfg()
