@@ -33,6 +33,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch, from one ncu capture of the
+# current build of each kernel (`ncu --set full`, decode bench command); None for a kernel
+# changed since its counters were taken.
+NCU_TRAFFIC = {"gemv_kernel<Q4_0, M=1>": 28340224, "gemv_kernel<Q4_0, M=8>": 28397824,
+               "gemv_kernel<Q4_0, M=32>": 28590592}
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -259,7 +265,7 @@ def run_decode(args, world, device, peaks):
     roof = {"bound": "hbm", "kernel": f"gemv_kernel<Q4_0, M={dom}>",
             "achieved": per_m[str(dom)]["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(per_m[str(dom)]["gbs"] / peaks["hbm_gbs"], 4),
-            "traffic": None, "algorithmic_bytes_per_launch": wbytes}
+            "traffic": NCU_TRAFFIC.get(f"gemv_kernel<Q4_0, M={dom}>"), "algorithmic_bytes_per_launch": wbytes}
 
     # end to end through the public API with host buffers: inputs H2D from pinned memory, y D2H
     e2e = None
