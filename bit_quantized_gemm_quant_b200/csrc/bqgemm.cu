@@ -191,24 +191,53 @@ int choose_bn(int64_t M, int64_t N, int num_sms, int max_bn, int overhead)
     return best_bn;
 }
 
-template <int MODE>
-bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void* a_src, const uint16_t* scales,
-                    const uint16_t* biases, uint16_t* y, int64_t M, int64_t N, int64_t K, cudaStream_t st)
+// Launch plan of the tensor-core kernel for one problem on one device.
+struct TcPlan {
+    int bn = 0, num_acc = 2, acc_stride = 0, stages = 0, splits = 1;
+    int64_t tiles = 0;
+    size_t ws_bytes = 0;      // fp32 partials needed when splits > 1
+};
+
+int64_t splitk_stride(int64_t M, int64_t N) { return (M * N + 3) / 4 * 4; }   // floats per split, 16-byte multiple
+
+// K splits for the fused kernel when its tiles do not fill the SMs: minimise
+// rounds(units) x (k-blocks per split + c) + r, with c the per-unit fixed cost
+// (pipeline fill, epilogue) and r the reduction pass, both in k-block units.
+int choose_splits(int64_t tiles, int64_t nk, int num_sms)
 {
-    using C = TcCfg<MODE>;
-    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return BQ_ERR_SHAPE;
+    if (tiles >= num_sms) return 1;
+    constexpr int64_t kUnitCost = 4, kReduceCost = 4, kMinKBlocks = 4;
+    auto cost = [&](int64_t sp) {
+        const int64_t rounds = (tiles * sp + num_sms - 1) / num_sms;
+        return rounds * ((nk + sp - 1) / sp + kUnitCost) + (sp > 1 ? kReduceCost : 0);
+    };
+    int best = 1;
+    int64_t best_cost = cost(1);
+    for (int sp = 2; sp <= 8 && nk / sp >= kMinKBlocks; ++sp) {
+        const int64_t c = cost(sp);
+        if (c < best_cost) {
+            best_cost = c;
+            best = sp;
+        }
+    }
+    return best;
+}
+
+template <int MODE>
+bool plan_tc(int64_t M, int64_t N, int64_t K, int num_sms, int smem_optin, TcPlan* pl)
+{
     constexpr bool kFused = MODE != kModeBF16;
     // TMEM (512 columns): two accumulators acc_stride columns apart and, in fused
     // modes, one 32-column dequantized weight tile per pipeline stage.  A fused
     // tile wider than 192 tokens leaves room for one accumulator only; it is taken
     // when it needs fewer rounds of tiles over the SMs than the best tile <= 192.
-    int bn = kFused ? choose_bn(M, N, di.num_sms, 192, 64) : choose_bn(M, N, di.num_sms, 256, 32);
+    int bn = kFused ? choose_bn(M, N, num_sms, 192, 64) : choose_bn(M, N, num_sms, 256, 32);
     int num_acc = 2;
+    const int64_t wtiles = (N + 127) / 128;
     if (kFused && M > 192) {
-        const int64_t wtiles = (N + 127) / 128;
         auto rounds = [&](int b) {
             const int64_t t = ((M + b - 1) / b) * wtiles;
-            return (t + di.num_sms - 1) / di.num_sms;
+            return (t + num_sms - 1) / num_sms;
         };
         const int wide = (int)std::min<int64_t>(256, (M + 15) / 16 * 16);
         if (wide > 192 && rounds(wide) < rounds(bn)) {
@@ -218,10 +247,54 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     }
     const int acc_stride = kFused ? (bn + 31) / 32 * 32 : 256;
     const uint32_t stage = tc_stage_bytes(MODE, bn);
-    const int budget = di.max_smem_optin - 1024 - 512;
+    const int budget = smem_optin - 1024 - 512;
     int stages = std::min<int>(8, budget / (int)stage);
     if (kFused) stages = std::min(stages, (512 - num_acc * acc_stride) / 32);
-    if (stages < 3) return BQ_ERR_UNSUPPORTED;
+    if (stages < 3) return false;
+    pl->bn = bn;
+    pl->num_acc = num_acc;
+    pl->acc_stride = acc_stride;
+    pl->stages = stages;
+    pl->tiles = ((M + bn - 1) / bn) * wtiles;
+    pl->splits = kFused ? choose_splits(pl->tiles, (K + 63) / 64, num_sms) : 1;
+    pl->ws_bytes = pl->splits > 1 ? (size_t)pl->splits * (size_t)splitk_stride(M, N) * 4u : 0u;
+    return true;
+}
+
+// y = bf16(sum over splits of ws[split]) in split order (deterministic).
+__global__ void splitk_reduce_kernel(const float* __restrict__ ws, uint16_t* __restrict__ y, int64_t mn,
+                                     int64_t stride, int splits)
+{
+    const int64_t n4 = mn / 4;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        float4 a = reinterpret_cast<const float4*>(ws)[i];
+        for (int sp = 1; sp < splits; ++sp) {
+            const float4 b = reinterpret_cast<const float4*>(ws + sp * stride)[i];
+            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        reinterpret_cast<uint2*>(y)[i] = make_uint2(pack_bf16x2_rn(a.x, a.y), pack_bf16x2_rn(a.z, a.w));
+    }
+    if (blockIdx.x == 0)
+        for (int64_t i = n4 * 4 + threadIdx.x; i < mn; i += blockDim.x) {
+            float a = ws[i];
+            for (int sp = 1; sp < splits; ++sp) a += ws[sp * stride + i];
+            y[i] = (uint16_t)f32_to_bf16_bits(a);
+        }
+}
+
+template <int MODE>
+bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void* a_src, const uint16_t* scales,
+                    const uint16_t* biases, uint16_t* y, int64_t M, int64_t N, int64_t K, cudaStream_t st,
+                    void* ws = nullptr, size_t ws_bytes = 0)
+{
+    using C = TcCfg<MODE>;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return BQ_ERR_SHAPE;
+    TcPlan pl;
+    if (!plan_tc<MODE>(M, N, K, di.num_sms, di.max_smem_optin, &pl)) return BQ_ERR_UNSUPPORTED;
+    // K splits only with a workspace that holds their partial sums
+    if (pl.splits > 1 && (!ws || ws_bytes < pl.ws_bytes)) pl.splits = 1;
+    const int bn = pl.bn, stages = pl.stages;
+    const uint32_t stage = tc_stage_bytes(MODE, bn);
     // one CTA per SM: the kernel allocates all 512 TMEM columns
     const size_t smem = std::max<size_t>(1024 + (size_t)stages * stage + 512, (size_t)di.max_smem_optin / 2 + 1024);
 
@@ -256,11 +329,21 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     const int64_t tiles = (int64_t)p.m_tiles * ((N + 127) / 128);
     if (tiles > INT32_MAX) return BQ_ERR_SHAPE;
     p.tiles = (int)tiles;
-    p.acc_stride = acc_stride;
-    p.num_acc = num_acc;
+    p.acc_stride = pl.acc_stride;
+    p.num_acc = pl.num_acc;
+    p.splits = pl.splits;
+    p.ws = pl.splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
+    p.ws_stride = splitk_stride(M, N);
     p.vec_scales = (K % 512 == 0) ? 1 : 0;
-    const unsigned grid = (unsigned)std::min<int64_t>(tiles, di.num_sms);
+    const unsigned grid = (unsigned)std::min<int64_t>(tiles * pl.splits, di.num_sms);
     tc_gemm_kernel<MODE><<<grid, C::kThreads, smem, st>>>(tm_x, tm_a, p);
+    if (pl.splits > 1) {
+        bq_status r = launch_status();
+        if (r != BQ_OK) return r;
+        const int64_t mn = M * N;
+        const unsigned rgrid = (unsigned)std::max<int64_t>(1, std::min<int64_t>((mn / 4 + 255) / 256, 4 * di.num_sms));
+        splitk_reduce_kernel<<<rgrid, 256, 0, st>>>(p.ws, y, mn, splitk_stride(M, N), pl.splits);
+    }
     return launch_status();
 }
 
@@ -315,9 +398,17 @@ bq_status library_workspace(int dev, size_t need, void** out)
     return BQ_OK;
 }
 
-size_t workspace_for(int path, int64_t N, int64_t K)
+// Workspace of a path: the bf16 copy of W for the pair; the K-split partial
+// sums for the fused kernel when its plan splits K (0 otherwise).
+size_t workspace_for(int path, WFmt fmt, int64_t M, int64_t N, int64_t K, int num_sms, int smem_optin)
 {
-    return path == BQ_PATH_DEQUANT_GEMM ? (size_t)N * (size_t)K * 2u : 0u;
+    if (path == BQ_PATH_DEQUANT_GEMM) return (size_t)N * (size_t)K * 2u;
+    if (path != BQ_PATH_TC_FUSED || K % 64 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return 0u;
+    TcPlan pl;
+    bool ok = fmt == WFmt::Q4_0  ? plan_tc<kModeQ4_0>(M, N, K, num_sms, smem_optin, &pl)
+              : fmt == WFmt::AFF4 ? plan_tc<kModeAff4>(M, N, K, num_sms, smem_optin, &pl)
+                                  : plan_tc<kModeAff8>(M, N, K, num_sms, smem_optin, &pl);
+    return ok ? pl.ws_bytes : 0u;
 }
 
 bq_status dequant_any(WFmt fmt, const void* wq, const void* scales, const void* biases, uint16_t* out, int64_t N,
@@ -367,10 +458,11 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
     if (path == BQ_PATH_AUTO) path = select_path(M, K, fmt);
     if (path == BQ_PATH_GEMV && M > kGemvMaxM) return BQ_ERR_UNSUPPORTED;
     if (path == BQ_PATH_TC_FUSED && K % 64 != 0) return BQ_ERR_UNSUPPORTED;
-    const size_t need = workspace_for(path, N, K);
-    if (workspace && workspace_bytes < need) return BQ_ERR_WORKSPACE;
+    if (path == BQ_PATH_DEQUANT_GEMM && workspace && workspace_bytes < (size_t)N * (size_t)K * 2u)
+        return BQ_ERR_WORKSPACE;
 
     if ((s = current_device(&dev, &di)) != BQ_OK) return s;
+    const size_t need = workspace_for(path, fmt, M, N, K, di.num_sms, di.max_smem_optin);
 
     const uint16_t* sc = reinterpret_cast<const uint16_t*>(scales);
     const uint16_t* bi = reinterpret_cast<const uint16_t*>(biases);
@@ -379,10 +471,20 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
         if (fmt == WFmt::Q4_0) return launch_gemv<Fmt::Q4_0>(x, wq, sc, bi, y, M, N, K, group_size, st);
         if (fmt == WFmt::AFF4) return launch_gemv<Fmt::AFF4>(x, wq, sc, bi, y, M, N, K, group_size, st);
         return launch_gemv<Fmt::AFF8>(x, wq, sc, bi, y, M, N, K, group_size, st);
-    case BQ_PATH_TC_FUSED:
-        if (fmt == WFmt::Q4_0) return launch_tc<kModeQ4_0>(di, dev, x, wq, sc, bi, y, M, N, K, st);
-        if (fmt == WFmt::AFF4) return launch_tc<kModeAff4>(di, dev, x, wq, sc, bi, y, M, N, K, st);
-        return launch_tc<kModeAff8>(di, dev, x, wq, sc, bi, y, M, N, K, st);
+    case BQ_PATH_TC_FUSED: {
+        // K splits take the caller's workspace when it is large enough, the
+        // library's per-device buffer when the caller passed none, and are
+        // dropped (one split) when a caller's workspace is too small.
+        void* ws = workspace;
+        size_t wsb = workspace_bytes;
+        if (!ws && need > 0) {
+            if ((s = library_workspace(dev, need, &ws)) != BQ_OK) return s;
+            wsb = need;
+        }
+        if (fmt == WFmt::Q4_0) return launch_tc<kModeQ4_0>(di, dev, x, wq, sc, bi, y, M, N, K, st, ws, wsb);
+        if (fmt == WFmt::AFF4) return launch_tc<kModeAff4>(di, dev, x, wq, sc, bi, y, M, N, K, st, ws, wsb);
+        return launch_tc<kModeAff8>(di, dev, x, wq, sc, bi, y, M, N, K, st, ws, wsb);
+    }
     default: {
         void* ws = workspace;
         if (!ws && (s = library_workspace(dev, need, &ws)) != BQ_OK) return s;
@@ -496,7 +598,15 @@ size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int group_si
     WFmt fmt;
     if (M < 0 || check_format(format_tag(group_size, bits), N, K, group_size, bits, &fmt) != BQ_OK) return 0;
     if (path == BQ_PATH_AUTO) path = select_path(M, K, fmt);
-    return workspace_for(path, N, K);
+    // the current device's SM count and shared memory when there is one, else a B200's
+    int dev, num_sms = 148, smem_optin = 232448;
+    DeviceInfo di;
+    if (cudaGetDevice(&dev) == cudaSuccess && current_device(&dev, &di) == BQ_OK) {
+        num_sms = di.num_sms;
+        smem_optin = di.max_smem_optin;
+    }
+    cudaGetLastError();
+    return workspace_for(path, fmt, M, N, K, num_sms, smem_optin);
 }
 
 int quant_matmul_select_path(int64_t M, int64_t N, int64_t K, int group_size, int bits)

@@ -66,6 +66,9 @@ struct TcParams {
     int acc_stride;           // TMEM columns between the two accumulators
     int num_acc;              // 2: the epilogue drains one tile while the next accumulates; 1: bn up to 256
     int vec_scales;           // scale rows are 16-byte aligned and hold whole 8-scale windows
+    int splits;               // K splits per tile (fused modes); > 1: fp32 partials to ws
+    float* ws;                // [splits][M][N] fp32 partial sums when splits > 1
+    int64_t ws_stride;        // floats between consecutive splits' partials
 };
 
 // Shared memory per pipeline stage: the activation tile (bn x 64 bf16, 128B
@@ -237,6 +240,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     volatile uint32_t* tmem_slot_ptr = reinterpret_cast<volatile uint32_t*>(smem_gen + (tmem_slot - base));
     auto tile_n0 = [&](int t) { return (t / p.m_tiles) * 128; };
     auto tile_m0 = [&](int t) { return (t % p.m_tiles) * p.bn; };
+    // Work units: unit u is tile u / splits over the k-blocks [kb_begin(u), kb_end(u))
+    // of K split u % splits (splits == 1: whole tiles).
+    const int units = p.tiles * p.splits;
+    auto unit_tile = [&](int u) { return u / p.splits; };
+    // (nk < 2^24 and splits <= 8: the products fit 32-bit arithmetic)
+    auto kb_begin = [&](int u) { return p.splits == 1 ? 0 : (u % p.splits) * nk / p.splits; };
+    auto kb_end = [&](int u) { return p.splits == 1 ? nk : (u % p.splits + 1) * nk / p.splits; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -271,9 +281,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             int s = 0, issued = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                const int t = unit_tile(u);
                 const int n0 = tile_n0(t), m0 = tile_m0(t);
-                for (int it = 0; it < nk; ++it) {
+                const int kb1 = kb_end(u);
+                for (int it = kb_begin(u); it < kb1; ++it) {
                     if (!mbar_wait(empty_bar(s), ph ^ 1u)) { ok = false; break; }
                     mbar_arrive_expect_tx(full_bar(s), b_bytes + (MODE == kModeBF16 ? C::kABytes : C::kCBytes));
                     tma_load_2d(b_base + (uint32_t)s * b_bytes, &tm_x, full_bar(s), it * 64, m0);
@@ -300,12 +312,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             int s = 0, lt = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++lt) {
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++lt) {
                 const int acc = acc_of(lt);
+                const int kb0 = kb_begin(u), kb1 = kb_end(u);
                 if (!mbar_wait(tempty_bar(acc), acc_phase(lt) ^ 1u)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.acc_stride);
-                for (int it = 0; it < nk; ++it) {
+                for (int it = kb0; it < kb1; ++it) {
                     if (!mbar_wait(full_bar(s), ph)) { ok = false; break; }
                     if constexpr (MODE != kModeBF16) {
                         if (!mbar_wait(afull_bar(s), ph)) { ok = false; break; }
@@ -317,12 +330,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             umma_f16_ss(d_tmem, umma_desc_k_sw128(a_addr + 32u * kk),
-                                        umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it | kk) != 0 ? 1u : 0u);
+                                        umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it != kb0 || kk != 0) ? 1u : 0u);
                     } else {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)   // K = 16 per MMA = 8 TMEM columns of A
                             umma_f16_ts(d_tmem, tmem_base + a_tmem_col(s) + 8u * kk,
-                                        umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it | kk) != 0 ? 1u : 0u);
+                                        umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it != kb0 || kk != 0) ? 1u : 0u);
                     }
                     umma_commit(empty_bar(s));
                     if (++s == S) { s = 0; ph ^= 1u; }
@@ -337,24 +350,48 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         // ---------------- epilogue ----------------
         const int q4 = warp & 3;                                       // TMEM lane quarter
         int lt = 0;
-        for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++lt) {
+        for (int u = blockIdx.x; u < units; u += gridDim.x, ++lt) {
+            const int t = unit_tile(u);
             const int acc = acc_of(lt);
             if (!mbar_wait_warp(tfull_bar(acc), acc_phase(lt))) break;
             tc_fence_after();
             const int row = tile_n0(t) + 32 * q4 + lane;
             const int m0 = tile_m0(t);
+            float* part = p.splits > 1 ? p.ws + (int64_t)(u % p.splits) * p.ws_stride : nullptr;
             const uint32_t lane_addr = tmem_base + ((uint32_t)(32 * q4) << 16) + (uint32_t)(acc * p.acc_stride);
-            for (int c0 = 0; c0 < p.bn; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(lane_addr + (uint32_t)c0, v);
-                tmem_wait_ld();
-                if (row < p.N) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int m = m0 + c0 + j;
-                        if (m < p.M) p.y[(int64_t)m * p.N + row] = (uint16_t)f32_to_bf16_bits(__uint_as_float(v[j]));
-                    }
+            // 16 columns (tokens) per TMEM load; the next load is in flight while
+            // this chunk is converted and stored (wait::ld waits for all loads).
+            auto drain = [&](auto&& store16) {
+                uint32_t va[16], vb[16];
+                tmem_ld_32x32b_x16(lane_addr, va);
+                for (int c0 = 0; c0 < p.bn; c0 += 32) {
+                    tmem_wait_ld();
+                    const bool more = c0 + 16 < p.bn;
+                    if (more) tmem_ld_32x32b_x16(lane_addr + (uint32_t)(c0 + 16), vb);
+                    store16(va, m0 + c0);
+                    if (!more) break;
+                    tmem_wait_ld();
+                    if (c0 + 32 < p.bn) tmem_ld_32x32b_x16(lane_addr + (uint32_t)(c0 + 32), va);
+                    store16(vb, m0 + c0 + 16);
                 }
+                tmem_wait_ld();
+            };
+            // The branch is warp-uniform (part is per unit): the TMEM loads are
+            // warp-collective, so every lane takes part; lanes past N only skip stores.
+            const bool row_ok = row < p.N;
+            if (part) {                                               // K split: fp32 partial sums
+                drain([&](const uint32_t (&v)[16], int mb) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (row_ok && mb + j < p.M) part[(int64_t)(mb + j) * p.N + row] = __uint_as_float(v[j]);
+                });
+            } else {
+                drain([&](const uint32_t (&v)[16], int mb) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (row_ok && mb + j < p.M)
+                            p.y[(int64_t)(mb + j) * p.N + row] = (uint16_t)f32_to_bf16_bits(__uint_as_float(v[j]));
+                });
             }
             tc_fence_before();
             mbar_arrive(tempty_bar(acc));
@@ -366,27 +403,35 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int h0 = (C::kDeqWarpsPerGroup == 8) ? ((warp >> 2) & 1) : 0;
         const int grp = warp / C::kDeqWarpsPerGroup;   // takes k-blocks kb with kb % groups == grp
         constexpr int kSpan = ScaleWindow<MODE>::kSpan;
-        const int nwin = (nk + kSpan - 1) / kSpan;
-        // Scale windows form one stream over this CTA's (tile, window) pairs, so
-        // the first window of the next tile is already in flight at a tile boundary.
-        auto load_q = [&](int q) {
-            const int t = blockIdx.x + (q / nwin) * gridDim.x;
-            const int row = t < p.tiles ? tile_n0(t) + r : p.N;
-            return load_scale_window<MODE>(p, row, q % nwin);
+        // The scale windows this CTA needs, in order: for each of its units, the
+        // windows over the unit's k-blocks.  The next one is always in flight, so a
+        // window is fetched a whole window ahead, also across unit boundaries.
+        struct WinPos { int u, w, w_last; };      // unit, window, the unit's last window
+        auto first_pos = [&](int u) {
+            return u < units ? WinPos{u, kb_begin(u) / kSpan, (kb_end(u) - 1) / kSpan} : WinPos{units, 0, 0};
         };
-        int q_cur = 0;
-        ScaleWindow<MODE> win_cur = load_q(0);
-        ScaleWindow<MODE> win_nxt = load_q(1);
-        int s = 0, ti = 0, kb = 0;
+        auto next_pos = [&](WinPos q) {
+            if (q.u < units && q.w < q.w_last) return WinPos{q.u, q.w + 1, q.w_last};
+            return first_pos(q.u < units ? q.u + (int)gridDim.x : units);
+        };
+        auto load_pos = [&](WinPos q) {
+            const int row = q.u < units ? tile_n0(unit_tile(q.u)) + r : p.N;   // past the end: nothing loaded
+            return load_scale_window<MODE>(p, row, q.w);
+        };
+        WinPos pos_cur = first_pos(blockIdx.x), pos_nxt = next_pos(pos_cur);
+        ScaleWindow<MODE> win_cur = load_pos(pos_cur);
+        ScaleWindow<MODE> win_nxt = load_pos(pos_nxt);
+        int s = 0, kb = 0;
         uint32_t ph = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++ti) {
-            for (int it = 0; it < nk; ++it, ++kb) {
-                const int q = ti * nwin + it / kSpan;
-                if (q_cur < q) {                                  // advance one window, fetch the one after
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            const int kb1 = kb_end(u);
+            for (int it = kb_begin(u); it < kb1; ++it, ++kb) {
+                if (pos_cur.u != u || pos_cur.w != it / kSpan) {   // advance one window, fetch the one after
                     win_cur = win_nxt;
-                    ++q_cur;
-                    win_nxt = load_q(q_cur + 1);
+                    pos_cur = pos_nxt;
+                    pos_nxt = next_pos(pos_nxt);
+                    win_nxt = load_pos(pos_nxt);
                 }
                 if (C::kDeqGroups > 1 && kb % C::kDeqGroups != grp) {   // another group's k-block
                     if (++s == S) { s = 0; ph ^= 1u; }

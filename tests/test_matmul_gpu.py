@@ -181,3 +181,22 @@ def test_bf16_matmul(M, N, K):
 
 def test_device_status_clean():
     assert bq.bq_device_status() == 0
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "affine4", "affine8"])
+@pytest.mark.parametrize("N,K", [(250, 1024), (1000, 2048), (130, 4096), (520, 8192)])
+def test_gemv_shapes(fmt, N, K):
+    """Decode sizes over ragged row tiles (N % 32 != 0) and several K."""
+    p = Problem(fmt, N, K, seed=N + K)
+    for M in (1, 3, 8, 17, 32):
+        check(p, M, "gemv")
+
+
+def test_gemv_many_rows_sampled():
+    p = Problem("q4_0", 12288, 1024, seed=21)
+    rows = list(range(0, 12288, 97)) + [12287]
+    for M in (1, 8, 32):
+        x = p.x(M)
+        y = run(p, x, "gemv")
+        y_ref, a_ref = reference(x, p.wb[rows])
+        assert_within_tolerance(y[:, torch.as_tensor(rows, device=y.device)], y_ref, a_ref, f"M={M}")
