@@ -9,10 +9,14 @@ Parity status of each function (what pins it, see ``tests/test_oracle_pins.py``)
   f32/f16/bf16 conversions  -- numpy / torch conversions, exhaustive or 1M+ values
   q4_0_quantize             -- closed forms: exact round trip, all-zero block,
                                max-abs element -> q = 0, q range, error bound
-  q4_0_dequantize           -- hand-worked golden block, round trip
+  q4_0_dequantize           -- closed form over every code value with both signs
+                               of d, exact round trip of quantize
+  q4_0_import_aos           -- blocks assembled byte by byte with numpy from
+                               random codes and scales
   affine_quantize           -- closed forms: exact round trip, constant group,
                                min -> 0 / max -> L, error bound
-  affine_dequantize         -- hand-worked golden groups (4 and 8 bit), round trip
+  affine_dequantize         -- closed form over every code value (4 and 8 bit),
+                               exact round trip of quantize
   matmul_ref                -- exact rational (fractions.Fraction) brute force
                                on tiny non-square shapes, one-hot identities
 """
@@ -45,6 +49,7 @@ def _load():
     lib.oracle_f16_to_f32_array.argtypes = [P, P, I64]
     lib.oracle_q4_0_quantize.argtypes = [P, I64, I64, P, P]
     lib.oracle_q4_0_dequantize.argtypes = [P, P, I64, I64, P]
+    lib.oracle_q4_0_import_aos.argtypes = [P, I64, I64, P, P]
     lib.oracle_affine_quantize.argtypes = [P, I64, I64, I, I, P, P, P]
     lib.oracle_affine_dequantize.argtypes = [P, P, P, I64, I64, I, I, P]
     lib.oracle_matmul_ref.argtypes = [P, P, I64, I64, I64, P, I64, P, P, I]
@@ -115,6 +120,18 @@ def q4_0_dequantize(wq, d) -> np.ndarray:
     out = np.empty((N, K), np.uint16)
     _load().oracle_q4_0_dequantize(_ptr(wq), _ptr(d), N, K, _ptr(out))
     return out
+
+
+def q4_0_import_aos(blocks) -> tuple[np.ndarray, np.ndarray]:
+    """Array-of-structs Q4_0 blocks u8 [N][K/32 * 18] (fp16 d, then 16 code bytes)
+    -> (wq u8 [N][K/2], d fp16 bits u16 [N][K/32])."""
+    blocks = _c(blocks, np.uint8)
+    N, K = blocks.shape[0], blocks.shape[1] // 18 * 32
+    assert blocks.shape[1] == K // 32 * 18
+    wq = np.empty((N, K // 2), np.uint8)
+    d = np.empty((N, K // 32), np.uint16)
+    _load().oracle_q4_0_import_aos(_ptr(blocks), N, K, _ptr(wq), _ptr(d))
+    return wq, d
 
 
 # -------------------------------------------------------------------- affine

@@ -179,6 +179,23 @@ void oracle_q4_0_dequantize(const uint8_t* wq, const uint16_t* d16, int64_t N, i
     }
 }
 
+/* Split array-of-structs Q4_0 blocks into the separate code and scale arrays.
+ * Block layout (ggml's Q4_0 block, which the SYCL page's "reordered" Q4_0
+ * kernels start from): the fp16 scale d (2 bytes, little-endian), then the 16
+ * code bytes in the same nibble order as wq.  Row n holds K/32 consecutive
+ * 18-byte blocks. */
+void oracle_q4_0_import_aos(const uint8_t* blocks, int64_t N, int64_t K, uint8_t* wq, uint16_t* d16)
+{
+    const int64_t nb = K / 32;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const uint8_t* blk = blocks + (n * nb + b) * 18;
+            d16[n * nb + b] = (uint16_t)(blk[0] | (blk[1] << 8));
+            for (int j = 0; j < 16; ++j) wq[n * (K / 2) + b * 16 + j] = blk[2 + j];
+        }
+    }
+}
+
 /* ------------------------------------------------------------------ */
 /* Affine (MLX-style) b-bit, b in {4, 8}                               */
 /* ------------------------------------------------------------------ */

@@ -403,3 +403,24 @@ def test_pins_catch_planted_mistakes():
     assert not np.allclose(y, yt)
     ydrop, _, _ = oracle.matmul_ref(x[:, :31], w[:, :31])
     assert not np.allclose(y, ydrop)
+
+
+def test_q4_0_import_aos_matches_hand_assembled_blocks():
+    """Array-of-structs blocks (fp16 d little-endian, then 16 code bytes) built
+    with numpy from random codes and scales split back into exactly those arrays."""
+    rng = np.random.default_rng(11)
+    N, K = 7, 96
+    wq = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    d = rng.integers(0, 65536, (N, K // 32), dtype=np.uint16)
+    blocks = np.empty((N, K // 32, 18), np.uint8)
+    blocks[:, :, 0] = d & 0xFF
+    blocks[:, :, 1] = d >> 8
+    blocks[:, :, 2:] = wq.reshape(N, K // 32, 16)
+    got_wq, got_d = oracle.q4_0_import_aos(blocks.reshape(N, -1))
+    assert np.array_equal(got_wq, wq)
+    assert np.array_equal(got_d, d)
+    # a planted byte swap of the scale is caught
+    swapped = blocks.copy()
+    swapped[:, :, [0, 1]] = swapped[:, :, [1, 0]]
+    _, bad_d = oracle.q4_0_import_aos(swapped.reshape(N, -1))
+    assert not np.array_equal(bad_d, d)
