@@ -45,6 +45,7 @@ def lib() -> ctypes.CDLL:
     P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     sigs = {
         "q4_0_dequantize": [P, P, P, I64, I64, P],
+        "q4_0_import_aos": [P, P, P, I64, I64, P],
         "affine_dequantize": [P, P, P, P, I64, I64, I, I, P],
         "quant_matmul": [P, P, P, P, P, I64, I64, I64, I, I, I, P],
         "quant_matmul_ex": [P, P, P, P, P, I64, I64, I64, I, I, I, I, P, SZ, P],
@@ -110,6 +111,18 @@ def q4_0_dequantize(wq: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | 
     _check(lib().q4_0_dequantize(_ptr(wq), _ptr(_bits16(scales)), _ptr(out), N, K, _stream(stream)),
            "q4_0_dequantize")
     return out
+
+
+def q4_0_import_aos(blocks: torch.Tensor, stream=None):
+    """Array-of-structs Q4_0 blocks u8 [N][K/32 * 18] (fp16 d, then 16 code bytes)
+    -> (wq u8 [N][K/2], scales fp16 [N][K/32])."""
+    N, K = blocks.shape[0], blocks.shape[1] // 18 * 32
+    if blocks.dtype != torch.uint8 or blocks.shape[1] != K // 32 * 18:
+        raise ValueError("blocks must be u8 [N][K/32 * 18]")
+    wq = torch.empty(N, K // 2, dtype=torch.uint8, device=blocks.device)
+    scales = torch.empty(N, K // 32, dtype=torch.float16, device=blocks.device)
+    _check(lib().q4_0_import_aos(_ptr(blocks), _ptr(wq), _ptr(scales), N, K, _stream(stream)), "q4_0_import_aos")
+    return wq, scales
 
 
 def affine_dequantize(wq: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor, group_size: int = 64,

@@ -539,6 +539,25 @@ bq_status q4_0_dequantize(const uint8_t* wq, const uint16_t* scales_f16, uint16_
     return dequant_any(WFmt::Q4_0, wq, scales_f16, nullptr, out_bf16, N, K, 32, di, (cudaStream_t)stream);
 }
 
+bq_status q4_0_import_aos(const uint8_t* blocks, uint8_t* wq, uint16_t* scales_f16, int64_t N, int64_t K,
+                          bq_stream_t stream)
+{
+    if (N < 0 || K < 0 || K % 32 != 0) return BQ_ERR_SHAPE;
+    const int64_t nb = N * (K / 32);
+    if (nb == 0) return BQ_OK;
+    if (!blocks || !wq || !scales_f16) return BQ_ERR_NULL;
+    if (!aligned16(blocks) || !aligned16(wq) || !aligned16(scales_f16)) return BQ_ERR_ALIGN;
+    int dev;
+    DeviceInfo di;
+    bq_status s = current_device(&dev, &di);
+    if (s != BQ_OK) return s;
+    const int64_t nchunks = (nb + 31) / 32;
+    const int64_t grid = std::min<int64_t>((nchunks + kImportWarps - 1) / kImportWarps, (int64_t)di.num_sms * 8);
+    q4_0_import_aos_kernel<<<(unsigned)std::max<int64_t>(grid, 1), 32 * kImportWarps, 0, (cudaStream_t)stream>>>(
+        blocks, wq, scales_f16, nb);
+    return launch_status();
+}
+
 bq_status affine_dequantize(const uint32_t* wq, const uint16_t* scales_bf16, const uint16_t* biases_bf16,
                             uint16_t* out_bf16, int64_t N, int64_t K, int group_size, int bits, bq_stream_t stream)
 {

@@ -171,4 +171,43 @@ affine_quant_kernel(const float* __restrict__ w, uint32_t* __restrict__ wq, uint
     }
 }
 
+// Array-of-structs Q4_0 import: blocks of 18 bytes (fp16 d little-endian, then
+// the 16 code bytes) -> separate code and scale arrays.  One warp moves 32
+// consecutive blocks (576 bytes, 16-byte aligned when the base is) per step:
+// 16-byte loads into shared memory, then each lane splits out its own block.
+constexpr int kImportWarps = 8;
+
+__global__ void __launch_bounds__(32 * kImportWarps) q4_0_import_aos_kernel(const uint8_t* __restrict__ blocks,
+                                                                           uint8_t* __restrict__ wq,
+                                                                           uint16_t* __restrict__ d16, int64_t nb)
+{
+    __shared__ __align__(16) uint8_t buf[kImportWarps][576];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t* sb = buf[warp];
+    const int64_t nchunks = (nb + 31) / 32;
+    for (int64_t c = (int64_t)blockIdx.x * kImportWarps + warp; c < nchunks; c += (int64_t)gridDim.x * kImportWarps) {
+        const int64_t b0 = c * 32;
+        const int cnt = (int)(nb - b0 < 32 ? nb - b0 : 32);
+        const uint8_t* src = blocks + b0 * 18;
+        if (cnt == 32) {
+            reinterpret_cast<uint4*>(sb)[lane] = ldg_stream(src + 16 * lane);
+            if (lane < 4) reinterpret_cast<uint4*>(sb)[32 + lane] = ldg_stream(src + 512 + 16 * lane);
+        } else {
+            for (int i = lane; i < cnt * 18; i += 32) sb[i] = src[i];
+        }
+        __syncwarp();
+        if (lane < cnt) {
+            const uint8_t* blk = sb + lane * 18;
+            d16[b0 + lane] = (uint16_t)(blk[0] | (blk[1] << 8));
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                w[k] = (uint32_t)blk[2 + 4 * k] | ((uint32_t)blk[3 + 4 * k] << 8) | ((uint32_t)blk[4 + 4 * k] << 16) |
+                       ((uint32_t)blk[5 + 4 * k] << 24);
+            reinterpret_cast<uint4*>(wq)[b0 + lane] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        __syncwarp();
+    }
+}
+
 }  // namespace bq

@@ -108,6 +108,22 @@ BQ_API bq_status affine_dequantize(const uint32_t* wq, const uint16_t* scales_bf
                             bq_stream_t stream);
 
 /*
+ * q4_0_import_aos -- split array-of-structs Q4_0 blocks into the separate code
+ * and scale arrays every other call here takes.  Reading of the pages: the
+ * SYCL page "2026-05-06 Q4 sync-after focused repro" (Important source touch
+ * points) runs its decode kernels on "reordered" Q4_0, i.e. on ggml's Q4_0
+ * blocks moved into separate arrays; the block read here is ggml's: the fp16
+ * scale d (little-endian), then the 16 code bytes in the nibble order of wq.
+ *   blocks      device u8 [N][K/32][18], read
+ *   wq          device u8 [N][K/2], written (16 bytes per block)
+ *   scales_f16  device u16 [N][K/32], written
+ *   K % 32 == 0; all pointers 16-byte aligned (BQ_ERR_ALIGN otherwise).
+ * Bit-exact byte moves; stream-ordered; the caller owns every buffer.
+ */
+BQ_API bq_status q4_0_import_aos(const uint8_t* blocks, uint8_t* wq, uint16_t* scales_f16, int64_t N, int64_t K,
+                                 bq_stream_t stream);
+
+/*
  * quant_matmul -- y[M][N] = bf16_rne(sum_k x[m][k] * dequant(W)[n][k]), fp32
  * accumulation.  mx.quantized_matmul(x, wq, scales, biases, transpose=True,
  * group_size, bits) on the MLX issue page (Repro); its result equals

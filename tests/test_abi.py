@@ -141,3 +141,10 @@ def test_empty_problems_need_no_pointers(L):
     assert L.affine_dequantize(None, None, None, None, 4, 0, 64, 8, None) == 0
     assert L.bf16_matmul(None, None, None, 0, 4, 16, None) == 0
     assert L.q4_0_quantize(None, None, None, 0, 64, None) == 0
+
+
+def test_q4_0_import_aos_validation(L):
+    assert L.q4_0_import_aos(ALIGNED, ALIGNED, ALIGNED, 4, 48, None) == 2        # K % 32
+    assert L.q4_0_import_aos(None, ALIGNED, ALIGNED, 4, 64, None) == 1
+    assert L.q4_0_import_aos(MISALIGNED, ALIGNED, ALIGNED, 4, 64, None) == 4
+    assert L.q4_0_import_aos(None, None, None, 0, 64, None) == 0                  # empty: nothing touched

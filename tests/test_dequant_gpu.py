@@ -99,3 +99,36 @@ def test_affine_quantize_bit_exact(bits, N, K):
     assert np.array_equal(wq.cpu().numpy().view(np.uint32), wq_ref)
     assert np.array_equal(u16(s), s_ref)
     assert np.array_equal(u16(b), b_ref)
+
+
+@pytest.mark.parametrize("N,K", [(1, 32), (3, 96), (250, 1024), (37, 4096), (12288, 4096)])
+def test_q4_0_import_aos_bit_exact(N, K):
+    """Random 18-byte blocks (random fp16 scale bits and code bytes), split on the GPU
+    and by the oracle: identical bytes.  Block counts cover whole 32-block warp
+    chunks and ragged tails."""
+    g = inputs.generator(N + K)
+    blocks = inputs.random_bytes((N, K // 32 * 18), g)
+    wq_ref, d_ref = oracle.q4_0_import_aos(blocks.numpy())
+    wq, d = bq.q4_0_import_aos(blocks.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(wq.cpu().numpy(), wq_ref)
+    assert np.array_equal(d.view(torch.int16).cpu().numpy().view(np.uint16), d_ref)
+
+
+def test_q4_0_import_aos_then_matmul():
+    """Blocks assembled from an oracle quantization feed quant_matmul after import."""
+    N, K, M = 300, 1024, 16
+    g = inputs.generator(4)
+    w = inputs.weights_fp32(N, K, g).numpy()
+    wq, d = oracle.q4_0_quantize(w)
+    blocks = np.empty((N, K // 32, 18), np.uint8)
+    blocks[:, :, 0] = d & 0xFF
+    blocks[:, :, 1] = d >> 8
+    blocks[:, :, 2:] = wq.reshape(N, K // 32, 16)
+    wq_d, d_d = bq.q4_0_import_aos(torch.from_numpy(blocks.reshape(N, -1)).cuda())
+    x = inputs.activations_bf16(M, K, g)
+    y = bq.quant_matmul(x.cuda(), wq_d, d_d, None, 32, 4)
+    torch.cuda.synchronize()
+    y_ref, a_ref, _ = oracle.matmul_ref(x.view(torch.int16).numpy().view(np.uint16), oracle.q4_0_dequantize(wq, d))
+    tol = oracle.tolerance(a_ref, y_ref)
+    assert np.all(np.abs(y.float().cpu().numpy().astype(np.float64) - y_ref) <= tol)
