@@ -358,7 +358,9 @@ def run_prefill(args, world, device, peaks, fmt, Ms):
 def run_stack(args, world, device, peaks):
     """Llama-3.2-1B-shaped projection stack, Q4_0: the 112 matmuls of 16 layers (q, k, v, o,
     gate, up, down), each layer with its own weights (547 MB packed > L2), at M = 512 and
-    M = 1.  One CUDA graph holds the whole stack; tokens/s = M / stack time."""
+    M = 1.  q/k/v and gate/up, which share an activation, go through quant_matmul_multi
+    (one launch each at decode sizes).  One CUDA graph holds the whole stack;
+    tokens/s = M / stack time."""
     import torch
     import bit_quantized_gemm_quant_b200 as bq
     from bit_quantized_gemm_quant_b200 import inputs, workloads
@@ -380,16 +382,31 @@ def run_stack(args, world, device, peaks):
         xs = {K: inputs.activations_bf16(M, K, gx).to(device) for K in sorted({K for _, K, _, _ in mats})}
         ys = [torch.empty(M, N, dtype=torch.bfloat16, device=device) for N, _, _, _ in mats]
 
+        # per layer: q, k, v share one activation (one quant_matmul_multi call), then
+        # o; gate and up share one (one call), then down
+        per_layer = len(wl.shapes)
+        calls = []
+        for l0 in range(0, len(mats), per_layer):
+            lm, ly = mats[l0:l0 + per_layer], ys[l0:l0 + per_layer]
+            calls.append(("multi", lm[0:3], ly[0:3]))
+            calls.append(("one", lm[3:4], ly[3:4]))
+            calls.append(("multi", lm[4:6], ly[4:6]))
+            calls.append(("one", lm[6:7], ly[6:7]))
+
         def stack():
-            for (N, K, wq, d), y in zip(mats, ys):
-                bq.quant_matmul(xs[K], wq, d, None, 32, 4, out=y)
+            for kind, ms, yl in calls:
+                K = ms[0][1]
+                if kind == "multi":
+                    bq.quant_matmul_multi(xs[K], [(wq, d, None) for _, _, wq, d in ms], 32, 4, outs=yl)
+                else:
+                    bq.quant_matmul(xs[K], ms[0][2], ms[0][3], None, 32, 4, out=yl[0])
         gt = GraphTimer(stack)
         for _ in range(max(3, args.warmup // 50)):
             gt.replay()
         reps = max(3, min(200, args.steps // 100))
         sec = max_over_ranks(time_graphs([gt], reps, world, device) / reps, world, device)
         paths = sorted({bq.quant_matmul_select_path(M, N, K, 32, 4) for N, K, _, _ in mats})
-        launches += reps * len(mats)
+        launches += reps * (len(calls) if M <= 32 else len(mats))
         per_m[str(M)] = {"us_per_stack": round(sec * 1e6, 2), "tokens_per_s": round(aggregate(M, world, sec), 1),
                          "tflops": round(2.0 * M * params / sec / 1e12, 2),
                          "frac_tensor": round(2.0 * M * params / sec / 1e12 / peaks["bf16_tflops"], 4),

@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
         "quant_matmul": [P, P, P, P, P, I64, I64, I64, I, I, I, P],
         "quant_matmul_ex": [P, P, P, P, P, I64, I64, I64, I, I, I, I, P, SZ, P],
         "quant_matmul_noalloc": [P, P, P, P, P, I64, I64, I64, I, I, I, P],
+        "quant_matmul_multi": [P, I, P, P, P, P, P, I64, I64, I, I, I, P],
         "quant_matmul_workspace_size": [I64, I64, I64, I, I, I],
         "quant_matmul_select_path": [I64, I64, I64, I, I],
         "bf16_matmul": [P, P, P, I64, I64, I64, P],
@@ -170,6 +171,32 @@ def quant_matmul_ex(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, bia
                 1 if transpose else 0, p, _ptr(workspace), ws_bytes, _stream(stream))
     _check(st, "quant_matmul")
     return out
+
+
+def quant_matmul_multi(x: torch.Tensor, weights, group_size: int = 32, bits: int = 4, transpose: bool = True,
+                       outs=None, stream=None):
+    """Several quantized matmuls sharing x: weights = [(wq, scales, biases|None), ...]
+    (at most 8, one format); returns [y_i bf16 [M][N_i]].  Decode sizes run as one launch."""
+    M, K = x.shape
+    count = len(weights)
+    q4 = weights[0][2] is None
+    if any((b is None) != q4 for _, _, b in weights):
+        raise ValueError("all matrices must be Q4_0 (biases None) or all affine")
+    Ns = [wq.shape[0] for wq, _, _ in weights]
+    for wq, _, b in weights:
+        if K != _k_of(wq, b, bits):
+            raise ValueError("K mismatch between x and a weight matrix")
+    if outs is None:
+        outs = [torch.empty(M, n, dtype=torch.bfloat16, device=x.device) for n in Ns]
+    VP = ctypes.c_void_p * max(count, 1)
+    wq_a = VP(*[_ptr(wq) for wq, _, _ in weights])
+    s_a = VP(*[_ptr(_bits16(sc)) for _, sc, _ in weights])
+    b_a = None if q4 else VP(*[_ptr(_bits16(b)) for _, _, b in weights])
+    y_a = VP(*[_ptr(y) for y in outs])
+    n_a = (ctypes.c_int64 * max(count, 1))(*Ns)
+    _check(lib().quant_matmul_multi(_ptr(x), count, wq_a, s_a, b_a, y_a, n_a, M, K, group_size, bits,
+                                    1 if transpose else 0, _stream(stream)), "quant_matmul_multi")
+    return outs
 
 
 NOALLOC_SCRATCH_BYTES = 32 << 20

@@ -373,6 +373,34 @@ bq_status launch_gemv(const uint16_t* x, const void* wq, const uint16_t* s, cons
     return launch_gemv_cfg<F, 4, 2, 8, 1, 1>(x, wq, s, b, y, M, N, K, group_size, st);
 }
 
+template <Fmt F, int NT, int RT, int KS, int PIPE, int MINB>
+bq_status launch_gemv_multi_cfg(const uint16_t* x, GemvMultiTable& tab, int64_t M, int64_t K, int group_size,
+                                cudaStream_t st)
+{
+    tab.tile_begin[0] = 0;
+    for (int i = 0; i < tab.count; ++i) {
+        const int64_t end = tab.tile_begin[i] + ((int64_t)tab.N[i] + 16 * RT - 1) / (16 * RT);
+        if (end > INT32_MAX) return BQ_ERR_SHAPE;
+        tab.tile_begin[i + 1] = (int)end;
+    }
+    const int grid = tab.tile_begin[tab.count];
+    if (grid == 0) return BQ_OK;
+    gemv_multi_kernel<F, NT, RT, KS, PIPE, MINB><<<(unsigned)grid, 32 * KS, 0, st>>>(x, tab, (int)M, (int)K,
+                                                                                  group_size);
+    return launch_status();
+}
+
+// Same launch shapes as launch_gemv, all matrices in one grid.
+template <Fmt F>
+bq_status launch_gemv_multi(const uint16_t* x, GemvMultiTable& tab, int64_t M, int64_t K, int group_size,
+                            cudaStream_t st)
+{
+    if (K > INT32_MAX) return BQ_ERR_SHAPE;
+    if (M <= 8) return launch_gemv_multi_cfg<F, 1, 2, 4, 2, 3>(x, tab, M, K, group_size, st);
+    if (M <= 16) return launch_gemv_multi_cfg<F, 2, 2, 4, 2, 2>(x, tab, M, K, group_size, st);
+    return launch_gemv_multi_cfg<F, 4, 2, 8, 1, 1>(x, tab, M, K, group_size, st);
+}
+
 // ------------------------------------------------------------------ library workspace
 struct Workspace {
     void* ptr = nullptr;
@@ -610,6 +638,56 @@ bq_status quant_matmul_noalloc(const uint16_t* x_bf16, const void* wq, const voi
     if ((s = noalloc_scratch(dev, &ws)) != BQ_OK) return s;
     return matmul_impl(x_bf16, wq, scales, biases, y_bf16, M, N, K, group_size, bits, transpose,
                        BQ_PATH_DEQUANT_GEMM, ws, BQ_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream);
+}
+
+bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const void* const* wq, const void* const* scales,
+                             const void* const* biases, uint16_t* const* y_bf16, const int64_t* N, int64_t M,
+                             int64_t K, int group_size, int bits, int transpose, bq_stream_t stream)
+{
+    if (transpose != 1) return BQ_ERR_UNSUPPORTED;
+    if (count < 0 || count > kMultiMax || M < 0 || K < 0) return count > kMultiMax ? BQ_ERR_UNSUPPORTED : BQ_ERR_SHAPE;
+    if (count == 0) return BQ_OK;
+    if (!wq || !scales || !y_bf16 || !N) return BQ_ERR_NULL;
+    WFmt fmt;
+    bq_status s;
+    for (int i = 0; i < count; ++i) {
+        if (N[i] < 0 || N[i] > INT32_MAX) return BQ_ERR_SHAPE;
+        if (biases && !biases[i]) return BQ_ERR_NULL;            // all affine or all Q4_0
+        if ((s = check_format(biases ? biases[i] : nullptr, N[i], K, group_size, bits, &fmt)) != BQ_OK) return s;
+    }
+    if (M == 0) return BQ_OK;
+    const int path = select_path(M, K, fmt);
+    if (path != BQ_PATH_GEMV || K == 0) {
+        // prefill sizes: each matrix through its own launch of the chosen path
+        for (int i = 0; i < count; ++i) {
+            s = matmul_impl(x_bf16, wq[i], scales[i], biases ? biases[i] : nullptr, y_bf16[i], M, N[i], K,
+                            group_size, bits, transpose, BQ_PATH_AUTO, nullptr, 0, (cudaStream_t)stream);
+            if (s != BQ_OK) return s;
+        }
+        return BQ_OK;
+    }
+    if (!x_bf16) return BQ_ERR_NULL;
+    if (!aligned16(x_bf16)) return BQ_ERR_ALIGN;
+    GemvMultiTable tab;
+    tab.count = count;
+    for (int i = 0; i < count; ++i) {
+        if (N[i] > 0 && (!wq[i] || !scales[i] || !y_bf16[i])) return BQ_ERR_NULL;
+        if (N[i] > 0 && (!aligned16(wq[i]) || !aligned16(scales[i]) || !aligned16(y_bf16[i]) ||
+                         (biases && !aligned16(biases[i]))))
+            return BQ_ERR_ALIGN;
+        tab.wq[i] = reinterpret_cast<const uint8_t*>(wq[i]);
+        tab.scales[i] = reinterpret_cast<const uint16_t*>(scales[i]);
+        tab.biases[i] = biases ? reinterpret_cast<const uint16_t*>(biases[i]) : nullptr;
+        tab.y[i] = y_bf16[i];
+        tab.N[i] = (int)N[i];
+    }
+    int dev;
+    DeviceInfo di;
+    if ((s = current_device(&dev, &di)) != BQ_OK) return s;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (fmt == WFmt::Q4_0) return launch_gemv_multi<Fmt::Q4_0>(x_bf16, tab, M, K, group_size, st);
+    if (fmt == WFmt::AFF4) return launch_gemv_multi<Fmt::AFF4>(x_bf16, tab, M, K, group_size, st);
+    return launch_gemv_multi<Fmt::AFF8>(x_bf16, tab, M, K, group_size, st);
 }
 
 size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int group_size, int bits, int path)

@@ -236,11 +236,10 @@ BQ_DEVINL void load_step(GemvStage<F, RT>& st, const uint8_t* __restrict__ wq, c
 // weight loads of step s + PIPE are issued before step s is computed, so every
 // load has PIPE steps of other work to hide behind and no warp ever waits a
 // full memory round trip between batches.
-template <Fmt F, int NT, int RT, int KSPLIT, int PIPE, int MINB>
-__global__ void __launch_bounds__(32 * KSPLIT, MINB)
-gemv_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
-            const uint16_t* __restrict__ scales, const uint16_t* __restrict__ biases,
-            uint16_t* __restrict__ y, int M, int N, int K, int group_size)
+template <Fmt F, int NT, int RT, int KSPLIT, int PIPE>
+__device__ __forceinline__ void gemv_body(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
+                                          const uint16_t* __restrict__ scales, const uint16_t* __restrict__ biases,
+                                          uint16_t* __restrict__ y, int M, int N, int K, int group_size, int row_base)
 {
     using T = FmtTraits<F>;
     constexpr int kCE = T::kChunkElems;
@@ -249,7 +248,6 @@ gemv_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
     constexpr int kXWords = kCE / 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int row_base = blockIdx.x * 16 * RT;
     const int64_t row_bytes = (int64_t)K * T::kBits / 8;
     const int nchunks = K / kCE;
     const int per_warp = (nchunks + KSPLIT - 1) / KSPLIT;
@@ -341,6 +339,40 @@ gemv_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
         if (m < M && row_base + row < N)
             y[(int64_t)m * N + row_base + row] = (uint16_t)f32_to_bf16_bits(s);
     }
+}
+
+// One matrix: CTA b owns rows [16*RT*b, 16*RT*(b+1)).
+template <Fmt F, int NT, int RT, int KSPLIT, int PIPE, int MINB>
+__global__ void __launch_bounds__(32 * KSPLIT, MINB)
+gemv_kernel(const uint16_t* __restrict__ x, const uint8_t* __restrict__ wq,
+            const uint16_t* __restrict__ scales, const uint16_t* __restrict__ biases,
+            uint16_t* __restrict__ y, int M, int N, int K, int group_size)
+{
+    gemv_body<F, NT, RT, KSPLIT, PIPE>(x, wq, scales, biases, y, M, N, K, group_size, blockIdx.x * 16 * RT);
+}
+
+// Several matrices that share x (and K, format, group size), one launch: the
+// CTAs of matrix i are [tile_begin[i], tile_begin[i+1]).
+constexpr int kMultiMax = 8;
+struct GemvMultiTable {
+    int count;
+    int tile_begin[kMultiMax + 1];
+    const uint8_t* wq[kMultiMax];
+    const uint16_t* scales[kMultiMax];
+    const uint16_t* biases[kMultiMax];
+    uint16_t* y[kMultiMax];
+    int N[kMultiMax];
+};
+
+template <Fmt F, int NT, int RT, int KSPLIT, int PIPE, int MINB>
+__global__ void __launch_bounds__(32 * KSPLIT, MINB)
+gemv_multi_kernel(const uint16_t* __restrict__ x, const __grid_constant__ GemvMultiTable tab, int M, int K,
+                  int group_size)
+{
+    int i = 0;
+    while (i + 1 < tab.count && (int)blockIdx.x >= tab.tile_begin[i + 1]) ++i;
+    gemv_body<F, NT, RT, KSPLIT, PIPE>(x, tab.wq[i], tab.scales[i], tab.biases[i], tab.y[i], M, tab.N[i], K,
+                                       group_size, ((int)blockIdx.x - tab.tile_begin[i]) * 16 * RT);
 }
 
 }  // namespace bq

@@ -175,6 +175,25 @@ BQ_API bq_status quant_matmul_noalloc(const uint16_t* x_bf16, const void* wq, co
                                       int group_size, int bits, int transpose, bq_stream_t stream);
 
 /*
+ * quant_matmul_multi -- count (<= 8) quantized matmuls that share one
+ * activation x: y[i] = quant_matmul(x, wq[i], scales[i], biases[i], N[i]) for
+ * every i, all with the same M, K, format and group size.  After the SYCL
+ * page "2026-05-06 Q4 sync-after focused repro" (Important source touch
+ * points), which fuses adjacent Q4_0 matrix-vector products sharing one
+ * token's activation (ffn_gate + ffn_up, Vcur + Kcur) into one kernel.
+ *   wq, scales, y_bf16, N: host arrays of count device pointers / row counts
+ *   biases: host array of count device pointers (affine), or NULL (Q4_0 for all)
+ * At decode sizes (the dispatcher's GEMV path) all matrices run in one launch
+ * and give the same bits as separate quant_matmul calls; at larger M each
+ * matrix runs its own quant_matmul path.  Errors as quant_matmul;
+ * count > 8 returns BQ_ERR_UNSUPPORTED, count == 0 or M == 0 does nothing.
+ */
+BQ_API bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const void* const* wq,
+                                    const void* const* scales, const void* const* biases, uint16_t* const* y_bf16,
+                                    const int64_t* N, int64_t M, int64_t K, int group_size, int bits, int transpose,
+                                    bq_stream_t stream);
+
+/*
  * quant_matmul_ex -- quant_matmul with an explicit path (bq_path) and an
  * optional caller-owned device workspace.  With workspace == NULL the library's
  * per-device buffer is used as in quant_matmul; otherwise workspace_bytes must

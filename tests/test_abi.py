@@ -148,3 +148,15 @@ def test_q4_0_import_aos_validation(L):
     assert L.q4_0_import_aos(None, ALIGNED, ALIGNED, 4, 64, None) == 1
     assert L.q4_0_import_aos(MISALIGNED, ALIGNED, ALIGNED, 4, 64, None) == 4
     assert L.q4_0_import_aos(None, None, None, 0, 64, None) == 0                  # empty: nothing touched
+
+
+def test_quant_matmul_multi_validation(L):
+    VP = ctypes.c_void_p * 2
+    ptrs = VP(ALIGNED, ALIGNED)
+    n = (ctypes.c_int64 * 2)(256, 128)
+    assert L.quant_matmul_multi(ALIGNED, 2, ptrs, ptrs, None, ptrs, n, 4, 48, 32, 4, 1, None) == 2     # K % 32
+    assert L.quant_matmul_multi(ALIGNED, 9, ptrs, ptrs, None, ptrs, n, 4, 64, 32, 4, 1, None) == 3     # count > 8
+    assert L.quant_matmul_multi(ALIGNED, 2, ptrs, ptrs, None, ptrs, n, 4, 64, 32, 4, 0, None) == 3     # transpose
+    assert L.quant_matmul_multi(ALIGNED, 2, None, ptrs, None, ptrs, n, 4, 64, 32, 4, 1, None) == 1
+    assert L.quant_matmul_multi(MISALIGNED, 2, ptrs, ptrs, None, ptrs, n, 4, 64, 32, 4, 1, None) == 4
+    assert L.quant_matmul_multi(None, 0, None, None, None, None, None, 4, 64, 32, 4, 1, None) == 0     # nothing

@@ -200,3 +200,23 @@ def test_gemv_many_rows_sampled():
         y = run(p, x, "gemv")
         y_ref, a_ref = reference(x, p.wb[rows])
         assert_within_tolerance(y[:, torch.as_tensor(rows, device=y.device)], y_ref, a_ref, f"M={M}")
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "affine4", "affine8"])
+@pytest.mark.parametrize("M", [1, 8, 32, 100])
+def test_multi_matches_separate_calls(fmt, M):
+    """quant_matmul_multi (Q/K/V-like: three matrices sharing x, ragged N) gives the
+    same bits as separate quant_matmul calls, and each is within the oracle's bound."""
+    K = 1024
+    probs = [Problem(fmt, n, K, seed=n) for n in (300, 64, 130)]
+    x = probs[0].x(M)
+    xd = x.cuda()
+    ws = [p.device() for p in probs]
+    ys = bq.quant_matmul_multi(xd, ws, probs[0].group_size, probs[0].bits)
+    torch.cuda.synchronize()
+    for p, (wq, s, b), y in zip(probs, ws, ys):
+        y1 = bq.quant_matmul(xd, wq, s, b, p.group_size, p.bits)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y1.view(torch.int16)), (fmt, M, p.N)
+        y_ref, a_ref = reference(x, p.wb)
+        assert_within_tolerance(y, y_ref, a_ref, f"multi {fmt} M={M} N={p.N}")
