@@ -211,10 +211,11 @@ def test_q4_0_invariants_random():
 # --------------------------------------------------------------------------
 # affine
 # --------------------------------------------------------------------------
+@pytest.mark.parametrize("G", [32, 64, 128])
 @pytest.mark.parametrize("bits", [4, 8])
-def test_affine_dequant_closed_form_layout(bits):
-    rng = np.random.default_rng(7 + bits)
-    N, K, G = 3, 256, 64
+def test_affine_dequant_closed_form_layout(bits, G):
+    rng = np.random.default_rng(7 + bits + G)
+    N, K = 3, 256
     L = (1 << bits) - 1
     q = rng.integers(0, L + 1, (N, K))
     s = rng.choice([0.25, 0.5, 0.0625], size=(N, K // G))      # b/s integer, q + b/s in [-48, 255]
@@ -244,10 +245,11 @@ def test_affine_dequant_rounding_reduces_to_library(bits):
     assert np.array_equal(got, torch_bf16_bits(exact.astype(np.float32)))
 
 
+@pytest.mark.parametrize("G", [32, 64, 128])
 @pytest.mark.parametrize("bits", [4, 8])
-def test_affine_round_trip_exact(bits):
-    rng = np.random.default_rng(9 + bits)
-    N, K, G = 8, 256, 64
+def test_affine_round_trip_exact(bits, G):
+    rng = np.random.default_rng(9 + bits + G)
+    N, K = 8, 256
     L = (1 << bits) - 1
     q = rng.integers(0, L + 1, (N, K))
     qg = q.reshape(N, K // G, G)
@@ -277,10 +279,11 @@ def test_affine_constant_group(bits):
     assert np.array_equal(back, w)
 
 
+@pytest.mark.parametrize("G", [32, 64, 128])
 @pytest.mark.parametrize("bits", [4, 8])
-def test_affine_invariants_random(bits):
-    g = inputs.generator(10 + bits)
-    N, K, G = 48, 1024, 64
+def test_affine_invariants_random(bits, G):
+    g = inputs.generator(10 + bits + G)
+    N, K = 48, 1024
     L = (1 << bits) - 1
     w = inputs.weights_bf16_valued(N, K, g).numpy()
     wq, s16, b16 = oracle.affine_quantize(w, G, bits)
