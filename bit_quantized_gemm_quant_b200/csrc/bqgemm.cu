@@ -70,7 +70,7 @@ bq_status check_format(const void* biases, int64_t N, int64_t K, int group_size,
         *fmt = WFmt::Q4_0;
     } else {
         if (bits != 4 && bits != 8) return BQ_ERR_UNSUPPORTED;
-        if (group_size != 64) return BQ_ERR_UNSUPPORTED;
+        if (group_size != 32 && group_size != 64 && group_size != 128) return BQ_ERR_UNSUPPORTED;
         if (K % group_size != 0) return BQ_ERR_SHAPE;
         *fmt = bits == 4 ? WFmt::AFF4 : WFmt::AFF8;
     }
@@ -285,7 +285,7 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ ws, uint16_t* __r
 template <int MODE>
 bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void* a_src, const uint16_t* scales,
                     const uint16_t* biases, uint16_t* y, int64_t M, int64_t N, int64_t K, cudaStream_t st,
-                    void* ws = nullptr, size_t ws_bytes = 0)
+                    void* ws = nullptr, size_t ws_bytes = 0, int group_size = 64)
 {
     using C = TcCfg<MODE>;
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return BQ_ERR_SHAPE;
@@ -334,7 +334,11 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     p.splits = pl.splits;
     p.ws = pl.splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
     p.ws_stride = splitk_stride(M, N);
-    p.vec_scales = (K % 512 == 0) ? 1 : 0;
+    {
+        const int gs = (MODE == kModeQ4_0 || MODE == kModeBF16) ? 32 : group_size;
+        p.gs_shift = gs == 32 ? 5 : gs == 64 ? 6 : 7;
+        p.vec_scales = ((K >> p.gs_shift) % 8 == 0) ? 1 : 0;   // every row starts and ends on whole windows
+    }
     const unsigned grid = (unsigned)std::min<int64_t>(tiles * pl.splits, di.num_sms);
     tc_gemm_kernel<MODE><<<grid, C::kThreads, smem, st>>>(tm_x, tm_a, p);
     if (pl.splits > 1) {
@@ -509,9 +513,9 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
             if ((s = library_workspace(dev, need, &ws)) != BQ_OK) return s;
             wsb = need;
         }
-        if (fmt == WFmt::Q4_0) return launch_tc<kModeQ4_0>(di, dev, x, wq, sc, bi, y, M, N, K, st, ws, wsb);
-        if (fmt == WFmt::AFF4) return launch_tc<kModeAff4>(di, dev, x, wq, sc, bi, y, M, N, K, st, ws, wsb);
-        return launch_tc<kModeAff8>(di, dev, x, wq, sc, bi, y, M, N, K, st, ws, wsb);
+        if (fmt == WFmt::Q4_0) return launch_tc<kModeQ4_0>(di, dev, x, wq, sc, bi, y, M, N, K, st, ws, wsb, group_size);
+        if (fmt == WFmt::AFF4) return launch_tc<kModeAff4>(di, dev, x, wq, sc, bi, y, M, N, K, st, ws, wsb, group_size);
+        return launch_tc<kModeAff8>(di, dev, x, wq, sc, bi, y, M, N, K, st, ws, wsb, group_size);
     }
     default: {
         void* ws = workspace;

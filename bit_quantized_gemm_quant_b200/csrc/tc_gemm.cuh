@@ -66,6 +66,7 @@ struct TcParams {
     int acc_stride;           // TMEM columns between the two accumulators
     int num_acc;              // 2: the epilogue drains one tile while the next accumulates; 1: bn up to 256
     int vec_scales;           // scale rows are 16-byte aligned and hold whole 8-scale windows
+    int gs_shift;             // log2 of the group size (Q4_0: 5; affine: 5, 6 or 7)
     int splits;               // K splits per tile (fused modes); > 1: fp32 partials to ws
     float* ws;                // [splits][M][N] fp32 partial sums when splits > 1
     int64_t ws_stride;        // floats between consecutive splits' partials
@@ -146,11 +147,10 @@ BQ_DEVINL void deq_aff8_half(uint4 raw0, uint4 raw1, float s, float b, uint32_t 
 struct DeqScale { uint32_t a, b; };
 
 // Scales of one dequant thread's row, fetched a whole window of k-blocks ahead:
-// one 16-byte vector holds 8 consecutive 16-bit scales = 4 k-blocks of Q4_0
-// (two blocks per k-block) or 8 k-blocks of affine (one group per k-block).
+// one 16-byte vector holds 8 consecutive 16-bit scales, i.e. group_size / 8
+// k-blocks (4 for Q4_0 and affine group 32, 8 for group 64, 16 for group 128).
 template <int MODE>
 struct ScaleWindow {
-    static constexpr int kSpan = (MODE == kModeQ4_0) ? 4 : 8;   // k-blocks per window
     uint4 s, b;
 };
 
@@ -166,7 +166,7 @@ BQ_DEVINL ScaleWindow<MODE> load_scale_window(const TcParams& p, int row, int wi
     ScaleWindow<MODE> w;
     w.s = w.b = make_uint4(0, 0, 0, 0);
     if (row >= p.N) return w;
-    const int per_row = (MODE == kModeQ4_0) ? p.K / 32 : p.K / 64;          // 16-bit scales per row
+    const int per_row = p.K >> p.gs_shift;                                    // 16-bit scales per row
     const int first = win * 8;
     const uint16_t* srow = p.scales + (int64_t)row * per_row;
     const uint16_t* brow = p.biases + (int64_t)row * per_row;
@@ -188,19 +188,23 @@ BQ_DEVINL ScaleWindow<MODE> load_scale_window(const TcParams& p, int row, int wi
     return w;
 }
 
-// Expanded scale of k-block `it` (half `h` for Q4_0) from its window.
+// Expanded scale of the 32-element half `h` of k-block `it` from its window:
+// the half starts at element 64 * (it mod span) + 32 * h of the window's K range,
+// which is group (that >> log2(group_size)) of the window.
 template <int MODE>
-BQ_DEVINL DeqScale window_scale(const ScaleWindow<MODE>& w, int it, int h)
+BQ_DEVINL DeqScale window_scale(const ScaleWindow<MODE>& w, int it, int h, int gs_shift)
 {
+    const int span_mask = (1 << (gs_shift - 3)) - 1;
+    const int k = (((it & span_mask) << 6) + 32 * h) >> gs_shift;
     DeqScale r;
     if constexpr (MODE == kModeQ4_0) {
-        const float d = f16_bits_to_f32(halfword(w.s, 2 * (it % 4) + h));
+        const float d = f16_bits_to_f32(halfword(w.s, k));
         r.a = pack_bf16x2_rn(d, d);                                            // d_hi
         const float lo = __fsub_rn(d, __uint_as_float(r.a << 16));           // d - d_hi, exact
         r.b = pack_bf16x2_rn(lo, lo);
     } else {
-        r.a = halfword(w.s, it % 8);
-        r.b = halfword(w.b, it % 8);
+        r.a = halfword(w.s, k);
+        r.b = halfword(w.b, k);
     }
     return r;
 }
@@ -402,13 +406,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         constexpr int kHalves = 8 / C::kDeqWarpsPerGroup;   // 32-element halves of a k-block per thread
         const int h0 = (C::kDeqWarpsPerGroup == 8) ? ((warp >> 2) & 1) : 0;
         const int grp = warp / C::kDeqWarpsPerGroup;   // takes k-blocks kb with kb % groups == grp
-        constexpr int kSpan = ScaleWindow<MODE>::kSpan;
+        const int span_shift = p.gs_shift - 3;   // log2(k-blocks per scale window)
         // The scale windows this CTA needs, in order: for each of its units, the
         // windows over the unit's k-blocks.  The next one is always in flight, so a
         // window is fetched a whole window ahead, also across unit boundaries.
         struct WinPos { int u, w, w_last; };      // unit, window, the unit's last window
         auto first_pos = [&](int u) {
-            return u < units ? WinPos{u, kb_begin(u) / kSpan, (kb_end(u) - 1) / kSpan} : WinPos{units, 0, 0};
+            return u < units ? WinPos{u, kb_begin(u) >> span_shift, (kb_end(u) - 1) >> span_shift}
+                             : WinPos{units, 0, 0};
         };
         auto next_pos = [&](WinPos q) {
             if (q.u < units && q.w < q.w_last) return WinPos{q.u, q.w + 1, q.w_last};
@@ -427,7 +432,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             const int kb1 = kb_end(u);
             for (int it = kb_begin(u); it < kb1; ++it, ++kb) {
-                if (pos_cur.u != u || pos_cur.w != it / kSpan) {   // advance one window, fetch the one after
+                if (pos_cur.u != u || pos_cur.w != (it >> span_shift)) {   // advance one window, fetch the next
                     win_cur = win_nxt;
                     pos_cur = pos_nxt;
                     pos_nxt = next_pos(pos_nxt);
@@ -442,7 +447,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                 for (int hh = 0; hh < kHalves; ++hh) {
                     const int h = h0 + hh;
-                    const DeqScale sc = window_scale<MODE>(win_cur, it, h);
+                    const DeqScale sc = window_scale<MODE>(win_cur, it, h, p.gs_shift);
                     uint32_t wv[16];
                     if constexpr (MODE == kModeQ4_0) {
                         deq_q4_0_half(ld_shared_v4(codes + 16u * h), sc.a, sc.b, wv);

@@ -18,8 +18,9 @@
  *  - MLX-style affine, the format of mx.quantize / mx.dequantize /
  *    mx.quantized_matmul on "quantized_matmul takes 14-41% longer than
  *    dequantize + bf16 matmul at prefill sizes (> 512 tokens)" (Repro).
- *    Groups of group_size (= 64) weights along K share a bf16 scale and a bf16
- *    bias; w = scale * q + bias, q in [0, 2^bits - 1], bits in {4, 8}.
+ *    Groups of group_size weights along K share a bf16 scale and a bf16 bias;
+ *    w = scale * q + bias, q in [0, 2^bits - 1], bits in {4, 8}, group_size in
+ *    {32, 64, 128} (the sizes mx.quantize accepts; the workloads use 64).
  *      wq      u32  [N][K*bits/32]  element k at bits bits*(k % (32/bits)) of
  *                                   word k / (32/bits) (lowest bits first)
  *      scales  bf16 [N][K/group_size]
@@ -101,7 +102,7 @@ BQ_API bq_status q4_0_dequantize(const uint8_t* wq, const uint16_t* scales_f16, 
  *   scales_bf16 device u16 [N][K/group_size]
  *   biases_bf16 device u16 [N][K/group_size]
  *   out_bf16    device u16 [N][K], written
- *   group_size  64;  bits  4 or 8;  K % group_size == 0
+ *   group_size  32, 64 or 128;  bits  4 or 8;  K % group_size == 0
  */
 BQ_API bq_status affine_dequantize(const uint32_t* wq, const uint16_t* scales_bf16, const uint16_t* biases_bf16,
                             uint16_t* out_bf16, int64_t N, int64_t K, int group_size, int bits,

@@ -68,7 +68,7 @@ def test_quant_matmul_rejects_before_launch(L):
     assert qmm(L, K=48) == 2                                  # Q4_0 needs K % 32 == 0
     assert qmm(L, bits=8) == 3                                # Q4_0 is 4-bit only
     assert qmm(L, g=64) == 3                                  # ... with group 32
-    assert qmm(L, b=ALIGNED, g=32, bits=4) == 3               # affine needs group 64
+    assert qmm(L, b=ALIGNED, g=16, bits=4) == 3               # affine groups: 32, 64 or 128
     assert qmm(L, b=ALIGNED, g=64, bits=3) == 3               # bits in {4, 8}
     assert qmm(L, b=ALIGNED, g=64, bits=4, K=96) == 2         # K % group
     assert qmm(L, x=None) == 1
@@ -94,7 +94,7 @@ def test_other_entry_points_reject_before_launch(L):
     assert L.bf16_matmul(ALIGNED, ALIGNED, ALIGNED, 4, 4, 12, None) == 2
     assert L.bf16_matmul(None, ALIGNED, ALIGNED, 4, 4, 16, None) == 1
     assert L.q4_0_quantize(ALIGNED, ALIGNED, MISALIGNED, 4, 64, None) == 4
-    assert L.affine_quantize(ALIGNED, ALIGNED, ALIGNED, ALIGNED, 4, 64, 32, 4, None) == 3
+    assert L.affine_quantize(ALIGNED, ALIGNED, ALIGNED, ALIGNED, 4, 64, 16, 4, None) == 3
 
 
 BOUNDARY_M = [1, 2, 8, 19, 31, 32, 33, 63, 64, 65, 127, 128, 129, 511, 512, 513, 1023, 1024, 1025, 8192]

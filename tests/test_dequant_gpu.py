@@ -132,3 +132,28 @@ def test_q4_0_import_aos_then_matmul():
     y_ref, a_ref, _ = oracle.matmul_ref(x.view(torch.int16).numpy().view(np.uint16), oracle.q4_0_dequantize(wq, d))
     tol = oracle.tolerance(a_ref, y_ref)
     assert np.all(np.abs(y.float().cpu().numpy().astype(np.float64) - y_ref) <= tol)
+
+
+GROUP_FORMATS = ["affine4_g32", "affine4_g128", "affine8_g32", "affine8_g128"]
+
+
+@pytest.mark.parametrize("fmt", GROUP_FORMATS)
+@pytest.mark.parametrize("N,K", [(3, 128), (250, 512), (64, 4096)])
+def test_dequant_bit_exact_group_sizes(fmt, N, K):
+    p = Problem(fmt, N, K, seed=N + K + 3)
+    assert np.array_equal(_gpu_dequant(p), p.wb)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("G", [32, 128])
+def test_affine_quantize_bit_exact_group_sizes(bits, G):
+    N, K = 250, 1024
+    g = inputs.generator(N + bits + G)
+    w = inputs.weights_bf16_valued(N, K, g)
+    w[0, :G] = -0.375                    # constant group: scale 0
+    wq_ref, s_ref, b_ref = oracle.affine_quantize(w.numpy(), G, bits)
+    wq, s, b = bq.affine_quantize(w.cuda(), G, bits)
+    torch.cuda.synchronize()
+    assert np.array_equal(wq.cpu().numpy().view(np.uint32), wq_ref)
+    assert np.array_equal(u16(s), s_ref)
+    assert np.array_equal(u16(b), b_ref)

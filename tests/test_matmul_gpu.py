@@ -220,3 +220,17 @@ def test_multi_matches_separate_calls(fmt, M):
         assert torch.equal(y.view(torch.int16), y1.view(torch.int16)), (fmt, M, p.N)
         y_ref, a_ref = reference(x, p.wb)
         assert_within_tolerance(y, y_ref, a_ref, f"multi {fmt} M={M} N={p.N}")
+
+
+@pytest.mark.parametrize("fmt", ["affine4_g32", "affine4_g128", "affine8_g32", "affine8_g128"])
+@pytest.mark.parametrize("N,K", [(300, 1024), (130, 4096)])
+def test_group_sizes_all_paths(fmt, N, K):
+    """Affine group sizes 32 and 128 (mx.quantize's other sizes) on every path,
+    including K-split fused tiles (few tiles) and windows of 4 or 16 k-blocks."""
+    p = Problem(fmt, N, K, seed=N * 3 + K)
+    for M in (1, 8, 32):
+        check(p, M, "gemv")
+    for M in (33, 100, 300):
+        check(p, M, "tc_fused")
+        check(p, M, "dequant_gemm")
+        check(p, M, "auto")
