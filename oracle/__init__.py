@@ -17,6 +17,11 @@ Parity status of each function (what pins it, see ``tests/test_oracle_pins.py``)
                                min -> 0 / max -> L, error bound
   affine_dequantize         -- closed form over every code value (4 and 8 bit),
                                exact round trip of quantize
+  q8_1_quantize             -- closed forms: power-of-two scales with exact codes,
+                               half-away-from-zero ties, all-zero block, |q| <= 127,
+                               qsum, reconstruction error <= d/2
+  q4_0_q8_matmul            -- unit scales give numpy's exact integer dot product;
+                               within the x-quantization error bound of matmul_ref
   matmul_ref                -- exact rational (fractions.Fraction) brute force
                                on tiny non-square shapes, one-hot identities
 """
@@ -50,6 +55,8 @@ def _load():
     lib.oracle_q4_0_quantize.argtypes = [P, I64, I64, P, P]
     lib.oracle_q4_0_dequantize.argtypes = [P, P, I64, I64, P]
     lib.oracle_q4_0_import_aos.argtypes = [P, I64, I64, P, P]
+    lib.oracle_q8_1_quantize.argtypes = [P, I64, I64, P, P, P]
+    lib.oracle_q4_0_q8_matmul.argtypes = [P, P, P, P, I64, I64, I64, P, P]
     lib.oracle_affine_quantize.argtypes = [P, I64, I64, I, I, P, P, P]
     lib.oracle_affine_dequantize.argtypes = [P, P, P, I64, I64, I, I, P]
     lib.oracle_matmul_ref.argtypes = [P, P, I64, I64, I64, P, I64, P, P, I]
@@ -132,6 +139,35 @@ def q4_0_import_aos(blocks) -> tuple[np.ndarray, np.ndarray]:
     d = np.empty((N, K // 32), np.uint16)
     _load().oracle_q4_0_import_aos(_ptr(blocks), N, K, _ptr(wq), _ptr(d))
     return wq, d
+
+
+# ------------------------------------------------------- quantized activations
+def q8_1_quantize(x_bf16_bits) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """bf16 bits u16 [M][K] -> (xq int8 [M][K], dx f32 [M][K/32], qsum int32 [M][K/32])."""
+    x = _c(x_bf16_bits, np.uint16)
+    M, K = x.shape
+    assert K % 32 == 0
+    xq = np.empty((M, K), np.int8)
+    dx = np.empty((M, K // 32), np.float32)
+    qs = np.empty((M, K // 32), np.int32)
+    _load().oracle_q8_1_quantize(_ptr(x), M, K, _ptr(xq), _ptr(dx), _ptr(qs))
+    return xq, dx, qs
+
+
+def q4_0_q8_matmul(xq, dx, wq, d) -> tuple[np.ndarray, np.ndarray]:
+    """Q4_0 weights times Q8_1-style activations, float64 from the integer codes:
+    -> (y f64 [M][N], a f64 [M][N] = sum of |block terms|)."""
+    xq = _c(xq, np.int8)
+    dx = _c(dx, np.float32)
+    wq = _c(wq, np.uint8)
+    d = _c(d, np.uint16)
+    M, K = xq.shape
+    N = wq.shape[0]
+    assert wq.shape == (N, K // 2) and d.shape == (N, K // 32) and dx.shape == (M, K // 32)
+    y = np.empty((M, N), np.float64)
+    a = np.empty((M, N), np.float64)
+    _load().oracle_q4_0_q8_matmul(_ptr(xq), _ptr(dx), _ptr(wq), _ptr(d), M, N, K, _ptr(y), _ptr(a))
+    return y, a
 
 
 # -------------------------------------------------------------------- affine

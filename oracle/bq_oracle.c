@@ -197,6 +197,66 @@ void oracle_q4_0_import_aos(const uint8_t* blocks, int64_t N, int64_t K, uint8_t
 }
 
 /* ------------------------------------------------------------------ */
+/* Quantized activations (Q8_1 style) for the Q4_0 decode path         */
+/* ------------------------------------------------------------------ */
+
+/* Per block of 32 consecutive elements of a token row: amax = max |x|,
+ * d = amax / 127 in fp32, id = d != 0 ? 1 / d : 0, q = roundf(x * id) (half away
+ * from zero, in [-127, 127]), qsum = the sum of the block's q. */
+void oracle_q8_1_quantize(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* dx, int32_t* qsum)
+{
+    const int64_t nb = K / 32;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const uint16_t* xb = x + m * K + b * 32;
+            float amax = 0.0f;
+            for (int j = 0; j < 32; ++j) {
+                float v = fabsf(oracle_bf16_to_f32(xb[j]));
+                if (v > amax) amax = v;
+            }
+            const float d = amax / 127.0f;
+            const float id = d != 0.0f ? 1.0f / d : 0.0f;
+            int32_t sum = 0;
+            for (int j = 0; j < 32; ++j) {
+                const int q = (int)roundf(oracle_bf16_to_f32(xb[j]) * id);
+                xq[m * K + b * 32 + j] = (int8_t)q;
+                sum += q;
+            }
+            dx[m * nb + b] = d;
+            qsum[m * nb + b] = sum;
+        }
+    }
+}
+
+/* y[m][n] = sum over blocks b of d_w[n][b] * dx[m][b] * sum_j xq[m][32b+j] * (q_w[n][32b+j] - 8),
+ * in float64 from the integer codes; a[m][n] = the same sum of absolute values of the
+ * block terms (for the tolerance). */
+void oracle_q4_0_q8_matmul(const int8_t* xq, const float* dx, const uint8_t* wq, const uint16_t* d16,
+                           int64_t M, int64_t N, int64_t K, double* y, double* a)
+{
+    const int64_t nb = K / 32;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, abs_acc = 0.0;
+            for (int64_t b = 0; b < nb; ++b) {
+                const uint8_t* in = wq + n * (K / 2) + b * 16;
+                const int8_t* xb = xq + m * K + b * 32;
+                int64_t dot = 0;
+                for (int j = 0; j < 16; ++j) {
+                    dot += (int64_t)xb[j] * ((in[j] & 0x0f) - 8);
+                    dot += (int64_t)xb[j + 16] * ((in[j] >> 4) - 8);
+                }
+                const double term = (double)oracle_f16_to_f32(d16[n * nb + b]) * (double)dx[m * nb + b] * (double)dot;
+                acc += term;
+                abs_acc += fabs(term);
+            }
+            y[m * N + n] = acc;
+            a[m * N + n] = abs_acc;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* Affine (MLX-style) b-bit, b in {4, 8}                               */
 /* ------------------------------------------------------------------ */
 

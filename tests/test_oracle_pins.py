@@ -427,3 +427,91 @@ def test_q4_0_import_aos_matches_hand_assembled_blocks():
     swapped[:, :, [0, 1]] = swapped[:, :, [1, 0]]
     _, bad_d = oracle.q4_0_import_aos(swapped.reshape(N, -1))
     assert not np.array_equal(bad_d, d)
+
+
+# --------------------------------------------------------------------------
+# Q8_1-style activations for the quantized-activation decode path
+# --------------------------------------------------------------------------
+def _bf16_bits_of(v: np.ndarray) -> np.ndarray:
+    return torch_bf16_bits(np.asarray(v, np.float32))
+
+
+def test_q8_1_quantize_closed_forms():
+    """Blocks of integer multiples of 2^e with one |value| = 127 * 2^e: d = 2^e exactly
+    and every code is the integer itself; ties at .5 round away from zero; an all-zero
+    block has d = 0 and zero codes."""
+    rng = np.random.default_rng(21)
+    e = np.array([-3, 0, -7], np.float64)
+    ints = rng.integers(-127, 128, (3, 32))
+    ints[:, 5] = 127
+    ints[1, 9] = -127
+    x = ints * np.exp2(e)[:, None]
+    half = np.zeros((1, 32))
+    half[0, 0] = 127.0
+    half[0, 1:5] = [2.5, -2.5, 0.5, -0.5]          # exactly halfway after scaling by 1/d = 1
+    zero = np.zeros((1, 32))
+    xb = _bf16_bits_of(np.concatenate([x, half, zero]).reshape(1, -1))
+    xq, dx, qs = oracle.q8_1_quantize(xb)
+    q = xq.reshape(5, 32)
+    assert np.array_equal(dx[0], np.array([2 ** -3, 1.0, 2 ** -7, 1.0, 0.0], np.float32))
+    assert np.array_equal(q[:3], ints)
+    assert list(q[3, 1:5]) == [3, -3, 1, -1]
+    assert np.all(q[4] == 0)
+    assert np.array_equal(qs[0], q.sum(axis=1))
+
+
+def test_q8_1_quantize_invariants_random():
+    g = inputs.generator(22)
+    M, K = 5, 1024
+    x = inputs.activations_bf16(M, K, g)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    xf = x.float().numpy().astype(np.float64)
+    xq, dx, qs = oracle.q8_1_quantize(xb)
+    assert np.abs(xq.astype(np.int32)).max() <= 127
+    amax = np.abs(xf.reshape(M, K // 32, 32)).max(axis=2)
+    assert np.array_equal(dx, (amax.astype(np.float32) / np.float32(127)))
+    assert np.array_equal(qs, xq.reshape(M, K // 32, 32).astype(np.int32).sum(axis=2))
+    err = np.abs(xf - xq.astype(np.float64) * np.repeat(dx.astype(np.float64), 32, axis=1))
+    # half a step, plus the fp32 rounding of 1/d and of x * (1/d) near ties
+    # (at most |x| * 2^-22 <= 127 d * 2^-22)
+    assert np.all(err <= np.repeat(dx.astype(np.float64), 32, axis=1) * (0.5 + 127 * 2.0 ** -22))
+
+
+def test_q4_0_q8_matmul_unit_scales_is_integer_dot_product():
+    """Activations that are integers with block maximum 127 (dx = 1) and weight
+    scales 1.0: the result is numpy's exact int64 dot product of x and (q - 8)."""
+    rng = np.random.default_rng(23)
+    M, N, K = 3, 5, 128
+    xi = rng.integers(-127, 128, (M, K))
+    xi[:, ::32] = 127
+    wq = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    d = np.full((N, K // 32), 0x3C00, np.uint16)                 # fp16 1.0
+    xq, dx, _ = oracle.q8_1_quantize(_bf16_bits_of(xi))
+    assert np.all(dx == 1.0) and np.array_equal(xq, xi)
+    blk = wq.reshape(N, K // 32, 16)
+    q = np.concatenate([blk & 0x0F, blk >> 4], axis=2).reshape(N, K).astype(np.int64)   # element j, then j + 16
+    expect = xi.astype(np.int64) @ (q - 8).T
+    y, a = oracle.q4_0_q8_matmul(xq, dx, wq, d)
+    assert np.array_equal(y, expect.astype(np.float64))
+
+
+def test_q4_0_q8_matmul_within_activation_quantization_bound():
+    """Against the plain bf16 matmul of the same weights: the difference is bounded by
+    the activation quantization error (<= dx / 2 per element) times |w|, plus the bf16
+    rounding of the weights (<= 2^-9 |w|) that the q8 path does not apply."""
+    g = inputs.generator(24)
+    M, N, K = 4, 40, 512
+    w = inputs.weights_fp32(N, K, g).numpy()
+    wq, d = oracle.q4_0_quantize(w)
+    x = inputs.activations_bf16(M, K, g)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    xq, dx, _ = oracle.q8_1_quantize(xb)
+    y, _ = oracle.q4_0_q8_matmul(xq, dx, wq, d)
+    wb = oracle.q4_0_dequantize(wq, d)
+    y_ref, a_ref, _ = oracle.matmul_ref(xb, wb)
+    wabs = np.abs(f32_from_bf16_bits(wb).astype(np.float64))
+    bound = (np.repeat(dx.astype(np.float64), 32, axis=1) / 2) @ wabs.T + 2.0 ** -9 * a_ref * 1.01 + 1e-12
+    assert np.all(np.abs(y - y_ref) <= bound)
+    # and the bound is not vacuous: a planted sign error on the weights breaks it
+    y_bad, _ = oracle.q4_0_q8_matmul(xq, dx, wq ^ 0x88, d)
+    assert not np.all(np.abs(y_bad - y_ref) <= bound)
