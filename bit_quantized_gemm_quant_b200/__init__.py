@@ -46,6 +46,8 @@ def lib() -> ctypes.CDLL:
     sigs = {
         "q4_0_dequantize": [P, P, P, I64, I64, P],
         "q4_0_import_aos": [P, P, P, I64, I64, P],
+        "q8_1_quantize": [P, P, P, P, I64, I64, P],
+        "quant_matmul_q8": [P, P, P, P, P, P, I64, I64, I64, P],
         "affine_dequantize": [P, P, P, P, I64, I64, I, I, P],
         "quant_matmul": [P, P, P, P, P, I64, I64, I64, I, I, I, P],
         "quant_matmul_ex": [P, P, P, P, P, I64, I64, I64, I, I, I, I, P, SZ, P],
@@ -197,6 +199,30 @@ def quant_matmul_multi(x: torch.Tensor, weights, group_size: int = 32, bits: int
     _check(lib().quant_matmul_multi(_ptr(x), count, wq_a, s_a, b_a, y_a, n_a, M, K, group_size, bits,
                                     1 if transpose else 0, _stream(stream)), "quant_matmul_multi")
     return outs
+
+
+def q8_1_quantize(x: torch.Tensor, stream=None):
+    """bf16 x [M][K] -> (xq int8 [M][K], dx f32 [M][K/32], qsum int32 [M][K/32])."""
+    M, K = x.shape
+    xq = torch.empty(M, K, dtype=torch.int8, device=x.device)
+    dx = torch.empty(M, K // 32, dtype=torch.float32, device=x.device)
+    qs = torch.empty(M, K // 32, dtype=torch.int32, device=x.device)
+    _check(lib().q8_1_quantize(_ptr(x), _ptr(xq), _ptr(dx), _ptr(qs), M, K, _stream(stream)), "q8_1_quantize")
+    return xq, dx, qs
+
+
+def quant_matmul_q8(xq: torch.Tensor, dx: torch.Tensor, qsum: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor,
+                    out: torch.Tensor | None = None, stream=None):
+    """Q4_0 weights times quantized activations -> bf16 y [M][N]."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    if wq.shape[1] * 2 != K:
+        raise ValueError("K mismatch between activations and weights")
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=xq.device)
+    _check(lib().quant_matmul_q8(_ptr(xq), _ptr(dx), _ptr(qsum), _ptr(wq), _ptr(_bits16(scales)), _ptr(out), M, N,
+                                 K, _stream(stream)), "quant_matmul_q8")
+    return out
 
 
 NOALLOC_SCRATCH_BYTES = 32 << 20

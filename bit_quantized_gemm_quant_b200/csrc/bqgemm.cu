@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "dequant.cuh"
 #include "gemv.cuh"
+#include "gemv_q8.cuh"
 #include "tc_gemm.cuh"
 
 namespace bq {
@@ -588,6 +589,65 @@ bq_status q4_0_import_aos(const uint8_t* blocks, uint8_t* wq, uint16_t* scales_f
     q4_0_import_aos_kernel<<<(unsigned)std::max<int64_t>(grid, 1), 32 * kImportWarps, 0, (cudaStream_t)stream>>>(
         blocks, wq, scales_f16, nb);
     return launch_status();
+}
+
+bq_status q8_1_quantize(const uint16_t* x_bf16, int8_t* xq, float* dx, int32_t* qsum, int64_t M, int64_t K,
+                        bq_stream_t stream)
+{
+    if (M < 0 || K < 0 || K % 32 != 0) return BQ_ERR_SHAPE;
+    const int64_t nb = M * (K / 32);
+    if (nb == 0) return BQ_OK;
+    if (!x_bf16 || !xq || !dx || !qsum) return BQ_ERR_NULL;
+    if (!aligned16(x_bf16) || !aligned16(xq) || !aligned16(dx) || !aligned16(qsum)) return BQ_ERR_ALIGN;
+    int dev;
+    DeviceInfo di;
+    bq_status s = current_device(&dev, &di);
+    if (s != BQ_OK) return s;
+    q8_1_quantize_kernel<<<grid_for(nb, 128, di), 128, 0, (cudaStream_t)stream>>>(x_bf16, xq, dx, qsum, nb);
+    return launch_status();
+}
+
+bq_status quant_matmul_q8(const int8_t* xq, const float* dx, const int32_t* qsum, const uint8_t* wq,
+                          const uint16_t* scales_f16, uint16_t* y_bf16, int64_t M, int64_t N, int64_t K,
+                          bq_stream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0 || K % 32 != 0) return BQ_ERR_SHAPE;
+    if (M == 0 || N == 0) return BQ_OK;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return BQ_ERR_SHAPE;
+    if (!y_bf16) return BQ_ERR_NULL;
+    if (!aligned16(y_bf16)) return BQ_ERR_ALIGN;
+    int dev;
+    DeviceInfo di;
+    bq_status s = current_device(&dev, &di);
+    if (s != BQ_OK) return s;
+    if (K == 0)
+        return cudaMemsetAsync(y_bf16, 0, (size_t)M * (size_t)N * 2u, (cudaStream_t)stream) == cudaSuccess
+                   ? BQ_OK : BQ_ERR_CUDA;
+    if (!xq || !dx || !qsum || !wq || !scales_f16) return BQ_ERR_NULL;
+    if (!aligned16(xq) || !aligned16(dx) || !aligned16(qsum) || !aligned16(wq) || !aligned16(scales_f16))
+        return BQ_ERR_ALIGN;
+    const int64_t nb = K / 32;
+    const unsigned grid = (unsigned)((N + 7) / 8);
+    // at most 8 tokens per launch; larger M runs as consecutive token groups
+    for (int64_t m0 = 0; m0 < M; m0 += 8) {
+        const int mt = (int)std::min<int64_t>(8, M - m0);
+        const int8_t* xq_m = xq + m0 * K;
+        const float* dx_m = dx + m0 * nb;
+        const int32_t* qs_m = qsum + m0 * nb;
+        uint16_t* y_m = y_bf16 + m0 * N;
+        const cudaStream_t st = (cudaStream_t)stream;
+        constexpr int KS = 4;                      // warps per CTA, splitting K
+        if (mt == 1)
+            gemv_q8_kernel<1, KS><<<grid, 32 * KS, 0, st>>>(xq_m, dx_m, qs_m, wq, scales_f16, y_m, mt, (int)N, (int)K);
+        else if (mt == 2)
+            gemv_q8_kernel<2, KS><<<grid, 32 * KS, 0, st>>>(xq_m, dx_m, qs_m, wq, scales_f16, y_m, mt, (int)N, (int)K);
+        else if (mt <= 4)
+            gemv_q8_kernel<4, KS><<<grid, 32 * KS, 0, st>>>(xq_m, dx_m, qs_m, wq, scales_f16, y_m, mt, (int)N, (int)K);
+        else
+            gemv_q8_kernel<8, KS><<<grid, 32 * KS, 0, st>>>(xq_m, dx_m, qs_m, wq, scales_f16, y_m, mt, (int)N, (int)K);
+        if ((s = launch_status()) != BQ_OK) return s;
+    }
+    return BQ_OK;
 }
 
 bq_status affine_dequantize(const uint32_t* wq, const uint16_t* scales_bf16, const uint16_t* biases_bf16,

@@ -125,6 +125,35 @@ BQ_API bq_status q4_0_import_aos(const uint8_t* blocks, uint8_t* wq, uint16_t* s
                                  bq_stream_t stream);
 
 /*
+ * q8_1_quantize -- activations to the int8 form of the quantized-activation
+ * decode path.  Reading of the SYCL page "2026-05-06 Q4 sync-after focused
+ * repro" (Important source touch points: its Q4_0 x Q8_1 matrix-vector kernels;
+ * the page does not print the Q8_1 format).  Per block of 32 consecutive
+ * elements of a token row: amax = max |x|, d = amax / 127 (fp32),
+ * id = d != 0 ? 1 / d : 0, q = roundf(x * id) (half away from zero, in
+ * [-127, 127]), qsum = the sum of the block's q.
+ *   x_bf16  device u16 [M][K];  xq device i8 [M][K];  dx device f32 [M][K/32];
+ *   qsum device i32 [M][K/32].  K % 32 == 0; pointers 16-byte aligned.
+ * Bit-exact with the plain definition (IEEE division and product, one rounding each).
+ */
+BQ_API bq_status q8_1_quantize(const uint16_t* x_bf16, int8_t* xq, float* dx, int32_t* qsum, int64_t M, int64_t K,
+                               bq_stream_t stream);
+
+/*
+ * quant_matmul_q8 -- Q4_0 weights times quantized activations (q8_1_quantize):
+ *   y[m][n] = bf16( sum_b d[n][b] * dx[m][b] * sum_j xq[m][32b+j] * (q[n][32b+j] - 8) ).
+ * The block dot products are exact integers; the per-block scaling and the sum
+ * over blocks are fp32.  An approximation of quant_matmul (by the activation
+ * quantization: at most dx / 2 per activation), offered as a separate path.
+ *   xq, dx, qsum  as written by q8_1_quantize for the same M, K
+ *   wq device u8 [N][K/2];  scales_f16 device u16 [N][K/32];  y_bf16 device u16 [M][N]
+ *   Any M (8 tokens per launch); errors as quant_matmul.
+ */
+BQ_API bq_status quant_matmul_q8(const int8_t* xq, const float* dx, const int32_t* qsum, const uint8_t* wq,
+                                 const uint16_t* scales_f16, uint16_t* y_bf16, int64_t M, int64_t N, int64_t K,
+                                 bq_stream_t stream);
+
+/*
  * quant_matmul -- y[M][N] = bf16_rne(sum_k x[m][k] * dequant(W)[n][k]), fp32
  * accumulation.  mx.quantized_matmul(x, wq, scales, biases, transpose=True,
  * group_size, bits) on the MLX issue page (Repro); its result equals

@@ -160,3 +160,13 @@ def test_quant_matmul_multi_validation(L):
     assert L.quant_matmul_multi(ALIGNED, 2, None, ptrs, None, ptrs, n, 4, 64, 32, 4, 1, None) == 1
     assert L.quant_matmul_multi(MISALIGNED, 2, ptrs, ptrs, None, ptrs, n, 4, 64, 32, 4, 1, None) == 4
     assert L.quant_matmul_multi(None, 0, None, None, None, None, None, 4, 64, 32, 4, 1, None) == 0     # nothing
+
+
+def test_q8_path_validation(L):
+    assert L.q8_1_quantize(ALIGNED, ALIGNED, ALIGNED, ALIGNED, 2, 48, None) == 2             # K % 32
+    assert L.q8_1_quantize(None, ALIGNED, ALIGNED, ALIGNED, 2, 64, None) == 1
+    assert L.q8_1_quantize(ALIGNED, MISALIGNED, ALIGNED, ALIGNED, 2, 64, None) == 4
+    assert L.q8_1_quantize(None, None, None, None, 0, 64, None) == 0
+    assert L.quant_matmul_q8(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 2, 8, 40, None) == 2
+    assert L.quant_matmul_q8(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 2, 8, 64, None) == 1
+    assert L.quant_matmul_q8(None, None, None, None, None, None, 2, 0, 64, None) == 0
