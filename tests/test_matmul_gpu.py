@@ -234,3 +234,12 @@ def test_group_sizes_all_paths(fmt, N, K):
         check(p, M, "tc_fused")
         check(p, M, "dequant_gemm")
         check(p, M, "auto")
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "affine4"])
+def test_odd_n_tensor_core_paths(fmt):
+    """N odd: the epilogue's paired row stores do not apply and single stores are used."""
+    p = Problem(fmt, 77, 512, seed=13)
+    for M in (40, 300):
+        check(p, M, "tc_fused")
+        check(p, M, "dequant_gemm")
