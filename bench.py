@@ -37,8 +37,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from one ncu capture of the
 # current build of each kernel (`ncu --set full`, decode bench command); None for a kernel
 # changed since its counters were taken.
-NCU_TRAFFIC = {"gemv_kernel<Q4_0, M=1>": 28340224, "gemv_kernel<Q4_0, M=8>": 28397824,
-               "gemv_kernel<Q4_0, M=32>": 28590592}
+NCU_TRAFFIC = {"gemv_kernel<Q4_0, M=1>": 28340224, "gemv_kernel<Q4_0, M=8>": 28397568,
+               "gemv_kernel<Q4_0, M=32>": 28598784, "gemv_q8_kernel<M=1>": 28324608}
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -264,7 +264,7 @@ def run_decode(args, world, device, peaks):
     # the quantized-activation path (opt-in, approximate): activation quantization
     # plus the Q4_0 x int8 GEMV, same weights, rotation and graph timing
     q8 = {}
-    for M in Ms:
+    for M in Ms[:1]:                                  # a one-token path
         fns = [(lambda wq=wq, s=s, M=M: bq.quant_matmul_q8(*bq.q8_1_quantize(xs[M]), wq, s, out=ys[M]))
                for (wq, s) in copies]
         t_all = kernel_seconds(fns, 4)
@@ -273,7 +273,8 @@ def run_decode(args, world, device, peaks):
         t_g = kernel_seconds(fns_g, 4)
         q8[str(M)] = {"us": round(t_all * 1e6, 3), "gbs": round(wbytes / t_all / 1e9, 1),
                       "gemv_us": round(t_g * 1e6, 3), "gemv_gbs": round(wbytes / t_g / 1e9, 1),
-                      "gemv_frac_hbm": round(wbytes / t_g / 1e9 / peaks["hbm_gbs"], 4)}
+                      "gemv_frac_hbm": round(wbytes / t_g / 1e9 / peaks["hbm_gbs"], 4),
+                      "gemv_traffic": NCU_TRAFFIC.get(f"gemv_q8_kernel<M={M}>")}
     dom = max(Ms, key=lambda M: per_m[str(M)]["us"])
     roof = {"bound": "hbm", "kernel": f"gemv_kernel<Q4_0, M={dom}>",
             "achieved": per_m[str(dom)]["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
