@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
         "q4_0_quantize": [P, P, P, I64, I64, P],
         "affine_quantize": [P, P, P, P, I64, I64, I, I, P],
         "bq_device_status": [],
+        "bq_selftest_wait_timeout": [ctypes.c_longlong, P],
         "bq_status_string": [I],
         "bq_version": [],
     }

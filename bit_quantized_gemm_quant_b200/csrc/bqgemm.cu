@@ -373,7 +373,7 @@ bq_status launch_gemv(const uint16_t* x, const void* wq, const uint16_t* s, cons
     // Launch shapes measured on B200 at N = 12288, K = 4096: 32 weight rows per CTA,
     // K split over 4 (8 at M > 16) warps, 2-deep load pipeline; MINB CTAs per SM
     // keep the whole grid resident in one wave.
-    if (M <= 8) return launch_gemv_cfg<F, 1, 2, 4, 2, 3>(x, wq, s, b, y, M, N, K, group_size, st);
+    if (M <= 8) return launch_gemv_cfg<F, 1, 2, 8, 1, 2>(x, wq, s, b, y, M, N, K, group_size, st);
     if (M <= 16) return launch_gemv_cfg<F, 2, 2, 4, 2, 2>(x, wq, s, b, y, M, N, K, group_size, st);
     return launch_gemv_cfg<F, 4, 2, 8, 1, 1>(x, wq, s, b, y, M, N, K, group_size, st);
 }
@@ -401,7 +401,7 @@ bq_status launch_gemv_multi(const uint16_t* x, GemvMultiTable& tab, int64_t M, i
                             cudaStream_t st)
 {
     if (K > INT32_MAX) return BQ_ERR_SHAPE;
-    if (M <= 8) return launch_gemv_multi_cfg<F, 1, 2, 4, 2, 3>(x, tab, M, K, group_size, st);
+    if (M <= 8) return launch_gemv_multi_cfg<F, 1, 2, 8, 1, 2>(x, tab, M, K, group_size, st);
     if (M <= 16) return launch_gemv_multi_cfg<F, 2, 2, 4, 2, 2>(x, tab, M, K, group_size, st);
     return launch_gemv_multi_cfg<F, 4, 2, 8, 1, 1>(x, tab, M, K, group_size, st);
 }
@@ -832,6 +832,36 @@ bq_status affine_quantize(const float* w, uint32_t* wq, uint16_t* scales_bf16, u
     else
         affine_quant_kernel<8><<<grid_for(ng, 256, di), 256, 0, (cudaStream_t)stream>>>(w, wq, scales_bf16,
                                                                                          biases_bf16, ng, group_size);
+    return launch_status();
+}
+
+// Self-test of the bounded waits: one thread waits on an mbarrier that nothing
+// arrives on, with the same try_wait and error recording as the kernels' waits,
+// and gives up after limit_cycles SM clocks.
+__global__ void selftest_wait_kernel(long long limit_cycles)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    fence_barrier_init();
+    const long long t0 = clock64();
+    while (!mbar_try_wait(b, 0)) {
+        if (clock64() - t0 > limit_cycles) {
+            raise_device_error(kErrWaitTimeout);
+            return;
+        }
+    }
+}
+
+bq_status bq_selftest_wait_timeout(long long limit_cycles, bq_stream_t stream)
+{
+    if (limit_cycles < 1000 || limit_cycles > 4000000000LL) return BQ_ERR_SHAPE;
+    int dev;
+    DeviceInfo di;
+    bq_status s = current_device(&dev, &di);
+    if (s != BQ_OK) return s;
+    selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(limit_cycles);
     return launch_status();
 }
 

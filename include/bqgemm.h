@@ -289,6 +289,17 @@ BQ_API bq_status affine_quantize(const float* w, uint32_t* wq, uint16_t* scales_
                           int64_t N, int64_t K, int group_size, int bits, bq_stream_t stream);
 
 /*
+ * bq_selftest_wait_timeout -- exercises the failure detection of the device-side
+ * bounded waits (no page has a counterpart; it tests this library's own
+ * mechanism).  Launches one thread that waits on an mbarrier nothing will ever
+ * complete, with the kernels' try_wait, and gives up after limit_cycles SM
+ * clocks (1000 .. 4e9), recording the timeout in the device error word exactly
+ * as a kernel's timed-out wait does.  bq_device_status() then returns
+ * BQ_ERR_TIMEOUT (and clears it); the context stays usable.  No fault, no trap.
+ */
+BQ_API bq_status bq_selftest_wait_timeout(long long limit_cycles, bq_stream_t stream);
+
+/*
  * bq_device_status -- waits for the current device to finish its work, then
  * reads and clears the library's device error word: BQ_OK, or BQ_ERR_TIMEOUT
  * when a kernel's bounded wait on a shared-memory barrier ran out (the kernel
