@@ -293,9 +293,10 @@ def run_decode(args, world, device, peaks):
         e2e_steps = max(3, min(args.steps, 20))
 
         def e2e_step():
+            # the step's inputs: the weight matrix (once) and each M's activations
+            d_wq.copy_(h_wq, non_blocking=True)
+            d_s.copy_(h_s, non_blocking=True)
             for M in Ms:
-                d_wq.copy_(h_wq, non_blocking=True)
-                d_s.copy_(h_s, non_blocking=True)
                 d_x[M].copy_(h_x[M], non_blocking=True)
                 bq.quant_matmul(d_x[M], d_wq, d_s, None, gs, bits, out=ys[M])
                 h_y[M].copy_(ys[M], non_blocking=True)
@@ -309,7 +310,7 @@ def run_decode(args, world, device, peaks):
         t1.record()
         torch.cuda.synchronize()
         es = max_over_ranks(t0.elapsed_time(t1) / 1000.0, world, device)
-        h2d = sum(h_wq.numel() * h_wq.element_size() + h_s.numel() * 2 + h_x[M].numel() * 2 for M in Ms)
+        h2d = h_wq.numel() * h_wq.element_size() + h_s.numel() * 2 + sum(h_x[M].numel() * 2 for M in Ms)
         d2h = sum(M * N * 2 for M in Ms)
         e2e = {"value": round(aggregate(e2e_steps * len(Ms) * wbytes, world, es) / 1e9, 3), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": e2e_steps}

@@ -102,14 +102,15 @@ int grid_for(int64_t items, int threads, const DeviceInfo& di)
 }
 
 // ------------------------------------------------------------------ env config
-// Default fused/pair threshold, from B200 sweeps of the 12288 x 4096 projection
-// (affine 4/8-bit and Q4_0): the fused kernel is faster up to 768 tokens, the
-// unfused pair from about 1024 tokens (equal for affine4 there, 5% ahead for Q4_0).
-constexpr int64_t kDefaultPairMinM = 1024;
+// Default fused/pair thresholds per format, from B200 sweeps of the 12288 x 4096
+// projection at M = 512 .. 8192: the fused kernel leads up to 1024 tokens for
+// Q4_0 and affine 4-bit (the pair from 2048); for affine 8-bit the pair leads at
+// 512 and from 1024, the fused kernel only at 768, so the pair is taken from 512.
+constexpr int64_t kDefaultPairMinM[3] = {2048, 2048, 512};   // Q4_0, affine4, affine8
 
 struct DispatchCfg {
     int tc_min_m = kGemvMaxM + 1;
-    int64_t pair_min_m = kDefaultPairMinM;   // 0: never
+    int64_t pair_min_m[3] = {kDefaultPairMinM[0], kDefaultPairMinM[1], kDefaultPairMinM[2]};   // 0: never
 };
 
 const DispatchCfg& dispatch_cfg()
@@ -122,18 +123,19 @@ const DispatchCfg& dispatch_cfg()
         }
         if (const char* v = std::getenv("BQ_PAIR_MIN_M")) {
             long long t = std::strtoll(v, nullptr, 10);
-            c.pair_min_m = t > 0 ? t : 0;
+            for (int f = 0; f < 3; ++f) c.pair_min_m[f] = t > 0 ? t : 0;
         }
         return c;
     }();
     return cfg;
 }
 
-int select_path(int64_t M, int64_t K, WFmt)
+int select_path(int64_t M, int64_t K, WFmt fmt)
 {
     const DispatchCfg& c = dispatch_cfg();
     if (M < c.tc_min_m) return BQ_PATH_GEMV;
-    if (c.pair_min_m > 0 && M >= c.pair_min_m) return BQ_PATH_DEQUANT_GEMM;
+    const int64_t pair_min = c.pair_min_m[(int)fmt];
+    if (pair_min > 0 && M >= pair_min) return BQ_PATH_DEQUANT_GEMM;
     return (K % 64 == 0) ? BQ_PATH_TC_FUSED : BQ_PATH_DEQUANT_GEMM;
 }
 

@@ -249,13 +249,14 @@ BQ_API size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int g
  * "et-backend: Q4_0 matrix-engine GEMM rewrite for prefill" (Overview: decode
  * routes to the vector-dot kernel).  Returns a bq_path other than AUTO:
  *   M <  tc_min_m                 -> BQ_PATH_GEMV        (tc_min_m default 33)
- *   M >= pair_min_m               -> BQ_PATH_DEQUANT_GEMM (pair_min_m default 1024,
- *                                    the measured fused/unfused crossover on B200)
+ *   M >= pair_min_m               -> BQ_PATH_DEQUANT_GEMM (pair_min_m by format, from
+ *                                    the measured fused/unfused crossovers on B200:
+ *                                    2048 for Q4_0 and affine 4-bit, 512 for 8-bit)
  *   otherwise                     -> BQ_PATH_TC_FUSED when K % 64 == 0,
  *                                    else BQ_PATH_DEQUANT_GEMM
  * Environment overrides, read once per process: BQ_TC_MIN_M (clamped to
- * [1, 33]; the GEMV handles at most 32 tokens) and BQ_PAIR_MIN_M (0: never;
- * unset: 1024).  Returns -1 for arguments quant_matmul would reject.
+ * [1, 33]; the GEMV handles at most 32 tokens) and BQ_PAIR_MIN_M (all
+ * formats; 0: never).  Returns -1 for arguments quant_matmul would reject.
  */
 BQ_API int quant_matmul_select_path(int64_t M, int64_t N, int64_t K, int group_size, int bits);
 
