@@ -243,3 +243,23 @@ def test_odd_n_tensor_core_paths(fmt):
     for M in (40, 300):
         check(p, M, "tc_fused")
         check(p, M, "dequant_gemm")
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "affine8"])
+def test_split_k_with_caller_workspace(fmt):
+    """Few tiles (N = 300, M = 48): the fused kernel splits K.  With a caller
+    workspace of the reported size it splits, with one too small it runs unsplit;
+    with none it uses the library's.  All three agree with the oracle."""
+    p = Problem(fmt, 300, 2048, seed=17)
+    wq, s, b = p.device()
+    M = 48
+    x = p.x(M)
+    need = bq.quant_matmul_workspace_size(M, 300, 2048, p.group_size, p.bits, "tc_fused")
+    assert need > 0, "this shape is expected to split K"
+    y_ref, a_ref = reference(x, p.wb)
+    xd = x.cuda()
+    for ws in (torch.empty(need, dtype=torch.uint8, device="cuda"),
+               torch.empty(64, dtype=torch.uint8, device="cuda"), None):
+        y = bq.quant_matmul_ex(xd, wq, s, b, p.group_size, p.bits, True, "tc_fused", workspace=ws)
+        torch.cuda.synchronize()
+        assert_within_tolerance(y, y_ref, a_ref, f"{fmt} ws={None if ws is None else ws.numel()}")
