@@ -263,3 +263,28 @@ def test_split_k_with_caller_workspace(fmt):
         y = bq.quant_matmul_ex(xd, wq, s, b, p.group_size, p.bits, True, "tc_fused", workspace=ws)
         torch.cuda.synchronize()
         assert_within_tolerance(y, y_ref, a_ref, f"{fmt} ws={None if ws is None else ws.numel()}")
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "affine4", "affine8"])
+def test_minimal_shapes_every_path(fmt):
+    """One weight row, the smallest K of the format, and M at the path limits."""
+    gs = 32 if fmt == "q4_0" else 64
+    for N, K in ((1, max(gs, 64)), (1, 128), (17, 64 if fmt == "q4_0" else 128)):
+        p = Problem(fmt, N, K, seed=N + K)
+        for M in (1, 32):
+            check(p, M, "gemv")
+        for M in (1, 33, 129):
+            check(p, M, "tc_fused")
+            check(p, M, "dequant_gemm")
+        check(p, 7, "auto")
+
+
+def test_q4_0_smallest_k_gemv_and_pair():
+    """K = 32 (one Q4_0 block): no 64-wide tensor-core k-block exists, so the
+    auto path takes the GEMV or the pair."""
+    p = Problem("q4_0", 40, 32, seed=2)
+    for M in (1, 5, 32):
+        check(p, M, "gemv")
+    for M in (33, 200):
+        check(p, M, "auto")
+        check(p, M, "dequant_gemm")
