@@ -203,49 +203,47 @@ struct TcPlan {
 
 int64_t splitk_stride(int64_t M, int64_t N) { return (M * N + 3) / 4 * 4; }   // floats per split, 16-byte multiple
 
-// K splits for the fused kernel when its tiles do not fill the SMs: minimise
-// rounds(units) x (k-blocks per split + c) + r, with c the per-unit fixed cost
-// (pipeline fill, epilogue) and r the reduction pass, both in k-block units.
-int choose_splits(int64_t tiles, int64_t nk, int num_sms)
-{
-    if (tiles >= num_sms) return 1;
-    constexpr int64_t kUnitCost = 4, kReduceCost = 4, kMinKBlocks = 4;
-    auto cost = [&](int64_t sp) {
-        const int64_t rounds = (tiles * sp + num_sms - 1) / num_sms;
-        return rounds * ((nk + sp - 1) / sp + kUnitCost) + (sp > 1 ? kReduceCost : 0);
-    };
-    int best = 1;
-    int64_t best_cost = cost(1);
-    for (int sp = 2; sp <= 8 && nk / sp >= kMinKBlocks; ++sp) {
-        const int64_t c = cost(sp);
-        if (c < best_cost) {
-            best_cost = c;
-            best = sp;
-        }
-    }
-    return best;
-}
-
 template <int MODE>
 bool plan_tc(int64_t M, int64_t N, int64_t K, int num_sms, int smem_optin, TcPlan* pl)
 {
     constexpr bool kFused = MODE != kModeBF16;
-    // TMEM (512 columns): two accumulators acc_stride columns apart and, in fused
-    // modes, one 32-column dequantized weight tile per pipeline stage.  A fused
-    // tile wider than 192 tokens leaves room for one accumulator only; it is taken
-    // when it needs fewer rounds of tiles over the SMs than the best tile <= 192.
-    int bn = kFused ? choose_bn(M, N, num_sms, 192, 64) : choose_bn(M, N, num_sms, 256, 32);
-    int num_acc = 2;
     const int64_t wtiles = (N + 127) / 128;
-    if (kFused && M > 192) {
-        auto rounds = [&](int b) {
-            const int64_t t = ((M + b - 1) / b) * wtiles;
-            return (t + num_sms - 1) / num_sms;
-        };
-        const int wide = (int)std::min<int64_t>(256, (M + 15) / 16 * 16);
-        if (wide > 192 && rounds(wide) < rounds(bn)) {
-            bn = wide;
-            num_acc = 1;
+    const int64_t nk = (K + 63) / 64;
+    int bn, num_acc = 2, splits = 1;
+    if (!kFused) {
+        bn = choose_bn(M, N, num_sms, 256, 32);
+    } else {
+        // The fused kernel's cost per k-block of a unit is nearly independent of
+        // the token tile width (the dequantization of the weight tile and the
+        // hand-offs dominate, about 0.55 us on B200), so wide tiles are preferred
+        // and the SMs are filled by splitting K.  Joint search over the tile width
+        // (two TMEM accumulators up to 192 tokens, one at 256, whose epilogue does
+        // not overlap the next tile: weight 1.12) and the split count, in k-block
+        // units:
+        //   cost = rounds(units) x (k-blocks per unit + 4) x w
+        //        + [split] (4 + fp32 partial traffic 8 x splits x M x N bytes at HBM speed)
+        // Ties go to the wider tile.
+        double best = 1e300;
+        bn = 16;
+        const int64_t maxb = std::min<int64_t>(256, (M + 15) / 16 * 16);
+        for (int b = 16; b <= maxb; b += 16) {
+            if (b > 192 && b < maxb && b != 256) continue;      // one accumulator: only the widest tile
+            const int acc = b > 192 ? 1 : 2;
+            const double w = acc == 1 ? 1.12 : 1.0;
+            const int64_t tiles = ((M + b - 1) / b) * wtiles;
+            for (int sp = 1; sp <= 8; ++sp) {
+                if (sp > 1 && nk / sp < 4) break;
+                const int64_t units = tiles * sp;
+                const int64_t rounds = (units + num_sms - 1) / num_sms;
+                const double reduce = sp > 1 ? 4.0 + (double)sp * (double)M * (double)N * 2.24e-6 : 0.0;
+                const double c = (double)rounds * (double)((nk + sp - 1) / sp + 4) * w + reduce;
+                if (c < best - 1e-9 || (c < best + 1e-9 && b > bn)) {
+                    best = c;
+                    bn = b;
+                    num_acc = acc;
+                    splits = sp;
+                }
+            }
         }
     }
     const int acc_stride = kFused ? (bn + 31) / 32 * 32 : 256;
@@ -259,8 +257,8 @@ bool plan_tc(int64_t M, int64_t N, int64_t K, int num_sms, int smem_optin, TcPla
     pl->acc_stride = acc_stride;
     pl->stages = stages;
     pl->tiles = ((M + bn - 1) / bn) * wtiles;
-    pl->splits = kFused ? choose_splits(pl->tiles, (K + 63) / 64, num_sms) : 1;
-    pl->ws_bytes = pl->splits > 1 ? (size_t)pl->splits * (size_t)splitk_stride(M, N) * 4u : 0u;
+    pl->splits = splits;
+    pl->ws_bytes = splits > 1 ? (size_t)splits * (size_t)splitk_stride(M, N) * 4u : 0u;
     return true;
 }
 
