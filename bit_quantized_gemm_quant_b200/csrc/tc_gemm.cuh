@@ -65,8 +65,8 @@ struct TcParams {
     int tiles;                // total tiles
     int acc_stride;           // TMEM columns between the two accumulators
     int num_acc;              // 2: the epilogue drains one tile while the next accumulates; 1: bn up to 256
-    int vec_scales;           // scale rows are 16-byte aligned and hold whole 8-scale windows
     int gs_shift;             // log2 of the group size (Q4_0: 5; affine: 5, 6 or 7)
+    int vec_scales;           // scale rows are 16-byte aligned and hold whole 8-group windows
     int splits;               // K splits per tile (fused modes); > 1: fp32 partials to ws
     float* ws;                // [splits][M][N] fp32 partial sums when splits > 1
     int64_t ws_stride;        // floats between consecutive splits' partials
@@ -146,10 +146,9 @@ BQ_DEVINL void deq_aff8_half(uint4 raw0, uint4 raw1, float s, float b, uint32_t 
 
 struct DeqScale { uint32_t a, b; };
 
-// Scales of one dequant thread's row, fetched a whole window of k-blocks ahead:
-// one 16-byte vector holds 8 consecutive 16-bit scales, i.e. group_size / 8
-// k-blocks (4 for Q4_0 and affine group 32, 8 for group 64, 16 for group 128).
-template <int MODE>
+// Eight consecutive groups' scales (and biases) of one weight row: one 16-byte
+// vector each.  A window spans group_size / 8 k-blocks (4 for group 32, 8 for 64,
+// 16 for 128).
 struct ScaleWindow {
     uint4 s, b;
 };
@@ -160,27 +159,29 @@ BQ_DEVINL uint32_t halfword(const uint4& v, int k)
     return (w >> (16 * (k & 1))) & 0xFFFFu;
 }
 
+// Window `win` (groups 8 win .. 8 win + 7) of weight row `row`; zeros past the
+// row's end and for rows past N.  With vec_scales every row is 16-byte aligned
+// and holds whole windows, so one vector load per array suffices.
 template <int MODE>
-BQ_DEVINL ScaleWindow<MODE> load_scale_window(const TcParams& p, int row, int win)
+BQ_DEVINL ScaleWindow load_scale_window(const TcParams& p, int row, int win)
 {
-    ScaleWindow<MODE> w;
+    ScaleWindow w;
     w.s = w.b = make_uint4(0, 0, 0, 0);
-    if (row >= p.N) return w;
-    const int per_row = p.K >> p.gs_shift;                                    // 16-bit scales per row
+    const int per_row = p.K >> p.gs_shift;
     const int first = win * 8;
-    const uint16_t* srow = p.scales + (int64_t)row * per_row;
-    const uint16_t* brow = p.biases + (int64_t)row * per_row;
-    if (first >= per_row) return w;                                           // window past the row end
-    if (p.vec_scales) {                                                       // 16-byte aligned rows, whole windows
-        w.s = __ldg(reinterpret_cast<const uint4*>(srow + first));
-        if constexpr (MODE != kModeQ4_0) w.b = __ldg(reinterpret_cast<const uint4*>(brow + first));
+    if (row >= p.N || first >= per_row) return w;
+    const uint16_t* srow = p.scales + (int64_t)row * per_row + first;
+    const uint16_t* brow = p.biases + (int64_t)row * per_row + first;
+    if (p.vec_scales) {
+        w.s = __ldg(reinterpret_cast<const uint4*>(srow));
+        if constexpr (MODE != kModeQ4_0) w.b = __ldg(reinterpret_cast<const uint4*>(brow));
     } else {
         uint32_t sv[8], bv[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const bool in = first + k < per_row;
-            sv[k] = in ? __ldg(srow + first + k) : 0u;
-            bv[k] = (MODE != kModeQ4_0 && in) ? __ldg(brow + first + k) : 0u;
+            sv[k] = in ? __ldg(srow + k) : 0u;
+            bv[k] = (MODE != kModeQ4_0 && in) ? __ldg(brow + k) : 0u;
         }
         w.s = make_uint4(sv[0] | sv[1] << 16, sv[2] | sv[3] << 16, sv[4] | sv[5] << 16, sv[6] | sv[7] << 16);
         w.b = make_uint4(bv[0] | bv[1] << 16, bv[2] | bv[3] << 16, bv[4] | bv[5] << 16, bv[6] | bv[7] << 16);
@@ -188,14 +189,13 @@ BQ_DEVINL ScaleWindow<MODE> load_scale_window(const TcParams& p, int row, int wi
     return w;
 }
 
-// Expanded scale of the 32-element half `h` of k-block `it` from its window:
-// the half starts at element 64 * (it mod span) + 32 * h of the window's K range,
-// which is group (that >> log2(group_size)) of the window.
+// The packed bf16x2 operands of one 32-element half's dequantization from group
+// k of a window.  Q4_0: d splits exactly into d_hi = bf16(d) and d_lo = d - d_hi
+// (both representable in bf16), so that fma(q - 8, d_hi, (q - 8) * d_lo) rounds
+// once to bf16((q - 8) * d).  Affine: the bf16 scale and bias bits.
 template <int MODE>
-BQ_DEVINL DeqScale window_scale(const ScaleWindow<MODE>& w, int it, int h, int gs_shift)
+BQ_DEVINL DeqScale window_scale(const ScaleWindow& w, int k)
 {
-    const int span_mask = (1 << (gs_shift - 3)) - 1;
-    const int k = (((it & span_mask) << 6) + 32 * h) >> gs_shift;
     DeqScale r;
     if constexpr (MODE == kModeQ4_0) {
         const float d = f16_bits_to_f32(halfword(w.s, k));
@@ -311,8 +311,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         __syncwarp();
     } else if (warp == C::kMmaWarp) {
         // ---------------- MMA issuer ----------------
+        // One lane issues everything; its per-k-block path is kept short because
+        // it shares an issue slot scheduler with busy dequant warps.  Descriptor
+        // words, the A column and the barrier addresses of the current stage
+        // advance incrementally.  Fused modes wait only for the dequant group's
+        // barrier: the group arrives after it has itself waited for the stage's
+        // TMA, so the activation tile has landed too.
         if (lane == 0) {
             const uint32_t idesc = umma_idesc_bf16_f32(128, p.bn);
+            const uint64_t bd0 = umma_desc_k_sw128(b_base);
+            const uint32_t b_lo0 = (uint32_t)bd0, desc_hi = (uint32_t)(bd0 >> 32);
+            const uint32_t b_step = b_bytes >> 4;
+            const uint32_t a_lo0 = (uint32_t)umma_desc_k_sw128(a_base);          // kModeBF16
+            const uint32_t a_col0 = tmem_base + a_tmem_col(0);                    // fused modes
+            const uint32_t a_step = (MODE == kModeBF16) ? (C::kABytes >> 4) : 32u;
+            const uint32_t wait_off = 8u * (uint32_t)((MODE == kModeBF16) ? 0 : 2 * S);   // full / afull
+            const uint32_t empty_off = 8u * (uint32_t)S;
+            uint32_t b_lo = b_lo0, a_cur = (MODE == kModeBF16) ? a_lo0 : a_col0, bar_s = bar_base;
             int s = 0, lt = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -322,27 +337,27 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 if (!mbar_wait(tempty_bar(acc), acc_phase(lt) ^ 1u)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.acc_stride);
+                uint32_t accumulate = 0;
                 for (int it = kb0; it < kb1; ++it) {
-                    if (!mbar_wait(full_bar(s), ph)) { ok = false; break; }
-                    if constexpr (MODE != kModeBF16) {
-                        if (!mbar_wait(afull_bar(s), ph)) { ok = false; break; }
-                    }
+                    if (!mbar_wait(bar_s + wait_off, ph)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t b_addr = b_base + (uint32_t)s * b_bytes;
-                    if constexpr (MODE == kModeBF16) {
-                        const uint32_t a_addr = a_base + (uint32_t)s * C::kABytes;
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_f16_ss(d_tmem, umma_desc_k_sw128(a_addr + 32u * kk),
-                                        umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it != kb0 || kk != 0) ? 1u : 0u);
+                    if constexpr (MODE == kModeBF16)
+                        umma_kblock_ss(d_tmem, a_cur, b_lo, desc_hi, idesc, accumulate);
+                    else
+                        umma_kblock_ts(d_tmem, a_cur, b_lo, desc_hi, idesc, accumulate);
+                    accumulate = 1;
+                    umma_commit(bar_s + empty_off);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                        b_lo = b_lo0;
+                        a_cur = (MODE == kModeBF16) ? a_lo0 : a_col0;
+                        bar_s = bar_base;
                     } else {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)   // K = 16 per MMA = 8 TMEM columns of A
-                            umma_f16_ts(d_tmem, tmem_base + a_tmem_col(s) + 8u * kk,
-                                        umma_desc_k_sw128(b_addr + 32u * kk), idesc, (it != kb0 || kk != 0) ? 1u : 0u);
+                        b_lo += b_step;
+                        a_cur += a_step;
+                        bar_s += 8u;
                     }
-                    umma_commit(empty_bar(s));
-                    if (++s == S) { s = 0; ph ^= 1u; }
                 }
                 umma_commit(tfull_bar(acc));
             }
@@ -402,72 +417,78 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         }
     } else if (MODE != kModeBF16 && warp < C::kDeqWarps) {
         // ---------------- dequantization ----------------
-        const int r = 32 * (warp & 3) + lane;   // weight row within the tile = TMEM lane
+        // Group grp takes the k-blocks whose position in this CTA's sequence (all
+        // k-blocks of all its units, in order) is grp modulo the number of
+        // groups; a warp walks only those, with a cursor over (unit, k-block).
+        // Scales come in 8-group windows (one 16-byte load per array); the window
+        // the group needs next is always in flight.
+        constexpr int G = C::kDeqGroups;
         constexpr int kHalves = 8 / C::kDeqWarpsPerGroup;   // 32-element halves of a k-block per thread
+        const int r = 32 * (warp & 3) + lane;                // weight row within the tile = TMEM lane
         const int h0 = (C::kDeqWarpsPerGroup == 8) ? ((warp >> 2) & 1) : 0;
-        const int grp = warp / C::kDeqWarpsPerGroup;   // takes k-blocks kb with kb % groups == grp
-        const int span_shift = p.gs_shift - 3;   // log2(k-blocks per scale window)
-        // The scale windows this CTA needs, in order: for each of its units, the
-        // windows over the unit's k-blocks.  The next one is always in flight, so a
-        // window is fetched a whole window ahead, also across unit boundaries.
-        struct WinPos { int u, w, w_last; };      // unit, window, the unit's last window
-        auto first_pos = [&](int u) {
-            return u < units ? WinPos{u, kb_begin(u) >> span_shift, (kb_end(u) - 1) >> span_shift}
-                             : WinPos{units, 0, 0};
+        const int grp = warp / C::kDeqWarpsPerGroup;
+        const int span_shift = p.gs_shift - 3;               // log2(k-blocks per window)
+        const uint32_t lane_base = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16);
+        struct Cur { int u, it, kb1, row; };                  // row: this thread's weight row in the unit's tile
+        auto cur_at = [&](int u) {
+            return u < units ? Cur{u, kb_begin(u), kb_end(u), tile_n0(unit_tile(u)) + r} : Cur{units, 0, 0, p.N};
         };
-        auto next_pos = [&](WinPos q) {
-            if (q.u < units && q.w < q.w_last) return WinPos{q.u, q.w + 1, q.w_last};
-            return first_pos(q.u < units ? q.u + (int)gridDim.x : units);
-        };
-        auto load_pos = [&](WinPos q) {
-            const int row = q.u < units ? tile_n0(unit_tile(q.u)) + r : p.N;   // past the end: nothing loaded
-            return load_scale_window<MODE>(p, row, q.w);
-        };
-        WinPos pos_cur = first_pos(blockIdx.x), pos_nxt = next_pos(pos_cur);
-        ScaleWindow<MODE> win_cur = load_pos(pos_cur);
-        ScaleWindow<MODE> win_nxt = load_pos(pos_nxt);
-        int s = 0, kb = 0;
-        uint32_t ph = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-            const int kb1 = kb_end(u);
-            for (int it = kb_begin(u); it < kb1; ++it, ++kb) {
-                if (pos_cur.u != u || pos_cur.w != (it >> span_shift)) {   // advance one window, fetch the next
-                    win_cur = win_nxt;
-                    pos_cur = pos_nxt;
-                    pos_nxt = next_pos(pos_nxt);
-                    win_nxt = load_pos(pos_nxt);
-                }
-                if (C::kDeqGroups > 1 && kb % C::kDeqGroups != grp) {   // another group's k-block
-                    if (++s == S) { s = 0; ph ^= 1u; }
-                    continue;
-                }
-                if (!mbar_wait_warp(full_bar(s), ph)) { ok = false; break; }
-                const uint32_t codes = c_base + (uint32_t)s * C::kCBytes + (uint32_t)(r * C::kCodeBytesPerRow);
-#pragma unroll
-                for (int hh = 0; hh < kHalves; ++hh) {
-                    const int h = h0 + hh;
-                    const DeqScale sc = window_scale<MODE>(win_cur, it, h, p.gs_shift);
-                    uint32_t wv[16];
-                    if constexpr (MODE == kModeQ4_0) {
-                        deq_q4_0_half(ld_shared_v4(codes + 16u * h), sc.a, sc.b, wv);
-                    } else if constexpr (MODE == kModeAff4) {
-                        deq_aff4_half(ld_shared_v4(codes + 16u * h), sc.a | (sc.a << 16), sc.b | (sc.b << 16), wv);
-                    } else {
-                        deq_aff8_half(ld_shared_v4(codes + 32u * h), ld_shared_v4(codes + 32u * h + 16u),
-                                      bf16_bits_to_f32(sc.a), bf16_bits_to_f32(sc.b), wv);
-                    }
-                    // These 32 weights = 16 TMEM columns of lane r in stage s.  The
-                    // stage's previous tile was consumed by the MMA S k-blocks back:
-                    // its smem stage was freed before this one was filled.
-                    tmem_st_32x32b_x16(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + a_tmem_col(s) + 16u * h, wv);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(afull_bar(s));
-                if (++s == S) { s = 0; ph ^= 1u; }
+        auto step = [&](Cur c, int n) {                      // n positions further along the sequence
+            c.it += n;
+            while (c.u < units && c.it >= c.kb1) {
+                const int carry = c.it - c.kb1;
+                c = cur_at(c.u + (int)gridDim.x);
+                c.it += carry;
             }
+            return c;
+        };
+        Cur cur = step(cur_at(blockIdx.x), grp);            // first own k-block: position grp
+        // Window in use (cu, cw) and the one in flight (nu, nw).
+        int cu = -1, cw = -1, nu = cur.u, nw = cur.it >> span_shift;
+        ScaleWindow win_cur, win_nxt = load_scale_window<MODE>(p, cur.row, nw);
+        win_cur = win_nxt;
+        int s = grp % S;
+        uint32_t ph = (uint32_t)(grp / S) & 1u;
+        bool ok = true;
+        while (ok && cur.u < units) {
+            const int w = cur.it >> span_shift;
+            if (cur.u != cu || w != cw) {                    // entering a new window
+                win_cur = (cur.u == nu && w == nw) ? win_nxt : load_scale_window<MODE>(p, cur.row, w);
+                cu = cur.u;
+                cw = w;
+                Cur c = step(cur, G);                        // the group's first k-block past this window
+                while (c.u == cu && (c.it >> span_shift) == cw) c = step(c, G);
+                nu = c.u;
+                nw = c.it >> span_shift;
+                win_nxt = load_scale_window<MODE>(p, c.row, nw);   // rows past N / units past the end: zeros
+            }
+            if (!mbar_wait_warp(full_bar(s), ph)) { ok = false; break; }
+            const uint32_t codes = c_base + (uint32_t)s * C::kCBytes + (uint32_t)(r * C::kCodeBytesPerRow);
+#pragma unroll
+            for (int hh = 0; hh < kHalves; ++hh) {
+                const int h = h0 + hh;
+                const DeqScale e = window_scale<MODE>(win_cur, ((cur.it * 64 + 32 * h) >> p.gs_shift) & 7);
+                uint32_t wv[16];
+                if constexpr (MODE == kModeQ4_0) {
+                    deq_q4_0_half(ld_shared_v4(codes + 16u * h), e.a, e.b, wv);
+                } else if constexpr (MODE == kModeAff4) {
+                    deq_aff4_half(ld_shared_v4(codes + 16u * h), e.a | (e.a << 16), e.b | (e.b << 16), wv);
+                } else {
+                    deq_aff8_half(ld_shared_v4(codes + 32u * h), ld_shared_v4(codes + 32u * h + 16u),
+                                  bf16_bits_to_f32(e.a), bf16_bits_to_f32(e.b), wv);
+                }
+                // These 32 weights = 16 TMEM columns of lane r in stage s.  The
+                // stage's previous tile was consumed by the MMA S k-blocks back:
+                // its smem stage was freed before this one was filled.
+                tmem_st_32x32b_x16(lane_base + a_tmem_col(s) + 16u * h, wv);
+            }
+            cur = step(cur, G);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(afull_bar(s));
+            s += G;
+            if (s >= S) { s -= S; ph ^= 1u; }
         }
     }
 

@@ -158,6 +158,45 @@ BQ_DEVINL void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, ui
         ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
+// One 64-element k-block: four K = 16 MMAs into d_tmem.  The B descriptor of
+// sub-step kk is the stage's descriptor with its start address advanced 32 bytes
+// (2 in the descriptor's 16-byte units; the 14-bit field never carries).  The
+// first MMA accumulates only when `accumulate` is nonzero; the other three always
+// do.  A from TMEM (a_tmem: stage column, +8 columns per sub-step) or from shared
+// memory (a_lo: the low word of its descriptor, same high word as B).
+BQ_DEVINL void umma_kblock_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t.reg .b32 l1, l2, l3, a1, a2, a3;\n\t.reg .b64 d0, d1, d2, d3;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\tsetp.eq.b32 q, %5, %5;\n\t"
+        "add.u32 l1, %2, 2;\n\tadd.u32 l2, %2, 4;\n\tadd.u32 l3, %2, 6;\n\t"
+        "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+        "mov.b64 d0, {%2, %3};\n\tmov.b64 d1, {l1, %3};\n\tmov.b64 d2, {l2, %3};\n\tmov.b64 d3, {l3, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], d0, %4, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], d1, %4, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], d2, %4, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], d3, %4, q;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+BQ_DEVINL void umma_kblock_ss(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc,
+                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t.reg .b32 l1, l2, l3, m1, m2, m3;\n\t.reg .b64 a0, a1, a2, a3, d0, d1, d2, d3;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\tsetp.eq.b32 q, %5, %5;\n\t"
+        "add.u32 l1, %2, 2;\n\tadd.u32 l2, %2, 4;\n\tadd.u32 l3, %2, 6;\n\t"
+        "add.u32 m1, %1, 2;\n\tadd.u32 m2, %1, 4;\n\tadd.u32 m3, %1, 6;\n\t"
+        "mov.b64 d0, {%2, %3};\n\tmov.b64 d1, {l1, %3};\n\tmov.b64 d2, {l2, %3};\n\tmov.b64 d3, {l3, %3};\n\t"
+        "mov.b64 a0, {%1, %3};\n\tmov.b64 a1, {m1, %3};\n\tmov.b64 a2, {m2, %3};\n\tmov.b64 a3, {m3, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a0, d0, %4, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, d1, %4, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a2, d2, %4, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a3, d3, %4, q;\n\t}"
+        ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate) : "memory");
+}
+
 // Arrive once on `bar` when all previously issued tcgen05 ops of this thread complete.
 BQ_DEVINL void umma_commit(uint32_t bar)
 {
