@@ -97,15 +97,15 @@ def test_other_entry_points_reject_before_launch(L):
     assert L.affine_quantize(ALIGNED, ALIGNED, ALIGNED, ALIGNED, 4, 64, 16, 4, None) == 3
 
 
-BOUNDARY_M = [1, 2, 8, 19, 31, 32, 33, 63, 64, 65, 127, 128, 129, 511, 512, 513, 1023, 1024, 1025, 2047, 2048,
-              8192]
+BOUNDARY_M = [1, 2, 8, 19, 31, 32, 33, 63, 64, 65, 127, 128, 129, 383, 384, 385, 511, 512, 513, 1023, 1024, 1025,
+              2047, 2048, 8192]
 
 
 def test_dispatcher_boundaries(L):
     for M in BOUNDARY_M:
         for g, bits in ((32, 4), (64, 4), (64, 8)):
             p = L.quant_matmul_select_path(M, 12288, 4096, g, bits)
-            pair_min = 512 if bits == 8 else 2048
+            pair_min = 384 if bits == 8 else 2048
             assert p == (1 if M <= 32 else 2 if M < pair_min else 3), (M, g, bits, p)
     # K % 64 != 0 (Q4_0 only): prefill goes through the unfused pair
     assert L.quant_matmul_select_path(512, 256, 544, 32, 4) == 3
