@@ -14,9 +14,10 @@ Parity status of each function (what pins it, see ``tests/test_oracle_pins.py``)
   q4_0_import_aos           -- blocks assembled byte by byte with numpy from
                                random codes and scales
   affine_quantize           -- closed forms: exact round trip, constant group,
-                               min -> 0 / max -> L, error bound
-  affine_dequantize         -- closed form over every code value (4 and 8 bit),
-                               exact round trip of quantize
+                               min -> 0 / max -> L, error bound (2, 3, 4, 6, 8 bits)
+  affine_dequantize         -- closed form over every code value, codes laid out
+                               by an independent numpy bit-stream packer and a
+                               hand-derived 3-bit word; exact round trip of quantize
   q8_1_quantize             -- closed forms: power-of-two scales with exact codes,
                                half-away-from-zero ties, all-zero block, |q| <= 127,
                                qsum, reconstruction error <= d/2
@@ -171,9 +172,13 @@ def q4_0_q8_matmul(xq, dx, wq, d) -> tuple[np.ndarray, np.ndarray]:
 
 
 # -------------------------------------------------------------------- affine
+AFFINE_BITS = (2, 3, 4, 6, 8)
+
+
 def affine_quantize(w, group_size: int = 64, bits: int = 4):
-    """fp32 w[N][K] -> (wq u32 [N][K*bits/32], scales bf16 bits, biases bf16 bits [N][K/group])."""
-    assert bits in (4, 8)
+    """fp32 w[N][K] -> (wq u32 [N][K*bits/32], scales bf16 bits, biases bf16 bits [N][K/group]).
+    Codes are a little-endian bit stream per row (code k at stream bits bits*k ..)."""
+    assert bits in AFFINE_BITS
     w = _c(w, np.float32)
     N, K = w.shape
     assert K % group_size == 0 and (K * bits) % 32 == 0
@@ -185,7 +190,7 @@ def affine_quantize(w, group_size: int = 64, bits: int = 4):
 
 
 def affine_dequantize(wq, scales, biases, group_size: int = 64, bits: int = 4) -> np.ndarray:
-    assert bits in (4, 8)
+    assert bits in AFFINE_BITS
     wq = _c(wq, np.uint32)
     scales = _c(scales, np.uint16)
     biases = _c(biases, np.uint16)

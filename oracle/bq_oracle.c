@@ -257,10 +257,33 @@ void oracle_q4_0_q8_matmul(const int8_t* xq, const float* dx, const uint8_t* wq,
 }
 
 /* ------------------------------------------------------------------ */
-/* Affine (MLX-style) b-bit, b in {4, 8}                               */
+/* Affine (MLX-style) b-bit, b in {2, 3, 4, 6, 8}                      */
 /* ------------------------------------------------------------------ */
 
+/* Codes of a row form a little-endian bit stream over its 32-bit words: code k
+ * occupies stream bits bits*k .. bits*k + bits - 1, lowest first, and stream
+ * bit i is bit (i mod 32) of word i / 32.  For 2, 4 and 8 bits a code never
+ * crosses a word (32 / bits codes per word, lowest bits first); 3- and 6-bit
+ * codes may.  Rows hold K * bits / 32 whole words (K is a multiple of 32). */
 static int64_t affine_words_per_row(int64_t K, int bits) { return K * bits / 32; }
+
+static void put_code(uint32_t* row, int64_t k, int bits, uint32_t q)
+{
+    for (int i = 0; i < bits; ++i) {
+        const int64_t bit = k * bits + i;
+        if ((q >> i) & 1u) row[bit / 32] |= 1u << (int)(bit % 32);
+    }
+}
+
+static uint32_t get_code(const uint32_t* row, int64_t k, int bits)
+{
+    uint32_t q = 0;
+    for (int i = 0; i < bits; ++i) {
+        const int64_t bit = k * bits + i;
+        q |= ((row[bit / 32] >> (int)(bit % 32)) & 1u) << i;
+    }
+    return q;
+}
 
 /* Quantize w[N][K] (values already bf16-representable) per group:
  *   scale = bf16((max - min) / L), bias = bf16(min), L = 2^bits - 1;
@@ -272,7 +295,6 @@ void oracle_affine_quantize(const float* w, int64_t N, int64_t K, int group, int
     const int L = (1 << bits) - 1;
     const int64_t ng = K / group;
     const int64_t wpr = affine_words_per_row(K, bits);
-    const int per_word = 32 / bits;
     memset(wq, 0, (size_t)(N * wpr) * sizeof(uint32_t));
     for (int64_t n = 0; n < N; ++n) {
         for (int64_t g = 0; g < ng; ++g) {
@@ -300,8 +322,7 @@ void oracle_affine_quantize(const float* w, int64_t N, int64_t K, int group, int
                     if (r > (float)L) r = (float)L;
                     q = (int)r;
                 }
-                int64_t k = g * group + j;
-                wq[n * wpr + k / per_word] |= (uint32_t)q << (bits * (int)(k % per_word));
+                put_code(wq + n * wpr, g * group + j, bits, (uint32_t)q);
             }
         }
     }
@@ -314,12 +335,9 @@ void oracle_affine_dequantize(const uint32_t* wq, const uint16_t* scales, const 
 {
     const int64_t ng = K / group;
     const int64_t wpr = affine_words_per_row(K, bits);
-    const int per_word = 32 / bits;
-    const uint32_t mask = (1u << bits) - 1u;
     for (int64_t n = 0; n < N; ++n) {
         for (int64_t k = 0; k < K; ++k) {
-            uint32_t word = wq[n * wpr + k / per_word];
-            uint32_t q = (word >> (bits * (int)(k % per_word))) & mask;
+            uint32_t q = get_code(wq + n * wpr, k, bits);
             float s = oracle_bf16_to_f32(scales[n * ng + k / group]);
             float b = oracle_bf16_to_f32(biases[n * ng + k / group]);
             out[n * K + k] = oracle_f32_to_bf16(fmaf(s, (float)q, b));

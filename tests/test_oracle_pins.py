@@ -31,12 +31,23 @@ def pack_q4_0(q: np.ndarray) -> np.ndarray:
 
 
 def pack_affine(q: np.ndarray, bits: int) -> np.ndarray:
-    """q[N][K] -> u32 words, 32/bits codes per word, lowest bits first."""
+    """q[N][K] -> u32 words of a little-endian bit stream per row: the bits of
+    code k, lowest first, are stream bits bits*k ..; stream bit i is bit i%32 of
+    word i//32 (numpy bit arrays, independent of the oracle's loops)."""
     N, K = q.shape
-    per = 32 // bits
-    qw = q.reshape(N, K // per, per).astype(np.uint64)
-    shifts = (np.arange(per, dtype=np.uint64) * bits)
-    return (qw << shifts).sum(axis=2).astype(np.uint32)
+    code_bits = (q.astype(np.uint64)[..., None] >> np.arange(bits, dtype=np.uint64)) & 1   # [N][K][bits]
+    stream = code_bits.reshape(N, K * bits).astype(np.uint8)
+    return np.ascontiguousarray(np.packbits(stream, axis=1, bitorder="little")).view("<u4")
+
+
+def unpack_affine(wq: np.ndarray, bits: int, K: int) -> np.ndarray:
+    N = wq.shape[0]
+    stream = np.unpackbits(np.ascontiguousarray(wq).astype("<u4").view(np.uint8), axis=1, bitorder="little")
+    code_bits = stream[:, :K * bits].reshape(N, K, bits).astype(np.int64)
+    return (code_bits << np.arange(bits)).sum(axis=2)
+
+
+AFFINE_BITS = [2, 3, 4, 6, 8]
 
 
 def f32_from_bf16_bits(h: np.ndarray) -> np.ndarray:
@@ -211,8 +222,29 @@ def test_q4_0_invariants_random():
 # --------------------------------------------------------------------------
 # affine
 # --------------------------------------------------------------------------
+def test_affine_packing_hand_derived():
+    """Layout fixed by hand: eight 3-bit codes 0..7 are the octal number
+    76543210 = 0xFAC688, bytes 88 C6 FA repeating; four 6-bit codes 1, 2, 3, 4 are
+    1 + 2*64 + 3*4096 + 4*262144 = 0x103081, bytes 81 30 10 repeating; 4- and
+    8-bit codes fill each word lowest bits first."""
+    q3 = (np.arange(32) % 8)[None, :]
+    assert pack_affine(q3, 3).tolist() == [[0x88FAC688, 0xC688FAC6, 0xFAC688FA]]
+    q6 = np.tile([1, 2, 3, 4], 8)[None, :]
+    assert pack_affine(q6, 6).tolist() == [[0x81103081, 0x30811030, 0x10308110] * 2]
+    q4 = (np.arange(32) % 16)[None, :]
+    assert pack_affine(q4, 4).tolist() == [[0x76543210, 0xFEDCBA98, 0x76543210, 0xFEDCBA98]]
+    q2 = (np.arange(32) % 4)[None, :]
+    assert pack_affine(q2, 2).tolist() == [[0xE4E4E4E4, 0xE4E4E4E4]]
+    # the oracle reads codes from the same layout: unit scale, zero bias gives q itself
+    for q, bits in ((q3, 3), (q6, 6), (q4, 4), (q2, 2)):
+        one = torch_bf16_bits(np.ones((1, 1), np.float32))
+        zero = np.zeros((1, 1), np.uint16)
+        got = f32_from_bf16_bits(oracle.affine_dequantize(pack_affine(q, bits), one, zero, 32, bits))
+        assert np.array_equal(got, q.astype(np.float32))
+
+
 @pytest.mark.parametrize("G", [32, 64, 128])
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", AFFINE_BITS)
 def test_affine_dequant_closed_form_layout(bits, G):
     rng = np.random.default_rng(7 + bits + G)
     N, K = 3, 256
@@ -227,7 +259,7 @@ def test_affine_dequant_closed_form_layout(bits, G):
     assert np.array_equal(got.astype(np.float64), expect)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", AFFINE_BITS)
 def test_affine_dequant_rounding_reduces_to_library(bits):
     """Random bf16 scale/bias with exponents close enough that scale*q + bias is
     exact in fp32; the result is then the library's bf16 rounding of it."""
@@ -246,7 +278,7 @@ def test_affine_dequant_rounding_reduces_to_library(bits):
 
 
 @pytest.mark.parametrize("G", [32, 64, 128])
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", AFFINE_BITS)
 def test_affine_round_trip_exact(bits, G):
     rng = np.random.default_rng(9 + bits + G)
     N, K = 8, 256
@@ -268,7 +300,7 @@ def test_affine_round_trip_exact(bits, G):
     assert np.array_equal(back, w)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", AFFINE_BITS)
 def test_affine_constant_group(bits):
     w = np.full((2, 128), -0.375, np.float32)
     w[1, 64:] = 0.0
@@ -280,15 +312,15 @@ def test_affine_constant_group(bits):
 
 
 @pytest.mark.parametrize("G", [32, 64, 128])
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", AFFINE_BITS)
 def test_affine_invariants_random(bits, G):
     g = inputs.generator(10 + bits + G)
     N, K = 48, 1024
     L = (1 << bits) - 1
     w = inputs.weights_bf16_valued(N, K, g).numpy()
     wq, s16, b16 = oracle.affine_quantize(w, G, bits)
-    per = 32 // bits
-    q = ((wq[:, :, None] >> (np.arange(per, dtype=np.uint32) * bits)) & L).reshape(N, K)
+    assert wq.shape == (N, K * bits // 32)
+    q = unpack_affine(wq, bits, K)
     wg = w.reshape(N, K // G, G)
     qg = q.reshape(N, K // G, G)
     # min maps to 0, max to L; scale = (max-min)/L and bias = min
@@ -302,7 +334,7 @@ def test_affine_invariants_random(bits, G):
     s_stored = f32_from_bf16_bits(s16)
     assert np.all(q_max[s_stored <= s_exact] == L)
     assert np.all(q_max >= L - 1)
-    if bits == 4:
+    if bits <= 6:                       # L * 2^-8 < 1/2: the rounded scale cannot move the max's code
         assert np.all(q_max == L)
     s = f32_from_bf16_bits(s16).astype(np.float64)[..., None]
     deq = f32_from_bf16_bits(oracle.affine_dequantize(wq, s16, b16, G, bits)).reshape(N, K // G, G)
