@@ -147,10 +147,18 @@ def _k_of(wq: torch.Tensor, biases, bits: int) -> int:
     return wq.shape[1] * 32 // bits
 
 
+def _nk_of(wq: torch.Tensor, biases, bits: int, transpose: bool) -> tuple[int, int]:
+    """(N, K) of the weights: [N][K] packed along K (transpose), else [K][N] packed along N."""
+    if transpose:
+        return wq.shape[0], _k_of(wq, biases, bits)
+    return _k_of(wq, biases, bits), wq.shape[0]
+
+
 def quant_matmul(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor | None = None,
                  group_size: int = 32, bits: int = 4, transpose: bool = True, out: torch.Tensor | None = None,
                  stream=None):
-    """y[M][N] = x[M][K] . dequant(W)[N][K]^T (biases None: Q4_0)."""
+    """y[M][N] = x[M][K] . dequant(W)[N][K]^T (biases None: Q4_0); transpose=False:
+    y = x . dequant(W) with affine W [K][N] packed and grouped along N."""
     return quant_matmul_ex(x, wq, scales, biases, group_size, bits, transpose, "auto", out=out, stream=stream)
 
 
@@ -158,9 +166,9 @@ def quant_matmul_ex(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, bia
                     group_size: int = 32, bits: int = 4, transpose: bool = True, path="auto",
                     workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None):
     M, K = x.shape
-    N = wq.shape[0]
-    if K != _k_of(wq, biases, bits):
-        raise ValueError(f"K mismatch: x has {K}, weights hold {_k_of(wq, biases, bits)}")
+    N, Kw = _nk_of(wq, biases, bits, transpose)
+    if K != Kw:
+        raise ValueError(f"K mismatch: x has {K}, weights hold {Kw}")
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
     p = PATHS[path] if isinstance(path, str) else int(path)
@@ -235,9 +243,9 @@ def quant_matmul_noalloc(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor
     32 MiB device scratch (N * K <= 16 Mi weights) and allocates nothing.  `out`
     (bf16 [M][N]) is required, since creating it here would allocate."""
     M, K = x.shape
-    N = wq.shape[0]
-    if K != _k_of(wq, biases, bits):
-        raise ValueError(f"K mismatch: x has {K}, weights hold {_k_of(wq, biases, bits)}")
+    N, Kw = _nk_of(wq, biases, bits, transpose)
+    if K != Kw:
+        raise ValueError(f"K mismatch: x has {K}, weights hold {Kw}")
     if tuple(out.shape) != (M, N) or out.dtype != torch.bfloat16:
         raise ValueError("out must be a bf16 tensor of shape [M][N]")
     _check(lib().quant_matmul_noalloc(_ptr(x), _ptr(wq), _ptr(_bits16(scales)),

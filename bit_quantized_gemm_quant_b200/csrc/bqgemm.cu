@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -59,9 +60,14 @@ bq_status current_device(int* dev_out, DeviceInfo* info_out)
 // ------------------------------------------------------------------ checks
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-enum class WFmt { Q4_0, AFF4, AFF8 };
+// Q4_0, affine 4- and 8-bit (every path), affine 2-, 3- and 6-bit (dequantize,
+// quantize and the unfused pair).
+enum class WFmt { Q4_0, AFF4, AFF8, AFF2, AFF3, AFF6 };
 
-// Format and shape checks shared by quant_matmul and its helpers (host only).
+bool has_fast_paths(WFmt f) { return f == WFmt::Q4_0 || f == WFmt::AFF4 || f == WFmt::AFF8; }
+
+// Format and shape checks shared by quant_matmul and its helpers (host only):
+// the packed matrix has N rows of K codes, grouped along K.
 bq_status check_format(const void* biases, int64_t N, int64_t K, int group_size, int bits, WFmt* fmt)
 {
     if (N < 0 || K < 0) return BQ_ERR_SHAPE;
@@ -70,10 +76,16 @@ bq_status check_format(const void* biases, int64_t N, int64_t K, int group_size,
         if (K % 32 != 0) return BQ_ERR_SHAPE;
         *fmt = WFmt::Q4_0;
     } else {
-        if (bits != 4 && bits != 8) return BQ_ERR_UNSUPPORTED;
+        switch (bits) {
+        case 2: *fmt = WFmt::AFF2; break;
+        case 3: *fmt = WFmt::AFF3; break;
+        case 4: *fmt = WFmt::AFF4; break;
+        case 6: *fmt = WFmt::AFF6; break;
+        case 8: *fmt = WFmt::AFF8; break;
+        default: return BQ_ERR_UNSUPPORTED;
+        }
         if (group_size != 32 && group_size != 64 && group_size != 128) return BQ_ERR_UNSUPPORTED;
         if (K % group_size != 0) return BQ_ERR_SHAPE;
-        *fmt = bits == 4 ? WFmt::AFF4 : WFmt::AFF8;
     }
     return BQ_OK;
 }
@@ -133,6 +145,7 @@ const DispatchCfg& dispatch_cfg()
 
 int select_path(int64_t M, int64_t K, WFmt fmt)
 {
+    if (!has_fast_paths(fmt)) return BQ_PATH_DEQUANT_GEMM;
     const DispatchCfg& c = dispatch_cfg();
     if (M < c.tc_min_m) return BQ_PATH_GEMV;
     const int64_t pair_min = c.pair_min_m[(int)fmt];
@@ -437,7 +450,9 @@ bq_status library_workspace(int dev, size_t need, void** out)
 size_t workspace_for(int path, WFmt fmt, int64_t M, int64_t N, int64_t K, int num_sms, int smem_optin)
 {
     if (path == BQ_PATH_DEQUANT_GEMM) return (size_t)N * (size_t)K * 2u;
-    if (path != BQ_PATH_TC_FUSED || K % 64 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return 0u;
+    if (path != BQ_PATH_TC_FUSED || !has_fast_paths(fmt) || K % 64 != 0 || M > INT32_MAX || N > INT32_MAX ||
+        K > INT32_MAX)
+        return 0u;
     TcPlan pl;
     bool ok = fmt == WFmt::Q4_0  ? plan_tc<kModeQ4_0>(M, N, K, num_sms, smem_optin, &pl)
               : fmt == WFmt::AFF4 ? plan_tc<kModeAff4>(M, N, K, num_sms, smem_optin, &pl)
@@ -452,16 +467,46 @@ bq_status dequant_any(WFmt fmt, const void* wq, const void* scales, const void* 
         const int64_t nb = N * (K / 32);
         q4_0_dequant_kernel<<<grid_for(nb, 256, di), 256, 0, st>>>(
             reinterpret_cast<const uint8_t*>(wq), reinterpret_cast<const uint16_t*>(scales), out, nb);
-    } else if (fmt == WFmt::AFF4) {
-        const int64_t nc = N * (K / 32);
-        affine_dequant_kernel<4><<<grid_for(nc, 256, di), 256, 0, st>>>(
-            reinterpret_cast<const uint32_t*>(wq), reinterpret_cast<const uint16_t*>(scales),
-            reinterpret_cast<const uint16_t*>(biases), out, nc, K, group_size);
     } else {
-        const int64_t nc = N * (K / 16);
-        affine_dequant_kernel<8><<<grid_for(nc, 256, di), 256, 0, st>>>(
-            reinterpret_cast<const uint32_t*>(wq), reinterpret_cast<const uint16_t*>(scales),
-            reinterpret_cast<const uint16_t*>(biases), out, nc, K, group_size);
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(wq);
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(scales);
+        const uint16_t* bi = reinterpret_cast<const uint16_t*>(biases);
+        auto go = [&](auto bits_tag) {
+            constexpr int B = decltype(bits_tag)::value;
+            const int64_t nu = N * (K / AffUnit<B>::E);
+            affine_dequant_kernel<B><<<grid_for(nu, 256, di), 256, 0, st>>>(w, sc, bi, out, nu, K, group_size);
+        };
+        switch (fmt) {
+        case WFmt::AFF2: go(std::integral_constant<int, 2>()); break;
+        case WFmt::AFF3: go(std::integral_constant<int, 3>()); break;
+        case WFmt::AFF4: go(std::integral_constant<int, 4>()); break;
+        case WFmt::AFF6: go(std::integral_constant<int, 6>()); break;
+        default: go(std::integral_constant<int, 8>()); break;
+        }
+    }
+    return launch_status();
+}
+
+// Affine W stored as R rows of C codes grouped along C, dequantized into its
+// transpose out[C][R] (the weight operand of y = x . W for transpose = 0).
+bq_status dequant_affine_t(WFmt fmt, const void* wq, const void* scales, const void* biases, uint16_t* out,
+                           int64_t R, int64_t C, int group_size, const DeviceInfo& di, cudaStream_t st)
+{
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(wq);
+    const uint16_t* sc = reinterpret_cast<const uint16_t*>(scales);
+    const uint16_t* bi = reinterpret_cast<const uint16_t*>(biases);
+    const int64_t tiles = ((R + kTrRows - 1) / kTrRows) * ((C + kTrCols - 1) / kTrCols);
+    const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)di.num_sms * 8));
+    auto go = [&](auto bits_tag) {
+        constexpr int B = decltype(bits_tag)::value;
+        affine_dequant_t_kernel<B><<<grid, 256, 0, st>>>(w, sc, bi, out, R, C, group_size);
+    };
+    switch (fmt) {
+    case WFmt::AFF2: go(std::integral_constant<int, 2>()); break;
+    case WFmt::AFF3: go(std::integral_constant<int, 3>()); break;
+    case WFmt::AFF4: go(std::integral_constant<int, 4>()); break;
+    case WFmt::AFF6: go(std::integral_constant<int, 6>()); break;
+    default: go(std::integral_constant<int, 8>()); break;
     }
     return launch_status();
 }
@@ -470,13 +515,23 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
                       int64_t M, int64_t N, int64_t K, int group_size, int bits, int transpose, int path,
                       void* workspace, size_t workspace_bytes, cudaStream_t st)
 {
-    if (transpose != 1) return BQ_ERR_UNSUPPORTED;
+    if (transpose != 0 && transpose != 1) return BQ_ERR_UNSUPPORTED;
     if (path < BQ_PATH_AUTO || path > BQ_PATH_DEQUANT_GEMM) return BQ_ERR_UNSUPPORTED;
     if (M < 0 || N < 0 || K < 0) return BQ_ERR_SHAPE;
-    if (M == 0 || N == 0) return BQ_OK;      // empty problem: nothing is read or written
+    // transpose = 0: y = x . W with W stored [K][N], codes and groups along N
+    // (affine only: Q4_0 blocks run along K); it runs as the unfused pair with
+    // a transposing dequantize, and x's rows must be 16-byte multiples.
+    if (transpose == 0 && !biases) return BQ_ERR_UNSUPPORTED;
     WFmt fmt;
-    bq_status s = check_format(biases, N, K, group_size, bits, &fmt);
+    bq_status s = transpose ? check_format(biases, N, K, group_size, bits, &fmt)
+                            : check_format(biases, K, N, group_size, bits, &fmt);
     if (s != BQ_OK) return s;
+    if (transpose == 0) {
+        if (path == BQ_PATH_GEMV || path == BQ_PATH_TC_FUSED) return BQ_ERR_UNSUPPORTED;
+        if (K % 8 != 0) return BQ_ERR_SHAPE;
+        path = BQ_PATH_DEQUANT_GEMM;
+    }
+    if (M == 0 || N == 0) return BQ_OK;      // empty problem: nothing is read or written
     int dev;
     DeviceInfo di;
     if (K == 0) {                            // empty sum: y = 0
@@ -490,6 +545,7 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
         (workspace && !aligned16(workspace)))
         return BQ_ERR_ALIGN;
     if (path == BQ_PATH_AUTO) path = select_path(M, K, fmt);
+    if (path != BQ_PATH_DEQUANT_GEMM && !has_fast_paths(fmt)) return BQ_ERR_UNSUPPORTED;
     if (path == BQ_PATH_GEMV && M > kGemvMaxM) return BQ_ERR_UNSUPPORTED;
     if (path == BQ_PATH_TC_FUSED && K % 64 != 0) return BQ_ERR_UNSUPPORTED;
     if (path == BQ_PATH_DEQUANT_GEMM && workspace && workspace_bytes < (size_t)N * (size_t)K * 2u)
@@ -523,7 +579,9 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
         void* ws = workspace;
         if (!ws && (s = library_workspace(dev, need, &ws)) != BQ_OK) return s;
         uint16_t* wb = reinterpret_cast<uint16_t*>(ws);
-        if ((s = dequant_any(fmt, wq, scales, biases, wb, N, K, group_size, di, st)) != BQ_OK) return s;
+        s = transpose ? dequant_any(fmt, wq, scales, biases, wb, N, K, group_size, di, st)
+                      : dequant_affine_t(fmt, wq, scales, biases, wb, K, N, group_size, di, st);
+        if (s != BQ_OK) return s;
         return launch_tc<kModeBF16>(di, dev, x, wb, nullptr, nullptr, y, M, N, K, st);
     }
     }
@@ -687,10 +745,12 @@ bq_status quant_matmul_noalloc(const uint16_t* x_bf16, const void* wq, const voi
                                uint16_t* y_bf16, int64_t M, int64_t N, int64_t K, int group_size, int bits,
                                int transpose, bq_stream_t stream)
 {
-    if (transpose != 1) return BQ_ERR_UNSUPPORTED;
+    if (transpose != 0 && transpose != 1) return BQ_ERR_UNSUPPORTED;
     if (M < 0 || N < 0 || K < 0) return BQ_ERR_SHAPE;
+    if (transpose == 0 && !biases) return BQ_ERR_UNSUPPORTED;
     WFmt fmt;
-    bq_status s = check_format(biases, N, K, group_size, bits, &fmt);
+    bq_status s = transpose ? check_format(biases, N, K, group_size, bits, &fmt)
+                            : check_format(biases, K, N, group_size, bits, &fmt);
     if (s != BQ_OK) return s;
     if (M == 0 || N == 0 || K == 0)           // nothing to stage: no scratch involved
         return matmul_impl(x_bf16, wq, scales, biases, y_bf16, M, N, K, group_size, bits, transpose,
@@ -827,12 +887,15 @@ bq_status affine_quantize(const float* w, uint32_t* wq, uint16_t* scales_bf16, u
     int dev;
     DeviceInfo di;
     if ((s = current_device(&dev, &di)) != BQ_OK) return s;
-    if (bits == 4)
-        affine_quant_kernel<4><<<grid_for(ng, 256, di), 256, 0, (cudaStream_t)stream>>>(w, wq, scales_bf16,
-                                                                                         biases_bf16, ng, group_size);
-    else
-        affine_quant_kernel<8><<<grid_for(ng, 256, di), 256, 0, (cudaStream_t)stream>>>(w, wq, scales_bf16,
-                                                                                         biases_bf16, ng, group_size);
+    const int grid = grid_for(ng, 256, di);
+    const cudaStream_t st = (cudaStream_t)stream;
+    switch (bits) {
+    case 2: affine_quant_kernel<2><<<grid, 256, 0, st>>>(w, wq, scales_bf16, biases_bf16, ng, group_size); break;
+    case 3: affine_quant_kernel<3><<<grid, 256, 0, st>>>(w, wq, scales_bf16, biases_bf16, ng, group_size); break;
+    case 4: affine_quant_kernel<4><<<grid, 256, 0, st>>>(w, wq, scales_bf16, biases_bf16, ng, group_size); break;
+    case 6: affine_quant_kernel<6><<<grid, 256, 0, st>>>(w, wq, scales_bf16, biases_bf16, ng, group_size); break;
+    default: affine_quant_kernel<8><<<grid, 256, 0, st>>>(w, wq, scales_bf16, biases_bf16, ng, group_size); break;
+    }
     return launch_status();
 }
 

@@ -49,41 +49,132 @@ q4_0_dequant_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__
 }
 
 // ----------------------------------------------------------------------------
-// Affine dequantize: one thread per 16 packed bytes (32 codes at 4 bits, 16 at
-// 8 bits).  out = bf16_rne(fmaf(scale, q, bias)).
+// Affine codes: each row is a little-endian bit stream, code k at stream bits
+// BITS*k .. BITS*k + BITS - 1 (lowest first; stream bit i = bit i%32 of word
+// i/32).  For 2, 4 and 8 bits that is 32/BITS codes per word, lowest bits
+// first, as on the MLX issue page's 4- and 8-bit weights; 3- and 6-bit codes
+// may cross a word.  A unit of W words holds E whole codes, E divides every
+// group size (32, 64, 128), so a unit never straddles a group.
+// ----------------------------------------------------------------------------
+template <int BITS> struct AffUnit;
+template <> struct AffUnit<2> { static constexpr int W = 2, E = 32; };
+template <> struct AffUnit<3> { static constexpr int W = 3, E = 32; };
+template <> struct AffUnit<4> { static constexpr int W = 4, E = 32; };
+template <> struct AffUnit<6> { static constexpr int W = 3, E = 16; };
+template <> struct AffUnit<8> { static constexpr int W = 4, E = 16; };
+
+// Code e of a unit (e a compile-time constant after unrolling).
+template <int BITS>
+BQ_DEVINL uint32_t unit_code(const uint32_t (&w)[AffUnit<BITS>::W], int e)
+{
+    const int bit = BITS * e, i = bit >> 5, sh = bit & 31;
+    uint32_t q = w[i] >> sh;
+    if (sh + BITS > 32) q |= w[i + 1] << (32 - sh);
+    return q & ((1u << BITS) - 1u);
+}
+
+// The W words of unit u of a packed array (16-, 8- or 4-byte loads by W).
+template <int BITS>
+BQ_DEVINL void load_unit(const uint32_t* __restrict__ wq, int64_t u, uint32_t (&w)[AffUnit<BITS>::W])
+{
+    constexpr int W = AffUnit<BITS>::W;
+    const uint32_t* p = wq + u * W;
+    if constexpr (W == 4) {
+        const uint4 v = ldg_stream(p);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else if constexpr (W == 2) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+        w[0] = v.x; w[1] = v.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < W; ++i) w[i] = __ldg(p + i);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Affine dequantize: one thread per unit.  out = bf16_rne(fmaf(scale, q, bias)).
 // ----------------------------------------------------------------------------
 template <int BITS>
 __global__ void __launch_bounds__(256)
 affine_dequant_kernel(const uint32_t* __restrict__ wq, const uint16_t* __restrict__ scales,
                       const uint16_t* __restrict__ biases, uint16_t* __restrict__ out,
-                      int64_t nchunks, int64_t K, int group_size)
+                      int64_t nunits, int64_t K, int group_size)
 {
-    constexpr int kPer = 32 / BITS;          // codes per word
-    constexpr int kElems = 4 * kPer;         // codes per 16-byte chunk
-    constexpr uint32_t kMask = (1u << BITS) - 1u;
-    const int64_t chunks_per_row = K / kElems;
+    constexpr int W = AffUnit<BITS>::W, E = AffUnit<BITS>::E;
+    const int64_t units_per_row = K / E;
     const int64_t groups_per_row = K / group_size;
-    for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < nchunks;
-         c += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t n = c / chunks_per_row;
-        const int64_t k0 = (c % chunks_per_row) * kElems;
-        const uint4 raw = ldg_stream(wq + c * 4);
-        const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
-        // A chunk never straddles a group: kElems (32 or 16) divides group_size.
+    for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < nunits;
+         u += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = u / units_per_row;
+        const int64_t k0 = (u % units_per_row) * E;
+        uint32_t w[W];
+        load_unit<BITS>(wq, u, w);
         const int64_t gi = n * groups_per_row + k0 / group_size;
         const float s = bf16_bits_to_f32(__ldg(scales + gi));
         const float bb = bf16_bits_to_f32(__ldg(biases + gi));
-        uint32_t packed[kElems / 2];
+        uint32_t packed[E / 2];
 #pragma unroll
-        for (int e = 0; e < kElems; e += 2) {
-            const uint32_t q0 = (words[e / kPer] >> (BITS * (e % kPer))) & kMask;
-            const uint32_t q1 = (words[(e + 1) / kPer] >> (BITS * ((e + 1) % kPer))) & kMask;
-            packed[e / 2] = pack_bf16x2_rn(__fmaf_rn(s, (float)q0, bb), __fmaf_rn(s, (float)q1, bb));
-        }
+        for (int e = 0; e < E; e += 2)
+            packed[e / 2] = pack_bf16x2_rn(__fmaf_rn(s, (float)unit_code<BITS>(w, e), bb),
+                                           __fmaf_rn(s, (float)unit_code<BITS>(w, e + 1), bb));
         uint4* o = reinterpret_cast<uint4*>(out + n * K + k0);
 #pragma unroll
-        for (int v = 0; v < kElems / 8; ++v)
+        for (int v = 0; v < E / 8; ++v)
             o[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Affine dequantize with a transposed result: the packed matrix is W[R][C]
+// (codes along C, groups of C), the output its transpose out[C][R] in bf16.
+// One CTA per tile of 32 rows x 64 columns: units are dequantized into a
+// shared tile, which is then written out 16 bytes per thread along R.
+// ----------------------------------------------------------------------------
+constexpr int kTrRows = 32, kTrCols = 64;
+
+template <int BITS>
+__global__ void __launch_bounds__(256)
+affine_dequant_t_kernel(const uint32_t* __restrict__ wq, const uint16_t* __restrict__ scales,
+                        const uint16_t* __restrict__ biases, uint16_t* __restrict__ out, int64_t R, int64_t C,
+                        int group_size)
+{
+    constexpr int W = AffUnit<BITS>::W, E = AffUnit<BITS>::E;
+    constexpr int kUnitsPerTileRow = kTrCols / E;
+    __shared__ uint16_t tile[kTrCols][kTrRows + 2];      // [column][row], padded against bank conflicts
+    const int64_t units_per_row = C / E, groups_per_row = C / group_size;
+    const int64_t tiles_r = (R + kTrRows - 1) / kTrRows, tiles_c = (C + kTrCols - 1) / kTrCols;
+    for (int64_t t = blockIdx.x; t < tiles_r * tiles_c; t += gridDim.x) {
+        const int64_t r0 = (t / tiles_c) * kTrRows, c0 = (t % tiles_c) * kTrCols;
+        for (int i = threadIdx.x; i < kTrRows * kUnitsPerTileRow; i += blockDim.x) {
+            const int rr = i / kUnitsPerTileRow, cu = i % kUnitsPerTileRow;
+            const int64_t r = r0 + rr, c = c0 + (int64_t)cu * E;
+            if (r >= R || c >= C) continue;
+            uint32_t w[W];
+            load_unit<BITS>(wq, r * units_per_row + c / E, w);
+            const int64_t gi = r * groups_per_row + c / group_size;
+            const float s = bf16_bits_to_f32(__ldg(scales + gi));
+            const float bb = bf16_bits_to_f32(__ldg(biases + gi));
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                tile[cu * E + e][rr] = (uint16_t)f32_to_bf16_bits(__fmaf_rn(s, (float)unit_code<BITS>(w, e), bb));
+        }
+        __syncthreads();
+        // out[c][r0 .. r0 + 31]: 4 threads per column, 8 rows (16 bytes) each
+        for (int i = threadIdx.x; i < kTrCols * (kTrRows / 8); i += blockDim.x) {
+            const int cc = i / (kTrRows / 8), rq = (i % (kTrRows / 8)) * 8;
+            const int64_t c = c0 + cc, r = r0 + rq;
+            if (c >= C || r >= R) continue;
+            uint16_t* dst = out + c * R + r;
+            if (r + 8 <= R) {
+                uint32_t v[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) v[j] = (uint32_t)tile[cc][rq + 2 * j] | ((uint32_t)tile[cc][rq + 2 * j + 1] << 16);
+                *reinterpret_cast<uint4*>(dst) = make_uint4(v[0], v[1], v[2], v[3]);
+            } else {
+                for (int j = 0; j < 8 && r + j < R; ++j) dst[j] = tile[cc][rq + j];
+            }
+        }
+        __syncthreads();
     }
 }
 
@@ -128,7 +219,8 @@ q4_0_quant_kernel(const float* __restrict__ w, uint8_t* __restrict__ wq, uint16_
 // ----------------------------------------------------------------------------
 // Affine quantize: one thread per group.  scale = bf16((max - min) / L),
 // bias = bf16(min); q = clamp(rint((w - bias) / scale), 0, L) from the stored
-// bf16 values (q = 0 when scale == 0).
+// bf16 values (q = 0 when scale == 0).  Codes are packed unit by unit into the
+// row's bit stream (a group holds whole units).
 // ----------------------------------------------------------------------------
 template <int BITS>
 __global__ void __launch_bounds__(256)
@@ -136,7 +228,7 @@ affine_quant_kernel(const float* __restrict__ w, uint32_t* __restrict__ wq, uint
                     uint16_t* __restrict__ biases, int64_t ngroups, int group_size)
 {
     constexpr int L = (1 << BITS) - 1;
-    constexpr int kPer = 32 / BITS;
+    constexpr int W = AffUnit<BITS>::W, E = AffUnit<BITS>::E;
     for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < ngroups;
          g += (int64_t)gridDim.x * blockDim.x) {
         const float* grp = w + g * group_size;
@@ -153,20 +245,25 @@ affine_quant_kernel(const float* __restrict__ w, uint32_t* __restrict__ wq, uint
         biases[g] = (uint16_t)b16;
         const float s = bf16_bits_to_f32(s16);
         const float bb = bf16_bits_to_f32(b16);
-        uint32_t* out = wq + g * (group_size / kPer);
-        for (int j0 = 0; j0 < group_size; j0 += kPer) {
-            uint32_t word = 0u;
+        uint32_t* out = wq + g * (group_size / E) * W;
+        for (int j0 = 0; j0 < group_size; j0 += E) {
+            uint32_t word[W];
 #pragma unroll
-            for (int e = 0; e < kPer; ++e) {
-                int q = 0;
+            for (int i = 0; i < W; ++i) word[i] = 0u;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                uint32_t q = 0u;
                 if (s != 0.0f) {
                     float r = rintf(__fdiv_rn(__fsub_rn(grp[j0 + e], bb), s));
                     r = fminf(fmaxf(r, 0.0f), (float)L);
-                    q = (int)r;
+                    q = (uint32_t)r;
                 }
-                word |= (uint32_t)q << (BITS * e);
+                const int bit = BITS * e, i = bit >> 5, sh = bit & 31;
+                word[i] |= q << sh;
+                if (sh + BITS > 32) word[i + 1] |= q >> (32 - sh);
             }
-            out[j0 / kPer] = word;
+#pragma unroll
+            for (int i = 0; i < W; ++i) out[(j0 / E) * W + i] = word[i];
         }
     }
 }

@@ -19,10 +19,17 @@
  *    mx.quantized_matmul on "quantized_matmul takes 14-41% longer than
  *    dequantize + bf16 matmul at prefill sizes (> 512 tokens)" (Repro).
  *    Groups of group_size weights along K share a bf16 scale and a bf16 bias;
- *    w = scale * q + bias, q in [0, 2^bits - 1], bits in {4, 8}, group_size in
- *    {32, 64, 128} (the sizes mx.quantize accepts; the workloads use 64).
- *      wq      u32  [N][K*bits/32]  element k at bits bits*(k % (32/bits)) of
- *                                   word k / (32/bits) (lowest bits first)
+ *    w = scale * q + bias, q in [0, 2^bits - 1], bits in {2, 3, 4, 6, 8},
+ *    group_size in {32, 64, 128} (the widths and sizes mx.quantize accepts; the
+ *    page's workloads use 4 and 8 bits with groups of 64).
+ *      wq      u32  [N][K*bits/32]  each row a little-endian bit stream: element
+ *                                   k at stream bits bits*k .. bits*k + bits - 1,
+ *                                   stream bit i = bit i % 32 of word i / 32.
+ *                                   For 2, 4 and 8 bits: 32/bits elements per
+ *                                   word, lowest bits first; 3- and 6-bit
+ *                                   elements may cross a word (reading: the page
+ *                                   shows 4 and 8 bits only, whose packing is
+ *                                   exactly this stream)
  *      scales  bf16 [N][K/group_size]
  *      biases  bf16 [N][K/group_size]
  *
@@ -102,7 +109,10 @@ BQ_API bq_status q4_0_dequantize(const uint8_t* wq, const uint16_t* scales_f16, 
  *   scales_bf16 device u16 [N][K/group_size]
  *   biases_bf16 device u16 [N][K/group_size]
  *   out_bf16    device u16 [N][K], written
- *   group_size  32, 64 or 128;  bits  4 or 8;  K % group_size == 0
+ *   group_size  32, 64 or 128;  bits  2, 3, 4, 6 or 8;  K % group_size == 0
+ * (A matrix stored the other way round -- codes and groups along N, as
+ * quant_matmul's transpose = 0 takes it -- is dequantized by passing its rows
+ * as N and its codes per row as K.)
  */
 BQ_API bq_status affine_dequantize(const uint32_t* wq, const uint16_t* scales_bf16, const uint16_t* biases_bf16,
                             uint16_t* out_bf16, int64_t N, int64_t K, int group_size, int bits,
@@ -164,7 +174,16 @@ BQ_API bq_status quant_matmul_q8(const int8_t* xq, const float* dx, const int32_
  *   biases   device bf16 [N][K/group_size]; NULL selects Q4_0 (then bits must be
  *            4 and group_size 32)
  *   y_bf16   device u16 [M][N], written
- *   transpose  must be 1 (W stored [N][K]); 0 returns BQ_ERR_UNSUPPORTED
+ *   transpose  1: W stored [N][K] as above.  0 (affine only; Q4_0 returns
+ *            BQ_ERR_UNSUPPORTED): y = x . W with W stored [K][N], codes and
+ *            groups along N -- wq u32 [K][N*bits/32], scales/biases bf16
+ *            [K][N/group_size], N % group_size == 0 -- the transpose=False form
+ *            of mx.quantized_matmul; it always runs as the unfused pair, W
+ *            dequantized into its [N][K] transpose, and needs K % 8 == 0
+ *            (BQ_ERR_SHAPE otherwise).  Other values: BQ_ERR_UNSUPPORTED.
+ * Affine 2-, 3- and 6-bit weights (either orientation) run as the unfused
+ * pair at every M; 4- and 8-bit and Q4_0 have the decode GEMV and the fused
+ * kernel as well.
  * The path is chosen by quant_matmul_select_path.  A path that needs scratch
  * memory (the unfused pair) uses a per-device buffer that the library
  * allocates on first need, grows on demand and keeps until process exit; a
@@ -184,7 +203,8 @@ BQ_API bq_status quant_matmul(const uint16_t* x_bf16, const void* wq, const void
  * unfused pair (q4_0_dequantize / affine_dequantize into scratch, then the
  * bf16 tensor-core GEMM), with the bf16 copy of W staged in a fixed 32 MiB
  * array that is part of the library's device image.
- *   Arguments, layouts, validation and errors are those of quant_matmul.
+ *   Arguments, layouts, validation and errors are those of quant_matmul
+ *   (both orientations).
  *   Limit: N * K * 2 bytes must fit in BQ_NOALLOC_SCRATCH_BYTES (N * K at most
  *   16,777,216 weights, e.g. 4096 x 4096); larger problems return
  *   BQ_ERR_WORKSPACE before anything is launched.
@@ -215,8 +235,9 @@ BQ_API bq_status quant_matmul_noalloc(const uint16_t* x_bf16, const void* wq, co
  *   biases: host array of count device pointers (affine), or NULL (Q4_0 for all)
  * At decode sizes (the dispatcher's GEMV path) all matrices run in one launch
  * and give the same bits as separate quant_matmul calls; at larger M each
- * matrix runs its own quant_matmul path.  Errors as quant_matmul;
- * count > 8 returns BQ_ERR_UNSUPPORTED, count == 0 or M == 0 does nothing.
+ * matrix runs its own quant_matmul path.  Errors as quant_matmul; transpose
+ * must be 1 and count > 8 returns BQ_ERR_UNSUPPORTED, count == 0 or M == 0
+ * does nothing.
  */
 BQ_API bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const void* const* wq,
                                     const void* const* scales, const void* const* biases, uint16_t* const* y_bf16,
@@ -228,7 +249,8 @@ BQ_API bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const voi
  * optional caller-owned device workspace.  With workspace == NULL the library's
  * per-device buffer is used as in quant_matmul; otherwise workspace_bytes must
  * be >= quant_matmul_workspace_size(...) (BQ_ERR_WORKSPACE if not).  Forcing
- * BQ_PATH_GEMV with M > 32 returns BQ_ERR_UNSUPPORTED.
+ * BQ_PATH_GEMV with M > 32, or BQ_PATH_GEMV / BQ_PATH_TC_FUSED for 2-, 3- or
+ * 6-bit weights or with transpose = 0, returns BQ_ERR_UNSUPPORTED.
  */
 BQ_API bq_status quant_matmul_ex(const uint16_t* x_bf16, const void* wq, const void* scales, const void* biases,
                           uint16_t* y_bf16, int64_t M, int64_t N, int64_t K, int group_size, int bits,
@@ -248,6 +270,7 @@ BQ_API size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int g
  * pick the dequantize path above some M) and the decode/prefill split of
  * "et-backend: Q4_0 matrix-engine GEMM rewrite for prefill" (Overview: decode
  * routes to the vector-dot kernel).  Returns a bq_path other than AUTO:
+ * (transpose = 1; 2-, 3- and 6-bit affine weights always get DEQUANT_GEMM):
  *   M <  tc_min_m                 -> BQ_PATH_GEMV        (tc_min_m default 33)
  *   M >= pair_min_m               -> BQ_PATH_DEQUANT_GEMM (pair_min_m by format, from
  *                                    the measured fused/unfused crossovers on B200:
@@ -284,7 +307,8 @@ BQ_API bq_status q4_0_quantize(const float* w, uint8_t* wq, uint16_t* scales_f16
  * page, Repro).  Per group: scale = bf16((max - min) / (2^bits - 1)),
  * bias = bf16(min), q = clamp(round_half_even((w - bias) / scale), 0, 2^bits - 1)
  * from the stored bf16 scale and bias (q = 0 when scale == 0).
- *   w device f32 [N][K]; wq device u32 [N][K*bits/32]; scales/biases device bf16 [N][K/group_size].
+ *   w device f32 [N][K]; wq device u32 [N][K*bits/32] (the bit-stream layout
+ *   above); scales/biases device bf16 [N][K/group_size]; bits 2, 3, 4, 6 or 8.
  */
 BQ_API bq_status affine_quantize(const float* w, uint32_t* wq, uint16_t* scales_bf16, uint16_t* biases_bf16,
                           int64_t N, int64_t K, int group_size, int bits, bq_stream_t stream);

@@ -69,7 +69,16 @@ def test_quant_matmul_rejects_before_launch(L):
     assert qmm(L, bits=8) == 3                                # Q4_0 is 4-bit only
     assert qmm(L, g=64) == 3                                  # ... with group 32
     assert qmm(L, b=ALIGNED, g=16, bits=4) == 3               # affine groups: 32, 64 or 128
-    assert qmm(L, b=ALIGNED, g=64, bits=3) == 3               # bits in {4, 8}
+    assert qmm(L, b=ALIGNED, g=64, bits=5) == 3               # bits in {2, 3, 4, 6, 8}
+    assert qmm(L, b=ALIGNED, g=64, bits=7) == 3
+    assert qmm(L, tr=2) == 3
+    assert qmm(L, b=ALIGNED, g=64, bits=3, path=1) == 3       # 2/3/6-bit: the pair only
+    assert qmm(L, b=ALIGNED, g=64, bits=6, M=64, path=2) == 3
+    assert qmm(L, b=ALIGNED, g=64, bits=2, M=64, path=2) == 3
+    assert qmm(L, b=ALIGNED, g=64, tr=0, path=1) == 3         # transpose=0: the pair only
+    assert qmm(L, b=ALIGNED, g=64, tr=0, M=64, path=2) == 3
+    assert qmm(L, b=ALIGNED, g=64, tr=0, K=12) == 2           # transpose=0 needs K % 8 == 0
+    assert qmm(L, b=ALIGNED, g=64, tr=0, N=96) == 2           # ... and groups along N
     assert qmm(L, b=ALIGNED, g=64, bits=4, K=96) == 2         # K % group
     assert qmm(L, x=None) == 1
     assert qmm(L, wq=None) == 1
@@ -99,6 +108,14 @@ def test_other_entry_points_reject_before_launch(L):
 
 BOUNDARY_M = [1, 2, 8, 19, 31, 32, 33, 63, 64, 65, 127, 128, 129, 383, 384, 385, 511, 512, 513, 1023, 1024, 1025,
               2047, 2048, 8192]
+
+
+def test_dispatcher_pair_only_widths(L):
+    for bits in (2, 3, 6):
+        for M in (1, 8, 32, 33, 512, 4096):
+            assert L.quant_matmul_select_path(M, 12288, 4096, 64, bits) == 3
+        assert L.quant_matmul_workspace_size(8, 256, 512, 64, bits, 0) == 256 * 512 * 2
+        assert L.quant_matmul_workspace_size(8, 256, 512, 64, bits, 2) == 0
 
 
 def test_dispatcher_boundaries(L):

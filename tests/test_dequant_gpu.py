@@ -157,3 +157,43 @@ def test_affine_quantize_bit_exact_group_sizes(bits, G):
     assert np.array_equal(wq.cpu().numpy().view(np.uint32), wq_ref)
     assert np.array_equal(u16(s), s_ref)
     assert np.array_equal(u16(b), b_ref)
+
+
+NEW_WIDTHS = ["affine2", "affine3", "affine6", "affine2_g32", "affine3_g128", "affine6_g32"]
+
+
+@pytest.mark.parametrize("fmt", NEW_WIDTHS)
+@pytest.mark.parametrize("N,K", [(3, 128), (250, 512), (64, 4096)])
+def test_dequant_bit_exact_2_3_6_bits(fmt, N, K):
+    p = Problem(fmt, N, K, seed=N + K + 5)
+    assert np.array_equal(_gpu_dequant(p), p.wb)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 6])
+def test_affine_dequant_random_codes_2_3_6_bits(bits):
+    """Arbitrary code words (3- and 6-bit codes crossing words) and scale bits."""
+    g = inputs.generator(40 + bits)
+    N, K, G = 300, 1024, 64
+    wq = inputs.random_u32((N, K * bits // 32), g).numpy()
+    s = inputs.random_bf16_bits((N, K // G), g, 100, 140).numpy().view(np.uint16)
+    b = inputs.random_bf16_bits((N, K // G), g, 100, 140).numpy().view(np.uint16)
+    ref = oracle.affine_dequantize(wq.view(np.uint32), s, b, G, bits)
+    out = bq.affine_dequantize(torch.from_numpy(wq).cuda(), torch.from_numpy(s.view(np.int16)).cuda().view(torch.bfloat16),
+                               torch.from_numpy(b.view(np.int16)).cuda().view(torch.bfloat16), G, bits)
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(out), ref)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 6])
+@pytest.mark.parametrize("G", [32, 64, 128])
+def test_affine_quantize_bit_exact_2_3_6_bits(bits, G):
+    N, K = 250, 1024
+    g = inputs.generator(N + bits + G + 1)
+    w = inputs.weights_bf16_valued(N, K, g)
+    w[0, :G] = -0.375                    # constant group: scale 0
+    wq_ref, s_ref, b_ref = oracle.affine_quantize(w.numpy(), G, bits)
+    wq, s, b = bq.affine_quantize(w.cuda(), G, bits)
+    torch.cuda.synchronize()
+    assert np.array_equal(wq.cpu().numpy().view(np.uint32), wq_ref)
+    assert np.array_equal(u16(s), s_ref)
+    assert np.array_equal(u16(b), b_ref)

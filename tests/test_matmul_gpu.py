@@ -288,3 +288,59 @@ def test_q4_0_smallest_k_gemv_and_pair():
     for M in (33, 200):
         check(p, M, "auto")
         check(p, M, "dequant_gemm")
+
+
+# ---------------------------------------------------------------- 2-, 3-, 6-bit affine
+@pytest.mark.parametrize("fmt", ["affine2", "affine3", "affine6", "affine3_g128", "affine6_g32"])
+@pytest.mark.parametrize("M", [1, 8, 33, 300])
+def test_2_3_6_bit_pair(fmt, M):
+    """Widths without a GEMV or fused kernel run as the unfused pair at every M."""
+    N, K = 300, 1024
+    p = Problem(fmt, N, K, seed=M + 11)
+    wq, s, b = p.device()
+    x = p.x(M)
+    assert bq.quant_matmul_select_path(M, N, K, p.group_size, p.bits) == 3
+    y = bq.quant_matmul(x.cuda(), wq, s, b, p.group_size, p.bits)
+    torch.cuda.synchronize()
+    y_ref, a_ref = reference(x, p.wb)
+    assert_within_tolerance(y, y_ref, a_ref, f"{fmt} M={M}")
+
+
+# ---------------------------------------------------------------- transpose = 0
+def _transposed_problem(bits: int, G: int, N: int, K: int, seed: int):
+    """Affine W stored [K][N] (codes and groups along N), quantized by the oracle."""
+    g = inputs.generator(seed)
+    w = inputs.weights_bf16_valued(K, N, g).numpy()
+    wq, sc, bi = oracle.affine_quantize(w, G, bits)
+    wd = oracle.affine_dequantize(wq, sc, bi, G, bits)          # [K][N] bf16 bits
+    dev = (torch.from_numpy(wq.view(np.int32)).cuda(),
+           torch.from_numpy(sc.view(np.int16)).cuda().view(torch.bfloat16),
+           torch.from_numpy(bi.view(np.int16)).cuda().view(torch.bfloat16))
+    return dev, np.ascontiguousarray(wd.T), g                      # reference weight [N][K]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (17, 320, 200), (130, 128, 1032), (300, 192, 64)])
+def test_transpose0(bits, M, N, K):
+    """y = x . W for W stored [K][N]: the pair with a transposing dequantize; K is
+    any multiple of 8 (ragged tiles in both directions)."""
+    (wq, s, b), w_ref, g = _transposed_problem(bits, 64, N, K, seed=bits * 1000 + M + K)
+    x = inputs.activations_bf16(M, K, g)
+    y = bq.quant_matmul(x.cuda(), wq, s, b, 64, bits, transpose=False)
+    torch.cuda.synchronize()
+    assert tuple(y.shape) == (M, N)
+    y_ref, a_ref = reference(x, w_ref)
+    assert_within_tolerance(y, y_ref, a_ref, f"transpose=0 bits={bits} {M}x{N}x{K}")
+
+
+def test_transpose0_group_sizes_and_noalloc():
+    for G, bits in ((32, 4), (128, 8), (32, 3)):
+        (wq, s, b), w_ref, g = _transposed_problem(bits, G, 256, 136, seed=G + bits)
+        x = inputs.activations_bf16(40, 136, g)
+        y = bq.quant_matmul(x.cuda(), wq, s, b, G, bits, transpose=False)
+        out = torch.empty(40, 256, dtype=torch.bfloat16, device="cuda")
+        bq.quant_matmul_noalloc(x.cuda(), wq, s, b, out, G, bits, transpose=False)
+        torch.cuda.synchronize()
+        y_ref, a_ref = reference(x, w_ref)
+        assert_within_tolerance(y, y_ref, a_ref, f"transpose=0 G={G} bits={bits}")
+        assert torch.equal(out.view(torch.int16), y.view(torch.int16))
