@@ -37,8 +37,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from one ncu capture of the
 # current build of each kernel (`ncu --set full`, decode bench command); None for a kernel
 # changed since its counters were taken.
-NCU_TRAFFIC = {"gemv_kernel<Q4_0, M=1>": None, "gemv_kernel<Q4_0, M=8>": None,
-               "gemv_kernel<Q4_0, M=32>": 28598784, "gemv_q8_kernel<M=1>": 28324608}
+NCU_TRAFFIC = {"gemv_kernel<Q4_0, M=1>": 28332800, "gemv_kernel<Q4_0, M=8>": 28389888,
+               "gemv_kernel<Q4_0, M=32>": 28590592, "gemv_q8_kernel<M=1>": 28324608}
 L2_BYTES = 126 * 1024 * 1024
 
 
