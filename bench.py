@@ -372,6 +372,42 @@ def run_prefill(args, world, device, peaks, fmt, Ms):
     return res, total_flops / total_s / 1e12
 
 
+def run_widths(args, world, device, peaks):
+    """Affine 2/3/6-bit weights and transpose=False (W stored [K][N], grouped along N), which run
+    as the unfused pair: the dequantize (bytes moved, GB/s) and quant_matmul's auto path per M."""
+    import torch
+    import bit_quantized_gemm_quant_b200 as bq
+    from bit_quantized_gemm_quant_b200 import inputs
+
+    N, K, G = 12288, 4096, 64
+    ws = torch.empty(N * K, dtype=torch.bfloat16, device=device)
+    res = {}
+    for name, bits, transpose in (("affine2", 2, True), ("affine3", 3, True), ("affine6", 6, True),
+                                  ("affine4_transpose0", 4, False), ("affine3_transpose0", 3, False)):
+        g = inputs.generator(0)
+        w = inputs.weights_bf16_valued(N, K, g) if transpose else inputs.weights_bf16_valued(K, N, g)
+        wq, s, b = bq.affine_quantize(w.to(device), G, bits)
+        del w
+        packed = wq.numel() * 4 + 2 * s.numel() * 2
+        entry = {"bits": bits, "transpose": transpose, "packed_bytes": packed}
+        if transpose:
+            t_dq = kernel_seconds([lambda: bq.affine_dequantize(wq, s, b, G, bits, out=ws.view(N, K))], 20)
+            entry["dequant_us"] = round(t_dq * 1e6, 2)
+            entry["dequant_gbs"] = round((packed + N * K * 2) / t_dq / 1e9, 1)
+        xg = inputs.generator(1)
+        for M in (1, 512, 2048):
+            x = inputs.activations_bf16(M, K, xg).to(device)
+            y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+            flops = 2.0 * M * N * K
+            t = kernel_seconds([lambda: bq.quant_matmul_ex(x, wq, s, b, G, bits, transpose, "auto", workspace=ws,
+                                                           out=y)], max(2, min(50, int(2e13 / flops))))
+            entry[str(M)] = {"us": round(t * 1e6, 2), "tflops": round(flops / t / 1e12, 1),
+                             "frac_tensor": round(flops / t / 1e12 / peaks["bf16_tflops"], 4)}
+            del x, y
+        res[name] = entry
+    return res
+
+
 def run_stack(args, world, device, peaks):
     """Llama-3.2-1B-shaped projection stack, Q4_0: the 112 matmuls of 16 layers (q, k, v, o,
     gate, up, down), each layer with its own weights (547 MB packed > L2), at M = 512 and
@@ -471,7 +507,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["q4_0_decode", "affine4_prefill", "affine8_sweep", "q4_0_prefill",
-                                           "llama1b_stack"],
+                                           "llama1b_stack", "affine_widths"],
                     default="q4_0_decode")
     ap.add_argument("--ms", type=str, default=None, help="comma-separated M list for a prefill workload")
     ap.add_argument("--no-e2e", action="store_true")
@@ -525,6 +561,18 @@ def main(argv=None):
                           "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": per_m["512"]["frac_tensor"],
                           "traffic": None},
              "clocks": clk.summary(), "gpu_launches": launches, "e2e": None}
+    elif args.workload == "affine_widths":
+        with ClockSampler(local_rank) as clk:
+            res = run_widths(args, world, device, peaks)
+        mean = sum(v["2048"]["tflops"] for v in res.values()) / len(res)
+        r = {"value": round(mean, 1), "unit": "TFLOP/s", "ms_per_step": None,
+             "dtype": "affine 2/3/4/6-bit weights, bf16 activations, fp32 accumulate",
+             "config": {"workload": "affine_widths_and_transpose0_g64_n12288_k4096", "M": [1, 512, 2048],
+                        "value": "mean TFLOP/s at M=2048 over the five weight layouts"},
+             "per_format": res,
+             "roofline": {"bound": "tensor", "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                          "frac": round(mean / peaks["bf16_tflops"], 4), "achieved": round(mean, 1), "traffic": None},
+             "clocks": clk.summary(), "gpu_launches": None, "e2e": None}
     else:
         fmt, Ms = {"affine4_prefill": ("affine4", (512, 2048, 8192)),
                    "affine8_sweep": ("affine8", (1, 32, 512, 2048, 8192)),
@@ -548,7 +596,7 @@ def main(argv=None):
             "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": r["dtype"], "data": "synthetic (seeded N(0, 0.02) weights, N(0, 1) bf16 activations)",
             "config": dict(r["config"], parallelism=f"replicas x{world}")}
-    for k in ("per_m", "crossover_m", "roofline", "e2e", "gpu_launches", "clocks", "secondary"):
+    for k in ("per_m", "per_format", "crossover_m", "roofline", "e2e", "gpu_launches", "clocks", "secondary"):
         if k in r:
             line[k] = r[k]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -127,10 +127,11 @@ affine_dequant_kernel(const uint32_t* __restrict__ wq, const uint16_t* __restric
 // ----------------------------------------------------------------------------
 // Affine dequantize with a transposed result: the packed matrix is W[R][C]
 // (codes along C, groups of C), the output its transpose out[C][R] in bf16.
-// One CTA per tile of 32 rows x 64 columns: units are dequantized into a
-// shared tile, which is then written out 16 bytes per thread along R.
+// One CTA per tile of 64 rows x 128 columns: consecutive threads dequantize
+// the same unit column of consecutive rows into a shared tile kept as
+// [column][row], which is then written out 16 bytes per thread along R.
 // ----------------------------------------------------------------------------
-constexpr int kTrRows = 32, kTrCols = 64;
+constexpr int kTrRows = 64, kTrCols = 128;
 
 template <int BITS>
 __global__ void __launch_bounds__(256)
@@ -140,13 +141,13 @@ affine_dequant_t_kernel(const uint32_t* __restrict__ wq, const uint16_t* __restr
 {
     constexpr int W = AffUnit<BITS>::W, E = AffUnit<BITS>::E;
     constexpr int kUnitsPerTileRow = kTrCols / E;
-    __shared__ uint16_t tile[kTrCols][kTrRows + 2];      // [column][row], padded against bank conflicts
+    __shared__ __align__(16) uint16_t tile[kTrCols][kTrRows + 8];   // [column][row]; rows padded by 16 bytes
     const int64_t units_per_row = C / E, groups_per_row = C / group_size;
     const int64_t tiles_r = (R + kTrRows - 1) / kTrRows, tiles_c = (C + kTrCols - 1) / kTrCols;
     for (int64_t t = blockIdx.x; t < tiles_r * tiles_c; t += gridDim.x) {
         const int64_t r0 = (t / tiles_c) * kTrRows, c0 = (t % tiles_c) * kTrCols;
         for (int i = threadIdx.x; i < kTrRows * kUnitsPerTileRow; i += blockDim.x) {
-            const int rr = i / kUnitsPerTileRow, cu = i % kUnitsPerTileRow;
+            const int rr = i % kTrRows, cu = i / kTrRows;    // consecutive threads: consecutive rows
             const int64_t r = r0 + rr, c = c0 + (int64_t)cu * E;
             if (r >= R || c >= C) continue;
             uint32_t w[W];
@@ -159,17 +160,14 @@ affine_dequant_t_kernel(const uint32_t* __restrict__ wq, const uint16_t* __restr
                 tile[cu * E + e][rr] = (uint16_t)f32_to_bf16_bits(__fmaf_rn(s, (float)unit_code<BITS>(w, e), bb));
         }
         __syncthreads();
-        // out[c][r0 .. r0 + 31]: 4 threads per column, 8 rows (16 bytes) each
+        // out[c][r0 .. r0 + 63]: 8 threads per column, 8 rows (16 bytes) each
         for (int i = threadIdx.x; i < kTrCols * (kTrRows / 8); i += blockDim.x) {
             const int cc = i / (kTrRows / 8), rq = (i % (kTrRows / 8)) * 8;
             const int64_t c = c0 + cc, r = r0 + rq;
             if (c >= C || r >= R) continue;
             uint16_t* dst = out + c * R + r;
             if (r + 8 <= R) {
-                uint32_t v[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) v[j] = (uint32_t)tile[cc][rq + 2 * j] | ((uint32_t)tile[cc][rq + 2 * j + 1] << 16);
-                *reinterpret_cast<uint4*>(dst) = make_uint4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&tile[cc][rq]);
             } else {
                 for (int j = 0; j < 8 && r + j < R; ++j) dst[j] = tile[cc][rq + j];
             }

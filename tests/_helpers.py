@@ -11,7 +11,7 @@ from bit_quantized_gemm_quant_b200 import inputs
 FMT = {"q4_0": (32, 4), "affine4": (64, 4), "affine8": (64, 8),
        "affine4_g32": (32, 4), "affine4_g128": (128, 4), "affine8_g32": (32, 8), "affine8_g128": (128, 8),
        "affine2": (64, 2), "affine3": (64, 3), "affine6": (64, 6),
-       "affine2_g32": (32, 2), "affine3_g128": (128, 3), "affine6_g32": (32, 6)}
+       "affine2_g32": (32, 2), "affine3_g32": (32, 3), "affine3_g128": (128, 3), "affine6_g32": (32, 6)}
 
 
 def u16(t: torch.Tensor) -> np.ndarray:

@@ -344,3 +344,38 @@ def test_transpose0_group_sizes_and_noalloc():
         y_ref, a_ref = reference(x, w_ref)
         assert_within_tolerance(y, y_ref, a_ref, f"transpose=0 G={G} bits={bits}")
         assert torch.equal(out.view(torch.int16), y.view(torch.int16))
+
+
+def test_2_3_6_bit_and_transpose0_edges():
+    """Empty and minimal problems for the pair-only layouts; multi falls back to
+    per-matrix calls for 3-bit weights with the same bits as separate calls."""
+    dev = "cuda"
+    for bits in (2, 3, 6):
+        p = Problem(f"affine{bits}_g32", 5, 32, seed=bits)
+        wq, s, b = p.device()
+        for M in (0, 1, 3):
+            x = p.x(M)
+            y = bq.quant_matmul(x.cuda(), wq, s, b, 32, bits)
+            torch.cuda.synchronize()
+            assert tuple(y.shape) == (M, 5)
+            if M:
+                y_ref, a_ref = reference(x, p.wb)
+                assert_within_tolerance(y, y_ref, a_ref, f"bits={bits} M={M} K=32")
+    # transpose=0: empty M, N, and K = 0 (zeros)
+    (wq, s, b), w_ref, g = _transposed_problem(4, 64, 64, 8, seed=5)
+    y = bq.quant_matmul(torch.zeros(0, 8, dtype=torch.bfloat16, device=dev), wq, s, b, 64, 4, transpose=False)
+    assert tuple(y.shape) == (0, 64)
+    x = inputs.activations_bf16(3, 8, g)
+    y = bq.quant_matmul(x.cuda(), wq, s, b, 64, 4, transpose=False)
+    torch.cuda.synchronize()
+    y_ref, a_ref = reference(x, w_ref)
+    assert_within_tolerance(y, y_ref, a_ref, "transpose=0 K=8")
+    # multi with 3-bit weights: per-matrix pair launches, identical to separate calls
+    ps = [Problem("affine3", n, 256, seed=n) for n in (64, 128, 192)]
+    devs = [q.device() for q in ps]
+    x = ps[0].x(4).cuda()
+    outs = bq.quant_matmul_multi(x, devs, 64, 3)
+    for (wq, s, b), o in zip(devs, outs):
+        sep = bq.quant_matmul(x, wq, s, b, 64, 3)
+        torch.cuda.synchronize()
+        assert torch.equal(o.view(torch.int16), sep.view(torch.int16))
