@@ -87,13 +87,6 @@ BQ_DEVINL uint4 ld_shared_v4(uint32_t addr)
     return v;
 }
 
-BQ_DEVINL uint32_t ld_shared_u16(uint32_t addr)
-{
-    unsigned short v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
-    return v;
-}
-
 // ------------------------------------------------------------------ TMA
 BQ_DEVINL void tma_prefetch_desc(const CUtensorMap* map)
 {
@@ -107,14 +100,6 @@ BQ_DEVINL void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];"
         ::"r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y) : "memory");
-}
-
-// 1-D bulk copy global -> this CTA's shared memory (no multicast); completes
-// `bytes` on `bar`.  Addresses and size must be multiples of 16 bytes.
-BQ_DEVINL void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05
@@ -136,27 +121,6 @@ BQ_DEVINL void tmem_dealloc(uint32_t taddr, uint32_t ncols)
 
 BQ_DEVINL void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 BQ_DEVINL void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (bf16 inputs, fp32 accumulate).
-BQ_DEVINL void umma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16.  A (M = 128) occupies TMEM lane m
-// for row m, two bf16 K-consecutive elements per 32-bit column.
-BQ_DEVINL void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
-}
 
 // One 64-element k-block: four K = 16 MMAs into d_tmem.  The B descriptor of
 // sub-step kk is the stage's descriptor with its start address advanced 32 bytes
