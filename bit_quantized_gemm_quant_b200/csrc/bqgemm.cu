@@ -15,6 +15,7 @@
 #include "dequant.cuh"
 #include "gemv.cuh"
 #include "gemv_q8.cuh"
+#include "gemv_affine.cuh"
 #include "tc_gemm.cuh"
 
 namespace bq {
@@ -61,10 +62,12 @@ bq_status current_device(int* dev_out, DeviceInfo* info_out)
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Q4_0, affine 4- and 8-bit (every path), affine 2-, 3- and 6-bit (dequantize,
-// quantize and the unfused pair).
+// quantize, the decode GEMV up to kGaMaxM tokens and the unfused pair).
 enum class WFmt { Q4_0, AFF4, AFF8, AFF2, AFF3, AFF6 };
 
 bool has_fast_paths(WFmt f) { return f == WFmt::Q4_0 || f == WFmt::AFF4 || f == WFmt::AFF8; }
+
+constexpr int64_t kGaMaxM = 8;   // tokens of the decode GEMV for 2-, 3- and 6-bit weights
 
 // Format and shape checks shared by quant_matmul and its helpers (host only):
 // the packed matrix has N rows of K codes, grouped along K.
@@ -145,7 +148,7 @@ const DispatchCfg& dispatch_cfg()
 
 int select_path(int64_t M, int64_t K, WFmt fmt)
 {
-    if (!has_fast_paths(fmt)) return BQ_PATH_DEQUANT_GEMM;
+    if (!has_fast_paths(fmt)) return M <= kGaMaxM ? BQ_PATH_GEMV : BQ_PATH_DEQUANT_GEMM;
     const DispatchCfg& c = dispatch_cfg();
     if (M < c.tc_min_m) return BQ_PATH_GEMV;
     const int64_t pair_min = c.pair_min_m[(int)fmt];
@@ -392,6 +395,33 @@ bq_status launch_gemv(const uint16_t* x, const void* wq, const uint16_t* s, cons
     return launch_gemv_cfg<F, 4, 2, 8, 1, 1>(x, wq, s, b, y, M, N, K, group_size, st);
 }
 
+// Decode GEMV for affine weights of any width (2-, 3- and 6-bit use it), M <= 8.
+bq_status launch_gemv_affine(WFmt fmt, const uint16_t* x, const void* wq, const uint16_t* s, const uint16_t* b,
+                             uint16_t* y, int64_t M, int64_t N, int64_t K, int group_size, cudaStream_t st)
+{
+    if (N > INT32_MAX || K > INT32_MAX || M > kGaMaxM) return BQ_ERR_SHAPE;
+    const int64_t rows_per_cta = (int64_t)kGaRows * kGaWarps;
+    const unsigned grid = (unsigned)((N + rows_per_cta - 1) / rows_per_cta);
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(wq);
+    auto go = [&](auto bits_tag, auto mt_tag) {
+        constexpr int B = decltype(bits_tag)::value, MT = decltype(mt_tag)::value;
+        gemv_affine_kernel<B, MT><<<grid, 32 * kGaWarps, 0, st>>>(x, w, s, b, y, (int)M, (int)N, (int)K, group_size);
+    };
+    auto by_m = [&](auto bits_tag) {
+        if (M <= 1) go(bits_tag, std::integral_constant<int, 1>());
+        else if (M <= 2) go(bits_tag, std::integral_constant<int, 2>());
+        else if (M <= 4) go(bits_tag, std::integral_constant<int, 4>());
+        else go(bits_tag, std::integral_constant<int, 8>());
+    };
+    switch (fmt) {
+    case WFmt::AFF2: by_m(std::integral_constant<int, 2>()); break;
+    case WFmt::AFF3: by_m(std::integral_constant<int, 3>()); break;
+    case WFmt::AFF6: by_m(std::integral_constant<int, 6>()); break;
+    default: return BQ_ERR_UNSUPPORTED;
+    }
+    return launch_status();
+}
+
 template <Fmt F, int NT, int RT, int KS, int PIPE, int MINB>
 bq_status launch_gemv_multi_cfg(const uint16_t* x, GemvMultiTable& tab, int64_t M, int64_t K, int group_size,
                                 cudaStream_t st)
@@ -545,7 +575,8 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
         (workspace && !aligned16(workspace)))
         return BQ_ERR_ALIGN;
     if (path == BQ_PATH_AUTO) path = select_path(M, K, fmt);
-    if (path != BQ_PATH_DEQUANT_GEMM && !has_fast_paths(fmt)) return BQ_ERR_UNSUPPORTED;
+    if (!has_fast_paths(fmt) && (path == BQ_PATH_TC_FUSED || (path == BQ_PATH_GEMV && M > kGaMaxM)))
+        return BQ_ERR_UNSUPPORTED;
     if (path == BQ_PATH_GEMV && M > kGemvMaxM) return BQ_ERR_UNSUPPORTED;
     if (path == BQ_PATH_TC_FUSED && K % 64 != 0) return BQ_ERR_UNSUPPORTED;
     if (path == BQ_PATH_DEQUANT_GEMM && workspace && workspace_bytes < (size_t)N * (size_t)K * 2u)
@@ -558,6 +589,7 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
     const uint16_t* bi = reinterpret_cast<const uint16_t*>(biases);
     switch (path) {
     case BQ_PATH_GEMV:
+        if (!has_fast_paths(fmt)) return launch_gemv_affine(fmt, x, wq, sc, bi, y, M, N, K, group_size, st);
         if (fmt == WFmt::Q4_0) return launch_gemv<Fmt::Q4_0>(x, wq, sc, bi, y, M, N, K, group_size, st);
         if (fmt == WFmt::AFF4) return launch_gemv<Fmt::AFF4>(x, wq, sc, bi, y, M, N, K, group_size, st);
         return launch_gemv<Fmt::AFF8>(x, wq, sc, bi, y, M, N, K, group_size, st);
@@ -782,7 +814,7 @@ bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const void* cons
     }
     if (M == 0) return BQ_OK;
     const int path = select_path(M, K, fmt);
-    if (path != BQ_PATH_GEMV || K == 0) {
+    if (path != BQ_PATH_GEMV || K == 0 || !has_fast_paths(fmt)) {
         // prefill sizes: each matrix through its own launch of the chosen path
         for (int i = 0; i < count; ++i) {
             s = matmul_impl(x_bf16, wq[i], scales[i], biases ? biases[i] : nullptr, y_bf16[i], M, N[i], K,

@@ -181,7 +181,9 @@ BQ_API bq_status quant_matmul_q8(const int8_t* xq, const float* dx, const int32_
  *            of mx.quantized_matmul; it always runs as the unfused pair, W
  *            dequantized into its [N][K] transpose, and needs K % 8 == 0
  *            (BQ_ERR_SHAPE otherwise).  Other values: BQ_ERR_UNSUPPORTED.
- * Affine 2-, 3- and 6-bit weights (either orientation) run as the unfused
+ * Affine 2-, 3- and 6-bit weights have a decode GEMV up to 8 tokens (over the
+ * exact weights scale*q + bias, within the GEMM tolerance of their bf16
+ * roundings) and run as the unfused pair above that; transpose = 0 runs as the
  * pair at every M; 4- and 8-bit and Q4_0 have the decode GEMV and the fused
  * kernel as well.
  * The path is chosen by quant_matmul_select_path.  A path that needs scratch
@@ -249,8 +251,9 @@ BQ_API bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const voi
  * optional caller-owned device workspace.  With workspace == NULL the library's
  * per-device buffer is used as in quant_matmul; otherwise workspace_bytes must
  * be >= quant_matmul_workspace_size(...) (BQ_ERR_WORKSPACE if not).  Forcing
- * BQ_PATH_GEMV with M > 32, or BQ_PATH_GEMV / BQ_PATH_TC_FUSED for 2-, 3- or
- * 6-bit weights or with transpose = 0, returns BQ_ERR_UNSUPPORTED.
+ * BQ_PATH_GEMV with M > 32 (M > 8 for 2-, 3- or 6-bit weights), BQ_PATH_TC_FUSED
+ * for 2-, 3- or 6-bit weights, or either with transpose = 0, returns
+ * BQ_ERR_UNSUPPORTED.
  */
 BQ_API bq_status quant_matmul_ex(const uint16_t* x_bf16, const void* wq, const void* scales, const void* biases,
                           uint16_t* y_bf16, int64_t M, int64_t N, int64_t K, int group_size, int bits,
@@ -270,7 +273,8 @@ BQ_API size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int g
  * pick the dequantize path above some M) and the decode/prefill split of
  * "et-backend: Q4_0 matrix-engine GEMM rewrite for prefill" (Overview: decode
  * routes to the vector-dot kernel).  Returns a bq_path other than AUTO:
- * (transpose = 1; 2-, 3- and 6-bit affine weights always get DEQUANT_GEMM):
+ * (transpose = 1; 2-, 3- and 6-bit affine weights get GEMV up to M = 8 and
+ * DEQUANT_GEMM above):
  *   M <  tc_min_m                 -> BQ_PATH_GEMV        (tc_min_m default 33)
  *   M >= pair_min_m               -> BQ_PATH_DEQUANT_GEMM (pair_min_m by format, from
  *                                    the measured fused/unfused crossovers on B200:

@@ -72,7 +72,7 @@ def test_quant_matmul_rejects_before_launch(L):
     assert qmm(L, b=ALIGNED, g=64, bits=5) == 3               # bits in {2, 3, 4, 6, 8}
     assert qmm(L, b=ALIGNED, g=64, bits=7) == 3
     assert qmm(L, tr=2) == 3
-    assert qmm(L, b=ALIGNED, g=64, bits=3, path=1) == 3       # 2/3/6-bit: the pair only
+    assert qmm(L, b=ALIGNED, g=64, bits=3, path=1) == 3       # 2/3/6-bit: GEMV to M = 8, then the pair
     assert qmm(L, b=ALIGNED, g=64, bits=6, M=64, path=2) == 3
     assert qmm(L, b=ALIGNED, g=64, bits=2, M=64, path=2) == 3
     assert qmm(L, b=ALIGNED, g=64, tr=0, path=1) == 3         # transpose=0: the pair only
@@ -112,9 +112,10 @@ BOUNDARY_M = [1, 2, 8, 19, 31, 32, 33, 63, 64, 65, 127, 128, 129, 383, 384, 385,
 
 def test_dispatcher_pair_only_widths(L):
     for bits in (2, 3, 6):
-        for M in (1, 8, 32, 33, 512, 4096):
-            assert L.quant_matmul_select_path(M, 12288, 4096, 64, bits) == 3
-        assert L.quant_matmul_workspace_size(8, 256, 512, 64, bits, 0) == 256 * 512 * 2
+        for M in (1, 8, 9, 32, 33, 512, 4096):
+            assert L.quant_matmul_select_path(M, 12288, 4096, 64, bits) == (1 if M <= 8 else 3)
+        assert L.quant_matmul_workspace_size(8, 256, 512, 64, bits, 0) == 0              # GEMV
+        assert L.quant_matmul_workspace_size(9, 256, 512, 64, bits, 0) == 256 * 512 * 2  # the pair
         assert L.quant_matmul_workspace_size(8, 256, 512, 64, bits, 2) == 0
 
 

@@ -292,18 +292,34 @@ def test_q4_0_smallest_k_gemv_and_pair():
 
 # ---------------------------------------------------------------- 2-, 3-, 6-bit affine
 @pytest.mark.parametrize("fmt", ["affine2", "affine3", "affine6", "affine3_g128", "affine6_g32"])
-@pytest.mark.parametrize("M", [1, 8, 33, 300])
+@pytest.mark.parametrize("M", [1, 8, 9, 33, 300])
 def test_2_3_6_bit_pair(fmt, M):
-    """Widths without a GEMV or fused kernel run as the unfused pair at every M."""
+    """2/3/6-bit widths: the any-width decode GEMV up to 8 tokens, the unfused pair
+    above (and at every M when forced)."""
     N, K = 300, 1024
     p = Problem(fmt, N, K, seed=M + 11)
     wq, s, b = p.device()
     x = p.x(M)
-    assert bq.quant_matmul_select_path(M, N, K, p.group_size, p.bits) == 3
-    y = bq.quant_matmul(x.cuda(), wq, s, b, p.group_size, p.bits)
+    assert bq.quant_matmul_select_path(M, N, K, p.group_size, p.bits) == (1 if M <= 8 else 3)
+    y_ref, a_ref = reference(x, p.wb)
+    for path in (["auto", "gemv", "dequant_gemm"] if M <= 8 else ["auto"]):
+        y = bq.quant_matmul_ex(x.cuda(), wq, s, b, p.group_size, p.bits, True, path)
+        torch.cuda.synchronize()
+        assert_within_tolerance(y, y_ref, a_ref, f"{fmt} M={M} {path}")
+
+
+@pytest.mark.parametrize("bits", [2, 3, 6])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("N,K", [(1, 32), (17, 96), (250, 2048)])
+def test_affine_any_width_gemv(bits, M, N, K):
+    """Every token-count template and ragged row groups of the any-width GEMV."""
+    p = Problem(f"affine{bits}_g32", N, K, seed=bits * 100 + M + N)
+    wq, s, b = p.device()
+    x = p.x(M)
+    y = bq.quant_matmul_ex(x.cuda(), wq, s, b, 32, bits, True, "gemv")
     torch.cuda.synchronize()
     y_ref, a_ref = reference(x, p.wb)
-    assert_within_tolerance(y, y_ref, a_ref, f"{fmt} M={M}")
+    assert_within_tolerance(y, y_ref, a_ref, f"bits={bits} M={M} {N}x{K}")
 
 
 # ---------------------------------------------------------------- transpose = 0

@@ -47,7 +47,7 @@ def test_random_transpose1(case):
     y_ref, a_ref = reference(x, wb)
     fast = kind == "q4_0" or bits in (4, 8)
     paths = ["auto", "dequant_gemm"]
-    if fast and M <= 32:
+    if (fast and M <= 32) or (not fast and M <= 8):
         paths.append("gemv")
     if fast and K % 64 == 0:
         paths.append("tc_fused")
