@@ -329,8 +329,11 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
 
     static bool attr_done[kMaxDevices] = {};
     if (!attr_done[dev]) {
-        if (cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 di.max_smem_optin) != cudaSuccess)
+        if (cudaFuncSetAttribute(tc_gemm_kernel<MODE, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 di.max_smem_optin) != cudaSuccess ||
+            (MODE != kModeBF16 && cudaFuncSetAttribute(tc_gemm_kernel<MODE, MODE != kModeBF16>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       di.max_smem_optin) != cudaSuccess))
             return BQ_ERR_CUDA;
         attr_done[dev] = true;
     }
@@ -358,7 +361,10 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
         p.vec_scales = ((K >> p.gs_shift) % 8 == 0) ? 1 : 0;   // every row starts and ends on whole windows
     }
     const unsigned grid = (unsigned)std::min<int64_t>(tiles * pl.splits, di.num_sms);
-    tc_gemm_kernel<MODE><<<grid, C::kThreads, smem, st>>>(tm_x, tm_a, p);
+    if (MODE != kModeBF16 && pl.num_acc == 1)
+        tc_gemm_kernel<MODE, MODE != kModeBF16><<<grid, C::kThreads, smem, st>>>(tm_x, tm_a, p);
+    else
+        tc_gemm_kernel<MODE, false><<<grid, C::kThreads, smem, st>>>(tm_x, tm_a, p);
     if (pl.splits > 1) {
         bq_status r = launch_status();
         if (r != BQ_OK) return r;

@@ -209,7 +209,10 @@ BQ_DEVINL DeqScale window_scale(const ScaleWindow& w, int k)
     return r;
 }
 
-template <int MODE>
+// ONE_ACC: one TMEM accumulator (p.num_acc == 1), the next tile waiting for
+// each drain; otherwise two, the drain overlapping the next tile.  A template
+// argument, so that each kernel carries only its own epilogue.
+template <int MODE, bool ONE_ACC>
 __global__ void __launch_bounds__(TcCfg<MODE>::kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a, TcParams p)
 {
@@ -235,10 +238,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     const uint32_t mma_done_bar = bar_base + 8u * (uint32_t)(3 * S + 4);
     // TMEM columns: accumulators at 0 (and acc_stride); fused modes keep stage s of
     // the dequantized weight tile (128 lanes x 64 bf16 = 32 columns) after them.
-    auto a_tmem_col = [&](int s) { return (uint32_t)(p.num_acc * p.acc_stride) + 32u * (uint32_t)s; };
+    constexpr int kNumAcc = ONE_ACC ? 1 : 2;
+    auto a_tmem_col = [&](int s) { return (uint32_t)(kNumAcc * p.acc_stride) + 32u * (uint32_t)s; };
     // Accumulator of the lt-th local tile and the parity of its use count.
-    auto acc_of = [&](int lt) { return p.num_acc == 2 ? (lt & 1) : 0; };
-    auto acc_phase = [&](int lt) { return (uint32_t)(p.num_acc == 2 ? (lt >> 1) : lt) & 1u; };
+    auto acc_of = [&](int lt) { return ONE_ACC ? 0 : (lt & 1); };
+    auto acc_phase = [&](int lt) { return (uint32_t)(ONE_ACC ? lt : (lt >> 1)) & 1u; };
     const uint32_t tmem_slot = mma_done_bar + 8u;
     uint8_t* smem_gen = smem_raw + (base - smem_u32(smem_raw));
     volatile uint32_t* tmem_slot_ptr = reinterpret_cast<volatile uint32_t*>(smem_gen + (tmem_slot - base));
@@ -403,6 +407,32 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         if (row_ok && mb + j < p.M) part[(int64_t)(mb + j) * p.N + row] = __uint_as_float(v[j]);
+                });
+            } else if constexpr (ONE_ACC) {
+                // One accumulator: the next tile waits for this drain, so it is kept
+                // short -- two tokens per conversion, and a whole 16-token chunk
+                // (the warp-uniform common case) stores without per-token checks.
+                // (With two accumulators the drain overlaps the next tile, and the
+                // per-token form below, which issues its stores more evenly,
+                // measured faster.)
+                const uint64_t ld_bytes = (uint64_t)p.N * 2u;
+                drain([&](const uint32_t (&v)[16], int mb) {
+                    if (!row_ok) return;
+                    uint16_t* py = p.y + (int64_t)mb * p.N + row;
+                    if (mb + 16 <= p.M) {
+#pragma unroll
+                        for (int j = 0; j < 16; j += 2) {
+                            const uint32_t pk = pack_bf16x2_rn(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                            char* a = reinterpret_cast<char*>(py) + (uint64_t)j * ld_bytes;
+                            *reinterpret_cast<uint16_t*>(a) = (uint16_t)(pk & 0xFFFFu);
+                            *reinterpret_cast<uint16_t*>(a + ld_bytes) = (uint16_t)(pk >> 16);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (mb + j < p.M)
+                                py[(int64_t)j * p.N] = (uint16_t)f32_to_bf16_bits(__uint_as_float(v[j]));
+                    }
                 });
             } else {
                 drain([&](const uint32_t (&v)[16], int mb) {
