@@ -118,11 +118,11 @@ int grid_for(int64_t items, int threads, const DeviceInfo& di)
 
 // ------------------------------------------------------------------ env config
 // Default fused/pair thresholds per format, from B200 sweeps of the 12288 x 4096
-// projection at M = 256 .. 8192: the fused kernel leads up to 2048 tokens for
-// Q4_0 and affine 4-bit (180 / 183 vs 187 us at 2048), ties the pair at 2560
-// and trails from 3072; for affine 8-bit the fused kernel leads at 256 and 768,
-// the pair at 384, 512 and from 1024, so the pair is taken from 384.
-constexpr int64_t kDefaultPairMinM[3] = {2560, 2560, 384};   // Q4_0, affine4, affine8
+// projection at M = 256 .. 8192: the fused kernel leads up to 3072 tokens for
+// Q4_0 and affine 4-bit (241 / 247 vs 252 us at 3072) and trails from 4096;
+// for affine 8-bit it leads at 256, 512, 768 and 1024 and trails from 2048 (and
+// at 384, where 192-token tiles fill 1.3 rounds of the SMs: 69 vs 66 us).
+constexpr int64_t kDefaultPairMinM[3] = {4096, 4096, 2048};   // Q4_0, affine4, affine8
 
 struct DispatchCfg {
     int tc_min_m = kGemvMaxM + 1;

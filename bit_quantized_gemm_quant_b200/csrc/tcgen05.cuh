@@ -68,15 +68,15 @@ BQ_DEVINL bool mbar_wait(uint32_t bar, uint32_t parity)
     return true;
 }
 
-// Warp-level wait: lane 0 polls the barrier, then __syncwarp orders every lane
-// of the warp after lane 0's acquire; 32 pollers per warp become one.
+// Warp-level wait: every lane polls.  A poll is one warp instruction either way,
+// all lanes see the same phase state from it (so they leave the loop together and
+// each lane holds its own acquire), and no result has to be broadcast -- a lane-0
+// poll followed by a shuffle measured 6-14% slower in the fused kernel.
 BQ_DEVINL bool mbar_wait_warp(uint32_t bar, uint32_t parity)
 {
-    uint32_t ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity) ? 1u : 0u;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
+    const bool ok = mbar_wait(bar, parity);
     __syncwarp();
-    return ok != 0;
+    return ok;
 }
 
 BQ_DEVINL uint4 ld_shared_v4(uint32_t addr)

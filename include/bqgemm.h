@@ -278,7 +278,7 @@ BQ_API size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int g
  *   M <  tc_min_m                 -> BQ_PATH_GEMV        (tc_min_m default 33)
  *   M >= pair_min_m               -> BQ_PATH_DEQUANT_GEMM (pair_min_m by format, from
  *                                    the measured fused/unfused crossovers on B200:
- *                                    2560 for Q4_0 and affine 4-bit, 384 for 8-bit)
+ *                                    4096 for Q4_0 and affine 4-bit, 2048 for 8-bit)
  *   otherwise                     -> BQ_PATH_TC_FUSED when K % 64 == 0,
  *                                    else BQ_PATH_DEQUANT_GEMM
  * Environment overrides, read once per process: BQ_TC_MIN_M (clamped to

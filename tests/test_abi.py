@@ -107,7 +107,7 @@ def test_other_entry_points_reject_before_launch(L):
 
 
 BOUNDARY_M = [1, 2, 8, 19, 31, 32, 33, 63, 64, 65, 127, 128, 129, 383, 384, 385, 511, 512, 513, 1023, 1024, 1025,
-              2047, 2048, 2559, 2560, 2561, 8192]
+              2047, 2048, 2049, 4095, 4096, 4097, 8192]
 
 
 def test_dispatcher_pair_only_widths(L):
@@ -123,7 +123,7 @@ def test_dispatcher_boundaries(L):
     for M in BOUNDARY_M:
         for g, bits in ((32, 4), (64, 4), (64, 8)):
             p = L.quant_matmul_select_path(M, 12288, 4096, g, bits)
-            pair_min = 384 if bits == 8 else 2560
+            pair_min = 2048 if bits == 8 else 4096
             assert p == (1 if M <= 32 else 2 if M < pair_min else 3), (M, g, bits, p)
     # K % 64 != 0 (Q4_0 only): prefill goes through the unfused pair
     assert L.quant_matmul_select_path(512, 256, 544, 32, 4) == 3
@@ -145,7 +145,7 @@ def _select_in_subprocess(env_extra, Ms):
 
 def test_dispatcher_env_overrides(L):
     Ms = [1, 8, 19, 32, 33, 512, 4096]
-    assert _select_in_subprocess({}, Ms) == [1, 1, 1, 1, 2, 2, 3]             # affine 4-bit: pair from 2560
+    assert _select_in_subprocess({}, Ms) == [1, 1, 1, 1, 2, 2, 3]             # affine 4-bit: pair from 4096
     assert _select_in_subprocess({"BQ_TC_MIN_M": "8"}, Ms) == [1, 2, 2, 2, 2, 2, 3]
     assert _select_in_subprocess({"BQ_TC_MIN_M": "1000"}, Ms) == [1, 1, 1, 1, 2, 2, 3]   # clamped to 33
     assert _select_in_subprocess({"BQ_PAIR_MIN_M": "512"}, Ms) == [1, 1, 1, 1, 2, 3, 3]
