@@ -344,7 +344,7 @@ def run_prefill(args, world, device, peaks, fmt, Ms):
         x = inputs.activations_bf16(M, K, g).to(device)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
         flops = 2.0 * M * N * K
-        reps = max(2, min(50, int(2e13 / flops)))
+        reps = max(10, min(50, int(2e13 / flops)))
         fused_path = "tc_fused" if M > 32 else "gemv"
         t_fused = kernel_seconds([lambda: bq.quant_matmul_ex(x, wq, s, b, gs, bits, True, fused_path, out=y)], reps)
         t_auto = kernel_seconds([lambda: bq.quant_matmul_ex(x, wq, s, b, gs, bits, True, "auto", workspace=ws,
@@ -400,7 +400,7 @@ def run_widths(args, world, device, peaks):
             y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
             flops = 2.0 * M * N * K
             t = kernel_seconds([lambda: bq.quant_matmul_ex(x, wq, s, b, G, bits, transpose, "auto", workspace=ws,
-                                                           out=y)], max(2, min(50, int(2e13 / flops))))
+                                                           out=y)], max(10, min(50, int(2e13 / flops))))
             entry[str(M)] = {"us": round(t * 1e6, 2), "tflops": round(flops / t / 1e12, 1),
                              "frac_tensor": round(flops / t / 1e12 / peaks["bf16_tflops"], 4)}
             del x, y
