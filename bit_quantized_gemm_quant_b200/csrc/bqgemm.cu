@@ -118,10 +118,10 @@ int grid_for(int64_t items, int threads, const DeviceInfo& di)
 
 // ------------------------------------------------------------------ env config
 // Default fused/pair thresholds per format, from B200 sweeps of the 12288 x 4096
-// projection at M = 256 .. 8192: the fused kernel leads up to 3072 tokens for
-// Q4_0 and affine 4-bit (241 / 247 vs 252 us at 3072) and trails from 4096;
-// for affine 8-bit it leads at 256, 512, 768 and 1024 and trails from 2048 (and
-// at 384, where 192-token tiles fill 1.3 rounds of the SMs: 69 vs 66 us).
+// projection at M = 256 .. 8192 (20 graph-captured calls per timing): the fused
+// kernel leads up to 3072 tokens for Q4_0 and affine 4-bit (230 / 236 vs 243 us
+// at 3072), ties or trails from 4096; for affine 8-bit it leads up to 1024 tokens
+// and trails from 2048 (192 vs 182 us).
 constexpr int64_t kDefaultPairMinM[3] = {4096, 4096, 2048};   // Q4_0, affine4, affine8
 
 struct DispatchCfg {
@@ -215,10 +215,15 @@ int choose_bn(int64_t M, int64_t N, int num_sms, int max_bn, int overhead)
 struct TcPlan {
     int bn = 0, num_acc = 2, acc_stride = 0, stages = 0, splits = 1;
     int64_t tiles = 0;
+    int64_t dp_tiles = 0;     // tiles run whole; the rest are split `splits` ways
     size_t ws_bytes = 0;      // fp32 partials needed when splits > 1
 };
 
-int64_t splitk_stride(int64_t M, int64_t N) { return (M * N + 3) / 4 * 4; }   // floats per split, 16-byte multiple
+// fp32 partial sums of the split tiles: one bn x 128 tile per split and tile
+size_t splitk_ws_bytes(int splits, int64_t split_tiles, int bn)
+{
+    return splits > 1 ? (size_t)splits * (size_t)split_tiles * (size_t)bn * 128u * 4u : 0u;
+}
 
 template <int MODE>
 bool plan_tc(int64_t M, int64_t N, int64_t K, int num_sms, int smem_optin, TcPlan* pl)
@@ -227,6 +232,7 @@ bool plan_tc(int64_t M, int64_t N, int64_t K, int num_sms, int smem_optin, TcPla
     const int64_t wtiles = (N + 127) / 128;
     const int64_t nk = (K + 63) / 64;
     int bn, num_acc = 2, splits = 1;
+    int64_t dp_tiles = 0;
     if (!kFused) {
         bn = choose_bn(M, N, num_sms, 256, 32);
     } else {
@@ -235,31 +241,49 @@ bool plan_tc(int64_t M, int64_t N, int64_t K, int num_sms, int smem_optin, TcPla
         // hand-offs dominate, about 0.55 us on B200), so wide tiles are preferred
         // and the SMs are filled by splitting K.  Joint search over the tile width
         // (two TMEM accumulators up to 192 tokens, one at 256, whose epilogue does
-        // not overlap the next tile: weight 1.12) and the split count, in k-block
-        // units:
-        //   cost = rounds(units) x (k-blocks per unit + 4) x w
-        //        + [split] (4 + fp32 partial traffic 8 x splits x M x N bytes at HBM speed)
-        // Ties go to the wider tile.
+        // not overlap the next tile: weight 1.12) and the K split, in k-block units.
+        // Two forms of split: every tile split sp ways, or whole tiles for the
+        // whole rounds of the grid and only the remaining tiles split (sp x their
+        // count <= one round), so that they fill the last round instead of leaving
+        // most SMs idle in it.
+        //   cost = rounds x (k-blocks per unit + 4) x w
+        //        + [split] (4 + fp32 partial traffic 8 x sp x split tiles x bn x 128 bytes at HBM speed)
+        // The second form's cost carries 5% more: a last round that leaves most
+        // SMs idle runs faster per tile than a full one, which the rounds count
+        // does not see (on B200 it paid at 512 and 2048 tokens of the 12288 x 4096
+        // projection, predicted 12% and 9% cheaper, and not at 4096, predicted 3%).
+        // Ties go to the wider tile, then to the form found first.
         double best = 1e300;
         bn = 16;
         const int64_t maxb = std::min<int64_t>(256, (M + 15) / 16 * 16);
+        auto consider = [&](double c, int b, int acc, int sp, int64_t dp) {
+            if (c < best - 1e-9 || (c < best + 1e-9 && b > bn)) {
+                best = c;
+                bn = b;
+                num_acc = acc;
+                splits = sp;
+                dp_tiles = dp;
+            }
+        };
         for (int b = 16; b <= maxb; b += 16) {
             if (b > 192 && b < maxb && b != 256) continue;      // one accumulator: only the widest tile
             const int acc = b > 192 ? 1 : 2;
             const double w = acc == 1 ? 1.12 : 1.0;
             const int64_t tiles = ((M + b - 1) / b) * wtiles;
-            for (int sp = 1; sp <= 8; ++sp) {
+            const double tile_elems = (double)b * 128.0;
+            for (int sp = 1; sp <= 8; ++sp) {                   // every tile split sp ways
                 if (sp > 1 && nk / sp < 4) break;
-                const int64_t units = tiles * sp;
-                const int64_t rounds = (units + num_sms - 1) / num_sms;
-                const double reduce = sp > 1 ? 4.0 + (double)sp * (double)M * (double)N * 2.24e-6 : 0.0;
-                const double c = (double)rounds * (double)((nk + sp - 1) / sp + 4) * w + reduce;
-                if (c < best - 1e-9 || (c < best + 1e-9 && b > bn)) {
-                    best = c;
-                    bn = b;
-                    num_acc = acc;
-                    splits = sp;
-                }
+                const int64_t rounds = (tiles * sp + num_sms - 1) / num_sms;
+                const double reduce = sp > 1 ? 4.0 + (double)sp * (double)tiles * tile_elems * 2.24e-6 : 0.0;
+                consider((double)rounds * (double)((nk + sp - 1) / sp + 4) * w + reduce, b, acc, sp,
+                         sp > 1 ? 0 : tiles);
+            }
+            const int64_t dp = tiles / num_sms * num_sms, tail = tiles - dp;
+            for (int sp = 2; dp > 0 && tail > 0 && sp <= 8 && tail * sp <= num_sms; ++sp) {   // only the tail split
+                if (nk / sp < 4) break;
+                const double c = (double)(dp / num_sms) * (double)(nk + 4) * w + (double)((nk + sp - 1) / sp + 4) * w +
+                                 4.0 + (double)sp * (double)tail * tile_elems * 2.24e-6;
+                consider(c * 1.05, b, acc, sp, dp);
             }
         }
     }
@@ -275,29 +299,42 @@ bool plan_tc(int64_t M, int64_t N, int64_t K, int num_sms, int smem_optin, TcPla
     pl->stages = stages;
     pl->tiles = ((M + bn - 1) / bn) * wtiles;
     pl->splits = splits;
-    pl->ws_bytes = splits > 1 ? (size_t)splits * (size_t)splitk_stride(M, N) * 4u : 0u;
+    pl->dp_tiles = splits > 1 ? dp_tiles : pl->tiles;
+    pl->ws_bytes = splitk_ws_bytes(splits, pl->tiles - pl->dp_tiles, bn);
     return true;
 }
 
-// y = bf16(sum over splits of ws[split]) in split order (deterministic).
-__global__ void splitk_reduce_kernel(const float* __restrict__ ws, uint16_t* __restrict__ y, int64_t mn,
-                                     int64_t stride, int splits)
+// y = bf16(sum over splits of the partials) for the split tiles, in split order
+// (deterministic).  Partials: [split][split tile][token of the tile][weight row of
+// the tile]; one thread per 4 rows of one token (16-byte loads; 8-byte stores
+// when N % 4 == 0 -- y and ws are 16-byte aligned).
+__global__ void splitk_reduce_kernel(const float* __restrict__ ws, uint16_t* __restrict__ y, int M, int N, int bn,
+                                     int m_tiles, int dp_tiles, int split_tiles, int splits)
 {
-    const int64_t n4 = mn / 4;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
-        float4 a = reinterpret_cast<const float4*>(ws)[i];
+    const int64_t per_tile = (int64_t)bn * 32;                       // 4-row groups per tile
+    const int64_t total = (int64_t)split_tiles * per_tile;
+    const int64_t split_stride = (int64_t)split_tiles * bn * 128;   // floats
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int j = (int)(i / per_tile);
+        const int e = (int)(i - (int64_t)j * per_tile);
+        const int m = e >> 5, r4 = (e & 31) * 4;
+        const int t = dp_tiles + j;
+        const int tok = (t % m_tiles) * bn + m, row = (t / m_tiles) * 128 + r4;
+        if (tok >= M || row >= N) continue;
+        const float* src = ws + ((int64_t)j * bn + m) * 128 + r4;
+        float4 a = *reinterpret_cast<const float4*>(src);
         for (int sp = 1; sp < splits; ++sp) {
-            const float4 b = reinterpret_cast<const float4*>(ws + sp * stride)[i];
+            const float4 b = *reinterpret_cast<const float4*>(src + sp * split_stride);
             a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
         }
-        reinterpret_cast<uint2*>(y)[i] = make_uint2(pack_bf16x2_rn(a.x, a.y), pack_bf16x2_rn(a.z, a.w));
-    }
-    if (blockIdx.x == 0)
-        for (int64_t i = n4 * 4 + threadIdx.x; i < mn; i += blockDim.x) {
-            float a = ws[i];
-            for (int sp = 1; sp < splits; ++sp) a += ws[sp * stride + i];
-            y[i] = (uint16_t)f32_to_bf16_bits(a);
+        uint16_t* dst = y + (int64_t)tok * N + row;
+        if ((N & 3) == 0) {                                          // then row + 4 <= N
+            *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2_rn(a.x, a.y), pack_bf16x2_rn(a.z, a.w));
+        } else {
+            const float v[4] = {a.x, a.y, a.z, a.w};
+            for (int k = 0; k < 4 && row + k < N; ++k) dst[k] = (uint16_t)f32_to_bf16_bits(v[k]);
         }
+    }
 }
 
 template <int MODE>
@@ -310,7 +347,10 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     TcPlan pl;
     if (!plan_tc<MODE>(M, N, K, di.num_sms, di.max_smem_optin, &pl)) return BQ_ERR_UNSUPPORTED;
     // K splits only with a workspace that holds their partial sums
-    if (pl.splits > 1 && (!ws || ws_bytes < pl.ws_bytes)) pl.splits = 1;
+    if (pl.splits > 1 && (!ws || ws_bytes < pl.ws_bytes)) {
+        pl.splits = 1;
+        pl.dp_tiles = pl.tiles;
+    }
     const int bn = pl.bn, stages = pl.stages;
     const uint32_t stage = tc_stage_bytes(MODE, bn);
     // one CTA per SM: the kernel allocates all 512 TMEM columns
@@ -353,14 +393,15 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     p.acc_stride = pl.acc_stride;
     p.num_acc = pl.num_acc;
     p.splits = pl.splits;
+    p.dp_tiles = (int)pl.dp_tiles;
     p.ws = pl.splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
-    p.ws_stride = splitk_stride(M, N);
     {
         const int gs = (MODE == kModeQ4_0 || MODE == kModeBF16) ? 32 : group_size;
         p.gs_shift = gs == 32 ? 5 : gs == 64 ? 6 : 7;
         p.vec_scales = ((K >> p.gs_shift) % 8 == 0) ? 1 : 0;   // every row starts and ends on whole windows
     }
-    const unsigned grid = (unsigned)std::min<int64_t>(tiles * pl.splits, di.num_sms);
+    const int64_t units = pl.dp_tiles + (tiles - pl.dp_tiles) * pl.splits;
+    const unsigned grid = (unsigned)std::min<int64_t>(units, di.num_sms);
     if (MODE != kModeBF16 && pl.num_acc == 1)
         tc_gemm_kernel<MODE, MODE != kModeBF16><<<grid, C::kThreads, smem, st>>>(tm_x, tm_a, p);
     else
@@ -368,9 +409,11 @@ bq_status launch_tc(const DeviceInfo& di, int dev, const uint16_t* x, const void
     if (pl.splits > 1) {
         bq_status r = launch_status();
         if (r != BQ_OK) return r;
-        const int64_t mn = M * N;
-        const unsigned rgrid = (unsigned)std::max<int64_t>(1, std::min<int64_t>((mn / 4 + 255) / 256, 4 * di.num_sms));
-        splitk_reduce_kernel<<<rgrid, 256, 0, st>>>(p.ws, y, mn, splitk_stride(M, N), pl.splits);
+        const int64_t split_tiles = tiles - pl.dp_tiles;
+        const int64_t groups = split_tiles * bn * 32;
+        const unsigned rgrid = (unsigned)std::max<int64_t>(1, std::min<int64_t>((groups + 255) / 256, 4 * di.num_sms));
+        splitk_reduce_kernel<<<rgrid, 256, 0, st>>>(p.ws, y, (int)M, (int)N, bn, p.m_tiles, p.dp_tiles,
+                                                    (int)split_tiles, pl.splits);
     }
     return launch_status();
 }

@@ -67,9 +67,10 @@ struct TcParams {
     int num_acc;              // 2: the epilogue drains one tile while the next accumulates; 1: bn up to 256
     int gs_shift;             // log2 of the group size (Q4_0: 5; affine: 5, 6 or 7)
     int vec_scales;           // scale rows are 16-byte aligned and hold whole 8-group windows
-    int splits;               // K splits per tile (fused modes); > 1: fp32 partials to ws
-    float* ws;                // [splits][M][N] fp32 partial sums when splits > 1
-    int64_t ws_stride;        // floats between consecutive splits' partials
+    int dp_tiles;             // tiles [0, dp_tiles) run whole, one unit each
+    int splits;               // K splits of each later tile (fused modes); > 1: fp32 partials to ws
+    float* ws;                // fp32 partials of the split tiles when splits > 1:
+                              // [split][tile - dp_tiles][token of the tile (bn)][weight row of the tile (128)]
 };
 
 // Shared memory per pipeline stage: the activation tile (bn x 64 bf16, 128B
@@ -248,13 +249,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     volatile uint32_t* tmem_slot_ptr = reinterpret_cast<volatile uint32_t*>(smem_gen + (tmem_slot - base));
     auto tile_n0 = [&](int t) { return (t / p.m_tiles) * 128; };
     auto tile_m0 = [&](int t) { return (t % p.m_tiles) * p.bn; };
-    // Work units: unit u is tile u / splits over the k-blocks [kb_begin(u), kb_end(u))
-    // of K split u % splits (splits == 1: whole tiles).
-    const int units = p.tiles * p.splits;
-    auto unit_tile = [&](int u) { return u / p.splits; };
+    // Work units: units [0, dp_tiles) are whole tiles.  Each later tile t is split
+    // over K into p.splits units; unit dp_tiles + (t - dp_tiles) * splits + s takes
+    // the k-blocks [kb_begin, kb_end) of split s.  With dp_tiles a whole number of
+    // rounds of the grid, the split tiles fill the last round (dp_tiles == 0: every
+    // tile is split; splits == 1: every tile is whole).
+    const int units = p.dp_tiles + (p.tiles - p.dp_tiles) * p.splits;
+    auto unit_tile = [&](int u) { return u < p.dp_tiles ? u : p.dp_tiles + (u - p.dp_tiles) / p.splits; };
+    auto unit_split = [&](int u) { return u < p.dp_tiles ? 0 : (u - p.dp_tiles) % p.splits; };
     // (nk < 2^24 and splits <= 8: the products fit 32-bit arithmetic)
-    auto kb_begin = [&](int u) { return p.splits == 1 ? 0 : (u % p.splits) * nk / p.splits; };
-    auto kb_end = [&](int u) { return p.splits == 1 ? nk : (u % p.splits + 1) * nk / p.splits; };
+    auto kb_begin = [&](int u) { return u < p.dp_tiles ? 0 : unit_split(u) * nk / p.splits; };
+    auto kb_end = [&](int u) { return u < p.dp_tiles ? nk : (unit_split(u) + 1) * nk / p.splits; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -380,7 +385,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc_fence_after();
             const int row = tile_n0(t) + 32 * q4 + lane;
             const int m0 = tile_m0(t);
-            float* part = p.splits > 1 ? p.ws + (int64_t)(u % p.splits) * p.ws_stride : nullptr;
+            // a split unit's partial tile: [token of the tile][weight row of the tile]
+            float* part = (p.splits > 1 && u >= p.dp_tiles)
+                              ? p.ws + ((int64_t)unit_split(u) * (p.tiles - p.dp_tiles) + (t - p.dp_tiles)) *
+                                           ((int64_t)p.bn * 128) + 32 * q4 + lane
+                              : nullptr;
             const uint32_t lane_addr = tmem_base + ((uint32_t)(32 * q4) << 16) + (uint32_t)(acc * p.acc_stride);
             // 16 columns (tokens) per TMEM load; the next load is in flight while
             // this chunk is converted and stored (wait::ld waits for all loads).
@@ -403,10 +412,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             // warp-collective, so every lane takes part; lanes past N only skip stores.
             const bool row_ok = row < p.N;
             if (part) {                                               // K split: fp32 partial sums
+                // every token and row of the tile (the reduce skips those past M and N);
+                // a warp's 32 rows of one token are one 128-byte line
                 drain([&](const uint32_t (&v)[16], int mb) {
+                    float* pt = part + (int64_t)(mb - m0) * 128;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (row_ok && mb + j < p.M) part[(int64_t)(mb + j) * p.N + row] = __uint_as_float(v[j]);
+                    for (int j = 0; j < 16; ++j) pt[j * 128] = __uint_as_float(v[j]);
                 });
             } else if constexpr (ONE_ACC) {
                 // One accumulator: the next tile waits for this drain, so it is kept

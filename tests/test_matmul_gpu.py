@@ -70,11 +70,16 @@ def _sample_rows(M, n=64, seed=0):
     return rows
 
 
-@pytest.mark.parametrize("M", [512, 2048, 8192])
-def test_affine4_prefill_config_sampled(M):
-    p = Problem("affine4", 12288, 4096)
+@pytest.mark.parametrize("fmt,M", [("affine4", 512), ("affine4", 2048), ("affine4", 8192),
+                                   ("q4_0", 512), ("q4_0", 2048), ("q4_0", 4096)])
+def test_prefill_config_sampled(fmt, M):
+    """The 12288 x 4096 projection at prefill sizes: the fused kernel's plans
+    there (split tail tiles at 512 and 2048 tokens, whole tiles at 4096 and
+    8192) and the pair."""
+    p = Problem(fmt, 12288, 4096)
     rows = _sample_rows(M)
     check(p, M, "auto", rows)
+    check(p, M, "tc_fused", rows)
     check(p, M, "dequant_gemm", rows)
 
 
@@ -263,6 +268,41 @@ def test_split_k_with_caller_workspace(fmt):
         y = bq.quant_matmul_ex(xd, wq, s, b, p.group_size, p.bits, True, "tc_fused", workspace=ws)
         torch.cuda.synchronize()
         assert_within_tolerance(y, y_ref, a_ref, f"{fmt} ws={None if ws is None else ws.numel()}")
+
+
+@pytest.mark.parametrize("fmt,M,N,K,sampled", [
+    ("q4_0", 64, 19160, 1024, False),      # 150 tiles of 64 tokens: 148 whole, 2 split 4 ways
+    ("affine4", 100, 18950, 1024, False),  # 149 tiles of 112 tokens (ragged), N % 4 == 2
+    ("affine8", 400, 9750, 1024, True),    # one accumulator, 256-token tiles: 6 split tiles, ragged M and N
+    ("affine4", 400, 9750, 1024, True),
+    ("q4_0", 200, 19750, 1024, False),     # one accumulator, a 208-token tile
+])
+def test_split_tail_tiles(fmt, M, N, K, sampled):
+    """More tiles than SMs: whole tiles fill the whole rounds and only the last
+    round's tiles are split over K, their fp32 partials reduced in split order.
+    The reported workspace holds only the split tiles' partials (every-tile
+    splitting needs at least 2 x M x N x 4 bytes); with it, with one too small
+    (no split) and with the library's, the result agrees with the oracle, and
+    repeated runs are bit-identical."""
+    p = Problem(fmt, N, K, seed=M + N)
+    need = bq.quant_matmul_workspace_size(M, N, K, p.group_size, p.bits, "tc_fused")
+    assert 0 < need < 2 * M * N * 4, need
+    wq, s, b = p.device()
+    x = p.x(M)
+    rows = _sample_rows(M) if sampled else None
+    y_ref, a_ref = reference(x, p.wb, rows)
+    xd = x.cuda()
+    outs = []
+    for ws in (torch.empty(need, dtype=torch.uint8, device="cuda"),
+               torch.empty(64, dtype=torch.uint8, device="cuda"), None):
+        y = bq.quant_matmul_ex(xd, wq, s, b, p.group_size, p.bits, True, "tc_fused", workspace=ws)
+        torch.cuda.synchronize()
+        got = y if rows is None else y[torch.as_tensor(rows, device=y.device)]
+        assert_within_tolerance(got, y_ref, a_ref, f"{fmt} M={M} N={N} ws={None if ws is None else ws.numel()}")
+        outs.append(y)
+    assert torch.equal(outs[0], outs[2])
+    assert torch.equal(outs[0], bq.quant_matmul_ex(xd, wq, s, b, p.group_size, p.bits, True, "tc_fused"))
+    assert bq.bq_device_status() == 0
 
 
 @pytest.mark.parametrize("fmt", ["q4_0", "affine4", "affine8"])
