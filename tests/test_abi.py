@@ -135,6 +135,32 @@ def test_dispatcher_boundaries(L):
     assert L.quant_matmul_workspace_size(512, 256, 512, 64, 8, 3) == 256 * 512 * 2
 
 
+TILE_PARTIAL = 128 * 4          # fp32 bytes per token of one 128-row split tile
+
+
+@pytest.mark.parametrize("M,N,K,g,bits,want", [
+    # 12288 x 4096 projection (96 weight tiles), on a B200's 148 SMs
+    (64, 12288, 4096, 64, 4, 3 * 96 * 64 * TILE_PARTIAL),    # 96 tiles of 64 tokens, every one split 3 ways
+    (256, 12288, 4096, 64, 4, 0),                            # 96 whole 256-token tiles
+    (512, 12288, 4096, 64, 4, 3 * 44 * 256 * TILE_PARTIAL),  # 192 tiles: 148 whole, the other 44 split 3 ways
+    (512, 12288, 4096, 32, 4, 3 * 44 * 256 * TILE_PARTIAL),  # Q4_0: the same plan
+    (1024, 12288, 4096, 64, 4, 0),                           # 384 whole tiles: 88 left over, too many to split
+    (2048, 12288, 4096, 64, 4, 5 * 28 * 256 * TILE_PARTIAL), # 768 tiles: 740 whole, 28 split 5 ways
+    (3072, 12288, 4096, 64, 4, 0),
+    (4096, 12288, 4096, 32, 4, 0),                           # 1536 tiles: splitting the last 56 does not pay
+    (2048, 12288, 4096, 64, 8, 5 * 28 * 256 * TILE_PARTIAL), # affine 8-bit, fused path forced
+    # the split-tail parity cases of the GPU tests
+    (64, 19160, 1024, 32, 4, 4 * 2 * 64 * TILE_PARTIAL),     # 150 tiles: 2 split 4 ways
+    (100, 18950, 1024, 64, 4, 4 * 1 * 112 * TILE_PARTIAL),   # 149 tiles of 112 tokens: 1 split 4 ways
+    (400, 9750, 1024, 64, 8, 4 * 6 * 256 * TILE_PARTIAL),    # 154 tiles: 6 split 4 ways
+    (200, 19750, 1024, 32, 4, 4 * 7 * 208 * TILE_PARTIAL),   # 155 tiles of 208 tokens: 7 split 4 ways
+])
+def test_fused_plan_workspace(L, M, N, K, g, bits, want):
+    """The fused kernel's K-split plan, seen through the workspace it asks for:
+    fp32 partials only for the split tiles (splits x split tiles x bn x 128)."""
+    assert L.quant_matmul_workspace_size(M, N, K, g, bits, 2) == want
+
+
 def _select_in_subprocess(env_extra, Ms):
     code = ("import sys; sys.path.insert(0, %r); import bit_quantized_gemm_quant_b200 as bq; "
             "print([bq.quant_matmul_select_path(m, 4096, 4096, 64, 4) for m in %r])" % (ROOT, Ms))
