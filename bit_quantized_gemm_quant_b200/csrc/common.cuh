@@ -57,6 +57,50 @@ BQ_DEVINL uint32_t hsub2_bf16(uint32_t a, uint32_t b)
     return d;
 }
 
+// Packed fp32x2 arithmetic (sm_100): two independent lanes in one 64-bit
+// register, each rounded exactly as the scalar operation (sub.rn.f32x2 lane =
+// __fsub_rn, fma.rn.f32x2 lane = __fmaf_rn), so results are bit-identical to
+// the scalar forms at half the instruction count.
+BQ_DEVINL uint64_t f32x2_pack(uint32_t lo, uint32_t hi)
+{
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+    return d;
+}
+
+BQ_DEVINL uint64_t f32x2_splat(float v) { return f32x2_pack(__float_as_uint(v), __float_as_uint(v)); }
+
+BQ_DEVINL void f32x2_unpack(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+BQ_DEVINL uint64_t sub_f32x2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+BQ_DEVINL uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// Affine 8-bit: bytes e and e+1 of a code word to bf16x2 (bf16_rne(fmaf(scale,
+// q, bias)) per lane).  Each byte becomes the fp32 2^23 + q by a byte permute;
+// subtracting 2^23 is exact.
+template <int E>
+BQ_DEVINL uint32_t deq_aff8_pair(uint32_t word, uint64_t s2, uint64_t b2)
+{
+    const uint64_t f = f32x2_pack(prmt(word, 0x4B000000u, 0x7650u | E), prmt(word, 0x4B000000u, 0x7650u | (E + 1)));
+    float lo, hi;
+    f32x2_unpack(fma_f32x2(s2, sub_f32x2(f, f32x2_splat(8388608.0f)), b2), lo, hi);
+    return pack_bf16x2_rn(lo, hi);
+}
+
 // (a & mask) | magic in one LOP3.
 BQ_DEVINL uint32_t and_or(uint32_t a, uint32_t mask, uint32_t magic)
 {

@@ -145,12 +145,10 @@ BQ_DEVINL void dequant_word(uint32_t word, const ChunkScale& cs, uint32_t (&p)[4
             p[n] = hfma2_bf16(hsub2_bf16_i<0x43004300u>(r), cs.s2, cs.b2);   // (8i+n, 8i+n+4)
         }
     } else {
-        float f[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            f[e] = __fsub_rn(__uint_as_float(prmt(word, 0x4B000000u, 0x7650u | e)), 8388608.0f);   // byte e
-        p[0] = pack_bf16x2_rn(__fmaf_rn(cs.a[0], f[0], cs.c[0]), __fmaf_rn(cs.a[0], f[1], cs.c[0]));
-        p[1] = pack_bf16x2_rn(__fmaf_rn(cs.a[0], f[2], cs.c[0]), __fmaf_rn(cs.a[0], f[3], cs.c[0]));
+        // bytes (0, 1) and (2, 3), two weights per packed fp32x2 subtract and FMA
+        const uint64_t s2 = f32x2_splat(cs.a[0]), b2 = f32x2_splat(cs.c[0]);
+        p[0] = deq_aff8_pair<0>(word, s2, b2);
+        p[1] = deq_aff8_pair<2>(word, s2, b2);
         p[2] = p[3] = 0u;
     }
 }

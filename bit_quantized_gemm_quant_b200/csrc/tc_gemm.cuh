@@ -130,18 +130,16 @@ BQ_DEVINL void deq_aff4_half(uint4 raw, uint32_t s2, uint32_t b2, uint32_t (&out
     }
 }
 
-// Affine 8-bit: 8 words of bytes; w = bf16_rne(fmaf(scale, q, bias)).
+// Affine 8-bit: 8 words of bytes; w = bf16_rne(fmaf(scale, q, bias)), two
+// weights per packed fp32x2 subtract and FMA.
 BQ_DEVINL void deq_aff8_half(uint4 raw0, uint4 raw1, float s, float b, uint32_t (&out)[16])
 {
     const uint32_t words[8] = {raw0.x, raw0.y, raw0.z, raw0.w, raw1.x, raw1.y, raw1.z, raw1.w};
+    const uint64_t s2 = f32x2_splat(s), b2 = f32x2_splat(b);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        float f[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            f[e] = __fsub_rn(__uint_as_float(prmt(words[i], 0x4B000000u, 0x7650u | e)), 8388608.0f);
-        out[2 * i] = pack_bf16x2_rn(__fmaf_rn(s, f[0], b), __fmaf_rn(s, f[1], b));
-        out[2 * i + 1] = pack_bf16x2_rn(__fmaf_rn(s, f[2], b), __fmaf_rn(s, f[3], b));
+        out[2 * i] = deq_aff8_pair<0>(words[i], s2, b2);
+        out[2 * i + 1] = deq_aff8_pair<2>(words[i], s2, b2);
     }
 }
 
