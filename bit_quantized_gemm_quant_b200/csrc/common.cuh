@@ -82,6 +82,20 @@ BQ_DEVINL uint64_t sub_f32x2(uint64_t a, uint64_t b)
     return d;
 }
 
+BQ_DEVINL uint64_t add_f32x2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+BQ_DEVINL float f32x2_sum(uint64_t v)
+{
+    float lo, hi;
+    f32x2_unpack(v, lo, hi);
+    return __fadd_rn(lo, hi);
+}
+
 BQ_DEVINL uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c)
 {
     uint64_t d;

@@ -6,12 +6,14 @@
 // quantized kernel wins there) is a matrix-vector product over packed codes.
 // Here one warp owns kRows weight rows and its lanes take whole code units
 // (AffUnit<BITS>: W words holding E codes, never straddling a group).  Per unit
-// and token the lane forms the exact fp32 sums  sum_e x[e] * q[e]  and
-// sum_e x[e], and adds  scale * (first) + bias * (second)  to the row's result:
-// the dot product of x with the weights scale * q + bias, over the exact
-// weights rather than their bf16 roundings (within the GEMM tolerance, which
-// covers a 2^-9 relative difference per weight).  Codes become floats exactly
-// through the 2^23 magic number.  Lane partials are reduced with shuffles.
+// and token the lane forms the fp32 sums  sum_e x[e] * q[e]  and  sum_e x[e]
+// (even and odd e in the two lanes of packed fp32x2 operations, the lanes added
+// at the unit's end), and adds  scale * (first) + bias * (second)  to the row's
+// result: the dot product of x with the weights scale * q + bias, over the
+// exact weights rather than their bf16 roundings (within the GEMM tolerance,
+// which covers a 2^-9 relative difference per weight).  Codes become floats
+// exactly through the 2^23 magic number.  Lane partials are reduced with
+// shuffles; the summation order is fixed, so results are deterministic.
 #pragma once
 
 #include "common.cuh"
@@ -51,41 +53,44 @@ gemv_affine_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ 
             sc[r] = bf16_bits_to_f32(__ldg(scales + gi));
             bi[r] = bf16_bits_to_f32(__ldg(biases + gi));
         }
-        float xq[kGaRows][MT], xs[MT];
+        // (even, odd) element pairs: x, the codes and the sums in packed fp32x2
+        uint64_t xq[kGaRows][MT], xs[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-            xs[m] = 0.0f;
+            xs[m] = 0u;
 #pragma unroll
-            for (int r = 0; r < kGaRows; ++r) xq[r][m] = 0.0f;
+            for (int r = 0; r < kGaRows; ++r) xq[r][m] = 0u;
         }
+        const uint64_t magic2 = f32x2_splat(8388608.0f);
 #pragma unroll
         for (int e0 = 0; e0 < E; e0 += 8) {
-            float xv[MT][8];
+            uint64_t xv[MT][4];                               // (x[e0 + 2i], x[e0 + 2i + 1])
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 const uint4 v = (m < M) ? ldg_cached(x + (int64_t)m * K + k0 + e0) : make_uint4(0, 0, 0, 0);
                 const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    xv[m][2 * i] = __uint_as_float(vw[i] << 16);
-                    xv[m][2 * i + 1] = __uint_as_float(vw[i] & 0xFFFF0000u);
+                    xv[m][i] = f32x2_pack(vw[i] << 16, vw[i] & 0xFFFF0000u);
+                    xs[m] = add_f32x2(xs[m], xv[m][i]);
                 }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) xs[m] += xv[m][e];
             }
 #pragma unroll
             for (int r = 0; r < kGaRows; ++r)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float q = __fsub_rn(__uint_as_float(unit_code<BITS>(w[r], e0 + e) | 0x4B000000u), 8388608.0f);
+                for (int i = 0; i < 4; ++i) {
+                    const uint64_t q = sub_f32x2(f32x2_pack(unit_code<BITS>(w[r], e0 + 2 * i) | 0x4B000000u,
+                                                            unit_code<BITS>(w[r], e0 + 2 * i + 1) | 0x4B000000u),
+                                                 magic2);
 #pragma unroll
-                    for (int m = 0; m < MT; ++m) xq[r][m] = __fmaf_rn(xv[m][e], q, xq[r][m]);
+                    for (int m = 0; m < MT; ++m) xq[r][m] = fma_f32x2(xv[m][i], q, xq[r][m]);
                 }
         }
 #pragma unroll
         for (int r = 0; r < kGaRows; ++r)
 #pragma unroll
-            for (int m = 0; m < MT; ++m) acc[r][m] = __fmaf_rn(sc[r], xq[r][m], __fmaf_rn(bi[r], xs[m], acc[r][m]));
+            for (int m = 0; m < MT; ++m)
+                acc[r][m] = __fmaf_rn(sc[r], f32x2_sum(xq[r][m]), __fmaf_rn(bi[r], f32x2_sum(xs[m]), acc[r][m]));
     }
 #pragma unroll
     for (int r = 0; r < kGaRows; ++r)
