@@ -249,8 +249,10 @@ BQ_API bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const voi
 /*
  * quant_matmul_ex -- quant_matmul with an explicit path (bq_path) and an
  * optional caller-owned device workspace.  With workspace == NULL the library's
- * per-device buffer is used as in quant_matmul; otherwise workspace_bytes must
- * be >= quant_matmul_workspace_size(...) (BQ_ERR_WORKSPACE if not).  Forcing
+ * per-device buffer is used as in quant_matmul.  Otherwise, for the unfused
+ * pair workspace_bytes must be >= quant_matmul_workspace_size(...)
+ * (BQ_ERR_WORKSPACE if not); the fused path given a smaller workspace runs
+ * without K splits (same result within the tolerance, possibly slower).  Forcing
  * BQ_PATH_GEMV with M > 32 (M > 8 for 2-, 3- or 6-bit weights), BQ_PATH_TC_FUSED
  * for 2-, 3- or 6-bit weights, or either with transpose = 0, returns
  * BQ_ERR_UNSUPPORTED.
@@ -261,8 +263,12 @@ BQ_API bq_status quant_matmul_ex(const uint16_t* x_bf16, const void* wq, const v
                           bq_stream_t stream);
 
 /* Bytes of workspace quant_matmul_ex needs for this problem and path
- * (path AUTO: the dispatcher's choice).  0 when the path needs none or the
- * arguments are invalid.  Having no biases pointer, this call and
+ * (path AUTO: the dispatcher's choice).  The pair: the bf16 copy of W (N x K x
+ * 2).  The fused path: the fp32 partial sums of the tiles its plan splits over
+ * K (splits x split tiles x tile tokens x 128 x 4; with more tiles than SMs,
+ * only the tiles of the last, partly filled round are split), planned for the
+ * current device, or for a B200 when there is none.  0 when the path needs none or
+ * the arguments are invalid.  Having no biases pointer, this call and
  * quant_matmul_select_path take group_size 32 with bits 4 as Q4_0 and any
  * other combination as affine. */
 BQ_API size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int group_size, int bits, int path);
