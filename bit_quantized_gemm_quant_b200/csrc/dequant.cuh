@@ -199,13 +199,13 @@ q4_0_quant_kernel(const float* __restrict__ w, uint8_t* __restrict__ wq, uint16_
             if (a > amax) { amax = a; mx = v[j]; }
         }
         const float d = __fdiv_rn(mx, -8.0f);
-        const float id = (d != 0.0f) ? __fdiv_rn(1.0f, d) : 0.0f;
         d16[b] = __half_as_ushort(__float2half_rn(d));
         uint32_t out[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            int q0 = (int)__fadd_rn(__fmul_rn(v[j], id), 8.5f);
-            int q1 = (int)__fadd_rn(__fmul_rn(v[j + 16], id), 8.5f);
+            // IEEE division by the unrounded fp32 d (an all-zero block has d == 0 and q = 8)
+            int q0 = (int)__fadd_rn(d != 0.0f ? __fdiv_rn(v[j], d) : 0.0f, 8.5f);
+            int q1 = (int)__fadd_rn(d != 0.0f ? __fdiv_rn(v[j + 16], d) : 0.0f, 8.5f);
             q0 = min(15, max(0, q0));
             q1 = min(15, max(0, q1));
             out[j / 4] |= (uint32_t)(q0 | (q1 << 4)) << (8 * (j % 4));

@@ -8,13 +8,16 @@ contraction); this module only marshals numpy arrays into it.
 Parity status of each function (what pins it, see ``tests/test_oracle_pins.py``):
   f32/f16/bf16 conversions  -- numpy / torch conversions, exhaustive or 1M+ values
   q4_0_quantize             -- closed forms: exact round trip, all-zero block,
-                               max-abs element -> q = 0, q range, error bound
+                               max-abs element -> q = 0, q range, error bound;
+                               exact w/d = k - 1/2 ties and the first-max rule
+                               (planted variants of the source fail them)
   q4_0_dequantize           -- closed form over every code value with both signs
                                of d, exact round trip of quantize
   q4_0_import_aos           -- blocks assembled byte by byte with numpy from
                                random codes and scales
   affine_quantize           -- closed forms: exact round trip, constant group,
-                               min -> 0 / max -> L, error bound (2, 3, 4, 6, 8 bits)
+                               min -> 0 / max -> L, error bound (2, 3, 4, 6, 8 bits);
+                               exact half-way ties go to even (roundf fails)
   affine_dequantize         -- closed form over every code value, codes laid out
                                by an independent numpy bit-stream packer and a
                                hand-derived 3-bit word; exact round trip of quantize

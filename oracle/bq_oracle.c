@@ -122,11 +122,14 @@ void oracle_f16_to_f32_array(const uint16_t* in, float* out, int64_t n)
 /* Quantize one row-major fp32 matrix w[N][K] (K % 32 == 0) to Q4_0.
  * Per block of 32 weights along K:
  *   1. m = the weight with the largest |w| (first index wins a tie);
- *   2. d = m / -8 in fp32, so that m itself maps to q = 0; id = 1/d (0 if d == 0);
- *   3. q_j = min(15, trunc(w_j * id + 8.5)), the argument is >= 0.5 so trunc == floor;
+ *   2. d = m / -8 in fp32, so that m itself maps to q = 0;
+ *   3. q_j = clamp(trunc(w_j / d + 8.5), 0, 15) with an IEEE fp32 division and
+ *      addition (q_j = 8 when d == 0: the block is all zeros);
  *   4. the stored scale is fp16(d); byte j = q_j | q_{j+16} << 4.
- * Reading (the pages print no quantizer): q is taken from the unrounded fp32
- * d through its reciprocal, and fp16(d) is what is stored. */
+ * Reading (the pages print no quantizer; the Q4_0 workload statement gives
+ * "d = signed max-abs / -8 as fp16" and "q = clamp(int(w/d + 8.5), 0, 15)"):
+ * w/d is a true division by the unrounded fp32 d, and fp16(d) is what is
+ * stored. */
 void oracle_q4_0_quantize(const float* w, int64_t N, int64_t K, uint8_t* wq, uint16_t* d16)
 {
     const int64_t nb = K / 32;
@@ -139,12 +142,11 @@ void oracle_q4_0_quantize(const float* w, int64_t N, int64_t K, uint8_t* wq, uin
                 if (fabsf(v) > amax) { amax = fabsf(v); mx = v; }
             }
             float d = mx / -8.0f;
-            float id = (d != 0.0f) ? 1.0f / d : 0.0f;
             d16[n * nb + b] = oracle_f32_to_f16(d);
             uint8_t* out = wq + n * (K / 2) + b * 16;
             for (int j = 0; j < 16; ++j) {
-                float t0 = blk[j] * id;
-                float t1 = blk[j + 16] * id;
+                float t0 = (d != 0.0f) ? blk[j] / d : 0.0f;
+                float t1 = (d != 0.0f) ? blk[j + 16] / d : 0.0f;
                 t0 = t0 + 8.5f;
                 t1 = t1 + 8.5f;
                 int q0 = (int)t0, q1 = (int)t1;

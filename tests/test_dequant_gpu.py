@@ -9,6 +9,7 @@ import bit_quantized_gemm_quant_b200 as bq
 import oracle
 from bit_quantized_gemm_quant_b200 import inputs
 from _helpers import Problem, u16
+import _ties
 
 pytestmark = pytest.mark.gpu
 
@@ -95,6 +96,31 @@ def test_affine_quantize_bit_exact(bits, N, K):
     w[0, :64] = -0.375                   # constant group: scale 0
     wq_ref, s_ref, b_ref = oracle.affine_quantize(w.numpy(), 64, bits)
     wq, s, b = bq.affine_quantize(w.cuda(), 64, bits)
+    torch.cuda.synchronize()
+    assert np.array_equal(wq.cpu().numpy().view(np.uint32), wq_ref)
+    assert np.array_equal(u16(s), s_ref)
+    assert np.array_equal(u16(b), b_ref)
+
+
+def test_q4_0_quantize_division_ties():
+    """Blocks whose elements divide to k - 1/2 exactly (code k): the device
+    quantizer divides by the fp32 d exactly as the pinned oracle does."""
+    w, q = _ties.q4_0_tie_matrix()
+    wq_ref, d_ref = oracle.q4_0_quantize(w)
+    wq, d = bq.q4_0_quantize(torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(wq.cpu().numpy(), wq_ref)
+    assert np.array_equal(u16(d), d_ref)
+    got = wq.cpu().numpy()
+    assert np.array_equal(np.concatenate([got & 15, got >> 4], axis=1), q)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
+def test_affine_quantize_ties_to_even(bits):
+    """(w - bias)/scale = j + 1/2 exactly: the device quantizer takes the even code."""
+    w, _, q = _ties.affine_tie_matrix(bits)
+    wq_ref, s_ref, b_ref = oracle.affine_quantize(w, 64, bits)
+    wq, s, b = bq.affine_quantize(torch.from_numpy(w).cuda(), 64, bits)
     torch.cuda.synchronize()
     assert np.array_equal(wq.cpu().numpy().view(np.uint32), wq_ref)
     assert np.array_equal(u16(s), s_ref)

@@ -547,3 +547,130 @@ def test_q4_0_q8_matmul_within_activation_quantization_bound():
     # and the bound is not vacuous: a planted sign error on the weights breaks it
     y_bad, _ = oracle.q4_0_q8_matmul(xq, dx, wq ^ 0x88, d)
     assert not np.all(np.abs(y_bad - y_ref) <= bound)
+
+
+# --------------------------------------------------------------------------
+# quantizer rounding decisions: exact ties, and planted variants of the oracle
+# --------------------------------------------------------------------------
+import ctypes
+import os
+import subprocess
+
+import _ties
+from oracle import build as _oracle_build
+
+
+def _q4_0_quantize_with(lib, w):
+    w = np.ascontiguousarray(w, np.float32)
+    N, K = w.shape
+    wq = np.empty((N, K // 2), np.uint8)
+    d = np.empty((N, K // 32), np.uint16)
+    lib.oracle_q4_0_quantize(ctypes.c_void_p(w.ctypes.data), ctypes.c_int64(N), ctypes.c_int64(K),
+                             ctypes.c_void_p(wq.ctypes.data), ctypes.c_void_p(d.ctypes.data))
+    return wq, d
+
+
+def _affine_quantize_with(lib, w, group, bits):
+    w = np.ascontiguousarray(w, np.float32)
+    N, K = w.shape
+    wq = np.empty((N, K * bits // 32), np.uint32)
+    s = np.empty((N, K // group), np.uint16)
+    b = np.empty((N, K // group), np.uint16)
+    lib.oracle_affine_quantize(ctypes.c_void_p(w.ctypes.data), ctypes.c_int64(N), ctypes.c_int64(K),
+                               ctypes.c_int(group), ctypes.c_int(bits), ctypes.c_void_p(wq.ctypes.data),
+                               ctypes.c_void_p(s.ctypes.data), ctypes.c_void_p(b.ctypes.data))
+    return wq, s, b
+
+
+class _Oracle:
+    """The oracle's own library, or a copy of its source with one planted change."""
+
+    def __init__(self, lib):
+        self.lib = lib
+
+    def q4_0(self, w):
+        return _q4_0_quantize_with(self.lib, w)
+
+    def affine(self, w, group, bits):
+        return _affine_quantize_with(self.lib, w, group, bits)
+
+
+def _planted(tmp_path, name, old, new):
+    src = open(_oracle_build.SRC).read()
+    assert src.count(old) >= 1, f"planted change {name!r} no longer applies"
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(old, new))
+    lib = tmp_path / f"lib{name}.so"
+    subprocess.check_call(["gcc", *_oracle_build.CFLAGS, str(path), "-o", str(lib), "-lm"])
+    return _Oracle(ctypes.CDLL(str(lib)))
+
+
+def _q4_0_ties_hold(orc: _Oracle) -> bool:
+    w, q = _ties.q4_0_tie_matrix()
+    wq, d16 = orc.q4_0(w)
+    d = np.array([np.float32(d) for d, _ in _ties.Q4_0_TIE_BLOCKS], np.float32)
+    return np.array_equal(wq, pack_q4_0(q)) and np.array_equal(d16[:, 0], np_f16_bits(d))
+
+
+def _affine_ties_hold(orc: _Oracle, bits: int) -> bool:
+    w, s, q = _ties.affine_tie_matrix(bits)
+    wq, s16, b16 = orc.affine(w, 64, bits)
+    return (np.array_equal(f32_from_bf16_bits(s16).astype(np.float64), np.repeat(s[:, None], 2, axis=1))
+            and np.all(b16 == 0) and np.array_equal(wq, pack_affine(q, bits)))
+
+
+def test_q4_0_quantize_exact_division_ties():
+    """Elements with w/d = k - 1/2 exactly get code k (q = int(w/d + 8.5) with the
+    fp32 d); both the reciprocal form w·(1/d) and a division by the stored fp16
+    scale give k - 1 on these blocks."""
+    assert _ties.q4_0_tie_exactness()
+    assert _q4_0_ties_hold(_Oracle(oracle._load()))
+    # the blocks discriminate the alternative readings (numpy fp32 arithmetic)
+    w, q = _ties.q4_0_tie_matrix()
+    for r, (d, ties) in enumerate(_ties.Q4_0_TIE_BLOCKS):
+        d32 = np.float32(d)
+        for i, k in ties:
+            assert int(np.float32(w[r, i] * (np.float32(1) / d32)) + np.float32(8.5)) == k - 1
+            assert int(np.float32(w[r, i] / np.float32(np.float16(d32))) + np.float32(8.5)) == k - 1
+
+
+def test_q4_0_quantize_max_abs_tie_takes_first_element():
+    """+a before -a with |a| the block maximum: d = a / -8 (negative), the +a
+    element gets code 0 and the -a element clamps to 15."""
+    w = np.full((1, 32), 0.125, np.float32)
+    w[0, 2], w[0, 7] = 0.75, -0.75
+    wq, d16 = oracle.q4_0_quantize(w)
+    assert d16[0, 0] == np_f16_bits(np.array([-0.09375], np.float32))[0]
+    lo, hi = wq[0] & 15, wq[0] >> 4
+    assert lo[2] == 0 and lo[7] == 15
+    assert np.all(np.delete(lo, [2, 7]) == 7) and np.all(hi == 7)     # 0.125 / -0.09375 + 8.5 = 7.17
+
+
+@pytest.mark.parametrize("bits", AFFINE_BITS)
+def test_affine_quantize_ties_to_even(bits):
+    """(w - bias)/scale = j + 1/2 exactly: the code is the even neighbour."""
+    assert _affine_ties_hold(_Oracle(oracle._load()), bits)
+
+
+def test_quantizer_pins_catch_planted_oracle_variants(tmp_path):
+    """Copies of the oracle source with one rounding rule changed fail the pins above."""
+    variants = [
+        ("roundf", "float r = nearbyintf(t);", "float r = roundf(t);", "affine"),
+        ("trunc_half", "float r = nearbyintf(t);", "float r = floorf(t + 0.5f);", "affine"),
+        ("reciprocal", "float t0 = (d != 0.0f) ? blk[j] / d : 0.0f;",
+         "float t0 = (d != 0.0f) ? blk[j] * (1.0f / d) : 0.0f;", "q4_0"),
+        ("fp16_scale", "float t0 = (d != 0.0f) ? blk[j] / d : 0.0f;",
+         "float t0 = (d != 0.0f) ? blk[j] / oracle_f16_to_f32(oracle_f32_to_f16(d)) : 0.0f;", "q4_0"),
+        ("last_max", "if (fabsf(v) > amax)", "if (fabsf(v) >= amax)", "q4_0_max"),
+    ]
+    for name, old, new, kind in variants:
+        orc = _planted(tmp_path, name, old, new)
+        if kind == "affine":
+            assert not all(_affine_ties_hold(orc, b) for b in AFFINE_BITS), name
+        elif kind == "q4_0":
+            assert not _q4_0_ties_hold(orc), name
+        else:
+            w = np.full((1, 32), 0.125, np.float32)
+            w[0, 2], w[0, 7] = 0.75, -0.75
+            _, d16 = orc.q4_0(w)
+            assert d16[0, 0] != np_f16_bits(np.array([-0.09375], np.float32))[0], name
