@@ -1,24 +1,30 @@
 """Benchmark of the weight-only block-quantized matmul hot path on B200.
 
-Default workload (one JSON line on rank 0): the Q4_0 decode GEMV of the
-12288 x 4096 MLP up-projection (the micro-benchmark shape of the MLX issue
+Headline (one JSON line on rank 0): the Q4_0 decode GEMV, one token, of the
+12288 x 4096 MLP up-projection -- the micro-benchmark shape of the MLX issue
 "quantized_matmul takes 14-41% longer than dequantize + bf16 matmul at prefill
-sizes (> 512 tokens)", Repro) at M = 1, 8 and 32 tokens.  One step is one
-quant_matmul call per token count, each on its own copy of the packed weights;
-12 rotating copies (340 MB > 126 MB of L2) make every launch read its weights
-from HBM.  value = packed weight + scale bytes read per step / step time.
+sizes (> 512 tokens)" (Repro).  One step is one quant_matmul call; 12 rotating
+copies of the packed weights (340 MB > 126 MB of L2) make every launch read its
+weights from HBM.  value = packed weight + scale bytes read / time, and
+roofline.frac = that over the measured copy bandwidth.
 
-Other workloads (--workload): affine4_prefill, affine8_sweep (TFLOP/s of the
-fused kernel and of the unfused dequantize + bf16 GEMM pair), llama1b_stack
-(tokens/s of the 112 projection matmuls of a 16-layer Llama-3.2-1B shape).
+The default run also measures, under "secondary", every other workload of the
+scope: decode at 8, 16 and 32 tokens; prefill of Q4_0, affine 4-bit and affine
+8-bit at 512 / 2048 / 8192 tokens (fused kernel, unfused pair, our bf16 GEMM,
+cuBLAS for context, and the dispatcher's choice), the affine 8-bit sweep with
+its fused/unfused crossover, the 16 x 256 x 512 Q4_0 check problem, the
+Llama-3.2-1B-shaped projection stack at 512 tokens and 1 token, and the CPU
+oracle on prefill sizes (full at 512 tokens, a 64-token sample above).
 
-Multi-GPU (torchrun): every rank runs its own replica of the workload (the
-path has no exchange step), timing is the max over ranks, value is the sum.
+Multi-GPU (torchrun): the weight rows of one tall matrix are sharded across
+ranks, 12288 rows per rank, x replicated (weak scaling; no exchange is needed
+for the matmul itself, --gather adds an NCCL all-gather of y, timed apart).
 --impl reference times the CPU oracle on the host cores instead.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -32,14 +38,34 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+METRIC = "prefill TFLOP/s (% bf16 TC peak); M=1 GEMV GB/s (% HBM peak)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-
-# dram__bytes_read.sum + dram__bytes_write.sum of one launch, from one ncu capture of the
-# current build of each kernel (`ncu --set full`, decode bench command); None for a kernel
-# changed since its counters were taken.
-NCU_TRAFFIC = {"gemv_kernel<Q4_0, M=1>": 28332800, "gemv_kernel<Q4_0, M=8>": 28389888,
-               "gemv_kernel<Q4_0, M=32>": 28590592, "gemv_q8_kernel<M=1>": 28324608}
 L2_BYTES = 126 * 1024 * 1024
+CSRC = os.path.join(ROOT, "bit_quantized_gemm_quant_b200", "csrc")
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch from one ncu capture,
+# with the hash of the kernel's source file at that capture.  A kernel whose
+# source changed since reports traffic null.
+NCU_TRAFFIC = {
+    "gemv_stream_kernel<Q4_0> M=1": {"bytes": None, "source": "gemv_stream.cuh", "sha16": None,
+                                      "capture": None},
+}
+
+
+def source_sha16(name: str) -> str:
+    with open(os.path.join(CSRC, name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def stored_traffic(kernel: str):
+    """(bytes per launch or None, provenance) of the stored capture of `kernel`."""
+    e = NCU_TRAFFIC.get(kernel)
+    if not e or e["bytes"] is None:
+        return None, "no capture stored for this kernel build"
+    cur = source_sha16(e["source"])
+    if cur != e["sha16"]:
+        return None, f"stale: {e['source']} is {cur}, the capture was of {e['sha16']}"
+    return e["bytes"], f"ncu capture {e['capture']} of {e['source']} {e['sha16']}"
 
 
 # ----------------------------------------------------------------------------- helpers (host only)
@@ -217,129 +243,181 @@ def kernel_seconds(fn_list, reps):
     return s.elapsed_time(e) / 1000.0 / (reps * len(fn_list))
 
 
-def run_decode(args, world, device, peaks):
+
+
+# ----------------------------------------------------------------------------- row shards (multi-GPU)
+def shard_rows(rows_per_rank: int, rank: int) -> tuple:
+    """Rows [first, last) of the tall matrix that `rank` owns: each rank holds
+    rows_per_rank consecutive weight rows (with their scales), x is replicated."""
+    return rank * rows_per_rank, (rank + 1) * rows_per_rank
+
+
+def shard_seed(seed: int, rank: int) -> int:
+    """Seed of the generator of rank `rank`'s rows (rank 0 keeps the workload's seed)."""
+    return seed + 7919 * rank
+
+
+def assemble_shards(shards):
+    """y [M][N_total] from the per-rank y [M][rows_per_rank] in rank order (torch tensors)."""
+    import torch
+    return torch.cat(list(shards), dim=1)
+
+
+def decode_config(world: int) -> dict:
+    """The headline workload, identical in both arms."""
+    from bit_quantized_gemm_quant_b200 import workloads
+    wl = workloads.Q4_0_DECODE
+    return {"workload": "q4_0_decode_m1_n12288_k4096", "fmt": "q4_0", "N": wl.N * world, "K": wl.K, "M": 1,
+            "rows_per_rank": wl.N, "parallelism": f"weight-row shards x{world}"}
+
+
+# ----------------------------------------------------------------------------- GPU workloads
+def run_decode(args, world, rank, device, peaks):
+    """Headline: one-token Q4_0 GEMV over this rank's 12288 x 4096 shard, 12 rotating copies."""
     import torch
     import bit_quantized_gemm_quant_b200 as bq
     from bit_quantized_gemm_quant_b200 import inputs, workloads
 
     wl = workloads.Q4_0_DECODE
-    N, K, Ms = wl.N, wl.K, wl.Ms
+    N, K = wl.N, wl.K
     gs, bits = _fmt_args(wl.fmt)
-    wq0, s0, _ = make_weights(wl.fmt, N, K, wl.seed, device)
+    wq0, s0, _ = make_weights(wl.fmt, N, K, shard_seed(wl.seed, rank), device)
     n_copies = 12
     copies = [(wq0, s0)] + [(wq0.clone(), s0.clone()) for _ in range(n_copies - 1)]
-    g = inputs.generator(wl.seed + 1)
-    xs = {M: inputs.activations_bf16(M, K, g).to(device) for M in Ms}
-    ys = {M: torch.empty(M, N, dtype=torch.bfloat16, device=device) for M in Ms}
+    g = inputs.generator(wl.seed + 1)                      # x is replicated: the same on every rank
+    xs = {M: inputs.activations_bf16(M, K, g).to(device) for M in (1, 8, 16, 32)}
+    ys = {M: torch.empty(M, N, dtype=torch.bfloat16, device=device) for M in xs}
     wbytes = workloads.packed_weight_bytes(wl.fmt, N, K, gs)
     assert n_copies * wbytes > 2 * L2_BYTES
 
-    def step_fn(phase):
+    def steps_fn(n):
+        # n consecutive steps, each on the next copy: every copy is read once per 12 steps
         def f():
-            for j, M in enumerate(Ms):
-                wq, s = copies[rotation(n_copies, len(Ms), phase, j)]
-                bq.quant_matmul(xs[M], wq, s, None, gs, bits, out=ys[M])
+            for j in range(n):
+                wq, s = copies[j % n_copies]
+                bq.quant_matmul(xs[1], wq, s, None, gs, bits, out=ys[1])
         return f
 
-    n_phase = n_copies // math.gcd(n_copies, len(Ms))
-    graphs = [GraphTimer(step_fn(p)) for p in range(n_phase)]
-    for i in range(args.warmup):
-        graphs[i % n_phase].replay()
+    # the timed steps run as graphs of 12 launches (the launches of one graph may
+    # overlap their set-up with the previous kernel) plus one graph of the rest
+    full, rest = divmod(args.steps, n_copies)
+    g_full = GraphTimer(steps_fn(n_copies))
+    g_rest = GraphTimer(steps_fn(rest)) if rest else None
+    for _ in range(max(1, -(-args.warmup // n_copies))):
+        g_full.replay()
     torch.cuda.synchronize()
     with ClockSampler(device.index if device.index is not None else 0) as clk:
-        secs = time_graphs(graphs, args.steps, world, device)
+        secs = time_graphs([g_full] * full + ([g_rest] if g_rest else []), full + (1 if g_rest else 0), world,
+                           device)
     secs_max = max_over_ranks(secs, world, device)
-    units = args.steps * len(Ms) * wbytes                   # bytes of packed weights read by this rank
-    value = aggregate(units, world, secs_max) / 1e9
+    value = aggregate(args.steps * wbytes, world, secs_max) / 1e9
 
-    # per-kernel device time (each M is its own GEMV instantiation), same launch configuration
+    # per-launch device time of each token count, same launch configuration
     per_m = {}
-    for M in Ms:
+    for M in xs:
         fns = [(lambda wq=wq, s=s, M=M: bq.quant_matmul(xs[M], wq, s, None, gs, bits, out=ys[M]))
                for (wq, s) in copies]
         t = kernel_seconds(fns, 4)
         per_m[str(M)] = {"us": round(t * 1e6, 3), "gbs": round(wbytes / t / 1e9, 1),
                          "frac_hbm": round(wbytes / t / 1e9 / peaks["hbm_gbs"], 4),
-                         "tflops": round(2.0 * M * N * K / t / 1e12, 3)}
+                         "tflops": round(2.0 * M * N * K / t / 1e12, 3),
+                         "path": {v: k for k, v in bq.PATHS.items()}[bq.quant_matmul_select_path(M, N, K, gs, bits)]}
     # the quantized-activation path (opt-in, approximate): activation quantization
     # plus the Q4_0 x int8 GEMV, same weights, rotation and graph timing
-    q8 = {}
-    for M in Ms[:1]:                                  # a one-token path
-        fns = [(lambda wq=wq, s=s, M=M: bq.quant_matmul_q8(*bq.q8_1_quantize(xs[M]), wq, s, out=ys[M]))
-               for (wq, s) in copies]
-        t_all = kernel_seconds(fns, 4)
-        xq, dxq, qsq = bq.q8_1_quantize(xs[M])
-        fns_g = [(lambda wq=wq, s=s, M=M: bq.quant_matmul_q8(xq, dxq, qsq, wq, s, out=ys[M])) for (wq, s) in copies]
-        t_g = kernel_seconds(fns_g, 4)
-        q8[str(M)] = {"us": round(t_all * 1e6, 3), "gbs": round(wbytes / t_all / 1e9, 1),
-                      "gemv_us": round(t_g * 1e6, 3), "gemv_gbs": round(wbytes / t_g / 1e9, 1),
-                      "gemv_frac_hbm": round(wbytes / t_g / 1e9 / peaks["hbm_gbs"], 4),
-                      "gemv_traffic": NCU_TRAFFIC.get(f"gemv_q8_kernel<M={M}>")}
-    dom = max(Ms, key=lambda M: per_m[str(M)]["us"])
-    roof = {"bound": "hbm", "kernel": f"gemv_kernel<Q4_0, M={dom}>",
-            "achieved": per_m[str(dom)]["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(per_m[str(dom)]["gbs"] / peaks["hbm_gbs"], 4),
-            "traffic": NCU_TRAFFIC.get(f"gemv_kernel<Q4_0, M={dom}>"), "algorithmic_bytes_per_launch": wbytes}
+    fns = [(lambda wq=wq, s=s: bq.quant_matmul_q8(*bq.q8_1_quantize(xs[1]), wq, s, out=ys[1])) for (wq, s) in copies]
+    t_all = kernel_seconds(fns, 4)
+    xq, dxq, qsq = bq.q8_1_quantize(xs[1])
+    t_g = kernel_seconds([(lambda wq=wq, s=s: bq.quant_matmul_q8(xq, dxq, qsq, wq, s, out=ys[1]))
+                          for (wq, s) in copies], 4)
+    q8 = {"us": round(t_all * 1e6, 3), "gbs": round(wbytes / t_all / 1e9, 1), "gemv_us": round(t_g * 1e6, 3),
+          "gemv_gbs": round(wbytes / t_g / 1e9, 1), "gemv_frac_hbm": round(wbytes / t_g / 1e9 / peaks["hbm_gbs"], 4),
+          "note": "opt-in approximate path: q8_1_quantize + quant_matmul_q8; not the headline value"}
 
-    # end to end through the public API with host buffers: inputs H2D from pinned memory, y D2H
+    t1 = per_m["1"]["us"] * 1e-6
+    traffic, traffic_src = stored_traffic("gemv_stream_kernel<Q4_0> M=1")
+    roof = {"bound": "hbm", "kernel": "gemv_stream_kernel<Q4_0> (M=1)", "achieved": per_m["1"]["gbs"],
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": per_m["1"]["frac_hbm"], "traffic": traffic,
+            "traffic_source": traffic_src, "algorithmic_bytes_per_launch": wbytes,
+            "launch_us": round(t1 * 1e6, 3)}
+
+    # end to end through the public API with host buffers: the step's inputs (this
+    # rank's weight shard and x) copied in from pinned memory, y read back
     e2e = None
     if not args.no_e2e:
-        h_wq = wq0.cpu().pin_memory()
-        h_s = s0.cpu().pin_memory()
-        h_x = {M: xs[M].cpu().pin_memory() for M in Ms}
-        h_y = {M: torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for M in Ms}
-        d_wq, d_s = torch.empty_like(wq0), torch.empty_like(s0)
-        d_x = {M: torch.empty_like(xs[M]) for M in Ms}
+        h_wq, h_s, h_x = wq0.cpu().pin_memory(), s0.cpu().pin_memory(), xs[1].cpu().pin_memory()
+        h_y = torch.empty(1, N, dtype=torch.bfloat16).pin_memory()
+        d_wq, d_s, d_x = torch.empty_like(wq0), torch.empty_like(s0), torch.empty_like(xs[1])
         e2e_steps = max(3, min(args.steps, 20))
 
         def e2e_step():
-            # the step's inputs: the weight matrix (once) and each M's activations
             d_wq.copy_(h_wq, non_blocking=True)
             d_s.copy_(h_s, non_blocking=True)
-            for M in Ms:
-                d_x[M].copy_(h_x[M], non_blocking=True)
-                bq.quant_matmul(d_x[M], d_wq, d_s, None, gs, bits, out=ys[M])
-                h_y[M].copy_(ys[M], non_blocking=True)
+            d_x.copy_(h_x, non_blocking=True)
+            bq.quant_matmul(d_x, d_wq, d_s, None, gs, bits, out=ys[1])
+            h_y.copy_(ys[1], non_blocking=True)
         e2e_step()
         torch.cuda.synchronize()
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
+        t0, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0.record()
         for _ in range(e2e_steps):
             e2e_step()
-        t1.record()
+        t1e.record()
         torch.cuda.synchronize()
-        es = max_over_ranks(t0.elapsed_time(t1) / 1000.0, world, device)
-        h2d = h_wq.numel() * h_wq.element_size() + h_s.numel() * 2 + sum(h_x[M].numel() * 2 for M in Ms)
-        d2h = sum(M * N * 2 for M in Ms)
-        e2e = {"value": round(aggregate(e2e_steps * len(Ms) * wbytes, world, es) / 1e9, 3), "unit": "GB/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": e2e_steps}
+        es = max_over_ranks(t0.elapsed_time(t1e) / 1000.0, world, device)
+        h2d = h_wq.numel() * h_wq.element_size() + h_s.numel() * 2 + h_x.numel() * 2
+        e2e = {"value": round(aggregate(e2e_steps * wbytes, world, es) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(h_y.numel() * 2), "steps": e2e_steps}
 
-    launches = args.steps * len(Ms)
+    # optional: reassemble y of the whole tall matrix on every rank (NCCL all-gather), timed apart
+    gather = None
+    if args.gather and world > 1:
+        import torch.distributed as dist
+        y1 = ys[1].contiguous()
+        outs = [torch.empty_like(y1) for _ in range(world)]
+        dist.all_gather(outs, y1)
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        dist.barrier()
+        ev0.record()
+        for _ in range(reps):
+            dist.all_gather(outs, y1)
+        ev1.record()
+        torch.cuda.synchronize()
+        gsec = max_over_ranks(ev0.elapsed_time(ev1) / 1000.0 / reps, world, device)
+        full = assemble_shards(outs)
+        gather = {"us": round(gsec * 1e6, 3), "y_shape": list(full.shape), "collective": "NCCL all_gather of y"}
+
     return {
         "value": round(value, 2), "unit": "GB/s", "ms_per_step": secs_max / args.steps * 1e3,
+        "frac_hbm": round(value / world / peaks["hbm_gbs"], 4),
         "higher_is_better": True, "dtype": "q4_0 weights, bf16 activations, fp32 accumulate",
-        "config": {"workload": wl.name, "fmt": "q4_0", "N": N, "K": K, "M": list(Ms),
-                   "l2": f"{n_copies} rotating weight copies ({n_copies * wbytes / 1e6:.0f} MB > 126 MB L2)",
-                   "bytes_per_step": len(Ms) * wbytes, "path": "quant_matmul auto -> gemv"},
-        "per_m": per_m, "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
-        "secondary": {"q8_activation_path": dict(q8, note="opt-in approximate path: q8_1_quantize + "
-                                                          "quant_matmul_q8; not the headline value")},
+        "config": decode_config(world),
+        "notes": {"l2": f"{n_copies} rotating weight copies per rank ({n_copies * wbytes / 1e6:.0f} MB > 126 MB L2)",
+                  "bytes_per_step": wbytes * world, "path": "quant_matmul auto -> " + per_m["1"]["path"],
+                  "timing": "CUDA events around graph replays of back-to-back launches, max over ranks"},
+        "per_m": per_m, "roofline": roof, "e2e": e2e, "gpu_launches": args.steps, "clocks": clk.summary(),
+        "secondary": {"q8_activation_path_m1": q8}, "gather": gather,
     }
 
 
 def run_prefill(args, world, device, peaks, fmt, Ms):
+    """TFLOP/s per token count of the fused kernel (GEMV at decode sizes), the unfused
+    pair, our bf16 GEMM alone, cuBLAS bf16 (context) and the dispatcher's own choice,
+    on the 12288 x 4096 projection; the fused/pair crossover is the first measured M
+    from which the pair is faster."""
     import torch
     import bit_quantized_gemm_quant_b200 as bq
-    from bit_quantized_gemm_quant_b200 import inputs, workloads
+    from bit_quantized_gemm_quant_b200 import inputs
 
     N, K = 12288, 4096
     gs, bits = _fmt_args(fmt)
     wq, s, b = make_weights(fmt, N, K, 0, device)
     g = inputs.generator(1)
     ws = torch.empty(N * K, dtype=torch.bfloat16, device=device)
+    wb = ws.view(N, K)
     res = {}
-    total_flops, total_s = 0.0, 0.0
+    names = {v: k for k, v in bq.PATHS.items()}
     for M in Ms:
         x = inputs.activations_bf16(M, K, g).to(device)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
@@ -347,29 +425,60 @@ def run_prefill(args, world, device, peaks, fmt, Ms):
         reps = max(10, min(50, int(2e13 / flops)))
         fused_path = "tc_fused" if M > 32 else "gemv"
         t_fused = kernel_seconds([lambda: bq.quant_matmul_ex(x, wq, s, b, gs, bits, True, fused_path, out=y)], reps)
-        t_auto = kernel_seconds([lambda: bq.quant_matmul_ex(x, wq, s, b, gs, bits, True, "auto", workspace=ws,
-                                                           out=y)], reps)
+        if M <= 32:
+            # decode sizes: rotating weight copies (> 2x L2) so that every launch reads HBM
+            from bit_quantized_gemm_quant_b200 import workloads
+            nc = -(-3 * L2_BYTES // workloads.packed_weight_bytes(fmt, N, K, gs))
+            cps = [(wq.clone(), s.clone(), None if b is None else b.clone()) for _ in range(nc)]
+            t_auto = kernel_seconds([(lambda c=c: bq.quant_matmul(x, c[0], c[1], c[2], gs, bits, out=y))
+                                     for c in cps], 4)
+            del cps
+        else:
+            t_auto = kernel_seconds([lambda: bq.quant_matmul(x, wq, s, b, gs, bits, out=y)], reps)
         t_pair = kernel_seconds([lambda: bq.quant_matmul_ex(x, wq, s, b, gs, bits, True, "dequant_gemm",
                                                            workspace=ws, out=y)], reps)
-        wb = ws.view(N, K)
         if fmt == "q4_0":
             bq.q4_0_dequantize(wq, s, out=wb)
         else:
             bq.affine_dequantize(wq, s, b, gs, bits, out=wb)
         t_gemm = kernel_seconds([lambda: bq.bf16_matmul(x, wb, out=y)], reps)
         t_cublas = kernel_seconds([lambda: torch.matmul(x, wb.t(), out=y)], reps)
-        total_flops += flops
-        total_s += t_fused
-        res[str(M)] = {"fused_tflops": round(flops / t_fused / 1e12, 1),
-                       "fused_frac": round(flops / t_fused / 1e12 / peaks["bf16_tflops"], 4),
-                       "pair_tflops": round(flops / t_pair / 1e12, 1),
-                       "bf16_gemm_tflops": round(flops / t_gemm / 1e12, 1),
+        auto = names[bq.quant_matmul_select_path(M, N, K, gs, bits)]
+        tf = flops / t_auto / 1e12
+        res[str(M)] = {"fused_us": round(t_fused * 1e6, 2), "pair_us": round(t_pair * 1e6, 2),
+                       "auto_us": round(t_auto * 1e6, 2), "auto_path": auto,
+                       "fused_tflops": round(flops / t_fused / 1e12, 1), "pair_tflops": round(flops / t_pair / 1e12, 1),
+                       "auto_tflops": round(tf, 1), "bf16_gemm_tflops": round(flops / t_gemm / 1e12, 1),
                        "cublas_bf16_tflops": round(flops / t_cublas / 1e12, 1),
-                       "fused_us": round(t_fused * 1e6, 2), "pair_us": round(t_pair * 1e6, 2),
-                       "auto_path": bq.quant_matmul_select_path(M, N, K, gs, bits),
-                       "auto_tflops": round(flops / t_auto / 1e12, 1)}
+                       "roofline": {"bound": "tensor" if M > 32 else "hbm", "kernel": f"quant_matmul auto -> {auto}",
+                                    "achieved": round(tf, 1) if M > 32 else None,
+                                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                    "frac": round(tf / peaks["bf16_tflops"], 4)}}
+        if M <= 32:
+            from bit_quantized_gemm_quant_b200 import workloads
+            wbytes = workloads.packed_weight_bytes(fmt, N, K, gs)
+            res[str(M)]["roofline"] = {"bound": "hbm", "kernel": f"quant_matmul auto -> {auto}",
+                                       "achieved": round(wbytes / t_auto / 1e9, 1), "peak": peaks["hbm_gbs"],
+                                       "unit": "GB/s", "frac": round(wbytes / t_auto / 1e9 / peaks["hbm_gbs"], 4),
+                                       "note": "auto path over rotating weight copies (HBM reads)"}
         del x, y
-    return res, total_flops / total_s / 1e12
+    cross = next((int(m) for m, v in sorted(res.items(), key=lambda kv: int(kv[0]))
+                  if int(m) > 32 and v["pair_us"] < v["fused_us"]), None)
+    return res, cross
+
+
+def run_small(args, device, peaks):
+    """The 16 x 256 x 512 Q4_0 check problem (launch-bound): auto path time."""
+    import torch
+    import bit_quantized_gemm_quant_b200 as bq
+    from bit_quantized_gemm_quant_b200 import inputs, workloads
+    wl = workloads.Q4_0_SMALL
+    wq, s, _ = make_weights("q4_0", wl.N, wl.K, wl.seed, device)
+    x = inputs.activations_bf16(16, wl.K, inputs.generator(wl.seed + 1)).to(device)
+    y = torch.empty(16, wl.N, dtype=torch.bfloat16, device=device)
+    t = kernel_seconds([lambda: bq.quant_matmul(x, wq, s, None, 32, 4, out=y)], 50)
+    return {"us": round(t * 1e6, 3), "tflops": round(2.0 * 16 * wl.N * wl.K / t / 1e12, 4),
+            "path": {v: k for k, v in bq.PATHS.items()}[bq.quant_matmul_select_path(16, wl.N, wl.K, 32, 4)]}
 
 
 def run_widths(args, world, device, peaks):
@@ -471,32 +580,81 @@ def run_stack(args, world, device, peaks):
 
 
 # ----------------------------------------------------------------------------- CPU oracle (baseline / reference arm)
-def oracle_decode_sample(budget_s: float):
-    """Time the CPU oracle on the decode workload: per step, dequantize W and take the
-    float64 matmul for M = 1, 8, 32.  Runs whole steps until ~budget_s has passed."""
+def _decode_problem():
     import numpy as np
+    import torch
     import oracle
     from bit_quantized_gemm_quant_b200 import inputs, workloads
     wl = workloads.Q4_0_DECODE
     g = inputs.generator(wl.seed)
     w = inputs.weights_fp32(wl.N, wl.K, g).numpy()
     wq, d = oracle.q4_0_quantize(w)
-    xs = {M: inputs.activations_bf16(M, wl.K, g).view(dtype=__import__("torch").int16).numpy().view(np.uint16)
-          for M in wl.Ms}
-    wbytes = workloads.packed_weight_bytes("q4_0", wl.N, wl.K, 32)
-    steps, threads = 0, 1
+    x = inputs.activations_bf16(1, wl.K, inputs.generator(wl.seed + 1)).view(torch.int16).numpy().view(np.uint16)
+    return wl, wq, d, x
+
+
+def oracle_decode_step(wq, d, x, rows: int) -> int:
+    """One oracle decode step over the first `rows` weight rows: dequantize them and
+    take the float64 product with the one token.  Returns the host threads used."""
+    import os as _os
+    import oracle
+    wb = oracle.q4_0_dequantize(wq[:rows], d[:rows])
+    _, _, threads = oracle.matmul_ref(x, wb, nthreads=_os.cpu_count())
+    return threads
+
+
+def oracle_decode_timing(steps: int, warmup: int, budget_s: float):
+    """The oracle on the headline workload, exactly warmup + steps steps; each step a
+    row sample of the 12288 x 4096 matrix sized so that the run takes about
+    budget_s (all rows when that fits).  GB/s of the sampled rows' packed bytes."""
+    from bit_quantized_gemm_quant_b200 import workloads
+    wl, wq, d, x = _decode_problem()
     t0 = time.perf_counter()
-    while True:
-        for M in wl.Ms:
-            wb = oracle.q4_0_dequantize(wq, d)
-            _, _, threads = oracle.matmul_ref(xs[M], wb, nthreads=os.cpu_count())
-        steps += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s:
+    oracle_decode_step(wq, d, x, 512)
+    per_row = (time.perf_counter() - t0) / 512
+    rows = int(budget_s / max(1, steps + warmup) / per_row)
+    rows = max(16, min(wl.N, rows // 16 * 16))
+    for _ in range(warmup):
+        oracle_decode_step(wq, d, x, rows)
+    t0 = time.perf_counter()
+    threads = 1
+    for _ in range(steps):
+        threads = oracle_decode_step(wq, d, x, rows)
+    el = time.perf_counter() - t0
+    wbytes = workloads.packed_weight_bytes("q4_0", rows, wl.K, 32)
+    return {"value": round(steps * wbytes / el / 1e9, 5), "unit": "GB/s", "cores": int(threads), "kind": "oracle",
+            "sample": f"{steps} step(s) of a one-token decode over {rows} of the {wl.N} weight rows "
+                      f"(dequantize + float64 product), {el:.1f} s"}, el / steps
+
+
+def oracle_prefill_timing(budget_s: float):
+    """The oracle on prefill sizes of the affine 4-bit projection: 512 tokens in full,
+    2048 and 8192 tokens on a 64-token sample (rate extrapolated to the full size)."""
+    import numpy as np
+    import torch
+    import oracle
+    from bit_quantized_gemm_quant_b200 import inputs
+    N, K = 12288, 4096
+    g = inputs.generator(0)
+    w = inputs.weights_bf16_valued(N, K, g).numpy()
+    wq, s, b = oracle.affine_quantize(w, 64, 4)
+    t0 = time.perf_counter()
+    wb = oracle.affine_dequantize(wq, s, b, 64, 4)
+    t_deq = time.perf_counter() - t0
+    out = {"dequantize_s": round(t_deq, 3)}
+    xg = inputs.generator(1)
+    for M, sample in ((512, 512), (2048, 64), (8192, 64)):
+        if time.perf_counter() - t0 > budget_s:
             break
-    return {"value": round(steps * len(wl.Ms) * wbytes / el / 1e9, 5), "unit": "GB/s", "cores": int(threads),
-            "kind": "oracle", "sample": f"{steps} full decode step(s) (dequantize + float64 matmul at M=1,8,32) "
-                                        f"in {el:.1f} s"}, el / steps
+        x = inputs.activations_bf16(sample, K, xg).view(torch.int16).numpy().view(np.uint16)
+        t1 = time.perf_counter()
+        _, _, threads = oracle.matmul_ref(x, wb, nthreads=os.cpu_count())
+        el = time.perf_counter() - t1
+        rate = 2.0 * sample * N * K / el
+        out[str(M)] = {"gflops": round(rate / 1e9, 3), "cores": int(threads), "tokens_timed": sample,
+                       "full_s": round(2.0 * M * N * K / rate + t_deq, 2),
+                       "extrapolated": sample < M}
+    return out
 
 
 # ----------------------------------------------------------------------------- main
@@ -512,8 +670,9 @@ def main(argv=None):
     ap.add_argument("--ms", type=str, default=None, help="comma-separated M list for a prefill workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-prefill", action="store_true", help="skip the secondary prefill measurement")
-    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-secondary", action="store_true", help="only the headline decode measurement")
+    ap.add_argument("--gather", action="store_true", help="N > 1: all-gather y of the sharded matrix (timed apart)")
+    ap.add_argument("--cpu-budget", type=float, default=25.0)
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     rank, local_rank, world = dist_env()
@@ -522,12 +681,12 @@ def main(argv=None):
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cb, sec_per_step = oracle_decode_sample(args.cpu_budget)
-        line = {"metric": "prefill TFLOP/s (% bf16 TC peak); M=1 GEMV GB/s (% HBM peak)", "impl": "reference",
-                "value": cb["value"], "unit": cb["unit"], "n_gpus": args.gpus, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": sec_per_step * 1e3, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": "q4_0_decode_n12288_k4096", "M": [1, 8, 32]}, "cpu_baseline": cb,
+        cb, sec_per_step = oracle_decode_timing(args.steps, args.warmup, args.cpu_budget)
+        line = {"metric": METRIC, "impl": "reference", "value": cb["value"], "unit": cb["unit"],
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec_per_step * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded N(0, 0.02) weights, N(0, 1) bf16 activations)",
+                "config": decode_config(args.gpus), "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": cb["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
                 "gpu_launches": 0}
         print(json.dumps(line), flush=True)
@@ -544,18 +703,23 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
 
     if args.workload == "q4_0_decode":
-        r = run_decode(args, world, device, peaks)
-        if not args.no_prefill:
-            pre, _ = run_prefill(args, world, device, peaks, "affine4", (2048,))
-            r.setdefault("secondary", {})["prefill_affine4_n12288_k4096_m2048"] = pre["2048"]
+        r = run_decode(args, world, rank, device, peaks)
+        if not args.no_secondary and world == 1:
+            sec = r["secondary"]
+            for fmt, Ms in (("q4_0", (512, 2048, 8192)), ("affine4", (512, 2048, 8192)),
+                            ("affine8", (1, 32, 64, 128, 256, 512, 2048, 8192))):
+                res, cross = run_prefill(args, world, device, peaks, fmt, Ms)
+                sec[f"{fmt}_n12288_k4096"] = {"per_m": res, "crossover_m": cross}
+            sec["q4_0_m16_n256_k512"] = run_small(args, device, peaks)
+            per_m, packed, params, _ = run_stack(args, world, device, peaks)
+            sec["llama3.2_1b_q4_0_projection_stack"] = {"per_m": per_m, "packed_bytes": packed, "params": params}
     elif args.workload == "llama1b_stack":
         with ClockSampler(local_rank) as clk:
             per_m, packed, params, launches = run_stack(args, world, device, peaks)
         r = {"value": per_m["512"]["tokens_per_s"], "unit": "tokens/s", "ms_per_step": per_m["512"]["us_per_stack"] / 1e3,
              "dtype": "q4_0 weights, bf16 activations, fp32 accumulate",
              "config": {"workload": "llama3.2_1b_q4_0_projection_stack_16_layers", "M": [512, 1],
-                        "params": params, "packed_bytes": packed,
-                        "l2": f"{packed / 1e6:.0f} MB of distinct packed weights per stack (> 126 MB L2)"},
+                        "params": params, "packed_bytes": packed},
              "per_m": per_m,
              "roofline": {"bound": "tensor", "kernel": "whole stack at M=512", "achieved": per_m["512"]["tflops"],
                           "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": per_m["512"]["frac_tensor"],
@@ -575,33 +739,38 @@ def main(argv=None):
              "clocks": clk.summary(), "gpu_launches": None, "e2e": None}
     else:
         fmt, Ms = {"affine4_prefill": ("affine4", (512, 2048, 8192)),
-                   "affine8_sweep": ("affine8", (1, 32, 512, 2048, 8192)),
+                   "affine8_sweep": ("affine8", (1, 32, 64, 128, 256, 512, 2048, 8192)),
                    "q4_0_prefill": ("q4_0", (512, 2048, 8192))}[args.workload]
         if args.ms:
             Ms = tuple(int(v) for v in args.ms.split(","))
         with ClockSampler(local_rank) as clk:
-            res, tflops = run_prefill(args, world, device, peaks, fmt, Ms)
+            res, cross = run_prefill(args, world, device, peaks, fmt, Ms)
+        big = [m for m in Ms if m > 32]
+        tflops = (sum(2.0 * m * 12288 * 4096 for m in big) /
+                  sum(res[str(m)]["auto_us"] * 1e-6 for m in big) / 1e12) if big else 0.0
         r = {"value": round(tflops, 1), "unit": "TFLOP/s", "ms_per_step": None, "higher_is_better": True,
              "dtype": f"{fmt} weights, bf16 activations, fp32 accumulate",
              "config": {"workload": f"{fmt}_g{_fmt_args(fmt)[0]}_n12288_k4096", "M": list(Ms)}, "per_m": res,
-             "crossover_m": next((int(m) for m, v in res.items() if v["pair_us"] < v["fused_us"]), None),
+             "crossover_m": cross,
              "roofline": {"bound": "tensor", "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                           "frac": round(tflops / peaks["bf16_tflops"], 4), "achieved": round(tflops, 1),
                           "traffic": None},
              "clocks": clk.summary(), "gpu_launches": None, "e2e": None}
     r["roofline"]["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
 
-    line = {"metric": "prefill TFLOP/s (% bf16 TC peak); M=1 GEMV GB/s (% HBM peak)", "value": r["value"],
-            "unit": r["unit"], "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": r["dtype"], "data": "synthetic (seeded N(0, 0.02) weights, N(0, 1) bf16 activations)",
-            "config": dict(r["config"], parallelism=f"replicas x{world}")}
-    for k in ("per_m", "per_format", "crossover_m", "roofline", "e2e", "gpu_launches", "clocks", "secondary"):
-        if k in r:
+    line = {"metric": METRIC, "value": r["value"], "unit": r["unit"], "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": r["dtype"],
+            "data": "synthetic (seeded N(0, 0.02) weights, N(0, 1) bf16 activations)", "config": r["config"]}
+    for k in ("frac_hbm", "notes", "per_m", "per_format", "crossover_m", "roofline", "e2e", "gpu_launches", "clocks",
+              "gather", "secondary"):
+        if k in r and r[k] is not None:
             line[k] = r[k]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb, _ = oracle_decode_sample(args.cpu_budget)
+        cb, _ = oracle_decode_timing(max(1, int(args.cpu_budget / 2)), 1, args.cpu_budget / 2)
         line["cpu_baseline"] = cb
+        if args.workload == "q4_0_decode" and not args.no_secondary:
+            line.setdefault("secondary", {})["oracle_cpu_affine4_prefill"] = oracle_prefill_timing(args.cpu_budget)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

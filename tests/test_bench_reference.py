@@ -29,7 +29,8 @@ def test_reference_arm_line(monkeypatch):
     assert line["metric"] == "prefill TFLOP/s (% bf16 TC peak); M=1 GEMV GB/s (% HBM peak)"
     assert line["unit"] == "GB/s" and line["higher_is_better"] is True
     assert line["value"] > 0 and line["steps"] == 1 and line["warmup"] == 3
-    assert line["config"]["workload"] == "q4_0_decode_n12288_k4096"
+    assert line["config"] == bench.decode_config(1)           # the GPU arm's config, key for key
+    assert line["config"]["workload"] == "q4_0_decode_m1_n12288_k4096" and line["config"]["M"] == 1
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
