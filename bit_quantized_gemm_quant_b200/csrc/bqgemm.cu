@@ -8,7 +8,9 @@
 #include <type_traits>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <vector>
 
 #include "bqgemm.h"
 #include "common.cuh"
@@ -16,6 +18,7 @@
 #include "gemv.cuh"
 #include "gemv_q8.cuh"
 #include "gemv_affine.cuh"
+#include "gemv_stream.cuh"
 #include "tc_gemm.cuh"
 
 namespace bq {
@@ -444,6 +447,191 @@ bq_status launch_gemv(const uint16_t* x, const void* wq, const uint16_t* s, cons
     return launch_gemv_cfg<F, 4, 2, 8, 1, 1>(x, wq, s, b, y, M, N, K, group_size, st);
 }
 
+// ------------------------------------------------------------------ streamed decode GEMV
+// Plan of gemv_stream_kernel for one problem: K chunk, ring depth, grid and the
+// shared-memory carve-up.  Applies to 1..8 tokens, Q4_0 and affine 4/8-bit,
+// when K is a multiple of 8 groups (every row's codes and scales of a chunk are
+// then whole 16-byte runs that bulk copies can move); false otherwise.
+constexpr int kSgWarps = 8;
+constexpr int kSgStaticSmem = 2048;   // the kernel's static shared arrays, rounded up
+
+struct SgPlan {
+    SGemvParams prm{};
+    int grid = 0;
+    int su = 0;               // units of every warp's slice of a full chunk when equal and 8/16/32, else 0
+    size_t smem = 0;
+};
+
+// The matrices of one streamed launch: one, or up to kSgMaxMats sharing x.
+struct SgMats {
+    int count = 0;
+    const void* wq[kSgMaxMats] = {};
+    const uint16_t* scales[kSgMaxMats] = {};
+    const uint16_t* biases[kSgMaxMats] = {};
+    uint16_t* y[kSgMaxMats] = {};
+    int64_t N[kSgMaxMats] = {};
+};
+
+bool plan_stream_gemv(WFmt fmt, int group_size, int64_t M, const SgMats& mats, int64_t K, const DeviceInfo& di,
+                      SgPlan* pl)
+{
+    if (fmt != WFmt::Q4_0 && fmt != WFmt::AFF4 && fmt != WFmt::AFF8) return false;
+    if (M < 1 || M > kSgMaxTokens || K < 1 || K > INT32_MAX / 16 || mats.count < 1 || mats.count > kSgMaxMats)
+        return false;
+    const int gs = fmt == WFmt::Q4_0 ? 32 : group_size;
+    if (K % (8 * gs) != 0) return false;
+    const int bits = fmt == WFmt::AFF8 ? 8 : 4, E = bits == 8 ? 16 : 32;
+    const int upg = gs / E, atom_units = upg > 2 ? upg : 2;
+    const int kc = (int)std::min<int64_t>(K, 8192);                   // a multiple of 8 x 128
+    const int nchunks = (int)((K + kc - 1) / kc);
+    SGemvParams& p = pl->prm;
+    p = SGemvParams{};
+    int64_t ntiles = 0;
+    p.count = mats.count;
+    for (int i = 0; i < mats.count; ++i) {
+        if (mats.N[i] < 0 || mats.N[i] > INT32_MAX / 2) return false;
+        p.tile_begin[i] = (int)ntiles;
+        ntiles += (mats.N[i] + 15) / 16;
+        if (ntiles > INT32_MAX / 2) return false;
+        p.wq[i] = reinterpret_cast<const uint8_t*>(mats.wq[i]);
+        p.scales[i] = mats.scales[i];
+        p.biases[i] = mats.biases[i];
+        p.y[i] = mats.y[i];
+        p.N[i] = (int)mats.N[i];
+    }
+    p.tile_begin[mats.count] = (int)ntiles;
+    if (ntiles == 0) return false;
+    // one CTA per SM; at most 8 tiles per CTA (more CTAs, in waves, for very tall W)
+    const int64_t grid = ntiles <= 8 * (int64_t)di.num_sms ? std::min<int64_t>(ntiles, di.num_sms) : (ntiles + 7) / 8;
+    const int64_t tcap = (ntiles + grid - 1) / grid;
+    // a warp's slice of a full chunk: at most ceil(atoms / warps) atoms; its scale
+    // run covers 2 bytes per group plus up to 15 bytes of alignment on each side
+    const int64_t natoms = kc / E / atom_units;
+    const int64_t nc_max = (natoms + kSgWarps - 1) / kSgWarps * atom_units;       // 16-byte code units
+    const int64_t gpw = nc_max / upg;                                              // groups
+    const int64_t ns_max = (2 * gpw + 30) / 16;                                    // 16-byte scale runs
+    // row pitches: odd multiples of 16 bytes, so 8 rows fall in 8 distinct bank groups
+    auto odd16 = [](int64_t units) { return (units % 2 == 0 ? units + 1 : units) * 16; };
+    const int64_t code_pitch = odd16(nc_max + 1), scale_pitch = odd16(ns_max + 1);
+    const bool affine = fmt != WFmt::Q4_0;
+    const int64_t wstage = 16 * code_pitch + 16 * scale_pitch * (affine ? 2 : 1);
+    const int64_t nu = K / E, ng = K / gs;
+    const int64_t x_row = nu * 4 * (bits == 8 ? 8 : 16) + 64;            // activation-table bytes per token
+    int64_t off = 0;
+    const int64_t off_x = off;
+    off = (off + M * x_row + 127) / 128 * 128;
+    const int64_t off_c = off;
+    off = (off + ng * kSgMaxTokens * (affine ? 8 : 4) + 127) / 128 * 128;
+    const int64_t red_cols = (M + 1) / 2 * 2;
+    const int64_t red = std::max<int64_t>(tcap * kSgWarps * 16 * red_cols * 4, M * nu * 8);
+    const int64_t off_red = off;
+    off = (off + red + 127) / 128 * 128;
+    const int64_t off_ring = off;
+    const int64_t budget = (int64_t)di.max_smem_optin - kSgStaticSmem;
+    const int64_t stages = std::min<int64_t>(4, (budget - off_ring) / (kSgWarps * wstage));
+    if (stages < 2) return false;
+    p.M = (int)M;
+    p.K = (int)K;
+    p.kc = kc;
+    p.nchunks = nchunks;
+    p.ntiles = (int)ntiles;
+    p.stages = (int)stages;
+    p.code_pitch = (uint32_t)code_pitch;
+    p.scale_pitch = (uint32_t)scale_pitch;
+    p.wstage_bytes = (uint32_t)wstage;
+    p.x_row_bytes = (uint32_t)x_row;
+    p.red_cols = (int)red_cols;
+    p.mul24 = 1u << 24;
+    p.off_x = (uint32_t)off_x;
+    p.off_c = (uint32_t)off_c;
+    p.off_red = (uint32_t)off_red;
+    p.off_ring = (uint32_t)off_ring;
+    pl->grid = (int)grid;
+    const int64_t su = natoms % kSgWarps == 0 ? natoms / kSgWarps * atom_units : 0;
+    pl->su = (su == 8 || su == 16 || su == 32) ? (int)su : 0;
+    pl->smem = (size_t)(off_ring + stages * kSgWarps * wstage);
+    return true;
+}
+
+// Launch with programmatic stream serialization: the kernel's launch and
+// prologue may overlap the previous kernel on the stream; its reads of x, W and
+// scales and its writes of y come after griddepcontrol.wait.
+template <Fmt F, int GS, int SU>
+bq_status launch_stream_gemv_su(SgPlan& pl, int dev, const DeviceInfo& di, const uint16_t* x, cudaStream_t st)
+{
+    auto kern = gemv_stream_kernel<F, GS, kSgWarps, SU>;
+    static bool attr_done[kMaxDevices] = {};
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 di.max_smem_optin - kSgStaticSmem) != cudaSuccess)
+            return BQ_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    pl.prm.x = x;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)pl.grid);
+    cfg.blockDim = dim3(32 * kSgWarps);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, pl.prm) != cudaSuccess) {
+        cudaGetLastError();
+        return BQ_ERR_CUDA;
+    }
+    return launch_status();
+}
+
+template <Fmt F, int GS>
+bq_status launch_stream_gemv(SgPlan& pl, int dev, const DeviceInfo& di, const uint16_t* x, cudaStream_t st)
+{
+    switch (pl.su) {
+    case 8: return launch_stream_gemv_su<F, GS, 8>(pl, dev, di, x, st);
+    case 16: return launch_stream_gemv_su<F, GS, 16>(pl, dev, di, x, st);
+    case 32: return launch_stream_gemv_su<F, GS, 32>(pl, dev, di, x, st);
+    default: return launch_stream_gemv_su<F, GS, 0>(pl, dev, di, x, st);
+    }
+}
+
+// The streamed kernel when its plan applies (returns true and the launch status
+// in *out), else false and the caller takes the register-streaming GEMV.
+bool try_stream_gemv(WFmt fmt, int group_size, const uint16_t* x, const SgMats& mats, int64_t M, int64_t K, int dev,
+                     const DeviceInfo& di, cudaStream_t st, bq_status* out)
+{
+    SgPlan pl;
+    if (fmt != WFmt::AFF8) return false;    // the register-streaming GEMV is faster for the 4-bit formats
+    if (!plan_stream_gemv(fmt, group_size, M, mats, K, di, &pl)) return false;
+    switch (fmt) {
+    case WFmt::Q4_0: *out = launch_stream_gemv<Fmt::Q4_0, 32>(pl, dev, di, x, st); break;
+    case WFmt::AFF4:
+        *out = group_size == 32   ? launch_stream_gemv<Fmt::AFF4, 32>(pl, dev, di, x, st)
+               : group_size == 64 ? launch_stream_gemv<Fmt::AFF4, 64>(pl, dev, di, x, st)
+                                  : launch_stream_gemv<Fmt::AFF4, 128>(pl, dev, di, x, st);
+        break;
+    default:
+        *out = group_size == 32   ? launch_stream_gemv<Fmt::AFF8, 32>(pl, dev, di, x, st)
+               : group_size == 64 ? launch_stream_gemv<Fmt::AFF8, 64>(pl, dev, di, x, st)
+                                  : launch_stream_gemv<Fmt::AFF8, 128>(pl, dev, di, x, st);
+        break;
+    }
+    return true;
+}
+
+SgMats one_matrix(const void* wq, const uint16_t* s, const uint16_t* b, uint16_t* y, int64_t N)
+{
+    SgMats m;
+    m.count = 1;
+    m.wq[0] = wq;
+    m.scales[0] = s;
+    m.biases[0] = b;
+    m.y[0] = y;
+    m.N[0] = N;
+    return m;
+}
+
 // Decode GEMV for affine weights of any width (2-, 3- and 6-bit use it), M <= 8.
 bq_status launch_gemv_affine(WFmt fmt, const uint16_t* x, const void* wq, const uint16_t* s, const uint16_t* b,
                              uint16_t* y, int64_t M, int64_t N, int64_t K, int group_size, cudaStream_t st)
@@ -500,25 +688,38 @@ bq_status launch_gemv_multi(const uint16_t* x, GemvMultiTable& tab, int64_t M, i
 }
 
 // ------------------------------------------------------------------ library workspace
+// Scratch of the calls that get no caller workspace: one buffer per (device,
+// stream), so calls on different streams never share one.  A buffer only grows
+// (to the next power of two of the need), and a grown-out block is retired,
+// not freed: CUDA graphs captured earlier keep pointing at valid memory.
+// Retired blocks and live buffers are released when the process exits.
 struct Workspace {
     void* ptr = nullptr;
     size_t bytes = 0;
 };
-Workspace g_ws[kMaxDevices];
+struct WorkspaceKey {
+    int dev;
+    cudaStream_t stream;
+    bool operator<(const WorkspaceKey& o) const { return dev != o.dev ? dev < o.dev : stream < o.stream; }
+};
+std::map<WorkspaceKey, Workspace> g_ws;
+std::vector<void*> g_ws_retired;
 
-bq_status library_workspace(int dev, size_t need, void** out)
+bq_status library_workspace(int dev, cudaStream_t st, size_t need, void** out)
 {
     std::lock_guard<std::mutex> lk(g_mu);
-    Workspace& w = g_ws[dev];
+    Workspace& w = g_ws[WorkspaceKey{dev, st}];
     if (w.bytes < need) {
-        if (w.ptr) cudaFree(w.ptr);
-        w.ptr = nullptr;
-        w.bytes = 0;
-        if (cudaMalloc(&w.ptr, need) != cudaSuccess) {
-            w.ptr = nullptr;
+        size_t bytes = 1u << 20;
+        while (bytes < need) bytes <<= 1;
+        void* p = nullptr;
+        if (cudaMalloc(&p, bytes) != cudaSuccess) {
+            cudaGetLastError();
             return BQ_ERR_CUDA;
         }
-        w.bytes = need;
+        if (w.ptr) g_ws_retired.push_back(w.ptr);
+        w.ptr = p;
+        w.bytes = bytes;
     }
     *out = w.ptr;
     return BQ_OK;
@@ -639,6 +840,7 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
     switch (path) {
     case BQ_PATH_GEMV:
         if (!has_fast_paths(fmt)) return launch_gemv_affine(fmt, x, wq, sc, bi, y, M, N, K, group_size, st);
+        if (try_stream_gemv(fmt, group_size, x, one_matrix(wq, sc, bi, y, N), M, K, dev, di, st, &s)) return s;
         if (fmt == WFmt::Q4_0) return launch_gemv<Fmt::Q4_0>(x, wq, sc, bi, y, M, N, K, group_size, st);
         if (fmt == WFmt::AFF4) return launch_gemv<Fmt::AFF4>(x, wq, sc, bi, y, M, N, K, group_size, st);
         return launch_gemv<Fmt::AFF8>(x, wq, sc, bi, y, M, N, K, group_size, st);
@@ -649,7 +851,7 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
         void* ws = workspace;
         size_t wsb = workspace_bytes;
         if (!ws && need > 0) {
-            if ((s = library_workspace(dev, need, &ws)) != BQ_OK) return s;
+            if ((s = library_workspace(dev, st, need, &ws)) != BQ_OK) return s;
             wsb = need;
         }
         if (fmt == WFmt::Q4_0) return launch_tc<kModeQ4_0>(di, dev, x, wq, sc, bi, y, M, N, K, st, ws, wsb, group_size);
@@ -658,7 +860,7 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
     }
     default: {
         void* ws = workspace;
-        if (!ws && (s = library_workspace(dev, need, &ws)) != BQ_OK) return s;
+        if (!ws && (s = library_workspace(dev, st, need, &ws)) != BQ_OK) return s;
         uint16_t* wb = reinterpret_cast<uint16_t*>(ws);
         s = transpose ? dequant_any(fmt, wq, scales, biases, wb, N, K, group_size, di, st)
                       : dequant_affine_t(fmt, wq, scales, biases, wb, K, N, group_size, di, st);
@@ -672,22 +874,18 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
 // Scratch of quant_matmul_noalloc: the bf16 copy of W that the unfused pair
 // stages between its two kernels, as a fixed array of the device image.  Host
 // code must not pass the name itself to a kernel (on the host it is a stand-in,
-// not a device address); noalloc_scratch looks the address up per device.
+// not a device address); noalloc_scratch looks the address up on the current
+// device at every call (no allocation; never stale after a device reset).
 static __device__ __align__(256) uint8_t g_noalloc_scratch[BQ_NOALLOC_SCRATCH_BYTES];
-void* g_noalloc_ptr[kMaxDevices];
 
-bq_status noalloc_scratch(int dev, void** out)
+bq_status noalloc_scratch(void** out)
 {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_noalloc_ptr[dev]) {                // once per device, with `dev` current
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
-            cudaGetLastError();
-            return BQ_ERR_CUDA;
-        }
-        g_noalloc_ptr[dev] = p;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return BQ_ERR_CUDA;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = p;
     return BQ_OK;
 }
 
@@ -836,14 +1034,19 @@ bq_status quant_matmul_noalloc(const uint16_t* x_bf16, const void* wq, const voi
     if (M == 0 || N == 0 || K == 0)           // nothing to stage: no scratch involved
         return matmul_impl(x_bf16, wq, scales, biases, y_bf16, M, N, K, group_size, bits, transpose,
                            BQ_PATH_DEQUANT_GEMM, nullptr, 0, (cudaStream_t)stream);
-    if ((uint64_t)N > (uint64_t)(BQ_NOALLOC_SCRATCH_BYTES / 2u) / (uint64_t)K) return BQ_ERR_WORKSPACE;
+    // quant_matmul's own path, with the fixed array as its scratch: the decode
+    // GEMV needs none, the fused kernel keeps its K-split partial sums there (or
+    // runs unsplit if they do not fit), the unfused pair stages W there.
+    const int path = transpose ? select_path(M, K, fmt) : BQ_PATH_DEQUANT_GEMM;
+    if (path == BQ_PATH_DEQUANT_GEMM && (uint64_t)N > (uint64_t)(BQ_NOALLOC_SCRATCH_BYTES / 2u) / (uint64_t)K)
+        return BQ_ERR_WORKSPACE;
     int dev;
     DeviceInfo di;
     if ((s = current_device(&dev, &di)) != BQ_OK) return s;
     void* ws = nullptr;
-    if ((s = noalloc_scratch(dev, &ws)) != BQ_OK) return s;
-    return matmul_impl(x_bf16, wq, scales, biases, y_bf16, M, N, K, group_size, bits, transpose,
-                       BQ_PATH_DEQUANT_GEMM, ws, BQ_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream);
+    if ((s = noalloc_scratch(&ws)) != BQ_OK) return s;
+    return matmul_impl(x_bf16, wq, scales, biases, y_bf16, M, N, K, group_size, bits, transpose, path, ws,
+                       BQ_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream);
 }
 
 bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const void* const* wq, const void* const* scales,
@@ -891,6 +1094,16 @@ bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const void* cons
     DeviceInfo di;
     if ((s = current_device(&dev, &di)) != BQ_OK) return s;
     const cudaStream_t st = (cudaStream_t)stream;
+    SgMats mats;
+    mats.count = count;
+    for (int i = 0; i < count; ++i) {
+        mats.wq[i] = wq[i];
+        mats.scales[i] = tab.scales[i];
+        mats.biases[i] = tab.biases[i];
+        mats.y[i] = y_bf16[i];
+        mats.N[i] = N[i];
+    }
+    if (try_stream_gemv(fmt, group_size, x_bf16, mats, M, K, dev, di, st, &s)) return s;
     if (fmt == WFmt::Q4_0) return launch_gemv_multi<Fmt::Q4_0>(x_bf16, tab, M, K, group_size, st);
     if (fmt == WFmt::AFF4) return launch_gemv_multi<Fmt::AFF4>(x_bf16, tab, M, K, group_size, st);
     return launch_gemv_multi<Fmt::AFF8>(x_bf16, tab, M, K, group_size, st);

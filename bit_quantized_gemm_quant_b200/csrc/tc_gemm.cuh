@@ -86,11 +86,6 @@ __host__ __device__ constexpr uint32_t tc_stage_bytes(int mode, int bn)
 // UMMA descriptor describes): chunk c of row r sits at position c ^ (r mod 8).
 BQ_DEVINL uint32_t sw128_offset(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
-BQ_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
-{
-    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
 // --- dequantization of one thread's 32 weights (half a k-block of one row) ---
 // Each returns 16 bf16x2 registers in natural K order: out[j] = (2j, 2j+1).
 

@@ -87,6 +87,11 @@ BQ_DEVINL uint4 ld_shared_v4(uint32_t addr)
     return v;
 }
 
+BQ_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 BQ_DEVINL void tma_prefetch_desc(const CUtensorMap* map)
 {

@@ -187,9 +187,18 @@ BQ_API bq_status quant_matmul_q8(const int8_t* xq, const float* dx, const int32_
  * pair at every M; 4- and 8-bit and Q4_0 have the decode GEMV and the fused
  * kernel as well.
  * The path is chosen by quant_matmul_select_path.  A path that needs scratch
- * memory (the unfused pair) uses a per-device buffer that the library
- * allocates on first need, grows on demand and keeps until process exit; a
- * first call that allocates must therefore not be made during stream capture.
+ * memory (the unfused pair's bf16 copy of W, the fused kernel's split-K
+ * partial sums) uses a library buffer, one per (device, stream):
+ *   - it is allocated on first need and grows on demand; a call that
+ *     allocates must not be made during stream capture, so make one call per
+ *     stream and problem size before capturing;
+ *   - growing never frees the old block (it is kept until the process exits),
+ *     so graphs captured before a growth stay valid;
+ *   - calls on one stream are ordered and share the stream's buffer safely;
+ *     calls on different streams use different buffers and do not race;
+ *   - a captured graph keeps the buffer of the stream it was captured on:
+ *     replays of it must not overlap on the GPU with each other or with
+ *     other calls that use that stream's buffer.
  */
 BQ_API bq_status quant_matmul(const uint16_t* x_bf16, const void* wq, const void* scales, const void* biases,
                        uint16_t* y_bf16, int64_t M, int64_t N, int64_t K, int group_size, int bits,
@@ -201,21 +210,25 @@ BQ_API bq_status quant_matmul(const uint16_t* x_bf16, const void* wq, const void
  * library may not call cudaMalloc: hosts that own all device memory through
  * their own pool or that budget it once at start-up, and latency-critical
  * callers that cannot afford an allocation's implicit synchronization on a
- * first call.  It computes the same y as quant_matmul, always through the
- * unfused pair (q4_0_dequantize / affine_dequantize into scratch, then the
- * bf16 tensor-core GEMM), with the bf16 copy of W staged in a fixed 32 MiB
- * array that is part of the library's device image.
+ * first call.  It takes quant_matmul's own path, with a fixed 32 MiB array
+ * that is part of the library's device image as its scratch: the decode GEMV
+ * uses none; the fused tensor-core kernel keeps its K-split partial sums there
+ * (and runs without splitting K when they would not fit); the unfused pair
+ * (q4_0_dequantize / affine_dequantize, then the bf16 tensor-core GEMM) stages
+ * the bf16 copy of W there.  y is the same as quant_matmul's.
  *   Arguments, layouts, validation and errors are those of quant_matmul
  *   (both orientations).
- *   Limit: N * K * 2 bytes must fit in BQ_NOALLOC_SCRATCH_BYTES (N * K at most
- *   16,777,216 weights, e.g. 4096 x 4096); larger problems return
- *   BQ_ERR_WORKSPACE before anything is launched.
+ *   Limit: where the path is the unfused pair, N * K * 2 bytes must fit in
+ *   BQ_NOALLOC_SCRATCH_BYTES (N * K at most 16,777,216 weights, e.g. 4096 x
+ *   4096); larger problems there return BQ_ERR_WORKSPACE before anything is
+ *   launched.
  *   Memory: every device that loads the library holds the 32 MiB array until
  *   the process exits.  The call itself makes no cudaMalloc / cudaFree and calls
  *   no allocating library routine.
- *   Set-up: the first call on each device, with that device current, looks up
- *   the array's device address (cudaGetSymbolAddress) and caches it; make that
- *   first call before any stream capture.
+ *   Set-up: every call looks up the array's device address on the current
+ *   device (cudaGetSymbolAddress: no allocation), so the address is never
+ *   stale, also after cudaDeviceReset.  The first call on a device also loads
+ *   the library's device code there; make it before any stream capture.
  *   Sharing: all calls on a device use the same array and it keeps the last
  *   call's contents (each call overwrites the part it uses before reading it).
  *   Calls whose execution overlaps on the GPU -- on different streams without
