@@ -21,8 +21,9 @@ LIB_PATH = os.path.join(_PKG, "libbqgemm.so")
 BQ_OK = 0
 STATUS = {0: "BQ_OK", 1: "BQ_ERR_NULL", 2: "BQ_ERR_SHAPE", 3: "BQ_ERR_UNSUPPORTED", 4: "BQ_ERR_ALIGN",
           5: "BQ_ERR_CUDA", 6: "BQ_ERR_TIMEOUT", 7: "BQ_ERR_WORKSPACE", 8: "BQ_ERR_DEVICE"}
-PATH_AUTO, PATH_GEMV, PATH_TC_FUSED, PATH_DEQUANT_GEMM = 0, 1, 2, 3
-PATHS = {"auto": PATH_AUTO, "gemv": PATH_GEMV, "tc_fused": PATH_TC_FUSED, "dequant_gemm": PATH_DEQUANT_GEMM}
+PATH_AUTO, PATH_GEMV, PATH_TC_FUSED, PATH_DEQUANT_GEMM, PATH_GEMV_STREAM = 0, 1, 2, 3, 4
+PATHS = {"auto": PATH_AUTO, "gemv": PATH_GEMV, "tc_fused": PATH_TC_FUSED, "dequant_gemm": PATH_DEQUANT_GEMM,
+         "gemv_stream": PATH_GEMV_STREAM}
 
 _lib = None
 

@@ -447,19 +447,24 @@ bq_status launch_gemv(const uint16_t* x, const void* wq, const uint16_t* s, cons
     return launch_gemv_cfg<F, 4, 2, 8, 1, 1>(x, wq, s, b, y, M, N, K, group_size, st);
 }
 
+bq_status library_workspace(int dev, cudaStream_t st, size_t need, void** out);
+
 // ------------------------------------------------------------------ streamed decode GEMV
-// Plan of gemv_stream_kernel for one problem: K chunk, ring depth, grid and the
-// shared-memory carve-up.  Applies to 1..8 tokens, Q4_0 and affine 4/8-bit,
-// when K is a multiple of 8 groups (every row's codes and scales of a chunk are
-// then whole 16-byte runs that bulk copies can move); false otherwise.
+// Plan of gemv_stream_kernel for one problem: K chunk, ring depth, grid, the
+// shared-memory carve-up and the activation tables.  Applies to one or two
+// tokens, Q4_0 and affine 4/8-bit, when K is a multiple of 8 groups (every
+// row's codes and scales of a chunk are then whole 16-byte runs that 16-byte
+// copies can move); false otherwise.
 constexpr int kSgWarps = 8;
-constexpr int kSgStaticSmem = 2048;   // the kernel's static shared arrays, rounded up
+constexpr int kSgStaticSmem = 1024;   // the kernel's static shared arrays, rounded up
 
 struct SgPlan {
     SGemvParams prm{};
     int grid = 0;
     int su = 0;               // units of every warp's slice of a full chunk when equal and 8/16/32, else 0
     size_t smem = 0;
+    int prep_grid = 0;        // CTAs of gemv_int_prep_kernel
+    size_t tab_bytes = 0;     // device bytes of its tables and flags
 };
 
 // The matrices of one streamed launch: one, or up to kSgMaxMats sharing x.
@@ -472,17 +477,38 @@ struct SgMats {
     int64_t N[kSgMaxMats] = {};
 };
 
+// Activation-table bytes of the streamed GEMV (slices, group table, one flag
+// word per prep CTA), or 0 when it does not apply to (fmt, M, K).
+size_t stream_gemv_table_bytes(WFmt fmt, int group_size, int64_t M, int64_t K, int* prep_grid = nullptr)
+{
+    if (fmt != WFmt::Q4_0 && fmt != WFmt::AFF4 && fmt != WFmt::AFF8) return 0;
+    const int gs = fmt == WFmt::Q4_0 ? 32 : group_size;
+    if (M < 1 || M > kSgIntTokens || K < 1 || K > INT32_MAX / 16 || K % (8 * gs) != 0) return 0;
+    const int64_t items = M * (K / 32) * 4;
+    const int64_t grid = (items + kSgPrepThreads - 1) / kSgPrepThreads;
+    if (prep_grid) *prep_grid = (int)grid;
+    return (size_t)((K / 32) * kSgIntStepBytes + (K / gs) * kSgIntCtabBytes + (grid * 4 + 15) / 16 * 16);
+}
+
+// BQ_PATH_GEMV takes the streamed kernel where it measured faster than the
+// register-streaming one on B200 (N = 12288, K = 4096, graph-timed launches
+// over rotating weight copies): affine 8-bit with one or two tokens (17.4 against
+// 18.3 us).  For Q4_0 and affine 4-bit the register-streaming kernel is faster
+// (12.6 against 14.5 us at M = 1).
+bool stream_gemv_preferred(WFmt fmt, int64_t M) { return fmt == WFmt::AFF8 && M <= kSgIntTokens; }
+
 bool plan_stream_gemv(WFmt fmt, int group_size, int64_t M, const SgMats& mats, int64_t K, const DeviceInfo& di,
                       SgPlan* pl)
 {
-    if (fmt != WFmt::Q4_0 && fmt != WFmt::AFF4 && fmt != WFmt::AFF8) return false;
-    if (M < 1 || M > kSgMaxTokens || K < 1 || K > INT32_MAX / 16 || mats.count < 1 || mats.count > kSgMaxMats)
-        return false;
+    int prep_grid = 0;
+    const size_t tab_bytes = stream_gemv_table_bytes(fmt, group_size, M, K, &prep_grid);
+    if (tab_bytes == 0 || mats.count < 1 || mats.count > kSgMaxMats) return false;
     const int gs = fmt == WFmt::Q4_0 ? 32 : group_size;
-    if (K % (8 * gs) != 0) return false;
     const int bits = fmt == WFmt::AFF8 ? 8 : 4, E = bits == 8 ? 16 : 32;
     const int upg = gs / E, atom_units = upg > 2 ? upg : 2;
-    const int kc = (int)std::min<int64_t>(K, 8192);                   // a multiple of 8 x 128
+    // K chunk: whole rows up to 4096 elements (a multiple of 8 x 128); 8-bit codes in
+    // 2048-element chunks measured slower (21.4 against 17.4 us at N = 12288, K = 4096)
+    const int kc = (int)std::min<int64_t>(K, 4096);
     const int nchunks = (int)((K + kc - 1) / kc);
     SGemvParams& p = pl->prm;
     p = SGemvParams{};
@@ -501,7 +527,8 @@ bool plan_stream_gemv(WFmt fmt, int group_size, int64_t M, const SgMats& mats, i
     }
     p.tile_begin[mats.count] = (int)ntiles;
     if (ntiles == 0) return false;
-    // one CTA per SM; at most 8 tiles per CTA (more CTAs, in waves, for very tall W)
+    // one CTA per SM over a contiguous range of tiles; at most 8 tiles per CTA
+    // (more CTAs, in waves, for very tall W)
     const int64_t grid = ntiles <= 8 * (int64_t)di.num_sms ? std::min<int64_t>(ntiles, di.num_sms) : (ntiles + 7) / 8;
     const int64_t tcap = (ntiles + grid - 1) / grid;
     // a warp's slice of a full chunk: at most ceil(atoms / warps) atoms; its scale
@@ -512,20 +539,20 @@ bool plan_stream_gemv(WFmt fmt, int group_size, int64_t M, const SgMats& mats, i
     const int64_t ns_max = (2 * gpw + 30) / 16;                                    // 16-byte scale runs
     // row pitches: odd multiples of 16 bytes, so 8 rows fall in 8 distinct bank groups
     auto odd16 = [](int64_t units) { return (units % 2 == 0 ? units + 1 : units) * 16; };
-    const int64_t code_pitch = odd16(nc_max + 1), scale_pitch = odd16(ns_max + 1);
+    const int64_t code_pitch = odd16(nc_max + 1), scale_pitch = odd16(ns_max);
     const bool affine = fmt != WFmt::Q4_0;
     const int64_t wstage = 16 * code_pitch + 16 * scale_pitch * (affine ? 2 : 1);
-    const int64_t nu = K / E, ng = K / gs;
-    const int64_t x_row = nu * 4 * (bits == 8 ? 8 : 16) + 64;            // activation-table bytes per token
+    // shared memory: the activation tables ([K/32 steps] x 256 bytes, [groups] x
+    // 64 bytes), the per-warp partial sums of the CTA's tiles, the rings
+    const int64_t x_bytes = (K / 32) * kSgIntStepBytes, c_bytes = (K / gs) * kSgIntCtabBytes;
     int64_t off = 0;
     const int64_t off_x = off;
-    off = (off + M * x_row + 127) / 128 * 128;
+    off = (off + x_bytes + 127) / 128 * 128;
     const int64_t off_c = off;
-    off = (off + ng * kSgMaxTokens * (affine ? 8 : 4) + 127) / 128 * 128;
-    const int64_t red_cols = (M + 1) / 2 * 2;
-    const int64_t red = std::max<int64_t>(tcap * kSgWarps * 16 * red_cols * 4, M * nu * 8);
+    off = (off + c_bytes + 127) / 128 * 128;
+    const int64_t red_cols = 2;
     const int64_t off_red = off;
-    off = (off + red + 127) / 128 * 128;
+    off = (off + tcap * kSgWarps * 16 * red_cols * 4 + 127) / 128 * 128;
     const int64_t off_ring = off;
     const int64_t budget = (int64_t)di.max_smem_optin - kSgStaticSmem;
     const int64_t stages = std::min<int64_t>(4, (budget - off_ring) / (kSgWarps * wstage));
@@ -539,14 +566,17 @@ bool plan_stream_gemv(WFmt fmt, int group_size, int64_t M, const SgMats& mats, i
     p.code_pitch = (uint32_t)code_pitch;
     p.scale_pitch = (uint32_t)scale_pitch;
     p.wstage_bytes = (uint32_t)wstage;
-    p.x_row_bytes = (uint32_t)x_row;
     p.red_cols = (int)red_cols;
-    p.mul24 = 1u << 24;
     p.off_x = (uint32_t)off_x;
     p.off_c = (uint32_t)off_c;
     p.off_red = (uint32_t)off_red;
     p.off_ring = (uint32_t)off_ring;
+    p.tab_c_off = (uint32_t)x_bytes;
+    p.tab_f_off = (uint32_t)(x_bytes + c_bytes);
+    p.nflags = prep_grid;
     pl->grid = (int)grid;
+    pl->prep_grid = prep_grid;
+    pl->tab_bytes = tab_bytes;
     const int64_t su = natoms % kSgWarps == 0 ? natoms / kSgWarps * atom_units : 0;
     pl->su = (su == 8 || su == 16 || su == 32) ? (int)su : 0;
     pl->smem = (size_t)(off_ring + stages * kSgWarps * wstage);
@@ -554,10 +584,30 @@ bool plan_stream_gemv(WFmt fmt, int group_size, int64_t M, const SgMats& mats, i
 }
 
 // Launch with programmatic stream serialization: the kernel's launch and
-// prologue may overlap the previous kernel on the stream; its reads of x, W and
-// scales and its writes of y come after griddepcontrol.wait.
+// prologue may overlap the previous kernel on the stream; its reads of x,
+// tables, W and scales and its writes come after griddepcontrol.wait.
+template <typename KernelT, typename... Args>
+bq_status launch_pdl(KernelT kern, int grid, int threads, size_t smem, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess) {
+        cudaGetLastError();
+        return BQ_ERR_CUDA;
+    }
+    return launch_status();
+}
+
 template <Fmt F, int GS, int SU>
-bq_status launch_stream_gemv_su(SgPlan& pl, int dev, const DeviceInfo& di, const uint16_t* x, cudaStream_t st)
+bq_status launch_stream_gemv_su(SgPlan& pl, int dev, const DeviceInfo& di, cudaStream_t st)
 {
     auto kern = gemv_stream_kernel<F, GS, kSgWarps, SU>;
     static bool attr_done[kMaxDevices] = {};
@@ -567,54 +617,54 @@ bq_status launch_stream_gemv_su(SgPlan& pl, int dev, const DeviceInfo& di, const
             return BQ_ERR_CUDA;
         attr_done[dev] = true;
     }
-    pl.prm.x = x;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)pl.grid);
-    cfg.blockDim = dim3(32 * kSgWarps);
-    cfg.dynamicSmemBytes = pl.smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, pl.prm) != cudaSuccess) {
-        cudaGetLastError();
-        return BQ_ERR_CUDA;
-    }
-    return launch_status();
+    return launch_pdl(kern, pl.grid, 32 * kSgWarps, pl.smem, st, pl.prm);
 }
 
+// The activation tables, then the streamed kernel.
 template <Fmt F, int GS>
-bq_status launch_stream_gemv(SgPlan& pl, int dev, const DeviceInfo& di, const uint16_t* x, cudaStream_t st)
+bq_status launch_stream_gemv(SgPlan& pl, int dev, const DeviceInfo& di, const uint16_t* x, uint8_t* tab,
+                             cudaStream_t st)
 {
+    pl.prm.x = x;
+    pl.prm.tab = tab;
+    bq_status s = launch_pdl(gemv_int_prep_kernel<F, GS>, pl.prep_grid, kSgPrepThreads, 0, st, x, pl.prm.M,
+                             pl.prm.K, tab, pl.prm.tab_c_off, pl.prm.tab_f_off);
+    if (s != BQ_OK) return s;
     switch (pl.su) {
-    case 8: return launch_stream_gemv_su<F, GS, 8>(pl, dev, di, x, st);
-    case 16: return launch_stream_gemv_su<F, GS, 16>(pl, dev, di, x, st);
-    case 32: return launch_stream_gemv_su<F, GS, 32>(pl, dev, di, x, st);
-    default: return launch_stream_gemv_su<F, GS, 0>(pl, dev, di, x, st);
+    case 8: return launch_stream_gemv_su<F, GS, 8>(pl, dev, di, st);
+    case 16: return launch_stream_gemv_su<F, GS, 16>(pl, dev, di, st);
+    case 32: return launch_stream_gemv_su<F, GS, 32>(pl, dev, di, st);
+    default: return launch_stream_gemv_su<F, GS, 0>(pl, dev, di, st);
     }
 }
 
 // The streamed kernel when its plan applies (returns true and the launch status
-// in *out), else false and the caller takes the register-streaming GEMV.
+// in *out), else false and the caller takes the register-streaming GEMV.  Its
+// tables go in the caller's workspace when one is given (false if it is too
+// small), else in the library's buffer of this stream.
 bool try_stream_gemv(WFmt fmt, int group_size, const uint16_t* x, const SgMats& mats, int64_t M, int64_t K, int dev,
-                     const DeviceInfo& di, cudaStream_t st, bq_status* out)
+                     const DeviceInfo& di, cudaStream_t st, void* workspace, size_t workspace_bytes, bq_status* out)
 {
     SgPlan pl;
-    if (fmt != WFmt::AFF8) return false;    // the register-streaming GEMV is faster for the 4-bit formats
     if (!plan_stream_gemv(fmt, group_size, M, mats, K, di, &pl)) return false;
+    void* tab = workspace;
+    if (tab) {
+        if (workspace_bytes < pl.tab_bytes) return false;
+    } else if ((*out = library_workspace(dev, st, pl.tab_bytes, &tab)) != BQ_OK) {
+        return true;
+    }
+    uint8_t* t = reinterpret_cast<uint8_t*>(tab);
     switch (fmt) {
-    case WFmt::Q4_0: *out = launch_stream_gemv<Fmt::Q4_0, 32>(pl, dev, di, x, st); break;
+    case WFmt::Q4_0: *out = launch_stream_gemv<Fmt::Q4_0, 32>(pl, dev, di, x, t, st); break;
     case WFmt::AFF4:
-        *out = group_size == 32   ? launch_stream_gemv<Fmt::AFF4, 32>(pl, dev, di, x, st)
-               : group_size == 64 ? launch_stream_gemv<Fmt::AFF4, 64>(pl, dev, di, x, st)
-                                  : launch_stream_gemv<Fmt::AFF4, 128>(pl, dev, di, x, st);
+        *out = group_size == 32   ? launch_stream_gemv<Fmt::AFF4, 32>(pl, dev, di, x, t, st)
+               : group_size == 64 ? launch_stream_gemv<Fmt::AFF4, 64>(pl, dev, di, x, t, st)
+                                  : launch_stream_gemv<Fmt::AFF4, 128>(pl, dev, di, x, t, st);
         break;
     default:
-        *out = group_size == 32   ? launch_stream_gemv<Fmt::AFF8, 32>(pl, dev, di, x, st)
-               : group_size == 64 ? launch_stream_gemv<Fmt::AFF8, 64>(pl, dev, di, x, st)
-                                  : launch_stream_gemv<Fmt::AFF8, 128>(pl, dev, di, x, st);
+        *out = group_size == 32   ? launch_stream_gemv<Fmt::AFF8, 32>(pl, dev, di, x, t, st)
+               : group_size == 64 ? launch_stream_gemv<Fmt::AFF8, 64>(pl, dev, di, x, t, st)
+                                  : launch_stream_gemv<Fmt::AFF8, 128>(pl, dev, di, x, t, st);
         break;
     }
     return true;
@@ -726,10 +776,16 @@ bq_status library_workspace(int dev, cudaStream_t st, size_t need, void** out)
 }
 
 // Workspace of a path: the bf16 copy of W for the pair; the K-split partial
-// sums for the fused kernel when its plan splits K (0 otherwise).
-size_t workspace_for(int path, WFmt fmt, int64_t M, int64_t N, int64_t K, int num_sms, int smem_optin)
+// sums for the fused kernel when its plan splits K; the activation tables of
+// the streamed decode GEMV (one or two tokens); 0 otherwise.
+size_t workspace_for(int path, WFmt fmt, int group_size, int64_t M, int64_t N, int64_t K, int num_sms,
+                     int smem_optin)
 {
     if (path == BQ_PATH_DEQUANT_GEMM) return (size_t)N * (size_t)K * 2u;
+    if (path == BQ_PATH_GEMV)
+        return has_fast_paths(fmt) && stream_gemv_preferred(fmt, M) ? stream_gemv_table_bytes(fmt, group_size, M, K)
+                                                                    : 0u;
+    if (path == BQ_PATH_GEMV_STREAM) return has_fast_paths(fmt) ? stream_gemv_table_bytes(fmt, group_size, M, K) : 0u;
     if (path != BQ_PATH_TC_FUSED || !has_fast_paths(fmt) || K % 64 != 0 || M > INT32_MAX || N > INT32_MAX ||
         K > INT32_MAX)
         return 0u;
@@ -796,7 +852,7 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
                       void* workspace, size_t workspace_bytes, cudaStream_t st)
 {
     if (transpose != 0 && transpose != 1) return BQ_ERR_UNSUPPORTED;
-    if (path < BQ_PATH_AUTO || path > BQ_PATH_DEQUANT_GEMM) return BQ_ERR_UNSUPPORTED;
+    if (path < BQ_PATH_AUTO || path > BQ_PATH_GEMV_STREAM) return BQ_ERR_UNSUPPORTED;
     if (M < 0 || N < 0 || K < 0) return BQ_ERR_SHAPE;
     // transpose = 0: y = x . W with W stored [K][N], codes and groups along N
     // (affine only: Q4_0 blocks run along K); it runs as the unfused pair with
@@ -807,7 +863,8 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
                             : check_format(biases, K, N, group_size, bits, &fmt);
     if (s != BQ_OK) return s;
     if (transpose == 0) {
-        if (path == BQ_PATH_GEMV || path == BQ_PATH_TC_FUSED) return BQ_ERR_UNSUPPORTED;
+        if (path == BQ_PATH_GEMV || path == BQ_PATH_TC_FUSED || path == BQ_PATH_GEMV_STREAM)
+            return BQ_ERR_UNSUPPORTED;
         if (K % 8 != 0) return BQ_ERR_SHAPE;
         path = BQ_PATH_DEQUANT_GEMM;
     }
@@ -833,14 +890,23 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
         return BQ_ERR_WORKSPACE;
 
     if ((s = current_device(&dev, &di)) != BQ_OK) return s;
-    const size_t need = workspace_for(path, fmt, M, N, K, di.num_sms, di.max_smem_optin);
+    const size_t need = workspace_for(path, fmt, group_size, M, N, K, di.num_sms, di.max_smem_optin);
 
     const uint16_t* sc = reinterpret_cast<const uint16_t*>(scales);
     const uint16_t* bi = reinterpret_cast<const uint16_t*>(biases);
     switch (path) {
+    case BQ_PATH_GEMV_STREAM:
+        if (!has_fast_paths(fmt) || stream_gemv_table_bytes(fmt, group_size, M, K) == 0) return BQ_ERR_UNSUPPORTED;
+        if (try_stream_gemv(fmt, group_size, x, one_matrix(wq, sc, bi, y, N), M, K, dev, di, st, workspace,
+                            workspace_bytes, &s))
+            return s;
+        return workspace && workspace_bytes < need ? BQ_ERR_WORKSPACE : BQ_ERR_UNSUPPORTED;
     case BQ_PATH_GEMV:
         if (!has_fast_paths(fmt)) return launch_gemv_affine(fmt, x, wq, sc, bi, y, M, N, K, group_size, st);
-        if (try_stream_gemv(fmt, group_size, x, one_matrix(wq, sc, bi, y, N), M, K, dev, di, st, &s)) return s;
+        if (stream_gemv_preferred(fmt, M) &&
+            try_stream_gemv(fmt, group_size, x, one_matrix(wq, sc, bi, y, N), M, K, dev, di, st, workspace,
+                            workspace_bytes, &s))
+            return s;
         if (fmt == WFmt::Q4_0) return launch_gemv<Fmt::Q4_0>(x, wq, sc, bi, y, M, N, K, group_size, st);
         if (fmt == WFmt::AFF4) return launch_gemv<Fmt::AFF4>(x, wq, sc, bi, y, M, N, K, group_size, st);
         return launch_gemv<Fmt::AFF8>(x, wq, sc, bi, y, M, N, K, group_size, st);
@@ -1103,7 +1169,8 @@ bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const void* cons
         mats.y[i] = y_bf16[i];
         mats.N[i] = N[i];
     }
-    if (try_stream_gemv(fmt, group_size, x_bf16, mats, M, K, dev, di, st, &s)) return s;
+    if (stream_gemv_preferred(fmt, M) && try_stream_gemv(fmt, group_size, x_bf16, mats, M, K, dev, di, st, nullptr, 0, &s))
+        return s;
     if (fmt == WFmt::Q4_0) return launch_gemv_multi<Fmt::Q4_0>(x_bf16, tab, M, K, group_size, st);
     if (fmt == WFmt::AFF4) return launch_gemv_multi<Fmt::AFF4>(x_bf16, tab, M, K, group_size, st);
     return launch_gemv_multi<Fmt::AFF8>(x_bf16, tab, M, K, group_size, st);
@@ -1122,7 +1189,7 @@ size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int group_si
         smem_optin = di.max_smem_optin;
     }
     cudaGetLastError();
-    return workspace_for(path, fmt, M, N, K, num_sms, smem_optin);
+    return workspace_for(path, fmt, group_size, M, N, K, num_sms, smem_optin);
 }
 
 int quant_matmul_select_path(int64_t M, int64_t N, int64_t K, int group_size, int bits)

@@ -1,49 +1,65 @@
-// gemv_stream.cuh -- decode path for 1..8 tokens: the packed weights stream
-// once from HBM into per-warp shared-memory rings (16-byte asynchronous
-// copies), and warp-level bf16 MMAs multiply the exact integer codes against
-// the activations; each block's (or group's) scale is applied once to its fp32
-// partial sum.
+// gemv_stream.cuh -- decode path for one or two tokens.  The packed weights
+// stream once from HBM through per-warp shared-memory rings (16-byte
+// asynchronous copies) into integer tensor-core MMAs that multiply the codes,
+// as unsigned bytes, with the activations split into signed bytes: every inner
+// sum is an exact integer, and each block's (or group's) scale is applied once.
 //
 // The pages' decode kernels are prior art for this path: decode routes to a
 // vector-dot kernel in "et-backend: Q4_0 matrix-engine GEMM rewrite for
 // prefill" (Overview), and the SYCL page "2026-05-06 Q4 sync-after focused
-// repro" runs MMVQ kernels over "reordered" Q4_0 (Important source touch
-// points).  The operation is the MLX issue's quantized_matmul ("Repro"): y =
-// x . dequant(W)^T, which is
+// repro" runs MMVQ kernels, which take the activations as 8-bit integers, over
+// "reordered" Q4_0 (Important source touch points).  Here the integer form of
+// x is exact, not a quantization.  The operation is the MLX issue's
+// quantized_matmul ("Repro"): y = x . dequant(W)^T, which is
 //
 //   y[m][n] = sum over blocks b of  d[n][b] * sum_{j in b} x[m][j] * (q[n][j] - 8)      (Q4_0)
 //   y[m][n] = sum over groups g of  s[n][g] * sum_{j in g} x[m][j] * q[n][j]
 //                                 + z[n][g] * sum_{j in g} x[m][j]                  (affine)
 //
-// computed in that order: the inner sums exactly in the tensor core (codes
-// and activations are exact bf16, products exact, fp32 accumulation), the
-// scale once per block.  The result differs from a product with the
+// computed in that order; the result differs from a product with the
 // bf16-rounded dequantized weights only by those weights' roundings.
 //
-// Codes enter the MMA without arithmetic: OR-ing a nibble into the bf16
-// pattern 0x4300 gives the value 128 + q exactly, so one LOP3 (plus a shift)
-// turns two nibbles into an A-operand register.  The constant 128 (and Q4_0's
-// -8) is removed through the activation sums: for Q4_0 the accumulator starts
-// at C = -136 * sum_j x[j] (MMA addend), so it ends at sum_j x[j] (q[j] - 8).
-// 8-bit codes are split into nibbles q = lo + 16 hi; the high nibbles multiply
-// 16 x (exact in bf16), and the offset is 128 + 16 * 128 = 2176.
+// Activations.  With one or two tokens most of an n8 MMA's columns would carry
+// nothing; they hold the tokens' activations split into signed bytes instead.
+// With S = 8 slices for one token, 4 for each of two:
 //
-// Layout of the work: one CTA per SM walks a contiguous range of 16-row
-// weight tiles (of one matrix, or of up to eight matrices that share x, as the
-// fused pairs of one-token MMVQ nodes on the SYCL page; a tile is computed the
-// same way whichever launch it is in, so the bits do not depend on it).  Each
-// of the CTA's KW warps owns a fixed K slice of every tile and streams exactly
+//   per token and scale group, e = the exponent of the group's largest |x|, P = 8 S - 3;
+//   v_k = x_k * 2^(P - e), an integer whenever x_k's exponent is >= e - (P - 7);
+//   v_k = sum_j 2^(8 j) l_j,k, l_j in [-128, 127] below the top slice, |l_top| <= 64;
+//   the MMA column of slice j holds l_j, and its sum is scaled by 2^(e - P + 8 j).
+//
+// So every bf16 activation within 2^54 (one token) or 2^22 (two tokens) of its
+// group's largest is held exactly.  A launch whose activations are not all held
+// exactly computes plain fp32 dot products instead (gemv_exact): the integer
+// route never rounds x.  Q4_0's -8 enters as the MMA addend -8 * sum_k l_j,k
+// (an exact integer), the affine bias as z * sum_g x (the fp32 sum of the bf16
+// activations).  A group holding Inf or NaN gives NaN.
+//
+// Codes.  An m16n8k32 step covers 32 elements of 16 rows: a Q4_0 block or an
+// affine-4 code unit (one 16-byte unit per row), or two affine-8 units, so the
+// codes reach the MMA with no arithmetic at all (affine 8-bit) or one AND and
+// one shift-AND per word (the two nibbles of each byte become separate bytes).
+// The k-slot order this gives is folded into the activation table:
+//   Q4_0, affine 8-bit: lane t's bytes are elements 4t..4t+3 (register 0) and 16+4t..16+4t+3 (register 1)
+//   affine 4-bit:       register 0 holds elements 8t, 8t+2, 8t+4, 8t+6 and register 1 elements 8t+1, +3, +5, +7
+//
+// Work.  gemv_int_prep_kernel builds the activation tables once per call, in a
+// device buffer; gemv_stream_kernel runs one CTA per SM over a contiguous range
+// of 16-row weight tiles (of one matrix, or of up to eight matrices that share
+// x, as the fused one-token MMVQ nodes on the SYCL page; a tile is computed
+// the same way whichever launch it is in, so the bits do not depend on it).
+// Each of its KW warps owns a fixed K slice of every tile and streams exactly
 // that slice (codes and scales of its 16 rows) into its own ring of S stages
-// with cp.async, so no warp waits for another and no registers hold data in
-// flight.  Rows are padded by 16 bytes so that ldmatrix reads them without
-// bank conflicts; ldmatrix hands each thread the 4-byte word of a 16-byte code
-// unit that its MMA fragment needs.  The activations are staged once per CTA
-// into a table permuted to the fragment order.  Per-warp partial sums of each
-// tile are summed in warp order at the end, so the result is deterministic.
+// with cp.async, so no warp waits for another; its part of the activation
+// tables travels with its first stage.  Rows are padded by 16 bytes so that
+// ldmatrix reads them without bank conflicts; ldmatrix hands each thread the
+// 4-byte word of a 16-byte code unit that its MMA fragment needs.  Per-warp
+// partial sums of each tile are summed in warp order at the end, so the
+// result is deterministic.
 //
-// Launch: with programmatic stream serialization the kernel's set-up overlaps
-// the previous kernel; every global read of the data and every write of y
-// happen after griddepcontrol.wait.
+// Launch: both kernels use programmatic stream serialization, so each launch
+// overlaps the tail of the kernel before it; each reads x, the tables, W and
+// scales, and writes its outputs, only after griddepcontrol.wait.
 #pragma once
 
 #include "gemv.cuh"
@@ -71,14 +87,14 @@ BQ_DEVINL void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, 
         : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr) : "memory");
 }
 
-// D = A x B + C, m16n8k16, fp16 inputs, fp32 accumulate (a pure function of its operands).
-BQ_DEVINL void mma_f16_16816_c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                               uint32_t b1, float c0, float c1, float c2, float c3)
+// D = A x B + C, m16n8k32, A unsigned bytes, B signed bytes, s32 accumulate: exact.
+BQ_DEVINL void mma_u8s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                              uint32_t b1, int c0, int c1, int c2, int c3)
 {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2), "f"(c3));
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c0), "r"(c1), "r"(c2), "r"(c3));
 }
 
 BQ_DEVINL uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
@@ -117,56 +133,19 @@ BQ_DEVINL void copy_block(uint32_t dst, uint32_t dpitch, const uint8_t* src, int
     }
 }
 
-// Right shift by 8 on the FMA pipe: the high word of w * 2^24.  The multiplier
-// comes from the launch parameters, so the compiler cannot turn it back into a
-// shift (which would load the ALU pipe that the LOP3s of the unpack need).
-BQ_DEVINL uint32_t shr8_fma(uint32_t w, uint32_t mul24) { return __umulhi(w, mul24); }
-
 // ------------------------------------------------------------------ formats
-// The codes enter the MMA as exact fp16 values, made by OR-ing them into fp16
-// patterns: a nibble in bits 0-3 under 0x6400 is 1024 + q, a nibble in bits
-// 4-7 under 0x5400 is 64 + q (exponent 6, 1/16 per mantissa step), a byte
-// under 0x64 (by a byte permute) is 1024 + q.  A 16-byte code unit of one row
-// holds E elements; ldmatrix gives thread t of a quad word t of the unit.
-//   Q4_0 (byte j: element j low nibble, j + 16 high): word t = bytes 4t..4t+3,
-//     r0 = 1024 + (4t, 4t+2)  r1 = 1024 + (4t+1, 4t+3)  r2 = 64 + (16+4t, 18+4t)  r3 = 64 + (17+4t, 19+4t)
-//   affine 4-bit (word i: elements 8i..8i+7, nibble n = element 8i+n)
-//     r0 = 1024 + (8t, 8t+4)  r1 = 64 + (8t+1, 8t+5)  r2 = 1024 + (8t+2, 8t+6)  r3 = 64 + (8t+3, 8t+7)
-//   affine 8-bit (word i: elements 4i..4i+3, one byte each)
-//     r0 = 1024 + (4t, 4t+2)  r1 = 1024 + (4t+1, 4t+3)
-// An MMA takes (r0, r1) as k-slots (2t, 2t+1) and (2t+8, 2t+9), a second one
-// (r2, r3); the activation table holds the matching fp16 pairs.  The offsets
-// (1024 or 64 per element) come out through per-unit activation sums.
+// A 16-byte code unit of one row holds E elements.
 template <Fmt F> struct SFmt;
-template <> struct SFmt<Fmt::Q4_0> { static constexpr int E = 32, kBits = 4, kMmas = 2; };
-template <> struct SFmt<Fmt::AFF4> { static constexpr int E = 32, kBits = 4, kMmas = 2; };
-template <> struct SFmt<Fmt::AFF8> { static constexpr int E = 16, kBits = 8, kMmas = 1; };
-
-template <Fmt F>
-BQ_DEVINL void unpack_unit_word(uint32_t w, uint32_t (&r)[4], uint32_t mul24)
-{
-    if constexpr (F == Fmt::AFF8) {
-        r[0] = prmt(w, 0x64646464u, 0x4240u);
-        r[1] = prmt(w, 0x64646464u, 0x4341u);
-    } else {
-        const uint32_t w8 = shr8_fma(w, mul24);
-        if constexpr (F == Fmt::Q4_0) {
-            r[0] = and_or_i<0x000F000Fu, 0x64006400u>(w);
-            r[1] = and_or_i<0x000F000Fu, 0x64006400u>(w8);
-            r[2] = and_or_i<0x00F000F0u, 0x54005400u>(w);
-            r[3] = and_or_i<0x00F000F0u, 0x54005400u>(w8);
-        } else {
-            r[0] = and_or_i<0x000F000Fu, 0x64006400u>(w);
-            r[1] = and_or_i<0x00F000F0u, 0x54005400u>(w);
-            r[2] = and_or_i<0x000F000Fu, 0x64006400u>(w8);
-            r[3] = and_or_i<0x00F000F0u, 0x54005400u>(w8);
-        }
-    }
-}
+template <> struct SFmt<Fmt::Q4_0> { static constexpr int E = 32, kBits = 4; };
+template <> struct SFmt<Fmt::AFF4> { static constexpr int E = 32, kBits = 4; };
+template <> struct SFmt<Fmt::AFF8> { static constexpr int E = 16, kBits = 8; };
 
 // ------------------------------------------------------------------ parameters
-constexpr int kSgMaxTokens = 8;      // one n8 MMA column group
-constexpr int kSgMaxMats = 8;        // matrices sharing x in one launch
+constexpr int kSgIntTokens = 2;                // 8 slices of one token, or 4 of each of two: one n8 MMA
+constexpr int kSgMaxMats = 8;                  // matrices sharing x in one launch
+constexpr int kSgIntCtabBytes = 64;            // group table: 4 quad positions x (c0, c1, X0, X1)
+constexpr uint32_t kSgIntStepBytes = 256;      // slice table per 32-element step: 8 columns x 4 x 8 bytes
+constexpr int kSgPrepThreads = 256;
 
 struct SGemvParams {
     const uint16_t* x;                   // bf16 [M][K], shared by every matrix
@@ -185,128 +164,320 @@ struct SGemvParams {
     uint32_t code_pitch;      // shared bytes per code row of a warp's stage (slice bytes + padding)
     uint32_t scale_pitch;     // shared bytes per scale (or bias) row of a warp's stage
     uint32_t wstage_bytes;    // one stage of one warp
-    uint32_t x_row_bytes;     // activation table bytes per token (units x 4 entries + 64)
-    uint32_t mul24;           // 2^24 (see shr8_fma)
-    int red_cols;             // token columns of the partial-sum buffer (M rounded up to even)
+    int red_cols;             // token columns of the partial-sum buffer
     uint32_t off_x, off_c, off_red, off_ring;   // offsets into dynamic shared memory
+    uint8_t* tab;             // activation tables built by gemv_int_prep_kernel: slices at 0,
+    uint32_t tab_c_off;       //   the group table at tab_c_off,
+    uint32_t tab_f_off;       //   one inexactness flag word per prep CTA at tab_f_off
+    int nflags;
 };
 
-// Activation-table entry bytes per (unit, quad position): the B registers of the unit's MMAs.
-template <Fmt F> constexpr int sg_entry_bytes() { return F == Fmt::AFF8 ? 8 : 16; }
-// C-table bytes per (group, token): Q4_0 the MMA addend C; affine (S, -T).
-template <Fmt F> constexpr int sg_ctab_bytes() { return F == Fmt::Q4_0 ? 4 : 8; }
+// fp32 bits of 2^n: normal, subnormal (n >= -149) or zero.
+BQ_DEVINL uint32_t pow2_bits(int n)
+{
+    return n >= -126 ? (uint32_t)(n + 127) << 23 : n >= -149 ? 1u << (n + 149) : 0u;
+}
 
-// ------------------------------------------------------------------ kernel pieces
-// The MMAs of one warp's K slice of one stage, NU code units (compile-time
-// count, fully unrolled) or nu_rt units (NU == 0).  ld: ldmatrix address of the
-// slice's first unit pair; sc: this thread's row-g scale run (row g + 8 is
-// 8 * pitch further, biases 16 rows further); xp: the slice's first
-// activation-table entry of this thread; cp: its first C-table pair.
+// MMA column of slice j of token m (slices per token: 8 for one token, 4 for two).
+BQ_DEVINL int int_column(int M, int m, int j) { return M == 1 ? j : 4 * m + j; }
+
+// ------------------------------------------------------------------ activation tables
+// One item (token m, 32-element step, quad position t) per thread: its eight
+// activations, their slices in the two B registers of column (m, j) for every
+// slice j, and -- by the first lane of each group -- the group's column scales
+// and addends.  Tables (in `tab`): slices [K / 32 steps][8 columns][4 quad
+// positions] x (register 0, register 1); groups [K / group][4 quad positions] x
+// (scale of column 2t, of column 2t + 1, Q4_0 addend or affine bias sum of
+// column 2t, of 2t + 1); then one flag word per CTA, nonzero when one of its
+// activations is not held exactly.
+//
+// Integer arithmetic on the bf16 bits: |x| = m 2^(E' - 134) with m = 128 + f
+// (E' = E) for normal values, m = f (E' = 1) for subnormal ones, so v = m 2^sh
+// with sh = E' - 134 - (e - P).  m << (sh mod 8) spans at most two bytes; its
+// signed-digit form (three digits, the last one 0 or +-1) lands at slice
+// sh / 8, and a byte transpose (prmt) gathers each slice's four bytes per MMA
+// register.  The top slice absorbs the carry, which keeps it within +-64.
+template <Fmt F, int GS>
+__global__ void __launch_bounds__(kSgPrepThreads)
+gemv_int_prep_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ tab, uint32_t c_off,
+                     uint32_t f_off)
+{
+    constexpr int SPG = GS / 32;                        // MMA steps per group
+    constexpr int GL = 4 * SPG;                         // lanes that hold one group
+    static_assert(GL <= 32, "a group's lanes lie in one warp");
+    grid_dependents_launch();                           // the GEMV may launch; it waits for this grid to finish
+    grid_dependency_wait();                             // x comes from the previous kernel
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int nsteps = K / 32;
+    const int S = M == 1 ? 8 : 4, P = 8 * S - 3;
+    const int items = M * nsteps * 4;                   // a multiple of 32 (K is a multiple of 256)
+    const int idx = blockIdx.x * kSgPrepThreads + tid;
+    int inexact = 0;
+    if (idx - lane < items) {                           // whole warps
+        const int t = idx & 3, step = (idx >> 2) % nsteps, m = (idx >> 2) / nsteps;
+        const uint16_t* xr = x + (int64_t)m * K + (int64_t)step * 32;
+        // the 8 activations as bf16 pairs: element i is half (i & 1) of word i >> 1
+        uint32_t raw[4];
+        if constexpr (F == Fmt::AFF4) {
+            // register 0 <- elements 8t + 2i (low halves), register 1 <- 8t + 2i + 1 (high halves)
+            const uint4 q = *reinterpret_cast<const uint4*>(xr + 8 * t);
+            raw[0] = __byte_perm(q.x, q.y, 0x5410);
+            raw[1] = __byte_perm(q.z, q.w, 0x5410);
+            raw[2] = __byte_perm(q.x, q.y, 0x7632);
+            raw[3] = __byte_perm(q.z, q.w, 0x7632);
+        } else {
+            const uint2 a = *reinterpret_cast<const uint2*>(xr + 4 * t);
+            const uint2 c = *reinterpret_cast<const uint2*>(xr + 16 + 4 * t);
+            raw[0] = a.x;
+            raw[1] = a.y;
+            raw[2] = c.x;
+            raw[3] = c.y;
+        }
+        uint32_t key[8];
+        uint32_t kmax = 0u;
+        int bad = 0;
+        float sum = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t bits = (raw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+            key[i] = bits;
+            bad |= (bits & 0x7FFFu) >= 0x7F80u;
+            kmax = max(kmax, bits & 0x7FFFu);
+            if constexpr (F != Fmt::Q4_0) sum += bf16_bits_to_f32(bits);
+        }
+#pragma unroll
+        for (int o = 1; o < GL; o <<= 1) {
+            kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
+            bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, o);
+            if constexpr (F != Fmt::Q4_0) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        }
+        // e = exponent of the group's largest |x| (0 for an all-zero or non-finite group)
+        const int emax = (int)(kmax >> 7);
+        const int e = (bad || kmax == 0u) ? 0 : emax > 0 ? emax - 127 : (31 - __clz((int)kmax)) - 133;
+        const int lsb = e - P;                          // exponent of v's unit
+        uint32_t lo[8], hi[8];                          // slices 0-3 and 4-7 of each element's v
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t bits = key[i];
+            const int E = (int)((bits >> 7) & 0xFFu);
+            const int mant = E ? (int)((bits & 0x7Fu) | 0x80u) : (int)(bits & 0x7Fu);
+            const int sh = (E ? E : 1) - 134 - lsb;
+            int W, j0;
+            if (sh >= 0) {
+                W = mant << (sh & 7);
+                j0 = sh >> 3;
+            } else {
+                const int rs = -sh;
+                W = rs >= 8 ? 0 : mant >> rs;
+                inexact |= (rs >= 8 ? mant : mant - (W << rs)) != 0;
+                j0 = 0;
+            }
+            if (bad) {
+                W = 0;
+                j0 = 0;
+            }
+            if (bits & 0x8000u) W = -W;
+            const int d0 = (W << 24) >> 24;
+            const int W1 = (W - d0) >> 8;
+            int d1 = (W1 << 24) >> 24, d2 = (W1 - d1) >> 8;
+            if (j0 + 2 >= S) {                          // top slice: keep the whole rest
+                d1 = W1;
+                d2 = 0;
+            }
+            const uint32_t D = ((uint32_t)d0 & 0xFFu) | (((uint32_t)d1 & 0xFFu) << 8) | (((uint32_t)d2 & 0xFFu) << 16);
+            const uint64_t T = (uint64_t)D << (8 * j0);
+            lo[i] = (uint32_t)T;
+            hi[i] = (uint32_t)(T >> 32);
+        }
+        // transpose: slice j of register r holds byte j of elements 4r .. 4r + 3
+        uint32_t r0[8], r1[8];
+        auto transpose4 = [](const uint32_t* a, uint32_t* out) {
+            const uint32_t t01l = __byte_perm(a[0], a[1], 0x5140), t01h = __byte_perm(a[0], a[1], 0x7362);
+            const uint32_t t23l = __byte_perm(a[2], a[3], 0x5140), t23h = __byte_perm(a[2], a[3], 0x7362);
+            out[0] = __byte_perm(t01l, t23l, 0x5410);
+            out[1] = __byte_perm(t01l, t23l, 0x7632);
+            out[2] = __byte_perm(t01h, t23h, 0x5410);
+            out[3] = __byte_perm(t01h, t23h, 0x7632);
+        };
+        transpose4(lo, r0);
+        transpose4(lo + 4, r1);
+        transpose4(hi, r0 + 4);
+        transpose4(hi + 4, r1 + 4);
+        int L[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (j < S) {
+                *reinterpret_cast<uint2*>(tab + (size_t)step * kSgIntStepBytes +
+                                          (size_t)(int_column(M, m, j) * 4 + t) * 8u) = make_uint2(r0[j], r1[j]);
+                L[j] = __dp4a((int)r0[j], 0x01010101, __dp4a((int)r1[j], 0x01010101, 0));
+#pragma unroll
+                for (int o = 1; o < GL; o <<= 1) L[j] += __shfl_xor_sync(0xFFFFFFFFu, L[j], o);
+            }
+        }
+        if ((lane & (GL - 1)) == 0) {
+            uint8_t* ct = tab + c_off + (size_t)(step / SPG) * kSgIntCtabBytes;
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                if (j < S) {
+                    uint32_t c[2], X[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        c[h] = bad ? 0x7FC00000u : pow2_bits(lsb + 8 * (j + h));
+                        if constexpr (F == Fmt::Q4_0) X[h] = (uint32_t)(-8 * L[j + h]);
+                        else X[h] = j + h == 0 ? __float_as_uint(sum) : 0u;
+                    }
+                    *reinterpret_cast<uint4*>(ct + (int_column(M, m, j) / 2) * 16) = make_uint4(c[0], c[1], X[0], X[1]);
+                }
+            }
+        }
+    }
+    inexact = __syncthreads_or(inexact);
+    if (tid == 0) reinterpret_cast<uint32_t*>(tab + f_off)[blockIdx.x] = inexact ? 1u : 0u;
+}
+
+// Exact fallback of the streamed GEMV for the CTA's tiles: fp32 dot products of
+// x with the weights dequantized in fp32 (d (q - 8) exactly, s q + z rounded
+// once), read straight from global memory; one warp per row, deterministic.
+template <Fmt F, int GS>
+BQ_DEVINL void gemv_exact(const SGemvParams& p, int t_begin, int t_end, int warp, int lane, int nwarps)
+{
+    const int M = p.M, K = p.K;
+    const int64_t row_bytes = (int64_t)K * SFmt<F>::kBits / 8, srow = K / GS;
+    for (int rl = warp; rl < (t_end - t_begin) * 16; rl += nwarps) {
+        const int tile = t_begin + (rl >> 4);
+        int mat = 0;
+        while (mat + 1 < p.count && tile >= p.tile_begin[mat + 1]) ++mat;
+        const int64_t row = (int64_t)(tile - p.tile_begin[mat]) * 16 + (rl & 15);
+        if (row >= p.N[mat]) continue;
+        const uint8_t* wr = p.wq[mat] + row * row_bytes;
+        const uint16_t* sr = p.scales[mat] + row * srow;
+        const uint16_t* br = F == Fmt::Q4_0 ? nullptr : p.biases[mat] + row * srow;
+        for (int m = 0; m < M; ++m) {
+            const uint16_t* xr = p.x + (int64_t)m * K;
+            float acc = 0.0f;
+            for (int k = lane; k < K; k += 32) {
+                float w;
+                if constexpr (F == Fmt::Q4_0) {
+                    const int j = k & 31;
+                    const uint32_t byte = wr[(k >> 5) * 16 + (j & 15)];
+                    const int q = (int)(j < 16 ? byte & 15u : byte >> 4);
+                    w = __half2float(__ushort_as_half(sr[k >> 5])) * (float)(q - 8);
+                } else {
+                    const uint32_t q = F == Fmt::AFF8 ? (uint32_t)wr[k] : (uint32_t)(wr[k >> 1] >> (4 * (k & 1))) & 15u;
+                    w = __fmaf_rn(bf16_bits_to_f32(sr[k / GS]), (float)q, bf16_bits_to_f32(br[k / GS]));
+                }
+                acc = __fmaf_rn(bf16_bits_to_f32(xr[k]), w, acc);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+            if (lane == 0) p.y[mat][(int64_t)m * p.N[mat] + row] = (uint16_t)f32_to_bf16_bits(acc);
+        }
+    }
+}
+
+// Scale (or bias) of row r's group `a` of the stage, as fp32: fp16 for Q4_0, bf16 for affine.
+template <Fmt F>
+BQ_DEVINL float stage_scale(const uint8_t* p)
+{
+    if constexpr (F == Fmt::Q4_0) return __half2float(*reinterpret_cast<const __half*>(p));
+    else return bf16_bits_to_f32(lds16(p));
+}
+
+
+// One warp's K slice of one stage, integer route: xp is this lane's slice-table
+// entry of the slice's first step, cp its group-table
+// entry of the slice's first group; sc as in slice_mma.
 template <Fmt F, int GS, int NU>
-BQ_DEVINL void slice_mma(float (&yv)[4], uint32_t ld, const uint8_t* sc, uint32_t pitch, const uint8_t* xp,
-                         const uint8_t* cp, int nu_rt, uint32_t mul24)
+BQ_DEVINL void slice_int(float (&yv)[4], uint32_t ld, const uint8_t* sc, uint32_t pitch, const uint8_t* xp,
+                         const uint8_t* cp, int nu_rt)
 {
     using T = SFmt<F>;
-    constexpr int UPG = GS / T::E;
-    constexpr int XU = 4 * sg_entry_bytes<F>();               // activation-table bytes per unit
-    constexpr int CG = kSgMaxTokens * sg_ctab_bytes<F>();     // C-table bytes per group
+    constexpr int UPG = GS / T::E;                      // code units per group
+    constexpr uint32_t kLo = 0x0F0F0F0Fu;
+    constexpr bool kAffine = F != Fmt::Q4_0;
     const int nu = NU > 0 ? NU : nu_rt;
-    if constexpr (UPG == 1) {
-        // Q4_0 or affine 4-bit with groups of 32: two groups per ldmatrix.x4
+    const uint8_t* sc8 = sc + 8 * pitch;
+    if constexpr (T::E == 32 && UPG == 1) {
+        // one group per unit (Q4_0, affine-4 with groups of 32): two per ldmatrix.x4
 #pragma unroll (NU > 0 ? NU / 2 : 2)
         for (int s = 0; s < nu / 2; ++s) {
             uint32_t w[4];                                      // (g, u) (g+8, u) (g, u+1) (g+8, u+1)
             ldsm_x4(ld + (uint32_t)s * 32u, w[0], w[1], w[2], w[3]);
-            const uint32_t sg = lds32(sc + 4 * s), sg8 = lds32(sc + 8 * pitch + 4 * s);
+            const uint32_t sg = lds32(sc + 4 * s), sg8 = lds32(sc8 + 4 * s);   // groups u, u + 1 of rows g, g + 8
             [[maybe_unused]] uint32_t bg = 0u, bg8 = 0u;
-            if constexpr (F != Fmt::Q4_0) {
+            if constexpr (kAffine) {
                 bg = lds32(sc + 16 * pitch + 4 * s);
-                bg8 = lds32(sc + 24 * pitch + 4 * s);
+                bg8 = lds32(sc8 + 16 * pitch + 4 * s);
             }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                uint32_t ra[4], rb[4];
-                unpack_unit_word<F>(w[2 * h], ra, mul24);
-                unpack_unit_word<F>(w[2 * h + 1], rb, mul24);
                 const int u = 2 * s + h;
-                const uint4 e = *reinterpret_cast<const uint4*>(xp + u * XU);
-                float acc[4];
-                if constexpr (F == Fmt::Q4_0) {
-                    const float2 c = *reinterpret_cast<const float2*>(cp + u * CG);
-                    mma_f16_16816_c(acc, ra[0], rb[0], ra[1], rb[1], e.x, e.y, c.x, c.y, c.x, c.y);
-                    mma_f16_16816_c(acc, ra[2], rb[2], ra[3], rb[3], e.z, e.w, acc[0], acc[1], acc[2], acc[3]);
+                const uint32_t wg = w[2 * h], wg8 = w[2 * h + 1];
+                const uint2 b = *reinterpret_cast<const uint2*>(xp + (uint32_t)u * kSgIntStepBytes);
+                const uint4 ce = *reinterpret_cast<const uint4*>(cp + u * kSgIntCtabBytes);
+                const int c0 = kAffine ? 0 : (int)ce.z, c1 = kAffine ? 0 : (int)ce.w;
+                int acc[4];
+                mma_u8s8_16832(acc, wg & kLo, wg8 & kLo, (wg >> 4) & kLo, (wg8 >> 4) & kLo, b.x, b.y, c0, c1, c0, c1);
+                float dg, dg8;
+                if constexpr (kAffine) {
+                    dg = __uint_as_float(h ? sg & 0xFFFF0000u : sg << 16);
+                    dg8 = __uint_as_float(h ? sg8 & 0xFFFF0000u : sg8 << 16);
+                } else {
                     const float2 d2 = __half22float2(*reinterpret_cast<const __half2*>(&sg));
                     const float2 d28 = __half22float2(*reinterpret_cast<const __half2*>(&sg8));
-                    const float dg = h ? d2.y : d2.x, dg8 = h ? d28.y : d28.x;
-                    yv[0] = __fmaf_rn(dg, acc[0], yv[0]);
-                    yv[1] = __fmaf_rn(dg, acc[1], yv[1]);
-                    yv[2] = __fmaf_rn(dg8, acc[2], yv[2]);
-                    yv[3] = __fmaf_rn(dg8, acc[3], yv[3]);
-                } else {
-                    const float4 c = *reinterpret_cast<const float4*>(cp + u * CG);   // (S, -T) of tokens 2t, 2t+1
-                    mma_f16_16816_c(acc, ra[0], rb[0], ra[1], rb[1], e.x, e.y, c.y, c.w, c.y, c.w);
-                    mma_f16_16816_c(acc, ra[2], rb[2], ra[3], rb[3], e.z, e.w, acc[0], acc[1], acc[2], acc[3]);
-                    const float dg = __uint_as_float(h ? sg & 0xFFFF0000u : sg << 16);
-                    const float dg8 = __uint_as_float(h ? sg8 & 0xFFFF0000u : sg8 << 16);
+                    dg = h ? d2.y : d2.x;
+                    dg8 = h ? d28.y : d28.x;
+                }
+                const float k0 = __uint_as_float(ce.x), k1 = __uint_as_float(ce.y);
+                if constexpr (kAffine) {
                     const float zg = __uint_as_float(h ? bg & 0xFFFF0000u : bg << 16);
                     const float zg8 = __uint_as_float(h ? bg8 & 0xFFFF0000u : bg8 << 16);
-                    yv[0] = __fmaf_rn(dg, acc[0], __fmaf_rn(zg, c.x, yv[0]));
-                    yv[1] = __fmaf_rn(dg, acc[1], __fmaf_rn(zg, c.z, yv[1]));
-                    yv[2] = __fmaf_rn(dg8, acc[2], __fmaf_rn(zg8, c.x, yv[2]));
-                    yv[3] = __fmaf_rn(dg8, acc[3], __fmaf_rn(zg8, c.z, yv[3]));
+                    const float b0 = __uint_as_float(ce.z), b1 = __uint_as_float(ce.w);
+                    yv[0] = __fmaf_rn(zg, b0, yv[0]);
+                    yv[1] = __fmaf_rn(zg, b1, yv[1]);
+                    yv[2] = __fmaf_rn(zg8, b0, yv[2]);
+                    yv[3] = __fmaf_rn(zg8, b1, yv[3]);
                 }
+                yv[0] = __fmaf_rn(dg * k0, (float)acc[0], yv[0]);
+                yv[1] = __fmaf_rn(dg * k1, (float)acc[1], yv[1]);
+                yv[2] = __fmaf_rn(dg8 * k0, (float)acc[2], yv[2]);
+                yv[3] = __fmaf_rn(dg8 * k1, (float)acc[3], yv[3]);
             }
         }
     } else {
-        // affine, one group of UPG >= 2 units per atom, every unit into the group's accumulator
+        // groups of two or more units, every MMA of a group into one accumulator
 #pragma unroll (NU > 0 ? NU / UPG : 1)
         for (int a = 0; a < nu / UPG; ++a) {
-            const float4 c = *reinterpret_cast<const float4*>(cp + a * CG);   // (S, -T) of tokens 2t, 2t+1
-            float gacc[4] = {c.y, c.w, c.y, c.w};
+            int acc[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int s = 0; s < UPG / 2; ++s) {
                 const int u = a * UPG + 2 * s;
                 uint32_t w[4];
                 ldsm_x4(ld + (uint32_t)u * 16u, w[0], w[1], w[2], w[3]);
+                if constexpr (F == Fmt::AFF8) {
+                    const uint2 b = *reinterpret_cast<const uint2*>(xp + (uint32_t)(u / 2) * kSgIntStepBytes);
+                    mma_u8s8_16832(acc, w[0], w[1], w[2], w[3], b.x, b.y, acc[0], acc[1], acc[2], acc[3]);
+                } else {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t ra[4], rb[4];
-                    unpack_unit_word<F>(w[2 * h], ra, mul24);
-                    unpack_unit_word<F>(w[2 * h + 1], rb, mul24);
-                    if constexpr (F == Fmt::AFF8) {
-                        const uint2 e = *reinterpret_cast<const uint2*>(xp + (u + h) * XU);
-                        mma_f16_16816_c(gacc, ra[0], rb[0], ra[1], rb[1], e.x, e.y, gacc[0], gacc[1], gacc[2],
-                                        gacc[3]);
-                    } else {
-                        const uint4 e = *reinterpret_cast<const uint4*>(xp + (u + h) * XU);
-                        mma_f16_16816_c(gacc, ra[0], rb[0], ra[1], rb[1], e.x, e.y, gacc[0], gacc[1], gacc[2],
-                                        gacc[3]);
-                        mma_f16_16816_c(gacc, ra[2], rb[2], ra[3], rb[3], e.z, e.w, gacc[0], gacc[1], gacc[2],
-                                        gacc[3]);
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t wg = w[2 * h], wg8 = w[2 * h + 1];
+                        const uint2 b = *reinterpret_cast<const uint2*>(xp + (uint32_t)(u + h) * kSgIntStepBytes);
+                        mma_u8s8_16832(acc, wg & kLo, wg8 & kLo, (wg >> 4) & kLo, (wg8 >> 4) & kLo, b.x, b.y, acc[0],
+                                       acc[1], acc[2], acc[3]);
                     }
                 }
             }
-            // group epilogue: y += s * acc + z * S
-            const float dg = bf16_bits_to_f32(lds16(sc + 2 * a));
-            const float dg8 = bf16_bits_to_f32(lds16(sc + 8 * pitch + 2 * a));
-            const float zg = bf16_bits_to_f32(lds16(sc + 16 * pitch + 2 * a));
-            const float zg8 = bf16_bits_to_f32(lds16(sc + 24 * pitch + 2 * a));
-            yv[0] = __fmaf_rn(dg, gacc[0], __fmaf_rn(zg, c.x, yv[0]));
-            yv[1] = __fmaf_rn(dg, gacc[1], __fmaf_rn(zg, c.z, yv[1]));
-            yv[2] = __fmaf_rn(dg8, gacc[2], __fmaf_rn(zg8, c.x, yv[2]));
-            yv[3] = __fmaf_rn(dg8, gacc[3], __fmaf_rn(zg8, c.z, yv[3]));
+            const uint4 ce = *reinterpret_cast<const uint4*>(cp + a * kSgIntCtabBytes);
+            const float dg = stage_scale<F>(sc + 2 * a), dg8 = stage_scale<F>(sc8 + 2 * a);
+            const float zg = stage_scale<F>(sc + 16 * pitch + 2 * a), zg8 = stage_scale<F>(sc8 + 16 * pitch + 2 * a);
+            const float k0 = __uint_as_float(ce.x), k1 = __uint_as_float(ce.y);
+            const float b0 = __uint_as_float(ce.z), b1 = __uint_as_float(ce.w);
+            yv[0] = __fmaf_rn(dg * k0, (float)acc[0], __fmaf_rn(zg, b0, yv[0]));
+            yv[1] = __fmaf_rn(dg * k1, (float)acc[1], __fmaf_rn(zg, b1, yv[1]));
+            yv[2] = __fmaf_rn(dg8 * k0, (float)acc[2], __fmaf_rn(zg8, b0, yv[2]));
+            yv[3] = __fmaf_rn(dg8 * k1, (float)acc[3], __fmaf_rn(zg8, b1, yv[3]));
         }
     }
-}
-
-// Scaled fp16 pair of two bf16 activations (lo and hi halves of v), and the
-// sum of the two fp16 values as the MMA sees them.
-BQ_DEVINL uint32_t x_pair_f16(uint32_t lo_bits, uint32_t hi_bits, float scale, float& sum)
-{
-    const __half2 h = __floats2half2_rn(bf16_bits_to_f32(lo_bits) * scale, bf16_bits_to_f32(hi_bits) * scale);
-    const float2 f = __half22float2(h);
-    sum += f.x + f.y;
-    return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -321,12 +492,9 @@ gemv_stream_kernel(const __grid_constant__ SGemvParams p)
     constexpr int UPG = GS / E;                          // code units per scale group
     constexpr bool kAffine = F != Fmt::Q4_0;
     constexpr int kAtomUnits = UPG > 2 ? UPG : 2;        // K-split atom: 2 units (one ldmatrix.x4), whole groups
-    constexpr int XE = sg_entry_bytes<F>();
-    constexpr int CB = sg_ctab_bytes<F>();
     static_assert(GS % E == 0, "group must hold whole code units");
 
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ float x_scale[kSgMaxTokens], x_unscale[kSgMaxTokens], warp_max[32][kSgMaxTokens];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sbase = smem_u32(smem);
     const int M = p.M, K = p.K, S = p.stages, nchunks = p.nchunks;
@@ -336,8 +504,6 @@ gemv_stream_kernel(const __grid_constant__ SGemvParams p)
     const int total = nt * nchunks;
     const int64_t row_bytes = (int64_t)K * T::kBits / 8;
     const int64_t srow = K / GS;                         // scale entries per row
-    const int nu_all = K / E;                            // code units per row
-    const int ng_all = K / GS;
     const uint32_t ring = sbase + p.off_ring + (uint32_t)warp * S * p.wstage_bytes;
 
     // This warp's slice of a chunk of kn elements (atoms [a_b, a_e)), with the
@@ -396,127 +562,37 @@ gemv_stream_kernel(const __grid_constant__ SGemvParams p)
 
     grid_dependency_wait();
     grid_dependents_launch();
-    for (int i = 0; i < S - 1; ++i) issue_next(i);
 
-    // ------------------------------------------------------------ activation tables
-    // Each token is scaled by a power of two 2^e so that its largest magnitude
-    // lies in [2^14, 2^15); the scaled bf16 values are then exact in fp16 (down to
-    // 2^-24 of that magnitude), and y is multiplied by 2^-e at the end, exactly.
-    const int nthreads = 32 * KW;
+    // A launch whose activations the slices do not hold exactly computes fp32
+    // dot products (every warp reads the same flags, so the choice is uniform).
     {
-        float mx[kSgMaxTokens];
-#pragma unroll
-        for (int m = 0; m < kSgMaxTokens; ++m) mx[m] = 0.0f;
-        const int nv = K / 8;                                           // 16-byte vectors per token
-#pragma unroll
-        for (int m = 0; m < kSgMaxTokens; ++m) {
-            if (m < M) {
-                const uint4* xr = reinterpret_cast<const uint4*>(p.x + (int64_t)m * K);
-#pragma unroll 4
-                for (int i = tid; i < nv; i += nthreads) {
-                    const uint4 v = xr[i];
-                    const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        mx[m] = fmaxf(mx[m], fmaxf(fabsf(bf16_bits_to_f32(vv[j] & 0xFFFFu)),
-                                                    fabsf(bf16_bits_to_f32(vv[j] >> 16))));
-                }
-            }
+        const uint32_t* flags = reinterpret_cast<const uint32_t*>(p.tab + p.tab_f_off);
+        uint32_t inexact = 0u;
+        for (int i = lane; i < p.nflags; i += 32) inexact |= flags[i];
+        if (__any_sync(0xFFFFFFFFu, inexact != 0u)) {
+            gemv_exact<F, GS>(p, t_begin, t_end, warp, lane, KW);
+            return;
         }
-#pragma unroll
-        for (int m = 0; m < kSgMaxTokens; ++m) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx[m] = fmaxf(mx[m], __shfl_xor_sync(0xFFFFFFFFu, mx[m], o));
-            if (lane == 0) warp_max[warp][m] = mx[m];
-        }
-        __syncthreads();
-        if (tid < kSgMaxTokens) {
-            float a = 0.0f;
-            for (int w = 0; w < KW; ++w) a = fmaxf(a, warp_max[w][tid]);
-            // exponent of a (normal range), clamped so that both 2^e and 2^-e are normal fp32
-            int e = 0;
-            if (a > 0.0f && a < 3.0e38f) {
-                const int ea = (int)((__float_as_uint(a) >> 23) & 0xFFu) - 127;
-                e = max(-120, min(120, 14 - ea));
-            }
-            x_scale[tid] = __uint_as_float((uint32_t)(e + 127) << 23);
-            x_unscale[tid] = __uint_as_float((uint32_t)(127 - e) << 23);
-        }
-        __syncthreads();
     }
-    // Entry (m, unit u, quad position t): the B registers of the unit's MMAs for
-    // token m, in the order unpack_unit_word produces the A registers.
-    // U[m][u] = (sum of the class-A elements, sum of the class-B elements) of the
-    // unit as fp16 values (class A: the 1024-offset codes, B: the 64-offset ones);
-    // then per group the C table: Q4_0 -(1032 A + 72 B), the MMA addend that
-    // leaves sum x (q - 8); affine (S, -T) with S = A + B and T = 1024 A + 64 B.
-    const uint32_t xtab = sbase + p.off_x;
-    float* usum = reinterpret_cast<float*>(smem + p.off_red);
-    {
-        const int entries = M * nu_all * 4;
-#pragma unroll 4
-        for (int base = warp * 32; base < entries; base += nthreads) {
-            const int idx = base + lane;
-            const bool valid = idx < entries;
-            const int t = idx & 3, u = (idx >> 2) % nu_all, m = (idx >> 2) / nu_all;
-            uint32_t e[4] = {0u, 0u, 0u, 0u};
-            float sa = 0.0f, sb = 0.0f;
-            if (valid) {
-                const float xs = x_scale[m];
-                const uint16_t* xr = p.x + (int64_t)m * K + (int64_t)u * E;
-                if constexpr (F == Fmt::AFF4) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(xr + 8 * t);   // elements 8t .. 8t+7
-                    e[0] = x_pair_f16(v.x & 0xFFFFu, v.z & 0xFFFFu, xs, sa);        // (8t, 8t+4)
-                    e[1] = x_pair_f16(v.x >> 16, v.z >> 16, xs, sb);                // (8t+1, 8t+5)
-                    e[2] = x_pair_f16(v.y & 0xFFFFu, v.w & 0xFFFFu, xs, sa);        // (8t+2, 8t+6)
-                    e[3] = x_pair_f16(v.y >> 16, v.w >> 16, xs, sb);                // (8t+3, 8t+7)
-                } else {
-                    const uint2 a = *reinterpret_cast<const uint2*>(xr + 4 * t);    // elements 4t .. 4t+3
-                    e[0] = x_pair_f16(a.x & 0xFFFFu, a.y & 0xFFFFu, xs, sa);        // (4t, 4t+2)
-                    e[1] = x_pair_f16(a.x >> 16, a.y >> 16, xs, sa);                // (4t+1, 4t+3)
-                    if constexpr (F == Fmt::Q4_0) {
-                        const uint2 b = *reinterpret_cast<const uint2*>(xr + 16 + 4 * t);   // 16+4t .. 16+4t+3
-                        e[2] = x_pair_f16(b.x & 0xFFFFu, b.y & 0xFFFFu, xs, sb);
-                        e[3] = x_pair_f16(b.x >> 16, b.y >> 16, xs, sb);
-                    }
-                }
-                const uint32_t at = xtab + (uint32_t)m * p.x_row_bytes + (uint32_t)(u * 4 + t) * (uint32_t)XE;
-                if constexpr (XE == 16)
-                    st_shared_v4(at, e[0], e[1], e[2], e[3]);
-                else
-                    *reinterpret_cast<uint2*>(smem + (at - sbase)) = make_uint2(e[0], e[1]);
-            }
-            sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 1);
-            sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 2);
-            sb += __shfl_xor_sync(0xFFFFFFFFu, sb, 1);
-            sb += __shfl_xor_sync(0xFFFFFFFFu, sb, 2);
-            if (valid && t == 0) *reinterpret_cast<float2*>(usum + 2 * (m * nu_all + u)) = make_float2(sa, sb);
-        }
-        __syncthreads();
-        for (int i = tid; i < ng_all * kSgMaxTokens; i += nthreads) {
-            const int gi = i / kSgMaxTokens, m = i % kSgMaxTokens;
-            float a = 0.0f, b = 0.0f;
-            if (m < M) {
-#pragma unroll
-                for (int j = 0; j < UPG; ++j) {
-                    const float2 v = *reinterpret_cast<const float2*>(usum + 2 * (m * nu_all + gi * UPG + j));
-                    a += v.x;
-                    b += v.y;
-                }
-            }
-            if constexpr (F == Fmt::Q4_0)
-                reinterpret_cast<float*>(smem + p.off_c)[i] = -1032.0f * a - 72.0f * b;
-            else
-                reinterpret_cast<float2*>(smem + p.off_c)[i] = make_float2(a + b, -(1024.0f * a + 64.0f * b));
-        }
-        __syncthreads();
+    // This warp's part of the activation tables -- the steps and groups of its
+    // slice in every chunk -- travels in the commit group of its first stage.
+    for (int c = 0; c < nchunks; ++c) {
+        const Slice& sl = c == nchunks - 1 ? sl_last : sl_full;
+        const int u0 = c * (p.kc / E) + sl.a_b * kAtomUnits;        // the slice's first unit in the row
+        const uint32_t xo = (uint32_t)(u0 * E / 32) * kSgIntStepBytes;
+        const uint32_t xn = (uint32_t)(sl.nu * E / 32) * kSgIntStepBytes;
+        const uint32_t co = (uint32_t)(u0 / UPG) * kSgIntCtabBytes;
+        const uint32_t cn = (uint32_t)(sl.nu / UPG) * kSgIntCtabBytes;
+        for (uint32_t o = (uint32_t)lane * 16u; o < xn; o += 512u) cp_async16(sbase + p.off_x + xo + o, p.tab + xo + o);
+        for (uint32_t o = (uint32_t)lane * 16u; o < cn; o += 512u)
+            cp_async16(sbase + p.off_c + co + o, p.tab + p.tab_c_off + co + o);
     }
+    for (int i = 0; i < S - 1; ++i) issue_next(i);
 
     // ------------------------------------------------------------ main loop
     const int g = lane >> 2, t = lane & 3;
-    // token column g of the MMA: columns g >= M read token M - 1 (their outputs are never stored)
-    const uint8_t* x_lane = smem + p.off_x + (size_t)min(g, M - 1) * p.x_row_bytes + (size_t)t * XE;
-    const uint8_t* c_lane = smem + p.off_c + (size_t)(2 * t) * CB;
+    const uint8_t* x_lane = smem + p.off_x + (size_t)((g * 4 + t) * 8);     // slice column g
+    const uint8_t* c_lane = smem + p.off_c + (size_t)t * 16;
     // ldmatrix.x4 row addresses: matrices (rows 0-7, unit u), (rows 8-15, unit u),
     // (rows 0-7, unit u+1), (rows 8-15, unit u+1)
     const uint32_t ld_lane =
@@ -540,16 +616,27 @@ gemv_stream_kernel(const __grid_constant__ SGemvParams p)
         const int g_b = u_b / UPG;                              // its first group
         const uint8_t* sc = smem + (st - sbase) + 16u * p.code_pitch + (size_t)g * p.scale_pitch +
                             ((2 * (g_b - k0 / GS)) & 15);
-        const uint8_t* xp = x_lane + (size_t)u_b * 4 * XE;
-        const uint8_t* cp = c_lane + (size_t)g_b * kSgMaxTokens * CB;
+        const uint8_t* xp = x_lane + (size_t)(u_b * E / 32) * kSgIntStepBytes;
+        const uint8_t* cp = c_lane + (size_t)g_b * kSgIntCtabBytes;
         if (SU > 0 && !(last && nchunks > 1))
-            slice_mma<F, GS, SU>(yv, st + ld_lane, sc, p.scale_pitch, xp, cp, SU, p.mul24);
+            slice_int<F, GS, SU>(yv, st + ld_lane, sc, p.scale_pitch, xp, cp, SU);
         else
-            slice_mma<F, GS, 0>(yv, st + ld_lane, sc, p.scale_pitch, xp, cp, sl.nu, p.mul24);
-        if (last && 2 * t < M) {
-            float* rp = red + ((tl * KW + warp) * 16 + g) * p.red_cols + 2 * t;
-            *reinterpret_cast<float2*>(rp) = make_float2(yv[0], yv[1]);
-            *reinterpret_cast<float2*>(rp + 8 * p.red_cols) = make_float2(yv[2], yv[3]);
+            slice_int<F, GS, 0>(yv, st + ld_lane, sc, p.scale_pitch, xp, cp, sl.nu);
+        if (last) {
+            // the slice columns of token m: all four lanes of the quad (one
+            // token), lanes t = 2m and 2m + 1 (two tokens)
+            float r = yv[0] + yv[1], r8 = yv[2] + yv[3];
+            r += __shfl_xor_sync(0xFFFFFFFFu, r, 1);
+            r8 += __shfl_xor_sync(0xFFFFFFFFu, r8, 1);
+            if (M == 1) {
+                r += __shfl_xor_sync(0xFFFFFFFFu, r, 2);
+                r8 += __shfl_xor_sync(0xFFFFFFFFu, r8, 2);
+            }
+            if ((t & 1) == 0 && (t >> 1) < M) {
+                float* rp = red + ((tl * KW + warp) * 16 + g) * p.red_cols + (t >> 1);
+                rp[0] = r;
+                rp[8 * p.red_cols] = r8;
+            }
         }
         if (++chunk == nchunks) {
             chunk = 0;
@@ -562,7 +649,7 @@ gemv_stream_kernel(const __grid_constant__ SGemvParams p)
     // ------------------------------------------------------------ cross-warp sum and store
     __syncthreads();
     const int rows_cta = nt * 16;
-    for (int o = tid; o < M * rows_cta; o += nthreads) {
+    for (int o = tid; o < M * rows_cta; o += 32 * KW) {
         const int m = o / rows_cta, rl = o - m * rows_cta;
         const int tl2 = rl >> 4, r = rl & 15;
         const int tile = t_begin + tl2;
@@ -573,7 +660,7 @@ gemv_stream_kernel(const __grid_constant__ SGemvParams p)
         float sum = 0.0f;
 #pragma unroll
         for (int w = 0; w < KW; ++w) sum += red[((tl2 * KW + w) * 16 + r) * p.red_cols + m];
-        p.y[mat][(int64_t)m * p.N[mat] + row] = (uint16_t)f32_to_bf16_bits(sum * x_unscale[m]);
+        p.y[mat][(int64_t)m * p.N[mat] + row] = (uint16_t)f32_to_bf16_bits(sum);
     }
 }
 

@@ -83,10 +83,24 @@ typedef enum {
 /* Kernel paths of quant_matmul_ex. */
 typedef enum {
     BQ_PATH_AUTO = 0,          /* the M-threshold dispatcher chooses (quant_matmul_select_path) */
-    BQ_PATH_GEMV = 1,          /* decode path: in-register dequant feeding warp-level MMA, M <= 32 */
+    BQ_PATH_GEMV = 1,          /* decode path, M <= 32: the faster of the two decode kernels below */
     BQ_PATH_TC_FUSED = 2,      /* prefill path: on-chip dequant feeding a tcgen05/TMEM GEMM */
-    BQ_PATH_DEQUANT_GEMM = 3   /* the unfused pair: *_dequantize into a bf16 workspace, then bf16_matmul */
+    BQ_PATH_DEQUANT_GEMM = 3,  /* the unfused pair: *_dequantize into a bf16 workspace, then bf16_matmul */
+    BQ_PATH_GEMV_STREAM = 4    /* the streamed integer-MMA decode kernel, forced (M <= 2) */
 } bq_path;
+
+/* The two decode kernels of BQ_PATH_GEMV (Q4_0, affine 4- and 8-bit):
+ *  - register-streaming: codes dequantized to bf16 in registers, warp MMAs, M <= 32;
+ *  - streamed integer-MMA (M <= 2, K a multiple of 8 groups): W streams through
+ *    shared memory into m16n8k32 integer MMAs that multiply the codes exactly by
+ *    the activations split into signed bytes, each group's scale applied once to
+ *    its sum; a small first kernel builds those activation tables.
+ * BQ_PATH_GEMV takes the streamed kernel for affine 8-bit with one or two tokens
+ * (measured faster on B200) and the register-streaming kernel otherwise.
+ * BQ_PATH_GEMV_STREAM forces the streamed kernel for any of the three formats
+ * (BQ_ERR_UNSUPPORTED where it does not apply).  Both give the product within
+ * the GEMM tolerance; the streamed kernel computes with the exact weights
+ * d (q - 8) or s q + z, the register-streaming one with their bf16 roundings. */
 
 /*
  * q4_0_dequantize -- out[n][k] = bf16_rne(fp32(d[n][k/32]) * (q[n][k] - 8)).
@@ -188,7 +202,8 @@ BQ_API bq_status quant_matmul_q8(const int8_t* xq, const float* dx, const int32_
  * kernel as well.
  * The path is chosen by quant_matmul_select_path.  A path that needs scratch
  * memory (the unfused pair's bf16 copy of W, the fused kernel's split-K
- * partial sums) uses a library buffer, one per (device, stream):
+ * partial sums, the decode GEMV's activation tables for one or two tokens)
+ * uses a library buffer, one per (device, stream):
  *   - it is allocated on first need and grows on demand; a call that
  *     allocates must not be made during stream capture, so make one call per
  *     stream and problem size before capturing;
@@ -212,7 +227,8 @@ BQ_API bq_status quant_matmul(const uint16_t* x_bf16, const void* wq, const void
  * callers that cannot afford an allocation's implicit synchronization on a
  * first call.  It takes quant_matmul's own path, with a fixed 32 MiB array
  * that is part of the library's device image as its scratch: the decode GEMV
- * uses none; the fused tensor-core kernel keeps its K-split partial sums there
+ * keeps its activation tables there (one or two tokens: 8 K + 64 K / group
+ * bytes and a few more); the fused tensor-core kernel keeps its K-split partial sums there
  * (and runs without splitting K when they would not fit); the unfused pair
  * (q4_0_dequantize / affine_dequantize, then the bf16 tensor-core GEMM) stages
  * the bf16 copy of W there.  y is the same as quant_matmul's.
@@ -249,7 +265,9 @@ BQ_API bq_status quant_matmul_noalloc(const uint16_t* x_bf16, const void* wq, co
  *   wq, scales, y_bf16, N: host arrays of count device pointers / row counts
  *   biases: host array of count device pointers (affine), or NULL (Q4_0 for all)
  * At decode sizes (the dispatcher's GEMV path) all matrices run in one launch
- * and give the same bits as separate quant_matmul calls; at larger M each
+ * and give the same bits as separate quant_matmul calls (with one or two
+ * tokens their activation tables go in the stream's library buffer, as in
+ * quant_matmul); at larger M each
  * matrix runs its own quant_matmul path.  Errors as quant_matmul; transpose
  * must be 1 and count > 8 returns BQ_ERR_UNSUPPORTED, count == 0 or M == 0
  * does nothing.
@@ -265,7 +283,9 @@ BQ_API bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const voi
  * per-device buffer is used as in quant_matmul.  Otherwise, for the unfused
  * pair workspace_bytes must be >= quant_matmul_workspace_size(...)
  * (BQ_ERR_WORKSPACE if not); the fused path given a smaller workspace runs
- * without K splits (same result within the tolerance, possibly slower).  Forcing
+ * without K splits (same result within the tolerance, possibly slower); the
+ * decode GEMV of one or two tokens given a smaller workspace runs the
+ * register-streaming GEMV of three and more tokens instead (same tolerance).  Forcing
  * BQ_PATH_GEMV with M > 32 (M > 8 for 2-, 3- or 6-bit weights), BQ_PATH_TC_FUSED
  * for 2-, 3- or 6-bit weights, or either with transpose = 0, returns
  * BQ_ERR_UNSUPPORTED.
@@ -280,7 +300,10 @@ BQ_API bq_status quant_matmul_ex(const uint16_t* x_bf16, const void* wq, const v
  * 2).  The fused path: the fp32 partial sums of the tiles its plan splits over
  * K (splits x split tiles x tile tokens x 128 x 4; with more tiles than SMs,
  * only the tiles of the last, partly filled round are split), planned for the
- * current device, or for a B200 when there is none.  0 when the path needs none or
+ * current device, or for a B200 when there is none.  The decode GEMV with one
+ * or two tokens: its activation tables, K / 32 x 256 bytes of byte slices of
+ * x, K / group x 64 bytes of per-group scales and sums, and a flag word per
+ * 2048 activations, rounded up to 16 bytes.  0 when the path needs none or
  * the arguments are invalid.  Having no biases pointer, this call and
  * quant_matmul_select_path take group_size 32 with bits 4 as Q4_0 and any
  * other combination as affine. */

@@ -216,3 +216,24 @@ def test_q8_path_validation(L):
     assert L.quant_matmul_q8(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 2, 8, 40, None) == 2
     assert L.quant_matmul_q8(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 2, 8, 64, None) == 1
     assert L.quant_matmul_q8(None, None, None, None, None, None, 2, 0, 64, None) == 0
+
+
+def test_decode_gemv_table_workspace(L):
+    """The streamed GEMV (one or two tokens) needs its activation tables: K/32 x
+    256 bytes of byte slices, K/group x 64 bytes of group scales and sums, a flag
+    word per 2048 activations rounded up to 16 bytes.  Forced (path 4) for every
+    format; through the GEMV path (1, and AUTO) only where it is the dispatcher's
+    choice, affine 8-bit; none from three tokens on."""
+    for g, bits in ((32, 4), (64, 4), (64, 8), (128, 8), (32, 8), (128, 4)):
+        for M in (1, 2):
+            for K in (4096, 2048 if g < 128 else 1024):
+                flags = -(-M * K // 2048)
+                want = K // 32 * 256 + K // g * 64 + (flags * 4 + 15) // 16 * 16
+                assert L.quant_matmul_workspace_size(M, 12288, K, g, bits, 4) == want, (g, bits, M, K)
+                via_gemv = want if bits == 8 else 0
+                assert L.quant_matmul_workspace_size(M, 12288, K, g, bits, 1) == via_gemv
+                assert L.quant_matmul_workspace_size(M, 12288, K, g, bits, 0) == via_gemv
+        assert L.quant_matmul_workspace_size(3, 12288, 4096, g, bits, 1) == 0
+        assert L.quant_matmul_workspace_size(3, 12288, 4096, g, bits, 4) == 0
+    assert L.quant_matmul_workspace_size(1, 256, 544, 32, 4, 4) == 0      # K not a multiple of 8 blocks
+    assert L.quant_matmul_workspace_size(1, 256, 512, 64, 3, 4) == 0      # 3-bit: no streamed kernel
