@@ -47,8 +47,8 @@ CSRC = os.path.join(ROOT, "bit_quantized_gemm_quant_b200", "csrc")
 # with the hash of the kernel's source file at that capture.  A kernel whose
 # source changed since reports traffic null.
 NCU_TRAFFIC = {
-    "gemv_stream_kernel<Q4_0> M=1": {"bytes": None, "source": "gemv_stream.cuh", "sha16": None,
-                                      "capture": None},
+    "gemv_kernel<Q4_0> M=1": {"bytes": 28332288, "source": "gemv.cuh", "sha16": "94efba42044385eb",
+                              "capture": "2026-12-02 ncu --set full, profiles/gemv_kernel_q4_0_decode_m1_n12288_k4096.md"},
 }
 
 
@@ -224,6 +224,18 @@ def time_graphs(graphs, n_replays, world, device):
     return start.elapsed_time(end) / 1000.0
 
 
+def decode_kernel(bq, M, N, K, gs, bits):
+    """Which kernel(s) quant_matmul runs for this shape: the dispatcher's path and, on
+    the GEMV path, the streamed integer-MMA kernel exactly when it needs its
+    activation tables (quant_matmul_workspace_size > 0), else the register-streaming one."""
+    path = {v: k for k, v in bq.PATHS.items()}[bq.quant_matmul_select_path(M, N, K, gs, bits)]
+    if path != "gemv":
+        return {"path": path, "kernel": path, "launches_per_call": None}
+    if bq.quant_matmul_workspace_size(M, N, K, gs, bits, "gemv") > 0:
+        return {"path": path, "kernel": "gemv_int_prep_kernel + gemv_stream_kernel", "launches_per_call": 2}
+    return {"path": path, "kernel": "gemv_kernel", "launches_per_call": 1}
+
+
 def kernel_seconds(fn_list, reps):
     """Average device time of one call of each fn (back-to-back in one graph, CUDA events)."""
     import torch
@@ -285,7 +297,7 @@ def run_decode(args, world, rank, device, peaks):
     n_copies = 12
     copies = [(wq0, s0)] + [(wq0.clone(), s0.clone()) for _ in range(n_copies - 1)]
     g = inputs.generator(wl.seed + 1)                      # x is replicated: the same on every rank
-    xs = {M: inputs.activations_bf16(M, K, g).to(device) for M in (1, 8, 16, 32)}
+    xs = {M: inputs.activations_bf16(M, K, g).to(device) for M in (1, 2, 8, 16, 32)}
     ys = {M: torch.empty(M, N, dtype=torch.bfloat16, device=device) for M in xs}
     wbytes = workloads.packed_weight_bytes(wl.fmt, N, K, gs)
     assert n_copies * wbytes > 2 * L2_BYTES
@@ -320,8 +332,17 @@ def run_decode(args, world, rank, device, peaks):
         t = kernel_seconds(fns, 4)
         per_m[str(M)] = {"us": round(t * 1e6, 3), "gbs": round(wbytes / t / 1e9, 1),
                          "frac_hbm": round(wbytes / t / 1e9 / peaks["hbm_gbs"], 4),
-                         "tflops": round(2.0 * M * N * K / t / 1e12, 3),
-                         "path": {v: k for k, v in bq.PATHS.items()}[bq.quant_matmul_select_path(M, N, K, gs, bits)]}
+                         "tflops": round(2.0 * M * N * K / t / 1e12, 3), **decode_kernel(bq, M, N, K, gs, bits)}
+    # the streamed integer-MMA kernel forced at one and two tokens (BQ_PATH_GEMV takes it
+    # for affine 8-bit only; for Q4_0 the register-streaming kernel above is faster)
+    forced = {}
+    for M in (1, 2):
+        fns = [(lambda wq=wq, s=s, M=M: bq.quant_matmul_ex(xs[M], wq, s, None, gs, bits, True, "gemv_stream",
+                                                             out=ys[M])) for (wq, s) in copies]
+        t = kernel_seconds(fns, 4)
+        forced[str(M)] = {"us": round(t * 1e6, 3), "gbs": round(wbytes / t / 1e9, 1),
+                          "frac_hbm": round(wbytes / t / 1e9 / peaks["hbm_gbs"], 4),
+                          "kernel": "gemv_int_prep_kernel + gemv_stream_kernel", "launches_per_call": 2}
     # the quantized-activation path (opt-in, approximate): activation quantization
     # plus the Q4_0 x int8 GEMV, same weights, rotation and graph timing
     fns = [(lambda wq=wq, s=s: bq.quant_matmul_q8(*bq.q8_1_quantize(xs[1]), wq, s, out=ys[1])) for (wq, s) in copies]
@@ -334,8 +355,9 @@ def run_decode(args, world, rank, device, peaks):
           "note": "opt-in approximate path: q8_1_quantize + quant_matmul_q8; not the headline value"}
 
     t1 = per_m["1"]["us"] * 1e-6
-    traffic, traffic_src = stored_traffic("gemv_stream_kernel<Q4_0> M=1")
-    roof = {"bound": "hbm", "kernel": "gemv_stream_kernel<Q4_0> (M=1)", "achieved": per_m["1"]["gbs"],
+    kname = per_m["1"]["kernel"]
+    traffic, traffic_src = stored_traffic(f"{kname.split(' ')[-1]}<Q4_0> M=1")
+    roof = {"bound": "hbm", "kernel": f"{kname} <Q4_0> (M=1)", "achieved": per_m["1"]["gbs"],
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": per_m["1"]["frac_hbm"], "traffic": traffic,
             "traffic_source": traffic_src, "algorithmic_bytes_per_launch": wbytes,
             "launch_us": round(t1 * 1e6, 3)}
@@ -396,8 +418,9 @@ def run_decode(args, world, rank, device, peaks):
         "notes": {"l2": f"{n_copies} rotating weight copies per rank ({n_copies * wbytes / 1e6:.0f} MB > 126 MB L2)",
                   "bytes_per_step": wbytes * world, "path": "quant_matmul auto -> " + per_m["1"]["path"],
                   "timing": "CUDA events around graph replays of back-to-back launches, max over ranks"},
-        "per_m": per_m, "roofline": roof, "e2e": e2e, "gpu_launches": args.steps, "clocks": clk.summary(),
-        "secondary": {"q8_activation_path_m1": q8}, "gather": gather,
+        "per_m": per_m, "roofline": roof, "e2e": e2e,
+        "gpu_launches": args.steps * per_m["1"]["launches_per_call"], "clocks": clk.summary(),
+        "secondary": {"q8_activation_path_m1": q8, "streamed_int_kernel_forced": forced}, "gather": gather,
     }
 
 

@@ -126,9 +126,15 @@ int grid_for(int64_t items, int threads, const DeviceInfo& di)
 // at 3072), ties or trails from 4096; for affine 8-bit it leads up to 1024 tokens
 // and trails from 2048 (192 vs 182 us).
 constexpr int64_t kDefaultPairMinM[3] = {4096, 4096, 2048};   // Q4_0, affine4, affine8
+// Default GEMV/fused thresholds per format, from B200 sweeps of the same
+// projection at M = 8 .. 32: the fused kernel stays near 21.1-21.8 us (Q4_0),
+// 22.0-22.4 (affine 4-bit), 22.5-23.3 (affine 8-bit) while the GEMV grows with M;
+// they meet at M = 20 for the 4-bit formats (21.8 / 21.7, 22.4 / 22.3 us) and
+// between 12 and 16 for affine 8-bit (22.4-23.0 / 23.0 us at 16).
+constexpr int kDefaultTcMinM[3] = {21, 21, 17};
 
 struct DispatchCfg {
-    int tc_min_m = kGemvMaxM + 1;
+    int tc_min_m[3] = {kDefaultTcMinM[0], kDefaultTcMinM[1], kDefaultTcMinM[2]};
     int64_t pair_min_m[3] = {kDefaultPairMinM[0], kDefaultPairMinM[1], kDefaultPairMinM[2]};   // 0: never
 };
 
@@ -138,7 +144,7 @@ const DispatchCfg& dispatch_cfg()
         DispatchCfg c;
         if (const char* v = std::getenv("BQ_TC_MIN_M")) {
             long t = std::strtol(v, nullptr, 10);
-            c.tc_min_m = (int)std::min<long>(std::max<long>(t, 1), kGemvMaxM + 1);
+            for (int f = 0; f < 3; ++f) c.tc_min_m[f] = (int)std::min<long>(std::max<long>(t, 1), kGemvMaxM + 1);
         }
         if (const char* v = std::getenv("BQ_PAIR_MIN_M")) {
             long long t = std::strtoll(v, nullptr, 10);
@@ -153,7 +159,8 @@ int select_path(int64_t M, int64_t K, WFmt fmt)
 {
     if (!has_fast_paths(fmt)) return M <= kGaMaxM ? BQ_PATH_GEMV : BQ_PATH_DEQUANT_GEMM;
     const DispatchCfg& c = dispatch_cfg();
-    if (M < c.tc_min_m) return BQ_PATH_GEMV;
+    if (M < c.tc_min_m[(int)fmt]) return BQ_PATH_GEMV;
+    if (M <= kGemvMaxM && K % 64 != 0) return BQ_PATH_GEMV;      // no fused tile: the GEMV, not the pair
     const int64_t pair_min = c.pair_min_m[(int)fmt];
     if (pair_min > 0 && M >= pair_min) return BQ_PATH_DEQUANT_GEMM;
     return (K % 64 == 0) ? BQ_PATH_TC_FUSED : BQ_PATH_DEQUANT_GEMM;

@@ -317,15 +317,18 @@ BQ_API size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int g
  * routes to the vector-dot kernel).  Returns a bq_path other than AUTO:
  * (transpose = 1; 2-, 3- and 6-bit affine weights get GEMV up to M = 8 and
  * DEQUANT_GEMM above):
- *   M <  tc_min_m                 -> BQ_PATH_GEMV        (tc_min_m default 33)
+ *   M <  tc_min_m                 -> BQ_PATH_GEMV        (tc_min_m by format, from the
+ *                                    measured GEMV/fused crossovers on B200: 21 for
+ *                                    Q4_0 and affine 4-bit, 17 for 8-bit; with
+ *                                    K % 64 != 0 the GEMV up to M = 32)
  *   M >= pair_min_m               -> BQ_PATH_DEQUANT_GEMM (pair_min_m by format, from
  *                                    the measured fused/unfused crossovers on B200:
  *                                    4096 for Q4_0 and affine 4-bit, 2048 for 8-bit)
  *   otherwise                     -> BQ_PATH_TC_FUSED when K % 64 == 0,
  *                                    else BQ_PATH_DEQUANT_GEMM
- * Environment overrides, read once per process: BQ_TC_MIN_M (clamped to
- * [1, 33]; the GEMV handles at most 32 tokens) and BQ_PAIR_MIN_M (all
- * formats; 0: never).  Returns -1 for arguments quant_matmul would reject.
+ * Environment overrides, read once per process: BQ_TC_MIN_M (all formats,
+ * clamped to [1, 33]; the GEMV handles at most 32 tokens) and BQ_PAIR_MIN_M
+ * (all formats; 0: never).  Returns -1 for arguments quant_matmul would reject.
  */
 BQ_API int quant_matmul_select_path(int64_t M, int64_t N, int64_t K, int group_size, int bits);
 

@@ -124,10 +124,13 @@ def test_dispatcher_boundaries(L):
         for g, bits in ((32, 4), (64, 4), (64, 8)):
             p = L.quant_matmul_select_path(M, 12288, 4096, g, bits)
             pair_min = 2048 if bits == 8 else 4096
-            assert p == (1 if M <= 32 else 2 if M < pair_min else 3), (M, g, bits, p)
+            tc_min = 17 if bits == 8 else 21
+            assert p == (1 if M < tc_min else 2 if M < pair_min else 3), (M, g, bits, p)
     # K % 64 != 0 (Q4_0 only): prefill goes through the unfused pair
     assert L.quant_matmul_select_path(512, 256, 544, 32, 4) == 3
     assert L.quant_matmul_select_path(8, 256, 544, 32, 4) == 1
+    assert L.quant_matmul_select_path(32, 256, 544, 32, 4) == 1     # no fused tile: GEMV up to 32
+    assert L.quant_matmul_select_path(33, 256, 544, 32, 4) == 3
     assert L.quant_matmul_select_path(-1, 256, 512, 32, 4) == -1
     assert L.quant_matmul_select_path(8, 256, 512, 64, 5) == -1
     assert L.quant_matmul_workspace_size(512, 256, 544, 32, 4, 0) == 256 * 544 * 2
@@ -171,11 +174,11 @@ def _select_in_subprocess(env_extra, Ms):
 
 def test_dispatcher_env_overrides(L):
     Ms = [1, 8, 19, 32, 33, 512, 4096]
-    assert _select_in_subprocess({}, Ms) == [1, 1, 1, 1, 2, 2, 3]             # affine 4-bit: pair from 4096
+    assert _select_in_subprocess({}, Ms) == [1, 1, 1, 2, 2, 2, 3]             # affine 4-bit: fused from 21, pair from 4096
     assert _select_in_subprocess({"BQ_TC_MIN_M": "8"}, Ms) == [1, 2, 2, 2, 2, 2, 3]
     assert _select_in_subprocess({"BQ_TC_MIN_M": "1000"}, Ms) == [1, 1, 1, 1, 2, 2, 3]   # clamped to 33
-    assert _select_in_subprocess({"BQ_PAIR_MIN_M": "512"}, Ms) == [1, 1, 1, 1, 2, 3, 3]
-    assert _select_in_subprocess({"BQ_PAIR_MIN_M": "0"}, Ms) == [1, 1, 1, 1, 2, 2, 2]
+    assert _select_in_subprocess({"BQ_PAIR_MIN_M": "512"}, Ms) == [1, 1, 1, 2, 2, 3, 3]
+    assert _select_in_subprocess({"BQ_PAIR_MIN_M": "0"}, Ms) == [1, 1, 1, 2, 2, 2, 2]
 
 
 def test_empty_problems_need_no_pointers(L):
