@@ -49,6 +49,8 @@ CSRC = os.path.join(ROOT, "bit_quantized_gemm_quant_b200", "csrc")
 NCU_TRAFFIC = {
     "gemv_kernel<Q4_0> M=1": {"bytes": 28332288, "source": "gemv.cuh", "sha16": "94efba42044385eb",
                               "capture": "2026-12-02 ncu --set full, profiles/gemv_kernel_q4_0_decode_m1_n12288_k4096.md"},
+    "gemv_tma_kernel<Q4_0> M=1": {"bytes": 28394496, "source": "gemv_stream.cuh", "sha16": "c2bbd7433e1793e3",
+                                  "capture": "2026-12-02 ncu --set full, profiles/gemv_tma_kernel_q4_0_decode_m1_n12288_k4096.md"},
 }
 
 
@@ -224,16 +226,16 @@ def time_graphs(graphs, n_replays, world, device):
     return start.elapsed_time(end) / 1000.0
 
 
-def decode_kernel(bq, M, N, K, gs, bits):
-    """Which kernel(s) quant_matmul runs for this shape: the dispatcher's path and, on
-    the GEMV path, the streamed integer-MMA kernel exactly when it needs its
-    activation tables (quant_matmul_workspace_size > 0), else the register-streaming one."""
-    path = {v: k for k, v in bq.PATHS.items()}[bq.quant_matmul_select_path(M, N, K, gs, bits)]
-    if path != "gemv":
+def decode_kernel(bq, M, N, K, gs, bits, path=None):
+    """Which kernel(s) quant_matmul runs for this shape (the library's own answer,
+    quant_matmul_gemv_kernel): the dispatcher's path, and on a decode path the kernel
+    and its launches per call."""
+    if path is None:
+        path = {v: k for k, v in bq.PATHS.items()}[bq.quant_matmul_select_path(M, N, K, gs, bits)]
+    k = bq.quant_matmul_gemv_kernel(M, N, K, gs, bits, path) if path in ("gemv", "gemv_stream") else -1
+    if k < 0:
         return {"path": path, "kernel": path, "launches_per_call": None}
-    if bq.quant_matmul_workspace_size(M, N, K, gs, bits, "gemv") > 0:
-        return {"path": path, "kernel": "gemv_int_prep_kernel + gemv_stream_kernel", "launches_per_call": 2}
-    return {"path": path, "kernel": "gemv_kernel", "launches_per_call": 1}
+    return {"path": path, "kernel": bq.GEMV_KERNELS[k], "launches_per_call": 2 if k == 2 else 1}
 
 
 def kernel_seconds(fn_list, reps):
@@ -334,7 +336,7 @@ def run_decode(args, world, rank, device, peaks):
                          "frac_hbm": round(wbytes / t / 1e9 / peaks["hbm_gbs"], 4),
                          "tflops": round(2.0 * M * N * K / t / 1e12, 3), **decode_kernel(bq, M, N, K, gs, bits)}
     # the streamed integer-MMA kernel forced at one and two tokens (BQ_PATH_GEMV takes it
-    # for affine 8-bit only; for Q4_0 the register-streaming kernel above is faster)
+    # at one token, and at two for the affine formats)
     forced = {}
     for M in (1, 2):
         fns = [(lambda wq=wq, s=s, M=M: bq.quant_matmul_ex(xs[M], wq, s, None, gs, bits, True, "gemv_stream",
@@ -342,7 +344,7 @@ def run_decode(args, world, rank, device, peaks):
         t = kernel_seconds(fns, 4)
         forced[str(M)] = {"us": round(t * 1e6, 3), "gbs": round(wbytes / t / 1e9, 1),
                           "frac_hbm": round(wbytes / t / 1e9 / peaks["hbm_gbs"], 4),
-                          "kernel": "gemv_int_prep_kernel + gemv_stream_kernel", "launches_per_call": 2}
+                          **decode_kernel(bq, M, N, K, gs, bits, "gemv_stream")}
     # the quantized-activation path (opt-in, approximate): activation quantization
     # plus the Q4_0 x int8 GEMV, same weights, rotation and graph timing
     fns = [(lambda wq=wq, s=s: bq.quant_matmul_q8(*bq.q8_1_quantize(xs[1]), wq, s, out=ys[1])) for (wq, s) in copies]

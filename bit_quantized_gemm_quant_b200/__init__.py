@@ -55,6 +55,7 @@ def lib() -> ctypes.CDLL:
         "quant_matmul_noalloc": [P, P, P, P, P, I64, I64, I64, I, I, I, P],
         "quant_matmul_multi": [P, I, P, P, P, P, P, I64, I64, I, I, I, P],
         "quant_matmul_workspace_size": [I64, I64, I64, I, I, I],
+        "quant_matmul_gemv_kernel": [I64, I64, I64, I, I, I],
         "quant_matmul_select_path": [I64, I64, I64, I, I],
         "bf16_matmul": [P, P, P, I64, I64, I64, P],
         "q4_0_quantize": [P, P, P, I64, I64, P],
@@ -258,6 +259,16 @@ def quant_matmul_noalloc(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor
 
 def quant_matmul_select_path(M: int, N: int, K: int, group_size: int, bits: int) -> int:
     return lib().quant_matmul_select_path(M, N, K, group_size, bits)
+
+
+GEMV_KERNELS = {0: "gemv_kernel", 1: "gemv_tma_kernel", 2: "gemv_int_prep_kernel + gemv_stream_kernel",
+                3: "gemv_affine_kernel"}
+
+
+def quant_matmul_gemv_kernel(M: int, N: int, K: int, group_size: int, bits: int, path="auto") -> int:
+    """Which decode kernel runs (GEMV_KERNELS), -1 off the decode path (host only)."""
+    p = PATHS[path] if isinstance(path, str) else int(path)
+    return lib().quant_matmul_gemv_kernel(M, N, K, group_size, bits, p)
 
 
 def quant_matmul_workspace_size(M: int, N: int, K: int, group_size: int, bits: int, path="auto") -> int:

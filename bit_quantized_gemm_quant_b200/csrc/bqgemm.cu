@@ -184,6 +184,37 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+// Packed code rows [rows][row_bytes] seen as 3-D [row_bytes / 128][rows][128 bytes]
+// (strides 128 and row_bytes bytes), box [chunks][16][128 bytes], 128-byte swizzle.
+bool make_code_map_3d(CUtensorMap* m, const void* ptr, int64_t rows, int64_t row_bytes, int chunks)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[3] = {128, (cuuint64_t)rows, (cuuint64_t)(row_bytes / 128)};
+    cuuint64_t gstride[2] = {(cuuint64_t)row_bytes, 128};
+    cuuint32_t box[3] = {128, 16, (cuuint32_t)chunks};
+    cuuint32_t estride[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), gdim, gstride, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 16-bit scale rows [rows][groups] seen as 3-D [groups / 8][rows][8 values]
+// (strides 16 and groups * 2 bytes), box [units][16][8 values], no swizzle: the
+// rows of one 16-byte unit land 16 bytes apart.
+bool make_scale_map_3d(CUtensorMap* m, const void* ptr, int64_t rows, int64_t groups, int units)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[3] = {8, (cuuint64_t)rows, (cuuint64_t)(groups / 8)};
+    cuuint64_t gstride[2] = {(cuuint64_t)(groups * 2), 16};
+    cuuint32_t box[3] = {8, 16, (cuuint32_t)units};
+    cuuint32_t estride[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(ptr), gdim, gstride, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Row-major 2-D [rows][cols] tensor, tile box [box_rows][box_cols].
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* ptr, int64_t rows, int64_t cols,
               int box_rows, int box_cols, CUtensorMapSwizzle sw)
@@ -499,10 +530,20 @@ size_t stream_gemv_table_bytes(WFmt fmt, int group_size, int64_t M, int64_t K, i
 
 // BQ_PATH_GEMV takes the streamed kernel where it measured faster than the
 // register-streaming one on B200 (N = 12288, K = 4096, graph-timed launches
-// over rotating weight copies): affine 8-bit with one or two tokens (17.4 against
-// 18.3 us).  For Q4_0 and affine 4-bit the register-streaming kernel is faster
-// (12.6 against 14.5 us at M = 1).
-bool stream_gemv_preferred(WFmt fmt, int64_t M) { return fmt == WFmt::AFF8 && M <= kSgIntTokens; }
+// over rotating weight copies, TMA-fed variant): one token for every format
+// (Q4_0 10.98 against 12.58 us, affine 4-bit 10.66 / 13.26, affine 8-bit 12.89 /
+// 18.3), two tokens for the affine formats (12.18 / 13.38, 14.31 / 18.3); Q4_0 at
+// two tokens ties (12.58 / 12.61) and keeps the register-streaming kernel.
+// It runs one CTA per SM and pays a fixed start per CTA (its activation slices,
+// the ring's fill), so it needs several 16-row tiles per SM: with the Llama-3.2-1B
+// stack's matrices (32 to 1024 tiles, K = 2048 or 8192) one token took 549 against
+// 441 us per stack.  It is taken where it was measured faster: K >= 4096 and at
+// least 4 tiles per SM.
+bool stream_gemv_preferred(WFmt fmt, int64_t M, int64_t ntiles, int64_t K, int num_sms)
+{
+    if (K < 4096 || ntiles < 4 * (int64_t)num_sms) return false;
+    return M == 1 || (M == 2 && fmt != WFmt::Q4_0);
+}
 
 bool plan_stream_gemv(WFmt fmt, int group_size, int64_t M, const SgMats& mats, int64_t K, const DeviceInfo& di,
                       SgPlan* pl)
@@ -645,13 +686,180 @@ bq_status launch_stream_gemv(SgPlan& pl, int dev, const DeviceInfo& di, const ui
     }
 }
 
+// Plan of the TMA-fed kernel: stages of CH = 16 (else 8) 128-byte code chunks
+// per row, whole rows split into nchunks stages; false when K does not split
+// that way or a stage's scales are not whole 16-byte rows.
+struct SgTmaPlan {
+    STmaParams prm{};
+    int grid = 0, ch = 0;
+    size_t smem = 0;
+};
+
+// The TMA kernel's stage shape and shared-memory carve-up for (fmt, M, K) and
+// ntiles 16-row tiles on a device with num_sms SMs and smem_optin bytes of
+// shared memory per block; false when it does not apply.
+struct SgTmaShape {
+    int ch = 0, stages = 0, nchunks = 0, grid = 0;
+    int64_t stage_elems = 0, stage_groups = 0, scale_row = 0, stage_pitch = 0;
+    int64_t off_x = 0, off_c = 0, off_red = 0, off_bar = 0, off_stage = 0, smem = 0;
+};
+
+bool tma_shape(WFmt fmt, int group_size, int64_t M, int64_t ntiles, int64_t K, int num_sms, int smem_optin,
+               SgTmaShape* sh)
+{
+    if (stream_gemv_table_bytes(fmt, group_size, M, K) == 0 || ntiles < 1) return false;
+    const int gs = fmt == WFmt::Q4_0 ? 32 : group_size;
+    const int bits = fmt == WFmt::AFF8 ? 8 : 4, E = bits == 8 ? 16 : 32;
+    const int upg = gs / E, atom_units = upg > 2 ? upg : 2;
+    const int64_t row_bytes = K * bits / 8;
+    if (row_bytes % 128 != 0) return false;
+    const int64_t row_chunks = row_bytes / 128;
+    const int ch = row_chunks % 16 == 0 ? 16 : row_chunks % 8 == 0 ? 8 : 0;
+    if (ch == 0 || ch % atom_units != 0) return false;
+    SgTmaShape& h = *sh;
+    h.ch = ch;
+    h.stage_elems = (int64_t)ch * 128 * 8 / bits;
+    h.stage_groups = h.stage_elems / gs;
+    h.scale_row = h.stage_groups * 2;
+    if (h.scale_row % 16 != 0) return false;
+    h.nchunks = (int)(row_chunks / ch);
+    h.grid = (int)(ntiles <= 8 * (int64_t)num_sms ? std::min<int64_t>(ntiles, num_sms) : (ntiles + 7) / 8);
+    const int64_t tcap = (ntiles + h.grid - 1) / h.grid;
+    const bool affine = fmt != WFmt::Q4_0;
+    auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
+    h.stage_pitch = up((int64_t)ch * 2048 + 16 * h.scale_row * (affine ? 2 : 1), 1024);
+    int64_t off = 0;
+    h.off_x = off;
+    off = up(off + (K / 32) * kSgIntStepBytes, 128);
+    h.off_c = off;
+    off = up(off + (K / gs) * kSgIntCtabBytes, 128);
+    h.off_red = off;
+    off = up(off + tcap * kSgWarpsTma * 16 * M * 4, 128);           // one column per token
+    h.off_bar = off;
+    off = up(off + (2 * kSgMaxStagesTma + 1) * 8, 1024);
+    h.off_stage = off;
+    const int64_t budget = (int64_t)smem_optin - 1024;               // 1 KB to align the base
+    // as many stages as fit, up to 4 (5 measured slower for the 4-bit formats: 13.2
+    // against 12.7 us for Q4_0 at M = 1)
+    h.stages = (int)std::min<int64_t>(kSgMaxStagesTma, (budget - off) / h.stage_pitch);
+    if (h.stages < 2) return false;
+    h.smem = off + h.stages * h.stage_pitch + 1024;
+    return true;
+}
+
+bool plan_stream_gemv_tma(WFmt fmt, int group_size, int64_t M, const SgMats& mats, int64_t K, const DeviceInfo& di,
+                          SgTmaPlan* pl)
+{
+    if (mats.count < 1 || mats.count > kSgMaxMats) return false;
+    int64_t nt_all = 0;
+    for (int i = 0; i < mats.count; ++i) nt_all += (std::max<int64_t>(mats.N[i], 0) + 15) / 16;
+    SgTmaShape h;
+    if (!tma_shape(fmt, group_size, M, nt_all, K, di.num_sms, di.max_smem_optin, &h)) return false;
+    const int gs = fmt == WFmt::Q4_0 ? 32 : group_size;
+    const int bits = fmt == WFmt::AFF8 ? 8 : 4;
+    const int64_t row_bytes = K * bits / 8;
+    const int ch = h.ch;
+    const int64_t stage_groups = h.stage_groups;
+    SgTmaPlan& P = *pl;
+    STmaParams& q = P.prm;
+    q = STmaParams{};
+    SGemvParams& p = q.g;
+    int64_t ntiles = 0;
+    p.count = mats.count;
+    for (int i = 0; i < mats.count; ++i) {
+        if (mats.N[i] < 0 || mats.N[i] > INT32_MAX / 2) return false;
+        p.tile_begin[i] = (int)ntiles;
+        ntiles += (mats.N[i] + 15) / 16;
+        if (ntiles > INT32_MAX / 2) return false;
+        p.wq[i] = reinterpret_cast<const uint8_t*>(mats.wq[i]);
+        p.scales[i] = mats.scales[i];
+        p.biases[i] = mats.biases[i];
+        p.y[i] = mats.y[i];
+        p.N[i] = (int)mats.N[i];
+        if (mats.N[i] == 0) continue;
+        if (!make_code_map_3d(&q.codes[i], mats.wq[i], mats.N[i], row_bytes, ch)) return false;
+        if (!make_scale_map_3d(&q.scales[i], mats.scales[i], mats.N[i], K / gs, (int)(stage_groups / 8)))
+            return false;
+        if (fmt != WFmt::Q4_0 &&
+            !make_scale_map_3d(&q.biases[i], mats.biases[i], mats.N[i], K / gs, (int)(stage_groups / 8)))
+            return false;
+    }
+    p.tile_begin[mats.count] = (int)ntiles;
+    if (ntiles == 0) return false;
+    const bool affine = fmt != WFmt::Q4_0;
+    p.M = (int)M;
+    p.K = (int)K;
+    p.kc = (int)h.stage_elems;
+    p.nchunks = h.nchunks;
+    p.ntiles = (int)ntiles;
+    p.stages = h.stages;
+    p.red_cols = (int)M;
+    p.off_x = (uint32_t)h.off_x;
+    p.off_c = (uint32_t)h.off_c;
+    p.off_red = (uint32_t)h.off_red;
+    q.off_stage = (uint32_t)h.off_stage;
+    q.stage_pitch = (uint32_t)h.stage_pitch;
+    q.scale_row_bytes = (uint32_t)h.scale_row;
+    q.stage_tx = (uint32_t)(ch * 2048 + 16 * h.scale_row * (affine ? 2 : 1));
+    q.off_bar = (uint32_t)h.off_bar;
+    P.grid = h.grid;
+    P.ch = ch;
+    P.smem = (size_t)h.smem;
+    return true;
+}
+
+template <Fmt F, int GS, int CH>
+bq_status launch_stream_gemv_tma_ch(SgTmaPlan& pl, int dev, const DeviceInfo& di, cudaStream_t st)
+{
+    auto kern = gemv_tma_kernel<F, GS, CH>;
+    static bool attr_done[kMaxDevices] = {};
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin) !=
+            cudaSuccess)
+            return BQ_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    return launch_pdl(kern, pl.grid, 32 * (kSgWarpsTma + 1), pl.smem, st, pl.prm);
+}
+
+// One launch: the kernel builds its activation tables itself.
+template <Fmt F, int GS>
+bq_status launch_stream_gemv_tma(SgTmaPlan& pl, int dev, const DeviceInfo& di, const uint16_t* x, cudaStream_t st)
+{
+    pl.prm.g.x = x;
+    pl.prm.g.tab = nullptr;
+    return pl.ch == 16 ? launch_stream_gemv_tma_ch<F, GS, 16>(pl, dev, di, st)
+                       : launch_stream_gemv_tma_ch<F, GS, 8>(pl, dev, di, st);
+}
+
 // The streamed kernel when its plan applies (returns true and the launch status
-// in *out), else false and the caller takes the register-streaming GEMV.  Its
+// in *out), else false and the caller takes the register-streaming GEMV.  The
+// TMA-fed variant runs where its stages fit K, the cp.async one otherwise.  Its
 // tables go in the caller's workspace when one is given (false if it is too
 // small), else in the library's buffer of this stream.
+std::mutex g_sg_mu;                        // the TMA plan's static storage
+
 bool try_stream_gemv(WFmt fmt, int group_size, const uint16_t* x, const SgMats& mats, int64_t M, int64_t K, int dev,
                      const DeviceInfo& di, cudaStream_t st, void* workspace, size_t workspace_bytes, bq_status* out)
 {
+    static SgTmaPlan tp;                   // large (tensor maps): not on the stack
+    std::lock_guard<std::mutex> lk(g_sg_mu);
+    if (plan_stream_gemv_tma(fmt, group_size, M, mats, K, di, &tp)) {     // needs no device scratch
+        switch (fmt) {
+        case WFmt::Q4_0: *out = launch_stream_gemv_tma<Fmt::Q4_0, 32>(tp, dev, di, x, st); break;
+        case WFmt::AFF4:
+            *out = group_size == 32   ? launch_stream_gemv_tma<Fmt::AFF4, 32>(tp, dev, di, x, st)
+                   : group_size == 64 ? launch_stream_gemv_tma<Fmt::AFF4, 64>(tp, dev, di, x, st)
+                                      : launch_stream_gemv_tma<Fmt::AFF4, 128>(tp, dev, di, x, st);
+            break;
+        default:
+            *out = group_size == 32   ? launch_stream_gemv_tma<Fmt::AFF8, 32>(tp, dev, di, x, st)
+                   : group_size == 64 ? launch_stream_gemv_tma<Fmt::AFF8, 64>(tp, dev, di, x, st)
+                                      : launch_stream_gemv_tma<Fmt::AFF8, 128>(tp, dev, di, x, st);
+            break;
+        }
+        return true;
+    }
     SgPlan pl;
     if (!plan_stream_gemv(fmt, group_size, M, mats, K, di, &pl)) return false;
     void* tab = workspace;
@@ -789,10 +997,16 @@ size_t workspace_for(int path, WFmt fmt, int group_size, int64_t M, int64_t N, i
                      int smem_optin)
 {
     if (path == BQ_PATH_DEQUANT_GEMM) return (size_t)N * (size_t)K * 2u;
-    if (path == BQ_PATH_GEMV)
-        return has_fast_paths(fmt) && stream_gemv_preferred(fmt, M) ? stream_gemv_table_bytes(fmt, group_size, M, K)
-                                                                    : 0u;
-    if (path == BQ_PATH_GEMV_STREAM) return has_fast_paths(fmt) ? stream_gemv_table_bytes(fmt, group_size, M, K) : 0u;
+    if ((path == BQ_PATH_GEMV && stream_gemv_preferred(fmt, M, (N + 15) / 16, K, num_sms)) ||
+        path == BQ_PATH_GEMV_STREAM) {
+        // the TMA-fed kernel builds its tables in shared memory; the cp.async one
+        // takes them from device scratch
+        if (!has_fast_paths(fmt)) return 0u;
+        SgTmaShape h;
+        if (tma_shape(fmt, group_size, M, (N + 15) / 16, K, num_sms, smem_optin, &h)) return 0u;
+        return stream_gemv_table_bytes(fmt, group_size, M, K);
+    }
+    if (path == BQ_PATH_GEMV) return 0u;
     if (path != BQ_PATH_TC_FUSED || !has_fast_paths(fmt) || K % 64 != 0 || M > INT32_MAX || N > INT32_MAX ||
         K > INT32_MAX)
         return 0u;
@@ -910,7 +1124,7 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
         return workspace && workspace_bytes < need ? BQ_ERR_WORKSPACE : BQ_ERR_UNSUPPORTED;
     case BQ_PATH_GEMV:
         if (!has_fast_paths(fmt)) return launch_gemv_affine(fmt, x, wq, sc, bi, y, M, N, K, group_size, st);
-        if (stream_gemv_preferred(fmt, M) &&
+        if (stream_gemv_preferred(fmt, M, (N + 15) / 16, K, di.num_sms) &&
             try_stream_gemv(fmt, group_size, x, one_matrix(wq, sc, bi, y, N), M, K, dev, di, st, workspace,
                             workspace_bytes, &s))
             return s;
@@ -1176,7 +1390,10 @@ bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const void* cons
         mats.y[i] = y_bf16[i];
         mats.N[i] = N[i];
     }
-    if (stream_gemv_preferred(fmt, M) && try_stream_gemv(fmt, group_size, x_bf16, mats, M, K, dev, di, st, nullptr, 0, &s))
+    int64_t ntiles_all = 0;
+    for (int i = 0; i < count; ++i) ntiles_all += (N[i] + 15) / 16;
+    if (stream_gemv_preferred(fmt, M, ntiles_all, K, di.num_sms) &&
+        try_stream_gemv(fmt, group_size, x_bf16, mats, M, K, dev, di, st, nullptr, 0, &s))
         return s;
     if (fmt == WFmt::Q4_0) return launch_gemv_multi<Fmt::Q4_0>(x_bf16, tab, M, K, group_size, st);
     if (fmt == WFmt::AFF4) return launch_gemv_multi<Fmt::AFF4>(x_bf16, tab, M, K, group_size, st);
@@ -1197,6 +1414,30 @@ size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int group_si
     }
     cudaGetLastError();
     return workspace_for(path, fmt, group_size, M, N, K, num_sms, smem_optin);
+}
+
+int quant_matmul_gemv_kernel(int64_t M, int64_t N, int64_t K, int group_size, int bits, int path)
+{
+    WFmt fmt;
+    if (M < 1 || check_format(format_tag(group_size, bits), N, K, group_size, bits, &fmt) != BQ_OK) return -1;
+    if (path == BQ_PATH_AUTO) path = select_path(M, K, fmt);
+    if (path != BQ_PATH_GEMV && path != BQ_PATH_GEMV_STREAM) return -1;
+    if (!has_fast_paths(fmt)) return path == BQ_PATH_GEMV && M <= kGaMaxM ? 3 : -1;
+    int dev, num_sms = 148, smem_optin = 232448;
+    DeviceInfo di;
+    if (cudaGetDevice(&dev) == cudaSuccess && current_device(&dev, &di) == BQ_OK) {
+        num_sms = di.num_sms;
+        smem_optin = di.max_smem_optin;
+    }
+    cudaGetLastError();
+    const bool streamed =
+        path == BQ_PATH_GEMV_STREAM || stream_gemv_preferred(fmt, M, (N + 15) / 16, K, num_sms);
+    if (streamed && stream_gemv_table_bytes(fmt, group_size, M, K) > 0) {
+        SgTmaShape h;
+        return tma_shape(fmt, group_size, M, (N + 15) / 16, K, num_sms, smem_optin, &h) ? 1 : 2;
+    }
+    if (path == BQ_PATH_GEMV_STREAM) return -1;
+    return M <= kGemvMaxM ? 0 : -1;
 }
 
 int quant_matmul_select_path(int64_t M, int64_t N, int64_t K, int group_size, int bits)

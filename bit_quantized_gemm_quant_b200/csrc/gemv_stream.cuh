@@ -57,9 +57,10 @@
 // partial sums of each tile are summed in warp order at the end, so the
 // result is deterministic.
 //
-// Launch: both kernels use programmatic stream serialization, so each launch
-// overlaps the tail of the kernel before it; each reads x, the tables, W and
-// scales, and writes its outputs, only after griddepcontrol.wait.
+// Launch: both kernels use programmatic stream serialization.  The prep kernel
+// reads x after its griddepcontrol.wait and lets the GEMV launch only then; the
+// cp.async GEMV reads everything after its own wait, the TMA-fed one streams W
+// before it (see there) and reads x's tables and writes y after it.
 #pragma once
 
 #include "gemv.cuh"
@@ -146,6 +147,8 @@ constexpr int kSgMaxMats = 8;                  // matrices sharing x in one laun
 constexpr int kSgIntCtabBytes = 64;            // group table: 4 quad positions x (c0, c1, X0, X1)
 constexpr uint32_t kSgIntStepBytes = 256;      // slice table per 32-element step: 8 columns x 4 x 8 bytes
 constexpr int kSgPrepThreads = 256;
+constexpr int kSgWarpsTma = 8;                 // compute warps of the TMA-fed kernel (plus one producer)
+constexpr int kSgMaxStagesTma = 4;
 
 struct SGemvParams {
     const uint16_t* x;                   // bf16 [M][K], shared by every matrix
@@ -197,42 +200,46 @@ BQ_DEVINL int int_column(int M, int m, int j) { return M == 1 ? j : 4 * m + j; }
 // signed-digit form (three digits, the last one 0 or +-1) lands at slice
 // sh / 8, and a byte transpose (prmt) gathers each slice's four bytes per MMA
 // register.  The top slice absorbs the carry, which keeps it within +-64.
+// One item of the activation tables (token m, 32-element step, quad position
+// t) by one lane of a warp whose lanes all take part (a lane with valid ==
+// false computes on clamped data and stores nothing): the slices of its eight
+// activations into `xt` (the slice table), and -- by the first lane of each
+// group -- the group's column scales and addends into `ct` (the group table).
+// A group's lanes must be consecutive lanes of the warp, aligned to 4 SPG.
+// Returns nonzero when one of its activations is not held exactly.
+// The item's eight activations as bf16 pairs in the order of the two MMA B
+// registers: element i is half (i & 1) of word i >> 1.
+template <Fmt F>
+BQ_DEVINL void int_item_load(const uint16_t* __restrict__ x, int K, int m, int step, int t, uint32_t (&raw)[4])
+{
+    const uint16_t* xr = x + (int64_t)m * K + (int64_t)step * 32;
+    if constexpr (F == Fmt::AFF4) {
+        // register 0 <- elements 8t + 2i (low halves), register 1 <- 8t + 2i + 1 (high halves)
+        const uint4 q = *reinterpret_cast<const uint4*>(xr + 8 * t);
+        raw[0] = __byte_perm(q.x, q.y, 0x5410);
+        raw[1] = __byte_perm(q.z, q.w, 0x5410);
+        raw[2] = __byte_perm(q.x, q.y, 0x7632);
+        raw[3] = __byte_perm(q.z, q.w, 0x7632);
+    } else {
+        const uint2 a = *reinterpret_cast<const uint2*>(xr + 4 * t);
+        const uint2 c = *reinterpret_cast<const uint2*>(xr + 16 + 4 * t);
+        raw[0] = a.x;
+        raw[1] = a.y;
+        raw[2] = c.x;
+        raw[3] = c.y;
+    }
+}
+
 template <Fmt F, int GS>
-__global__ void __launch_bounds__(kSgPrepThreads)
-gemv_int_prep_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ tab, uint32_t c_off,
-                     uint32_t f_off)
+BQ_DEVINL int int_table_item_raw(const uint32_t (&raw)[4], int M, int m, int step, int t, int lane, bool valid,
+                                 uint8_t* xt, uint8_t* ct)
 {
     constexpr int SPG = GS / 32;                        // MMA steps per group
     constexpr int GL = 4 * SPG;                         // lanes that hold one group
     static_assert(GL <= 32, "a group's lanes lie in one warp");
-    grid_dependents_launch();                           // the GEMV may launch; it waits for this grid to finish
-    grid_dependency_wait();                             // x comes from the previous kernel
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int nsteps = K / 32;
     const int S = M == 1 ? 8 : 4, P = 8 * S - 3;
-    const int items = M * nsteps * 4;                   // a multiple of 32 (K is a multiple of 256)
-    const int idx = blockIdx.x * kSgPrepThreads + tid;
     int inexact = 0;
-    if (idx - lane < items) {                           // whole warps
-        const int t = idx & 3, step = (idx >> 2) % nsteps, m = (idx >> 2) / nsteps;
-        const uint16_t* xr = x + (int64_t)m * K + (int64_t)step * 32;
-        // the 8 activations as bf16 pairs: element i is half (i & 1) of word i >> 1
-        uint32_t raw[4];
-        if constexpr (F == Fmt::AFF4) {
-            // register 0 <- elements 8t + 2i (low halves), register 1 <- 8t + 2i + 1 (high halves)
-            const uint4 q = *reinterpret_cast<const uint4*>(xr + 8 * t);
-            raw[0] = __byte_perm(q.x, q.y, 0x5410);
-            raw[1] = __byte_perm(q.z, q.w, 0x5410);
-            raw[2] = __byte_perm(q.x, q.y, 0x7632);
-            raw[3] = __byte_perm(q.z, q.w, 0x7632);
-        } else {
-            const uint2 a = *reinterpret_cast<const uint2*>(xr + 4 * t);
-            const uint2 c = *reinterpret_cast<const uint2*>(xr + 16 + 4 * t);
-            raw[0] = a.x;
-            raw[1] = a.y;
-            raw[2] = c.x;
-            raw[3] = c.y;
-        }
+    {
         uint32_t key[8];
         uint32_t kmax = 0u;
         int bad = 0;
@@ -269,7 +276,7 @@ gemv_int_prep_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t* __re
             } else {
                 const int rs = -sh;
                 W = rs >= 8 ? 0 : mant >> rs;
-                inexact |= (rs >= 8 ? mant : mant - (W << rs)) != 0;
+                inexact |= valid && (rs >= 8 ? mant : mant - (W << rs)) != 0;
                 j0 = 0;
             }
             if (bad) {
@@ -307,15 +314,16 @@ gemv_int_prep_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t* __re
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             if (j < S) {
-                *reinterpret_cast<uint2*>(tab + (size_t)step * kSgIntStepBytes +
-                                          (size_t)(int_column(M, m, j) * 4 + t) * 8u) = make_uint2(r0[j], r1[j]);
+                if (valid)
+                    *reinterpret_cast<uint2*>(xt + (size_t)step * kSgIntStepBytes +
+                                              (size_t)(int_column(M, m, j) * 4 + t) * 8u) = make_uint2(r0[j], r1[j]);
                 L[j] = __dp4a((int)r0[j], 0x01010101, __dp4a((int)r1[j], 0x01010101, 0));
 #pragma unroll
                 for (int o = 1; o < GL; o <<= 1) L[j] += __shfl_xor_sync(0xFFFFFFFFu, L[j], o);
             }
         }
-        if ((lane & (GL - 1)) == 0) {
-            uint8_t* ct = tab + c_off + (size_t)(step / SPG) * kSgIntCtabBytes;
+        if (valid && (lane & (GL - 1)) == 0) {
+            uint8_t* cg = ct + (size_t)(step / SPG) * kSgIntCtabBytes;
 #pragma unroll
             for (int j = 0; j < 8; j += 2) {
                 if (j < S) {
@@ -326,11 +334,40 @@ gemv_int_prep_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t* __re
                         if constexpr (F == Fmt::Q4_0) X[h] = (uint32_t)(-8 * L[j + h]);
                         else X[h] = j + h == 0 ? __float_as_uint(sum) : 0u;
                     }
-                    *reinterpret_cast<uint4*>(ct + (int_column(M, m, j) / 2) * 16) = make_uint4(c[0], c[1], X[0], X[1]);
+                    *reinterpret_cast<uint4*>(cg + (int_column(M, m, j) / 2) * 16) = make_uint4(c[0], c[1], X[0], X[1]);
                 }
             }
         }
     }
+    return inexact;
+}
+
+template <Fmt F, int GS>
+BQ_DEVINL int int_table_item(const uint16_t* __restrict__ x, int M, int K, int m, int step, int t, int lane,
+                             bool valid, uint8_t* xt, uint8_t* ct)
+{
+    uint32_t raw[4];
+    int_item_load<F>(x, K, m, step, t, raw);
+    return int_table_item_raw<F, GS>(raw, M, m, step, t, lane, valid, xt, ct);
+}
+
+template <Fmt F, int GS>
+__global__ void __launch_bounds__(kSgPrepThreads)
+gemv_int_prep_kernel(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ tab, uint32_t c_off,
+                     uint32_t f_off)
+{
+    grid_dependency_wait();                             // x comes from the previous kernel
+    // Only now may the GEMV launch: every kernel before this one has completed
+    // and its writes are visible.
+    grid_dependents_launch();
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int nsteps = K / 32;
+    const int items = M * nsteps * 4;                   // a multiple of 32 (K is a multiple of 256)
+    const int idx = blockIdx.x * kSgPrepThreads + tid;
+    int inexact = 0;
+    if (idx - lane < items)                             // whole warps
+        inexact = int_table_item<F, GS>(x, M, K, (idx >> 2) / nsteps, (idx >> 2) % nsteps, idx & 3, lane, true, tab,
+                                        tab + c_off);
     inexact = __syncthreads_or(inexact);
     if (tid == 0) reinterpret_cast<uint32_t*>(tab + f_off)[blockIdx.x] = inexact ? 1u : 0u;
 }
@@ -387,27 +424,25 @@ BQ_DEVINL float stage_scale(const uint8_t* p)
 // One warp's K slice of one stage, integer route: xp is this lane's slice-table
 // entry of the slice's first step, cp its group-table
 // entry of the slice's first group; sc as in slice_mma.
-template <Fmt F, int GS, int NU>
-BQ_DEVINL void slice_int(float (&yv)[4], uint32_t ld, const uint8_t* sc, uint32_t pitch, const uint8_t* xp,
-                         const uint8_t* cp, int nu_rt)
+template <Fmt F, int GS, int NU, typename LdAddr, typename ScAddr>
+BQ_DEVINL void slice_int(float (&yv)[4], LdAddr ld, ScAddr sa, const uint8_t* xp, const uint8_t* cp, int nu_rt)
 {
     using T = SFmt<F>;
     constexpr int UPG = GS / T::E;                      // code units per group
     constexpr uint32_t kLo = 0x0F0F0F0Fu;
     constexpr bool kAffine = F != Fmt::Q4_0;
     const int nu = NU > 0 ? NU : nu_rt;
-    const uint8_t* sc8 = sc + 8 * pitch;
     if constexpr (T::E == 32 && UPG == 1) {
         // one group per unit (Q4_0, affine-4 with groups of 32): two per ldmatrix.x4
 #pragma unroll (NU > 0 ? NU / 2 : 2)
         for (int s = 0; s < nu / 2; ++s) {
             uint32_t w[4];                                      // (g, u) (g+8, u) (g, u+1) (g+8, u+1)
-            ldsm_x4(ld + (uint32_t)s * 32u, w[0], w[1], w[2], w[3]);
-            const uint32_t sg = lds32(sc + 4 * s), sg8 = lds32(sc8 + 4 * s);   // groups u, u + 1 of rows g, g + 8
+            ldsm_x4(ld(2 * s), w[0], w[1], w[2], w[3]);
+            const uint32_t sg = lds32(sa(0, 0, 2 * s)), sg8 = lds32(sa(1, 0, 2 * s));   // groups u, u + 1, rows g, g + 8
             [[maybe_unused]] uint32_t bg = 0u, bg8 = 0u;
             if constexpr (kAffine) {
-                bg = lds32(sc + 16 * pitch + 4 * s);
-                bg8 = lds32(sc8 + 16 * pitch + 4 * s);
+                bg = lds32(sa(0, 1, 2 * s));
+                bg8 = lds32(sa(1, 1, 2 * s));
             }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -453,7 +488,7 @@ BQ_DEVINL void slice_int(float (&yv)[4], uint32_t ld, const uint8_t* sc, uint32_
             for (int s = 0; s < UPG / 2; ++s) {
                 const int u = a * UPG + 2 * s;
                 uint32_t w[4];
-                ldsm_x4(ld + (uint32_t)u * 16u, w[0], w[1], w[2], w[3]);
+                ldsm_x4(ld(u), w[0], w[1], w[2], w[3]);
                 if constexpr (F == Fmt::AFF8) {
                     const uint2 b = *reinterpret_cast<const uint2*>(xp + (uint32_t)(u / 2) * kSgIntStepBytes);
                     mma_u8s8_16832(acc, w[0], w[1], w[2], w[3], b.x, b.y, acc[0], acc[1], acc[2], acc[3]);
@@ -468,8 +503,8 @@ BQ_DEVINL void slice_int(float (&yv)[4], uint32_t ld, const uint8_t* sc, uint32_
                 }
             }
             const uint4 ce = *reinterpret_cast<const uint4*>(cp + a * kSgIntCtabBytes);
-            const float dg = stage_scale<F>(sc + 2 * a), dg8 = stage_scale<F>(sc8 + 2 * a);
-            const float zg = stage_scale<F>(sc + 16 * pitch + 2 * a), zg8 = stage_scale<F>(sc8 + 16 * pitch + 2 * a);
+            const float dg = stage_scale<F>(sa(0, 0, a)), dg8 = stage_scale<F>(sa(1, 0, a));
+            const float zg = stage_scale<F>(sa(0, 1, a)), zg8 = stage_scale<F>(sa(1, 1, a));
             const float k0 = __uint_as_float(ce.x), k1 = __uint_as_float(ce.y);
             const float b0 = __uint_as_float(ce.z), b1 = __uint_as_float(ce.w);
             yv[0] = __fmaf_rn(dg * k0, (float)acc[0], __fmaf_rn(zg, b0, yv[0]));
@@ -618,10 +653,14 @@ gemv_stream_kernel(const __grid_constant__ SGemvParams p)
                             ((2 * (g_b - k0 / GS)) & 15);
         const uint8_t* xp = x_lane + (size_t)(u_b * E / 32) * kSgIntStepBytes;
         const uint8_t* cp = c_lane + (size_t)g_b * kSgIntCtabBytes;
+        const uint32_t ld0 = st + ld_lane;
+        auto ld = [ld0](int u) { return ld0 + (uint32_t)u * 16u; };       // padded rows: units 16 bytes apart
+        const uint32_t sp = p.scale_pitch;
+        auto sa = [sc, sp](int h, int z, int G) { return sc + (uint32_t)(8 * h + 16 * z) * sp + 2 * G; };
         if (SU > 0 && !(last && nchunks > 1))
-            slice_int<F, GS, SU>(yv, st + ld_lane, sc, p.scale_pitch, xp, cp, SU);
+            slice_int<F, GS, SU>(yv, ld, sa, xp, cp, SU);
         else
-            slice_int<F, GS, 0>(yv, st + ld_lane, sc, p.scale_pitch, xp, cp, sl.nu);
+            slice_int<F, GS, 0>(yv, ld, sa, xp, cp, sl.nu);
         if (last) {
             // the slice columns of token m: all four lanes of the quad (one
             // token), lanes t = 2m and 2m + 1 (two tokens)
@@ -660,6 +699,235 @@ gemv_stream_kernel(const __grid_constant__ SGemvParams p)
         float sum = 0.0f;
 #pragma unroll
         for (int w = 0; w < KW; ++w) sum += red[((tl2 * KW + w) * 16 + r) * p.red_cols + m];
+        p.y[mat][(int64_t)m * p.N[mat] + row] = (uint16_t)f32_to_bf16_bits(sum);
+    }
+}
+
+
+// ------------------------------------------------------------------ TMA-fed variant
+// The same integer core, fed by the tensor-memory accelerator: one producer
+// warp (one elected lane) issues, per 16-row tile and stage, one 3-D box of
+// codes and one 2-D box of scales (and biases) that complete on the stage's
+// mbarrier, so the warps that compute never stall on issuing copies.
+//
+// Codes are viewed as a 3-D tensor [chunk][row][128 bytes] (strides 128 and
+// row_bytes), and a stage's box [CH chunks][16 rows][128 bytes] lands with the
+// 128-byte swizzle: byte chunk j of 128-byte line L is stored at chunk
+// j ^ (L mod 8).  Line L = 16 c + r for row r of chunk c, so the 8 rows that
+// one ldmatrix reads fall in 8 distinct bank groups.  Scales (and biases) are
+// viewed the same way with 16-byte lines, [8-group unit][row][16 bytes], so the
+// rows of one unit are 16 bytes apart, again in distinct banks.  Each of the 8
+// compute warps owns units [CH w, CH w + CH) of the stage (16-byte code units,
+// 8 per chunk); CH is the stage's chunk count.
+//
+// No table kernel runs ahead of it: after griddepcontrol.wait the producer
+// starts the ring while each compute warp builds, in shared memory, the slices
+// and group entries of its own K slice of x (int_table_item, the prep kernel's
+// per-item work), which overlaps the first stages' flight.  A CTA that finds an
+// activation the slices do not hold exactly drains the ring and computes its
+// tiles with fp32 dot products (gemv_exact); every CTA sees the same x, so all
+// make the same choice.
+struct STmaParams {
+    SGemvParams g;                          // shapes, tables, outputs (ring fields unused)
+    CUtensorMap codes[kSgMaxMats];
+    CUtensorMap scales[kSgMaxMats];
+    CUtensorMap biases[kSgMaxMats];
+    uint32_t off_stage;                     // first stage (1024-byte aligned)
+    uint32_t stage_pitch;                   // bytes between stages (multiple of 1024)
+    uint32_t scale_row_bytes;               // one row's scales of a stage (a multiple of 16): 16 rows x this per box
+    uint32_t stage_tx;                      // bytes a stage's copies complete
+    uint32_t off_bar;                       // 2 S mbarriers: full[S], empty[S] (S <= kSgMaxStagesTma)
+};
+
+template <Fmt F, int GS, int CH>
+__global__ void __launch_bounds__(32 * (kSgWarpsTma + 1), 1)
+gemv_tma_kernel(const __grid_constant__ STmaParams q)
+{
+    using T = SFmt<F>;
+    constexpr int E = T::E;
+    constexpr int UPG = GS / E;
+    constexpr bool kAffine = F != Fmt::Q4_0;
+    constexpr int KW = kSgWarpsTma;
+    constexpr int NU = CH;                               // units per warp per stage
+    constexpr int kStageElems = CH * 128 * 8 / T::kBits;
+    constexpr int kStageGroups = kStageElems / GS;
+    static_assert(NU % (UPG > 2 ? UPG : 2) == 0, "a warp's units are whole atoms");
+    static_assert(CH == 8 || CH == 16, "every warp's units start on a 128-byte chunk");
+    const SGemvParams& p = q.g;
+
+    // the swizzle pattern is relative to 1024-byte blocks: everything below
+    // lives at offsets from a 1024-byte aligned base (1 KB extra is allocated)
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t sbase = smem_u32(smem);
+    const int M = p.M, S = p.stages, nchunks = p.nchunks;
+    const int t_begin = (int)((int64_t)blockIdx.x * p.ntiles / gridDim.x);
+    const int t_end = (int)((int64_t)(blockIdx.x + 1) * p.ntiles / gridDim.x);
+    const int nt = t_end - t_begin;
+    const int total = nt * nchunks;
+    auto full_bar = [&](int s) { return sbase + q.off_bar + 8u * (uint32_t)s; };
+    auto empty_bar = [&](int s) { return sbase + q.off_bar + 8u * (uint32_t)(S + s); };
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), KW);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+    grid_dependency_wait();
+    grid_dependents_launch();
+
+    if (warp == KW) {
+        // ---------------------------------------------------------- producer
+        int tile = t_begin, chunk = 0, mat = 0;
+        while (mat + 1 < p.count && tile >= p.tile_begin[mat + 1]) ++mat;
+        auto issue = [&](int i) {
+            const int s = i % S;
+            const uint32_t st = sbase + q.off_stage + (uint32_t)s * q.stage_pitch;
+            const int row0 = (tile - p.tile_begin[mat]) * 16;
+            mbar_arrive_expect_tx(full_bar(s), q.stage_tx);
+            tma_load_3d(st, &q.codes[mat], full_bar(s), 0, row0, chunk * CH);
+            const uint32_t sdst = st + (uint32_t)CH * 2048u;
+            tma_load_3d(sdst, &q.scales[mat], full_bar(s), 0, row0, chunk * (kStageGroups / 8));
+            if constexpr (kAffine)
+                tma_load_3d(sdst + 16u * q.scale_row_bytes, &q.biases[mat], full_bar(s), 0, row0,
+                            chunk * (kStageGroups / 8));
+            if (++chunk == nchunks) {
+                chunk = 0;
+                ++tile;
+                while (mat + 1 < p.count && tile >= p.tile_begin[mat + 1]) ++mat;
+            }
+        };
+        if (lane == 0)
+            for (int i = 0; i < total; ++i) {
+                if (i >= S && !mbar_wait(empty_bar(i % S), (uint32_t)((i / S) - 1) & 1u)) break;
+                issue(i);
+            }
+        return;
+    }
+
+    // ------------------------------------------------------------ activation tables
+    // This warp's K slice of x, in every chunk: steps [st0, st0 + nst), items
+    // (token, step, quad position) 32 at a time; a group's lanes are consecutive.
+    // The loads of up to four batches go out together, then their arithmetic.
+    int inexact = 0;
+    {
+        constexpr int nst = NU * E / 32;
+        constexpr int kB = 4;
+        const int items = M * nst * 4;                  // per chunk
+        const int bpc = (items + 31) / 32;              // batches per chunk
+        const int nb = nchunks * bpc;
+        for (int b0 = 0; b0 < nb; b0 += kB) {
+            uint32_t raw[kB][4];
+            int mm[kB], stp[kB], tt[kB];
+            bool ok[kB];
+#pragma unroll
+            for (int j = 0; j < kB; ++j) {
+                const int b = b0 + j;
+                const int c = b / bpc, idx = (b - c * bpc) * 32 + lane;
+                ok[j] = b < nb && idx < items;
+                const int ic = idx < items ? idx : items - 1;
+                mm[j] = (ic >> 2) / nst;
+                stp[j] = (c * kStageElems + warp * NU * E) / 32 + (ic >> 2) % nst;
+                tt[j] = ic & 3;
+                if (b < nb) int_item_load<F>(p.x, p.K, mm[j], stp[j], tt[j], raw[j]);
+            }
+#pragma unroll
+            for (int j = 0; j < kB; ++j)
+                if (b0 + j < nb)                        // warp-uniform
+                    inexact |= int_table_item_raw<F, GS>(raw[j], M, mm[j], stp[j], tt[j], lane, ok[j], smem + p.off_x,
+                                                         smem + p.off_c);
+        }
+    }
+    // the same answer in every compute warp (and every CTA: they all read the same x)
+    int any_inexact;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\t"
+                 "bar.red.or.pred q, 2, %2, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
+                 : "=r"(any_inexact) : "r"(inexact), "n"(32 * KW) : "memory");
+    if (any_inexact) {
+        // release every stage so the producer finishes, then the fp32 path
+        for (int i = 0; i < total; ++i) {
+            if (!mbar_wait_warp(full_bar(i % S), (uint32_t)(i / S) & 1u)) break;
+            if (lane == 0) mbar_arrive(empty_bar(i % S));
+        }
+        gemv_exact<F, GS>(p, t_begin, t_end, warp, lane, KW);
+        return;
+    }
+
+    // -------------------------------------------------------------- consumers
+    const int g = lane >> 2, t = lane & 3;
+    const uint8_t* x_lane = smem + p.off_x + (size_t)((g * 4 + t) * 8);     // slice column g
+    const uint8_t* c_lane = smem + p.off_c + (size_t)t * 16;
+    // ldmatrix.x4 rows: lanes 0-7 rows 0-7 of unit u, 8-15 rows 8-15 of u, 16-31 the same of u + 1
+    const int r = (lane & 7) + ((lane >> 3) & 1) * 8, hi = lane >> 4;
+    uint32_t swz[4];                                     // swizzled byte offset of unit 2j + hi in its chunk
+#pragma unroll
+    for (int j = 0; j < 4; ++j) swz[j] = (uint32_t)(((2 * j + hi) ^ (r & 7)) << 4);
+    const uint32_t lane_row = (uint32_t)r * 128u + (uint32_t)(warp * NU / 8) * 2048u;
+    float* red = reinterpret_cast<float*>(smem + p.off_red);
+    float yv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+
+    int tl = 0, chunk = 0;
+    for (int i = 0; i < total; ++i) {
+        const int s = i % S;
+        if (!mbar_wait_warp(full_bar(s), (uint32_t)(i / S) & 1u)) break;
+        if (chunk == 0) yv[0] = yv[1] = yv[2] = yv[3] = 0.0f;
+        const bool last = chunk == nchunks - 1;
+        const uint32_t st = sbase + q.off_stage + (uint32_t)s * q.stage_pitch;
+        const int u_b = chunk * (kStageElems / E) + warp * NU;            // first unit of the slice (in the row)
+        const int g_b = u_b / UPG;                                        // its first group
+        // scales: [8-group unit][16 rows][16 bytes], biases the same after them
+        const uint8_t* sbox = smem + (st - sbase) + (size_t)CH * 2048u + (size_t)g * 16u;
+        const int G0 = warp * NU / UPG;                 // the warp's first group of the stage
+        const uint32_t zb = 16u * q.scale_row_bytes;
+        auto sa = [sbox, G0, zb](int h, int z, int G) {
+            const int Ga = G0 + G;
+            return sbox + (uint32_t)z * zb + (uint32_t)h * 128u + (uint32_t)(Ga >> 3) * 256u + (uint32_t)(Ga & 7) * 2u;
+        };
+        const uint8_t* xp = x_lane + (size_t)(u_b * E / 32) * kSgIntStepBytes;
+        const uint8_t* cp = c_lane + (size_t)g_b * kSgIntCtabBytes;
+        const uint32_t ld0 = st + lane_row;
+        // unit pair starting at relative unit u (even): chunk u / 8, pair (u mod 8) / 2
+        auto ld = [&](int u) { return ld0 + (uint32_t)(u >> 3) * 2048u + swz[(u & 7) >> 1]; };
+        slice_int<F, GS, NU>(yv, ld, sa, xp, cp, NU);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));       // this warp is done with stage s
+        if (last) {
+            float rr = yv[0] + yv[1], r8 = yv[2] + yv[3];
+            rr += __shfl_xor_sync(0xFFFFFFFFu, rr, 1);
+            r8 += __shfl_xor_sync(0xFFFFFFFFu, r8, 1);
+            if (M == 1) {
+                rr += __shfl_xor_sync(0xFFFFFFFFu, rr, 2);
+                r8 += __shfl_xor_sync(0xFFFFFFFFu, r8, 2);
+            }
+            if ((t & 1) == 0 && (t >> 1) < M) {
+                float* rp = red + ((tl * KW + warp) * 16 + g) * p.red_cols + (t >> 1);
+                rp[0] = rr;
+                rp[8 * p.red_cols] = r8;
+            }
+        }
+        if (++chunk == nchunks) {
+            chunk = 0;
+            ++tl;
+        }
+    }
+
+    // ------------------------------------------------------------ cross-warp sum and store
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * KW) : "memory");   // the compute warps only
+    const int rows_cta = nt * 16;
+    for (int o = tid; o < M * rows_cta; o += 32 * KW) {
+        const int m = o / rows_cta, rl = o - m * rows_cta;
+        const int tl2 = rl >> 4, rw = rl & 15;
+        const int tile = t_begin + tl2;
+        int mat = 0;
+        while (mat + 1 < p.count && tile >= p.tile_begin[mat + 1]) ++mat;
+        const int64_t row = (int64_t)(tile - p.tile_begin[mat]) * 16 + rw;
+        if (row >= p.N[mat]) continue;
+        float sum = 0.0f;
+#pragma unroll
+        for (int w = 0; w < KW; ++w) sum += red[((tl2 * KW + w) * 16 + rw) * p.red_cols + m];
         p.y[mat][(int64_t)m * p.N[mat] + row] = (uint16_t)f32_to_bf16_bits(sum);
     }
 }

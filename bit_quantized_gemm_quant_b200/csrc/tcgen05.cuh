@@ -107,6 +107,23 @@ BQ_DEVINL void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, i
         ::"r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y) : "memory");
 }
 
+// 3D tiled load (no multicast) into this CTA's shared memory; completes bytes on `bar`.
+BQ_DEVINL void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int32_t x, int32_t y, int32_t z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y), "r"(z) : "memory");
+}
+
+// Untiled bulk copy global -> this CTA's shared memory (16-byte aligned, a
+// multiple of 16 bytes); completes bytes on `bar`.
+BQ_DEVINL void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 BQ_DEVINL void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
 {

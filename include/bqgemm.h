@@ -309,6 +309,19 @@ BQ_API bq_status quant_matmul_ex(const uint16_t* x_bf16, const void* wq, const v
  * other combination as affine. */
 BQ_API size_t quant_matmul_workspace_size(int64_t M, int64_t N, int64_t K, int group_size, int bits, int path);
 
+/* Which decode kernel quant_matmul_ex runs for this problem on path (AUTO: the
+ * dispatcher's choice) -- host only, for tools and benchmarks:
+ *   0 the register-streaming GEMV (gemv_kernel), one launch;
+ *   1 the streamed integer-MMA GEMV fed by the tensor-memory accelerator
+ *     (gemv_tma_kernel), one launch, no workspace;
+ *   2 the streamed integer-MMA GEMV fed by cp.async, after the kernel that builds
+ *     its activation tables (gemv_int_prep_kernel, gemv_stream_kernel), two
+ *     launches, the tables in workspace;
+ *   3 the any-width affine GEMV (2-, 3- and 6-bit), one launch;
+ *  -1 the path is not a decode path, or the arguments are invalid.
+ * A caller workspace smaller than quant_matmul_workspace_size turns 2 into 0. */
+BQ_API int quant_matmul_gemv_kernel(int64_t M, int64_t N, int64_t K, int group_size, int bits, int path);
+
 /*
  * quant_matmul_select_path -- the M-threshold dispatcher (host only, no CUDA
  * call).  After the size threshold asked for on the MLX issue page (Question:

@@ -222,21 +222,50 @@ def test_q8_path_validation(L):
 
 
 def test_decode_gemv_table_workspace(L):
-    """The streamed GEMV (one or two tokens) needs its activation tables: K/32 x
-    256 bytes of byte slices, K/group x 64 bytes of group scales and sums, a flag
-    word per 2048 activations rounded up to 16 bytes.  Forced (path 4) for every
-    format; through the GEMV path (1, and AUTO) only where it is the dispatcher's
-    choice, affine 8-bit; none from three tokens on."""
+    """The streamed GEMV (one or two tokens): the TMA-fed kernel, which applies when a
+    row's codes split into stages of 8 or 16 128-byte chunks, builds its activation
+    tables in shared memory and needs no workspace; the cp.async kernel, which takes
+    the other shapes, needs its tables in device scratch: K/32 x 256 bytes of byte
+    slices, K/group x 64 bytes of group scales and sums, a flag word per 2048
+    activations rounded up to 16 bytes.  Forced (path 4) for every format; through
+    the GEMV path (1, and AUTO) only where it is the dispatcher's choice (one token,
+    or two for the affine formats, K >= 4096 and 4 tiles per SM); none from three
+    tokens on."""
+    def tables(M, K, g):
+        flags = -(-M * K // 2048)
+        return K // 32 * 256 + K // g * 64 + (flags * 4 + 15) // 16 * 16
     for g, bits in ((32, 4), (64, 4), (64, 8), (128, 8), (32, 8), (128, 4)):
         for M in (1, 2):
-            for K in (4096, 2048 if g < 128 else 1024):
-                flags = -(-M * K // 2048)
-                want = K // 32 * 256 + K // g * 64 + (flags * 4 + 15) // 16 * 16
-                assert L.quant_matmul_workspace_size(M, 12288, K, g, bits, 4) == want, (g, bits, M, K)
-                via_gemv = want if bits == 8 else 0
-                assert L.quant_matmul_workspace_size(M, 12288, K, g, bits, 1) == via_gemv
-                assert L.quant_matmul_workspace_size(M, 12288, K, g, bits, 0) == via_gemv
-        assert L.quant_matmul_workspace_size(3, 12288, 4096, g, bits, 1) == 0
+            assert L.quant_matmul_workspace_size(M, 12288, 4096, g, bits, 4) == 0, (g, bits, M)   # TMA-fed
+            assert L.quant_matmul_workspace_size(M, 12288, 4096, g, bits, 1) == 0
         assert L.quant_matmul_workspace_size(3, 12288, 4096, g, bits, 4) == 0
+    for M in (1, 2):
+        # K = 768: 384- or 768-byte rows, not whole 8-chunk stages: the cp.async kernel
+        assert L.quant_matmul_workspace_size(M, 300, 768, 32, 4, 4) == tables(M, 768, 32)
+        assert L.quant_matmul_workspace_size(M, 300, 768, 32, 8, 4) == tables(M, 768, 32)
+        # not the dispatcher's choice here (K < 4096, 19 tiles): the register-streaming GEMV
+        assert L.quant_matmul_workspace_size(M, 300, 768, 32, 4, 1) == 0
+        assert L.quant_matmul_workspace_size(M, 300, 768, 32, 8, 1) == 0
     assert L.quant_matmul_workspace_size(1, 256, 544, 32, 4, 4) == 0      # K not a multiple of 8 blocks
     assert L.quant_matmul_workspace_size(1, 256, 512, 64, 3, 4) == 0      # 3-bit: no streamed kernel
+
+
+def test_decode_kernel_query(L):
+    """quant_matmul_gemv_kernel names the decode kernel that runs (host only; B200
+    shared memory assumed without a device): 1 = TMA-fed streamed, 2 = cp.async
+    streamed with its table kernel, 0 = register-streaming, 3 = any-width, -1 = none."""
+    q = L.quant_matmul_gemv_kernel
+    assert q(1, 12288, 4096, 32, 4, 0) == 1                # Q4_0, one token: streamed
+    assert q(2, 12288, 4096, 32, 4, 0) == 0                # Q4_0, two tokens: register-streaming
+    assert q(2, 12288, 4096, 64, 4, 0) == 1                # affine 4-bit, two tokens: streamed
+    assert q(2, 12288, 4096, 64, 8, 0) == 1
+    assert q(8, 12288, 4096, 64, 8, 0) == 0
+    assert q(2, 12288, 4096, 32, 4, 4) == 1                # forced
+    assert q(1, 300, 768, 32, 8, 4) == 2                   # 768-byte rows: the cp.async kernel
+    assert q(1, 300, 768, 32, 8, 0) == 0                   # small: the register-streaming kernel
+    assert q(1, 2048, 4096, 32, 4, 0) == 0                 # 128 tiles on 148 SMs
+    assert q(1, 8192, 2048, 32, 4, 0) == 0                 # K < 4096
+    assert q(3, 12288, 4096, 32, 4, 4) == -1               # forced beyond two tokens
+    assert q(1, 12288, 4096, 64, 3, 0) == 3                # 3-bit: any-width GEMV
+    assert q(64, 12288, 4096, 32, 4, 0) == -1              # prefill: not a decode path
+    assert q(0, 12288, 4096, 32, 4, 0) == -1
