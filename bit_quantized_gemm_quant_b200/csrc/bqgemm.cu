@@ -530,10 +530,9 @@ size_t stream_gemv_table_bytes(WFmt fmt, int group_size, int64_t M, int64_t K, i
 
 // BQ_PATH_GEMV takes the streamed kernel where it measured faster than the
 // register-streaming one on B200 (N = 12288, K = 4096, graph-timed launches
-// over rotating weight copies, TMA-fed variant): one token for every format
-// (Q4_0 10.98 against 12.58 us, affine 4-bit 10.66 / 13.26, affine 8-bit 12.89 /
-// 18.3), two tokens for the affine formats (12.18 / 13.38, 14.31 / 18.3); Q4_0 at
-// two tokens ties (12.58 / 12.61) and keeps the register-streaming kernel.
+// over rotating weight copies, TMA-fed variant): one token (Q4_0 10.85 against
+// 12.58 us, affine 4-bit 10.28 / 13.26, affine 8-bit 12.44 / 18.3) and two
+// (12.30 / 12.60, 11.74 / 13.38, 13.79 / 18.3).
 // It runs one CTA per SM and pays a fixed start per CTA (its activation slices,
 // the ring's fill), so it needs several 16-row tiles per SM: with the Llama-3.2-1B
 // stack's matrices (32 to 1024 tiles, K = 2048 or 8192) one token took 549 against
@@ -541,8 +540,9 @@ size_t stream_gemv_table_bytes(WFmt fmt, int group_size, int64_t M, int64_t K, i
 // least 4 tiles per SM.
 bool stream_gemv_preferred(WFmt fmt, int64_t M, int64_t ntiles, int64_t K, int num_sms)
 {
+    (void)fmt;
     if (K < 4096 || ntiles < 4 * (int64_t)num_sms) return false;
-    return M == 1 || (M == 2 && fmt != WFmt::Q4_0);
+    return M <= kSgIntTokens;
 }
 
 bool plan_stream_gemv(WFmt fmt, int group_size, int64_t M, const SgMats& mats, int64_t K, const DeviceInfo& di,
@@ -701,7 +701,7 @@ struct SgTmaPlan {
 struct SgTmaShape {
     int ch = 0, stages = 0, nchunks = 0, grid = 0;
     int64_t stage_elems = 0, stage_groups = 0, scale_row = 0, stage_pitch = 0;
-    int64_t off_x = 0, off_c = 0, off_red = 0, off_bar = 0, off_stage = 0, smem = 0;
+    int64_t off_x = 0, off_c = 0, off_red = 0, off_bar = 0, off_raw = 0, off_stage = 0, smem = 0;
 };
 
 bool tma_shape(WFmt fmt, int group_size, int64_t M, int64_t ntiles, int64_t K, int num_sms, int smem_optin,
@@ -736,7 +736,9 @@ bool tma_shape(WFmt fmt, int group_size, int64_t M, int64_t ntiles, int64_t K, i
     h.off_red = off;
     off = up(off + tcap * kSgWarpsTma * 16 * M * 4, 128);           // one column per token
     h.off_bar = off;
-    off = up(off + (2 * kSgMaxStagesTma + 1) * 8, 1024);
+    off = up(off + (2 * kSgMaxStagesTma + 1) * 8, 128);
+    h.off_raw = off;                                                 // x itself, bf16 [M][K]
+    off = up(off + M * K * 2, 1024);
     h.off_stage = off;
     const int64_t budget = (int64_t)smem_optin - 1024;               // 1 KB to align the base
     // as many stages as fit, up to 4 (5 measured slower for the 4-bit formats: 13.2
@@ -798,6 +800,7 @@ bool plan_stream_gemv_tma(WFmt fmt, int group_size, int64_t M, const SgMats& mat
     p.off_c = (uint32_t)h.off_c;
     p.off_red = (uint32_t)h.off_red;
     q.off_stage = (uint32_t)h.off_stage;
+    q.off_raw = (uint32_t)h.off_raw;
     q.stage_pitch = (uint32_t)h.stage_pitch;
     q.scale_row_bytes = (uint32_t)h.scale_row;
     q.stage_tx = (uint32_t)(ch * 2048 + 16 * h.scale_row * (affine ? 2 : 1));

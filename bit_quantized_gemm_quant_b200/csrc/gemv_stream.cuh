@@ -736,7 +736,8 @@ struct STmaParams {
     uint32_t stage_pitch;                   // bytes between stages (multiple of 1024)
     uint32_t scale_row_bytes;               // one row's scales of a stage (a multiple of 16): 16 rows x this per box
     uint32_t stage_tx;                      // bytes a stage's copies complete
-    uint32_t off_bar;                       // 2 S mbarriers: full[S], empty[S] (S <= kSgMaxStagesTma)
+    uint32_t off_bar;                       // 2 S + 1 mbarriers: full[S], empty[S], x (S <= kSgMaxStagesTma)
+    uint32_t off_raw;                       // x, bf16 [M][K], copied in before the first stage
 };
 
 template <Fmt F, int GS, int CH>
@@ -768,11 +769,13 @@ gemv_tma_kernel(const __grid_constant__ STmaParams q)
     const int total = nt * nchunks;
     auto full_bar = [&](int s) { return sbase + q.off_bar + 8u * (uint32_t)s; };
     auto empty_bar = [&](int s) { return sbase + q.off_bar + 8u * (uint32_t)(S + s); };
+    const uint32_t x_bar = sbase + q.off_bar + 16u * (uint32_t)S;
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), KW);
         }
+        mbar_init(x_bar, 1);
         fence_barrier_init();
     }
     __syncthreads();
@@ -800,19 +803,27 @@ gemv_tma_kernel(const __grid_constant__ STmaParams q)
                 while (mat + 1 < p.count && tile >= p.tile_begin[mat + 1]) ++mat;
             }
         };
-        if (lane == 0)
+        if (lane == 0) {
+            // x first, so that it is ahead of the weights in the copy engine's queue
+            const uint32_t xbytes = (uint32_t)(M * p.K * 2);
+            mbar_arrive_expect_tx(x_bar, xbytes);
+            bulk_load(sbase + q.off_raw, p.x, xbytes, x_bar);
             for (int i = 0; i < total; ++i) {
                 if (i >= S && !mbar_wait(empty_bar(i % S), (uint32_t)((i / S) - 1) & 1u)) break;
                 issue(i);
             }
+        }
         return;
     }
 
     // ------------------------------------------------------------ activation tables
     // This warp's K slice of x, in every chunk: steps [st0, st0 + nst), items
     // (token, step, quad position) 32 at a time; a group's lanes are consecutive.
-    // The loads of up to four batches go out together, then their arithmetic.
+    // The loads of up to four batches go out together, then their arithmetic; x
+    // comes from this CTA's shared-memory copy.
     int inexact = 0;
+    if (!mbar_wait_warp(x_bar, 0u)) inexact = 1;         // timed out (device error set): the fp32 path
+    const uint16_t* xs = reinterpret_cast<const uint16_t*>(smem + q.off_raw);
     {
         constexpr int nst = NU * E / 32;
         constexpr int kB = 4;
@@ -832,7 +843,7 @@ gemv_tma_kernel(const __grid_constant__ STmaParams q)
                 mm[j] = (ic >> 2) / nst;
                 stp[j] = (c * kStageElems + warp * NU * E) / 32 + (ic >> 2) % nst;
                 tt[j] = ic & 3;
-                if (b < nb) int_item_load<F>(p.x, p.K, mm[j], stp[j], tt[j], raw[j]);
+                if (b < nb) int_item_load<F>(xs, p.K, mm[j], stp[j], tt[j], raw[j]);
             }
 #pragma unroll
             for (int j = 0; j < kB; ++j)

@@ -228,9 +228,8 @@ def test_decode_gemv_table_workspace(L):
     the other shapes, needs its tables in device scratch: K/32 x 256 bytes of byte
     slices, K/group x 64 bytes of group scales and sums, a flag word per 2048
     activations rounded up to 16 bytes.  Forced (path 4) for every format; through
-    the GEMV path (1, and AUTO) only where it is the dispatcher's choice (one token,
-    or two for the affine formats, K >= 4096 and 4 tiles per SM); none from three
-    tokens on."""
+    the GEMV path (1, and AUTO) only where it is the dispatcher's choice (one or two
+    tokens, K >= 4096 and 4 tiles per SM); none from three tokens on."""
     def tables(M, K, g):
         flags = -(-M * K // 2048)
         return K // 32 * 256 + K // g * 64 + (flags * 4 + 15) // 16 * 16
@@ -256,7 +255,7 @@ def test_decode_kernel_query(L):
     streamed with its table kernel, 0 = register-streaming, 3 = any-width, -1 = none."""
     q = L.quant_matmul_gemv_kernel
     assert q(1, 12288, 4096, 32, 4, 0) == 1                # Q4_0, one token: streamed
-    assert q(2, 12288, 4096, 32, 4, 0) == 0                # Q4_0, two tokens: register-streaming
+    assert q(2, 12288, 4096, 32, 4, 0) == 1                # Q4_0, two tokens: streamed
     assert q(2, 12288, 4096, 64, 4, 0) == 1                # affine 4-bit, two tokens: streamed
     assert q(2, 12288, 4096, 64, 8, 0) == 1
     assert q(8, 12288, 4096, 64, 8, 0) == 0
