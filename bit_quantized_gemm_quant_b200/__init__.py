@@ -108,13 +108,45 @@ def _bits16(t: torch.Tensor) -> torch.Tensor:
     return t
 
 
+BF16 = (torch.bfloat16, torch.int16, torch.uint16)      # bf16 values or their bit patterns
+BITS16 = (torch.bfloat16, torch.float16, torch.int16, torch.uint16)
+U8 = (torch.uint8, torch.int8)
+U32 = (torch.int32, torch.uint32)
+
+
+def _arg(t: torch.Tensor | None, dtypes, elems: int, name: str):
+    """The pointer of `t` after checking its type and that it holds at least `elems`
+    elements: the library reads and writes by the sizes it is given, so a tensor of
+    the wrong type or too small would be read or written out of bounds."""
+    if t is None:
+        return None
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: expected one of {[str(d) for d in dtypes]}, got {t.dtype}")
+    if t.numel() < elems:
+        raise ValueError(f"{name}: {t.numel()} elements, the call needs {elems}")
+    return _ptr(t)
+
+
+def _weights_args(wq, scales, biases, N: int, K: int, group_size: int, bits: int, transpose: bool, i=""):
+    """Checked pointers of one quantized matrix: Q4_0 (biases None) u8 codes [N][K/2]
+    with 16-bit scales [N][K/32]; affine u32 codes with bf16 scales and biases,
+    [N][K bits/32] and [N][K/group] (transpose), else [K][N bits/32] and [K][N/group]."""
+    if biases is None:
+        return (_arg(wq, U8, N * (K // 2), f"wq{i}"), _arg(scales, BITS16, N * (K // 32), f"scales{i}"), None)
+    g = max(group_size, 1)
+    ng = N * (K // g) if transpose else K * (N // g)
+    return (_arg(wq, U32, N * K * bits // 32, f"wq{i}"), _arg(scales, BITS16, ng, f"scales{i}"),
+            _arg(biases, BITS16, ng, f"biases{i}"))
+
+
 # ----------------------------------------------------------------- dequantize
 def q4_0_dequantize(wq: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None, stream=None):
     """wq u8 [N][K/2], scales fp16 [N][K/32] -> bf16 [N][K]."""
     N, K = wq.shape[0], wq.shape[1] * 2
     if out is None:
         out = torch.empty(N, K, dtype=torch.bfloat16, device=wq.device)
-    _check(lib().q4_0_dequantize(_ptr(wq), _ptr(_bits16(scales)), _ptr(out), N, K, _stream(stream)),
+    _check(lib().q4_0_dequantize(_arg(wq, U8, N * K // 2, "wq"), _arg(scales, BITS16, N * (K // 32), "scales"),
+                                 _arg(out, BF16, N * K, "out"), N, K, _stream(stream)),
            "q4_0_dequantize")
     return out
 
@@ -137,7 +169,9 @@ def affine_dequantize(wq: torch.Tensor, scales: torch.Tensor, biases: torch.Tens
     N, K = wq.shape[0], wq.shape[1] * 32 // bits
     if out is None:
         out = torch.empty(N, K, dtype=torch.bfloat16, device=wq.device)
-    _check(lib().affine_dequantize(_ptr(wq), _ptr(_bits16(scales)), _ptr(_bits16(biases)), _ptr(out), N, K,
+    ng = N * (K // max(group_size, 1))
+    _check(lib().affine_dequantize(_arg(wq, U32, N * K * bits // 32, "wq"), _arg(scales, BITS16, ng, "scales"),
+                                   _arg(biases, BITS16, ng, "biases"), _arg(out, BF16, N * K, "out"), N, K,
                                    group_size, bits, _stream(stream)), "affine_dequantize")
     return out
 
@@ -176,12 +210,14 @@ def quant_matmul_ex(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, bia
     p = PATHS[path] if isinstance(path, str) else int(path)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     fn = lib().quant_matmul_ex if (p != PATH_AUTO or workspace is not None) else None
+    xp, yp = _arg(x, BF16, M * K, "x"), _arg(out, BF16, M * N, "out")
+    wp, sp, bp = _weights_args(wq, scales, biases, N, K, group_size, bits, transpose)
     if fn is None:
-        st = lib().quant_matmul(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(out), M, N, K, group_size, bits,
-                                1 if transpose else 0, _stream(stream))
+        st = lib().quant_matmul(xp, wp, sp, bp, yp, M, N, K, group_size, bits, 1 if transpose else 0,
+                                _stream(stream))
     else:
-        st = fn(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(out), M, N, K, group_size, bits,
-                1 if transpose else 0, p, _ptr(workspace), ws_bytes, _stream(stream))
+        st = fn(xp, wp, sp, bp, yp, M, N, K, group_size, bits, 1 if transpose else 0, p, _ptr(workspace), ws_bytes,
+                _stream(stream))
     _check(st, "quant_matmul")
     return out
 
@@ -202,12 +238,14 @@ def quant_matmul_multi(x: torch.Tensor, weights, group_size: int = 32, bits: int
     if outs is None:
         outs = [torch.empty(M, n, dtype=torch.bfloat16, device=x.device) for n in Ns]
     VP = ctypes.c_void_p * max(count, 1)
-    wq_a = VP(*[_ptr(wq) for wq, _, _ in weights])
-    s_a = VP(*[_ptr(_bits16(sc)) for _, sc, _ in weights])
-    b_a = None if q4 else VP(*[_ptr(_bits16(b)) for _, _, b in weights])
-    y_a = VP(*[_ptr(y) for y in outs])
+    args = [_weights_args(wq, sc, b, n, K, group_size, bits, True, f"[{i}]")
+            for i, ((wq, sc, b), n) in enumerate(zip(weights, Ns))]
+    wq_a = VP(*[a[0] for a in args])
+    s_a = VP(*[a[1] for a in args])
+    b_a = None if q4 else VP(*[a[2] for a in args])
+    y_a = VP(*[_arg(y, BF16, M * n, f"outs[{i}]") for i, (y, n) in enumerate(zip(outs, Ns))])
     n_a = (ctypes.c_int64 * max(count, 1))(*Ns)
-    _check(lib().quant_matmul_multi(_ptr(x), count, wq_a, s_a, b_a, y_a, n_a, M, K, group_size, bits,
+    _check(lib().quant_matmul_multi(_arg(x, BF16, M * K, "x"), count, wq_a, s_a, b_a, y_a, n_a, M, K, group_size, bits,
                                     1 if transpose else 0, _stream(stream)), "quant_matmul_multi")
     return outs
 
@@ -218,7 +256,7 @@ def q8_1_quantize(x: torch.Tensor, stream=None):
     xq = torch.empty(M, K, dtype=torch.int8, device=x.device)
     dx = torch.empty(M, K // 32, dtype=torch.float32, device=x.device)
     qs = torch.empty(M, K // 32, dtype=torch.int32, device=x.device)
-    _check(lib().q8_1_quantize(_ptr(x), _ptr(xq), _ptr(dx), _ptr(qs), M, K, _stream(stream)), "q8_1_quantize")
+    _check(lib().q8_1_quantize(_arg(x, BF16, M * K, "x"), _ptr(xq), _ptr(dx), _ptr(qs), M, K, _stream(stream)), "q8_1_quantize")
     return xq, dx, qs
 
 
@@ -231,7 +269,9 @@ def quant_matmul_q8(xq: torch.Tensor, dx: torch.Tensor, qsum: torch.Tensor, wq: 
         raise ValueError("K mismatch between activations and weights")
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=xq.device)
-    _check(lib().quant_matmul_q8(_ptr(xq), _ptr(dx), _ptr(qsum), _ptr(wq), _ptr(_bits16(scales)), _ptr(out), M, N,
+    _check(lib().quant_matmul_q8(_arg(xq, (torch.int8,), M * K, "xq"), _arg(dx, (torch.float32,), M * (K // 32), "dx"),
+                                 _arg(qsum, (torch.int32,), M * (K // 32), "qsum"), _arg(wq, U8, N * K // 2, "wq"),
+                                 _arg(scales, BITS16, N * (K // 32), "scales"), _arg(out, BF16, M * N, "out"), M, N,
                                  K, _stream(stream)), "quant_matmul_q8")
     return out
 
@@ -250,8 +290,8 @@ def quant_matmul_noalloc(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor
         raise ValueError(f"K mismatch: x has {K}, weights hold {Kw}")
     if tuple(out.shape) != (M, N) or out.dtype != torch.bfloat16:
         raise ValueError("out must be a bf16 tensor of shape [M][N]")
-    _check(lib().quant_matmul_noalloc(_ptr(x), _ptr(wq), _ptr(_bits16(scales)),
-                                      None if biases is None else _ptr(_bits16(biases)), _ptr(out), M, N, K,
+    wp, sp, bp = _weights_args(wq, scales, biases, N, K, group_size, bits, transpose)
+    _check(lib().quant_matmul_noalloc(_arg(x, BF16, M * K, "x"), wp, sp, bp, _arg(out, BF16, M * N, "out"), M, N, K,
                                       group_size, bits, 1 if transpose else 0, _stream(stream)),
            "quant_matmul_noalloc")
     return out
@@ -282,7 +322,8 @@ def bf16_matmul(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = Non
     N = w.shape[0]
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
-    _check(lib().bf16_matmul(_ptr(x), _ptr(w), _ptr(out), M, N, K, _stream(stream)), "bf16_matmul")
+    _check(lib().bf16_matmul(_arg(x, BF16, M * K, "x"), _arg(w, BF16, N * K, "w"), _arg(out, BF16, M * N, "out"),
+                             M, N, K, _stream(stream)), "bf16_matmul")
     return out
 
 
@@ -292,7 +333,8 @@ def q4_0_quantize(w: torch.Tensor, stream=None):
     N, K = w.shape
     wq = torch.empty(N, K // 2, dtype=torch.uint8, device=w.device)
     d = torch.empty(N, K // 32, dtype=torch.float16, device=w.device)
-    _check(lib().q4_0_quantize(_ptr(w), _ptr(wq), _ptr(d), N, K, _stream(stream)), "q4_0_quantize")
+    _check(lib().q4_0_quantize(_arg(w, (torch.float32,), N * K, "w"), _ptr(wq), _ptr(d), N, K, _stream(stream)),
+           "q4_0_quantize")
     return wq, d
 
 
@@ -302,7 +344,8 @@ def affine_quantize(w: torch.Tensor, group_size: int = 64, bits: int = 4, stream
     wq = torch.empty(N, K * bits // 32, dtype=torch.int32, device=w.device)
     s = torch.empty(N, K // group_size, dtype=torch.bfloat16, device=w.device)
     b = torch.empty(N, K // group_size, dtype=torch.bfloat16, device=w.device)
-    _check(lib().affine_quantize(_ptr(w), _ptr(wq), _ptr(s), _ptr(b), N, K, group_size, bits, _stream(stream)),
+    _check(lib().affine_quantize(_arg(w, (torch.float32,), N * K, "w"), _ptr(wq), _ptr(s), _ptr(b), N, K, group_size,
+                                 bits, _stream(stream)),
            "affine_quantize")
     return wq, s, b
 

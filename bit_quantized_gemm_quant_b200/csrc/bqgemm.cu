@@ -927,6 +927,80 @@ bq_status launch_gemv_affine(WFmt fmt, const uint16_t* x, const void* wq, const 
     return launch_status();
 }
 
+// Decode GEMV over [K][N] affine weights (transpose = 0), 2-, 4- or 8-bit: up to
+// kGtMaxM tokens when forced, up to kGtAutoMaxM when the dispatcher chooses (the
+// measured crossover with the unfused pair on B200: the GEMV is ahead at 1 to 4
+// tokens, behind at 8).
+constexpr int64_t kGtMaxM = 8;
+constexpr int64_t kGtAutoMaxM = 4;
+
+// CTAs per cluster along K: as many as fit on the GPU at once beside the other
+// clusters (one wave), at most 8, with at least 32 rows of K per CTA.
+int gemv_t_split(int64_t N, int64_t K, int cols, int resident)
+{
+    const int64_t ncb = (N + cols - 1) / cols;
+    int64_t ks = std::min<int64_t>(kGtMaxSplit, std::max<int64_t>(1, (int64_t)resident / ncb));
+    while (ks > 1 && K < 32 * ks) --ks;
+    return (int)ks;
+}
+
+template <int BITS, int MT>
+bq_status launch_gemv_t_cfg(const uint16_t* x, const uint32_t* w, const uint16_t* s, const uint16_t* b, uint16_t* y,
+                            int64_t M, int64_t N, int64_t K, int group_size, const DeviceInfo& di, cudaStream_t st)
+{
+    constexpr int U = MT == 1 && BITS != 8 ? 8 : 4;   // rows per batch (two batches in registers)
+    constexpr int cols = 32 * gemv_t_cpl<MT>();
+    auto kern = gemv_t_kernel<BITS, MT, U, 2>;
+    static int per_sm = 0;                    // resident CTAs per SM (the same on every B200)
+    if (per_sm == 0) {
+        int v = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kern, 32 * kGtWarps, 0) != cudaSuccess) {
+            cudaGetLastError();
+            v = 1;
+        }
+        per_sm = std::max(v, 1);
+    }
+    const int ks = gemv_t_split(N, K, cols, per_sm * di.num_sms);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((N + cols - 1) / cols), (unsigned)ks);
+    cfg.blockDim = dim3(32 * kGtWarps);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = (unsigned)ks;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, x, w, s, b, y, (int)M, (int)N, (int)K, group_size) != cudaSuccess) {
+        cudaGetLastError();
+        return BQ_ERR_CUDA;
+    }
+    return launch_status();
+}
+
+bq_status launch_gemv_t(WFmt fmt, const uint16_t* x, const void* wq, const uint16_t* s, const uint16_t* b,
+                        uint16_t* y, int64_t M, int64_t N, int64_t K, int group_size, const DeviceInfo& di,
+                        cudaStream_t st)
+{
+    if (N > INT32_MAX || K > INT32_MAX || M > kGtMaxM) return BQ_ERR_SHAPE;
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(wq);
+    auto by_m = [&](auto bits_tag) {
+        constexpr int B = decltype(bits_tag)::value;
+        if (M <= 1) return launch_gemv_t_cfg<B, 1>(x, w, s, b, y, M, N, K, group_size, di, st);
+        if (M <= 2) return launch_gemv_t_cfg<B, 2>(x, w, s, b, y, M, N, K, group_size, di, st);
+        if (M <= 4) return launch_gemv_t_cfg<B, 4>(x, w, s, b, y, M, N, K, group_size, di, st);
+        return launch_gemv_t_cfg<B, 8>(x, w, s, b, y, M, N, K, group_size, di, st);
+    };
+    switch (fmt) {
+    case WFmt::AFF2: return by_m(std::integral_constant<int, 2>());
+    case WFmt::AFF4: return by_m(std::integral_constant<int, 4>());
+    case WFmt::AFF8: return by_m(std::integral_constant<int, 8>());
+    default: return BQ_ERR_UNSUPPORTED;
+    }
+}
+
 template <Fmt F, int NT, int RT, int KS, int PIPE, int MINB>
 bq_status launch_gemv_multi_cfg(const uint16_t* x, GemvMultiTable& tab, int64_t M, int64_t K, int group_size,
                                 cudaStream_t st)
@@ -1079,18 +1153,27 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
     if (path < BQ_PATH_AUTO || path > BQ_PATH_GEMV_STREAM) return BQ_ERR_UNSUPPORTED;
     if (M < 0 || N < 0 || K < 0) return BQ_ERR_SHAPE;
     // transpose = 0: y = x . W with W stored [K][N], codes and groups along N
-    // (affine only: Q4_0 blocks run along K); it runs as the unfused pair with
-    // a transposing dequantize, and x's rows must be 16-byte multiples.
+    // (affine only: Q4_0 blocks run along K).  Up to kGtAutoMaxM tokens of 2-, 4-
+    // or 8-bit codes (kGtMaxM when forced) run the decode GEMV over [K][N]
+    // (gemv_t_kernel); otherwise the unfused pair with a transposing dequantize,
+    // whose x rows must be 16-byte multiples.
     if (transpose == 0 && !biases) return BQ_ERR_UNSUPPORTED;
     WFmt fmt;
     bq_status s = transpose ? check_format(biases, N, K, group_size, bits, &fmt)
                             : check_format(biases, K, N, group_size, bits, &fmt);
     if (s != BQ_OK) return s;
+    bool gemv_t = false;
     if (transpose == 0) {
-        if (path == BQ_PATH_GEMV || path == BQ_PATH_TC_FUSED || path == BQ_PATH_GEMV_STREAM)
+        const bool gt_fmt = bits == 2 || bits == 4 || bits == 8;
+        if (path == BQ_PATH_TC_FUSED || path == BQ_PATH_GEMV_STREAM || (path == BQ_PATH_GEMV && !(gt_fmt && M <= kGtMaxM)))
             return BQ_ERR_UNSUPPORTED;
-        if (K % 8 != 0) return BQ_ERR_SHAPE;
-        path = BQ_PATH_DEQUANT_GEMM;
+        if (path == BQ_PATH_GEMV || (path == BQ_PATH_AUTO && gt_fmt && M <= kGtAutoMaxM)) {
+            gemv_t = true;
+            path = BQ_PATH_GEMV;
+        } else {
+            if (K % 8 != 0) return BQ_ERR_SHAPE;
+            path = BQ_PATH_DEQUANT_GEMM;
+        }
     }
     if (M == 0 || N == 0) return BQ_OK;      // empty problem: nothing is read or written
     int dev;
@@ -1118,6 +1201,7 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
 
     const uint16_t* sc = reinterpret_cast<const uint16_t*>(scales);
     const uint16_t* bi = reinterpret_cast<const uint16_t*>(biases);
+    if (gemv_t) return launch_gemv_t(fmt, x, wq, sc, bi, y, M, N, K, group_size, di, st);
     switch (path) {
     case BQ_PATH_GEMV_STREAM:
         if (!has_fast_paths(fmt) || stream_gemv_table_bytes(fmt, group_size, M, K) == 0) return BQ_ERR_UNSUPPORTED;
@@ -1327,7 +1411,8 @@ bq_status quant_matmul_noalloc(const uint16_t* x_bf16, const void* wq, const voi
     // quant_matmul's own path, with the fixed array as its scratch: the decode
     // GEMV needs none, the fused kernel keeps its K-split partial sums there (or
     // runs unsplit if they do not fit), the unfused pair stages W there.
-    const int path = transpose ? select_path(M, K, fmt) : BQ_PATH_DEQUANT_GEMM;
+    const bool gemv_t = transpose == 0 && M <= kGtAutoMaxM && (bits == 2 || bits == 4 || bits == 8);
+    const int path = transpose ? select_path(M, K, fmt) : gemv_t ? BQ_PATH_GEMV : BQ_PATH_DEQUANT_GEMM;
     if (path == BQ_PATH_DEQUANT_GEMM && (uint64_t)N > (uint64_t)(BQ_NOALLOC_SCRATCH_BYTES / 2u) / (uint64_t)K)
         return BQ_ERR_WORKSPACE;
     int dev;

@@ -192,14 +192,18 @@ BQ_API bq_status quant_matmul_q8(const int8_t* xq, const float* dx, const int32_
  *            BQ_ERR_UNSUPPORTED): y = x . W with W stored [K][N], codes and
  *            groups along N -- wq u32 [K][N*bits/32], scales/biases bf16
  *            [K][N/group_size], N % group_size == 0 -- the transpose=False form
- *            of mx.quantized_matmul; it always runs as the unfused pair, W
- *            dequantized into its [N][K] transpose, and needs K % 8 == 0
- *            (BQ_ERR_SHAPE otherwise).  Other values: BQ_ERR_UNSUPPORTED.
+ *            of mx.quantized_matmul.  Up to 4 tokens of 2-, 4- or 8-bit codes
+ *            run a decode GEMV over the [K][N] layout (any K; a cluster of up
+ *            to 8 CTAs splits K and sums its partials in a fixed order; up to
+ *            8 tokens when BQ_PATH_GEMV is forced); other sizes run the
+ *            unfused pair, W dequantized into its [N][K] transpose, which
+ *            needs K % 8 == 0 (BQ_ERR_SHAPE otherwise).
+ *            Other values: BQ_ERR_UNSUPPORTED.
  * Affine 2-, 3- and 6-bit weights have a decode GEMV up to 8 tokens (over the
  * exact weights scale*q + bias, within the GEMM tolerance of their bf16
- * roundings) and run as the unfused pair above that; transpose = 0 runs as the
- * pair at every M; 4- and 8-bit and Q4_0 have the decode GEMV and the fused
- * kernel as well.
+ * roundings) and run as the unfused pair above that; 4- and 8-bit and Q4_0 have
+ * the decode GEMV and the fused kernel as well.  With transpose = 0 only the
+ * GEMV over [K][N] (see transpose) and the pair exist.
  * The path is chosen by quant_matmul_select_path.  A path that needs scratch
  * memory (the unfused pair's bf16 copy of W, the fused kernel's split-K
  * partial sums, the decode GEMV's activation tables for one or two tokens)
@@ -287,8 +291,9 @@ BQ_API bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const voi
  * decode GEMV of one or two tokens given a smaller workspace runs the
  * register-streaming GEMV of three and more tokens instead (same tolerance).  Forcing
  * BQ_PATH_GEMV with M > 32 (M > 8 for 2-, 3- or 6-bit weights), BQ_PATH_TC_FUSED
- * for 2-, 3- or 6-bit weights, or either with transpose = 0, returns
- * BQ_ERR_UNSUPPORTED.
+ * for 2-, 3- or 6-bit weights, BQ_PATH_TC_FUSED or BQ_PATH_GEMV_STREAM with
+ * transpose = 0, or BQ_PATH_GEMV with transpose = 0 beyond 8 tokens or for 3-
+ * or 6-bit codes, returns BQ_ERR_UNSUPPORTED.
  */
 BQ_API bq_status quant_matmul_ex(const uint16_t* x_bf16, const void* wq, const void* scales, const void* biases,
                           uint16_t* y_bf16, int64_t M, int64_t N, int64_t K, int group_size, int bits,

@@ -75,9 +75,13 @@ def test_quant_matmul_rejects_before_launch(L):
     assert qmm(L, b=ALIGNED, g=64, bits=3, path=1) == 3       # 2/3/6-bit: GEMV to M = 8, then the pair
     assert qmm(L, b=ALIGNED, g=64, bits=6, M=64, path=2) == 3
     assert qmm(L, b=ALIGNED, g=64, bits=2, M=64, path=2) == 3
-    assert qmm(L, b=ALIGNED, g=64, tr=0, path=1) == 3         # transpose=0: the pair only
+    assert qmm(L, b=ALIGNED, g=64, tr=0, path=1) == 3         # transpose=0: GEMV to M = 8, then the pair
+    assert qmm(L, b=ALIGNED, g=64, tr=0, M=4, bits=3, path=1) == 3  # ... for 2-, 4- and 8-bit codes
+    assert qmm(L, b=ALIGNED, g=64, tr=0, M=4, path=2) == 3
+    assert qmm(L, b=ALIGNED, g=64, tr=0, M=1, path=4) == 3
     assert qmm(L, b=ALIGNED, g=64, tr=0, M=64, path=2) == 3
-    assert qmm(L, b=ALIGNED, g=64, tr=0, K=12) == 2           # transpose=0 needs K % 8 == 0
+    assert qmm(L, b=ALIGNED, g=64, tr=0, K=12) == 2           # the pair needs K % 8 == 0
+    assert qmm(L, b=ALIGNED, g=64, tr=0, M=4, bits=3, K=12) == 2
     assert qmm(L, b=ALIGNED, g=64, tr=0, N=96) == 2           # ... and groups along N
     assert qmm(L, b=ALIGNED, g=64, bits=4, K=96) == 2         # K % group
     assert qmm(L, x=None) == 1

@@ -435,3 +435,53 @@ def test_2_3_6_bit_and_transpose0_edges():
         sep = bq.quant_matmul(x, wq, s, b, 64, 3)
         torch.cuda.synchronize()
         assert torch.equal(o.view(torch.int16), sep.view(torch.int16))
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("G", [32, 64, 128])
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("K", [100, 300, 1000])
+def test_transpose0_decode_gemv(bits, G, M, K):
+    """transpose = 0 at decode sizes with 2-, 4- or 8-bit codes: the GEMV over
+    [K][N] (any K, split over a cluster of 3 CTAs at K = 100 and up to 8 at K = 300
+    and 1000, ragged per-CTA ranges; N a multiple of the group, ragged against the
+    256- and 512-column clusters) is the dispatcher's choice up to 4 tokens (auto
+    and forced give the same bits) and can be forced up to 8; quant_matmul_noalloc
+    takes quant_matmul's path."""
+    if K != 100 and M not in (1, 8):
+        pytest.skip("K = 300 and 1000 at one and eight tokens")
+    N = 6 * G + 32 if G == 32 else 3 * G
+    (wq, s, b), w_ref, g = _transposed_problem(bits, G, N, K, seed=bits * 100 + G + M)
+    x = inputs.activations_bf16(M, K, g)
+    y = bq.quant_matmul(x.cuda(), wq, s, b, G, bits, transpose=False)
+    y_g = bq.quant_matmul_ex(x.cuda(), wq, s, b, G, bits, False, "gemv")
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    bq.quant_matmul_noalloc(x.cuda(), wq, s, b, out, G, bits, transpose=False)
+    torch.cuda.synchronize()
+    y_ref, a_ref = reference(x, w_ref)
+    assert_within_tolerance(y, y_ref, a_ref, f"transpose=0 bits={bits} G={G} M={M}")
+    assert_within_tolerance(y_g, y_ref, a_ref, f"transpose=0 GEMV bits={bits} G={G} M={M}")
+    assert torch.equal(y.view(torch.int16), out.view(torch.int16))
+    if M <= 4:      # the dispatcher's own choice up to 4 tokens; forced above
+        assert torch.equal(y.view(torch.int16), y_g.view(torch.int16))
+
+
+def test_transpose0_decode_limits():
+    """3- and 6-bit codes and M > 8 keep the pair (forcing the GEMV there is
+    unsupported); the pair and the GEMV agree within the tolerance."""
+    (wq, s, b), w_ref, g = _transposed_problem(3, 64, 128, 64, seed=3)
+    x = inputs.activations_bf16(2, 64, g)
+    with pytest.raises(bq.BqError, match="UNSUPPORTED"):
+        bq.quant_matmul_ex(x.cuda(), wq, s, b, 64, 3, False, "gemv")
+    (wq, s, b), w_ref, g = _transposed_problem(4, 64, 128, 64, seed=4)
+    x9 = inputs.activations_bf16(9, 64, g)
+    with pytest.raises(bq.BqError, match="UNSUPPORTED"):
+        bq.quant_matmul_ex(x9.cuda(), wq, s, b, 64, 4, False, "gemv")
+    x = inputs.activations_bf16(4, 64, g)
+    y_pair = bq.quant_matmul_ex(x.cuda(), wq, s, b, 64, 4, False, "dequant_gemm")
+    y_gemv = bq.quant_matmul_ex(x.cuda(), wq, s, b, 64, 4, False, "gemv")
+    torch.cuda.synchronize()
+    y_ref, a_ref = reference(x, w_ref)
+    assert_within_tolerance(y_pair, y_ref, a_ref, "pair")
+    assert_within_tolerance(y_gemv, y_ref, a_ref, "gemv")
+    assert bq.bq_device_status() == 0
