@@ -49,7 +49,7 @@ CSRC = os.path.join(ROOT, "bit_quantized_gemm_quant_b200", "csrc")
 NCU_TRAFFIC = {
     "gemv_kernel<Q4_0> M=1": {"bytes": 28332288, "source": "gemv.cuh", "sha16": "94efba42044385eb",
                               "capture": "2026-12-02 ncu --set full, profiles/gemv_kernel_q4_0_decode_m1_n12288_k4096.md"},
-    "gemv_tma_kernel<Q4_0> M=1": {"bytes": 28394496, "source": "gemv_stream.cuh", "sha16": "c2bbd7433e1793e3",
+    "gemv_tma_kernel<Q4_0> M=1": {"bytes": 28392704, "source": "gemv_stream.cuh", "sha16": "1b64b04575034f32",
                                   "capture": "2026-12-02 ncu --set full, profiles/gemv_tma_kernel_q4_0_decode_m1_n12288_k4096.md"},
 }
 
@@ -345,6 +345,31 @@ def run_decode(args, world, rank, device, peaks):
         forced[str(M)] = {"us": round(t * 1e6, 3), "gbs": round(wbytes / t / 1e9, 1),
                           "frac_hbm": round(wbytes / t / 1e9 / peaks["hbm_gbs"], 4),
                           **decode_kernel(bq, M, N, K, gs, bits, "gemv_stream")}
+    # affine 4-bit weights stored [K][N] (transpose = 0, groups of 64 along N) at the
+    # same N and K: the dispatcher's decode GEMV over [K][N] (1 to 4 tokens) against
+    # the unfused pair (forced), same rotation over copies and graph timing
+    transpose0 = None
+    if not args.no_secondary:
+        gk = inputs.generator(wl.seed + 2)
+        w_kn = inputs.weights_bf16_valued(K, N, gk).to(device).float()
+        kq, ks_, kb_ = bq.affine_quantize(w_kn, 64, 4)
+        del w_kn
+        kbytes = kq.numel() * 4 + ks_.numel() * 2 + kb_.numel() * 2
+        kcopies = [(kq, ks_, kb_)] + [(kq.clone(), ks_.clone(), kb_.clone())
+                                      for _ in range(-(-2 * L2_BYTES // kbytes))]
+        transpose0 = {"weights": f"affine 4-bit [K={K}][N={N}], group 64 along N", "copies": len(kcopies)}
+        for M in (1, 2, 4):
+            xk = inputs.activations_bf16(M, K, gk).to(device)
+            yk = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+            tg = kernel_seconds([(lambda c=c: bq.quant_matmul(xk, c[0], c[1], c[2], 64, 4, False, out=yk))
+                                 for c in kcopies], 4)
+            tp = kernel_seconds([(lambda c=c: bq.quant_matmul_ex(xk, c[0], c[1], c[2], 64, 4, False, "dequant_gemm",
+                                                                 out=yk)) for c in kcopies[:4]], 2)
+            transpose0[str(M)] = {"gemv_us": round(tg * 1e6, 3), "gemv_gbs": round(kbytes / tg / 1e9, 1),
+                                  "gemv_frac_hbm": round(kbytes / tg / 1e9 / peaks["hbm_gbs"], 4),
+                                  "kernel": "gemv_t_kernel", "pair_us": round(tp * 1e6, 3)}
+        del kcopies
+
     # the quantized-activation path (opt-in, approximate): activation quantization
     # plus the Q4_0 x int8 GEMV, same weights, rotation and graph timing
     fns = [(lambda wq=wq, s=s: bq.quant_matmul_q8(*bq.q8_1_quantize(xs[1]), wq, s, out=ys[1])) for (wq, s) in copies]
@@ -422,7 +447,8 @@ def run_decode(args, world, rank, device, peaks):
                   "timing": "CUDA events around graph replays of back-to-back launches, max over ranks"},
         "per_m": per_m, "roofline": roof, "e2e": e2e,
         "gpu_launches": args.steps * per_m["1"]["launches_per_call"], "clocks": clk.summary(),
-        "secondary": {"q8_activation_path_m1": q8, "streamed_int_kernel_forced": forced}, "gather": gather,
+        "secondary": {"q8_activation_path_m1": q8, "streamed_int_kernel_forced": forced,
+                      "transpose0_affine4_decode": transpose0}, "gather": gather,
     }
 
 
@@ -507,8 +533,9 @@ def run_small(args, device, peaks):
 
 
 def run_widths(args, world, device, peaks):
-    """Affine 2/3/6-bit weights and transpose=False (W stored [K][N], grouped along N), which run
-    as the unfused pair: the dequantize (bytes moved, GB/s) and quant_matmul's auto path per M."""
+    """Affine 2/3/6-bit weights and transpose=False (W stored [K][N], grouped along N): the
+    dequantize (bytes moved, GB/s) and quant_matmul's auto path per M (the decode GEMV at one
+    token -- over [K][N] for affine4_transpose0 -- the unfused pair at 512 and 2048 tokens)."""
     import torch
     import bit_quantized_gemm_quant_b200 as bq
     from bit_quantized_gemm_quant_b200 import inputs
