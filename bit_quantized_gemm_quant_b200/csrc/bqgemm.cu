@@ -70,7 +70,9 @@ enum class WFmt { Q4_0, AFF4, AFF8, AFF2, AFF3, AFF6 };
 
 bool has_fast_paths(WFmt f) { return f == WFmt::Q4_0 || f == WFmt::AFF4 || f == WFmt::AFF8; }
 
-constexpr int64_t kGaMaxM = 8;   // tokens of the decode GEMV for 2-, 3- and 6-bit weights
+constexpr int64_t kGaMaxM = 8;   // tokens of one decode GEMV launch for 2-, 3- and 6-bit weights
+constexpr int64_t kGaAutoMaxM = 8;     // ... that the dispatcher sends to it
+constexpr int64_t kGaForcedMaxM = 32;  // ... that a forced BQ_PATH_GEMV takes (in passes of kGaMaxM)
 
 // Format and shape checks shared by quant_matmul and its helpers (host only):
 // the packed matrix has N rows of K codes, grouped along K.
@@ -157,7 +159,7 @@ const DispatchCfg& dispatch_cfg()
 
 int select_path(int64_t M, int64_t K, WFmt fmt)
 {
-    if (!has_fast_paths(fmt)) return M <= kGaMaxM ? BQ_PATH_GEMV : BQ_PATH_DEQUANT_GEMM;
+    if (!has_fast_paths(fmt)) return M <= kGaAutoMaxM ? BQ_PATH_GEMV : BQ_PATH_DEQUANT_GEMM;
     const DispatchCfg& c = dispatch_cfg();
     if (M < c.tc_min_m[(int)fmt]) return BQ_PATH_GEMV;
     if (M <= kGemvMaxM && K % 64 != 0) return BQ_PATH_GEMV;      // no fused tile: the GEMV, not the pair
@@ -900,11 +902,21 @@ SgMats one_matrix(const void* wq, const uint16_t* s, const uint16_t* b, uint16_t
     return m;
 }
 
-// Decode GEMV for affine weights of any width (2-, 3- and 6-bit use it), M <= 8.
+// Decode GEMV for affine weights of any width (2-, 3- and 6-bit use it): one
+// launch per kGaMaxM tokens (each pass a contiguous block of x's and y's rows,
+// reading W again), up to kGaForcedMaxM tokens.
 bq_status launch_gemv_affine(WFmt fmt, const uint16_t* x, const void* wq, const uint16_t* s, const uint16_t* b,
                              uint16_t* y, int64_t M, int64_t N, int64_t K, int group_size, cudaStream_t st)
 {
-    if (N > INT32_MAX || K > INT32_MAX || M > kGaMaxM) return BQ_ERR_SHAPE;
+    if (N > INT32_MAX || K > INT32_MAX || M > kGaForcedMaxM) return BQ_ERR_SHAPE;
+    if (M > kGaMaxM) {
+        for (int64_t m0 = 0; m0 < M; m0 += kGaMaxM) {
+            const bq_status r = launch_gemv_affine(fmt, x + m0 * K, wq, s, b, y + m0 * N,
+                                                   std::min<int64_t>(kGaMaxM, M - m0), N, K, group_size, st);
+            if (r != BQ_OK) return r;
+        }
+        return BQ_OK;
+    }
     const int64_t rows_per_cta = (int64_t)kGaRows * kGaWarps;
     const unsigned grid = (unsigned)((N + rows_per_cta - 1) / rows_per_cta);
     const uint32_t* w = reinterpret_cast<const uint32_t*>(wq);
@@ -1189,7 +1201,7 @@ bq_status matmul_impl(const uint16_t* x, const void* wq, const void* scales, con
         (workspace && !aligned16(workspace)))
         return BQ_ERR_ALIGN;
     if (path == BQ_PATH_AUTO) path = select_path(M, K, fmt);
-    if (!has_fast_paths(fmt) && (path == BQ_PATH_TC_FUSED || (path == BQ_PATH_GEMV && M > kGaMaxM)))
+    if (!has_fast_paths(fmt) && (path == BQ_PATH_TC_FUSED || (path == BQ_PATH_GEMV && M > kGaForcedMaxM)))
         return BQ_ERR_UNSUPPORTED;
     if (path == BQ_PATH_GEMV && M > kGemvMaxM) return BQ_ERR_UNSUPPORTED;
     if (path == BQ_PATH_TC_FUSED && K % 64 != 0) return BQ_ERR_UNSUPPORTED;
@@ -1510,7 +1522,7 @@ int quant_matmul_gemv_kernel(int64_t M, int64_t N, int64_t K, int group_size, in
     if (M < 1 || check_format(format_tag(group_size, bits), N, K, group_size, bits, &fmt) != BQ_OK) return -1;
     if (path == BQ_PATH_AUTO) path = select_path(M, K, fmt);
     if (path != BQ_PATH_GEMV && path != BQ_PATH_GEMV_STREAM) return -1;
-    if (!has_fast_paths(fmt)) return path == BQ_PATH_GEMV && M <= kGaMaxM ? 3 : -1;
+    if (!has_fast_paths(fmt)) return path == BQ_PATH_GEMV && M <= kGaForcedMaxM ? 3 : -1;
     int dev, num_sms = 148, smem_optin = 232448;
     DeviceInfo di;
     if (cudaGetDevice(&dev) == cudaSuccess && current_device(&dev, &di) == BQ_OK) {

@@ -201,7 +201,8 @@ BQ_API bq_status quant_matmul_q8(const int8_t* xq, const float* dx, const int32_
  *            Other values: BQ_ERR_UNSUPPORTED.
  * Affine 2-, 3- and 6-bit weights have a decode GEMV up to 8 tokens (over the
  * exact weights scale*q + bias, within the GEMM tolerance of their bf16
- * roundings) and run as the unfused pair above that; 4- and 8-bit and Q4_0 have
+ * roundings; forced with BQ_PATH_GEMV it takes up to 32 tokens, in launches of
+ * 8 tokens that each read W) and run as the unfused pair above that; 4- and 8-bit and Q4_0 have
  * the decode GEMV and the fused kernel as well.  With transpose = 0 only the
  * GEMV over [K][N] (see transpose) and the pair exist.
  * The path is chosen by quant_matmul_select_path.  A path that needs scratch
@@ -290,7 +291,7 @@ BQ_API bq_status quant_matmul_multi(const uint16_t* x_bf16, int count, const voi
  * without K splits (same result within the tolerance, possibly slower); the
  * decode GEMV of one or two tokens given a smaller workspace runs the
  * register-streaming GEMV of three and more tokens instead (same tolerance).  Forcing
- * BQ_PATH_GEMV with M > 32 (M > 8 for 2-, 3- or 6-bit weights), BQ_PATH_TC_FUSED
+ * BQ_PATH_GEMV with M > 32, BQ_PATH_TC_FUSED
  * for 2-, 3- or 6-bit weights, BQ_PATH_TC_FUSED or BQ_PATH_GEMV_STREAM with
  * transpose = 0, or BQ_PATH_GEMV with transpose = 0 beyond 8 tokens or for 3-
  * or 6-bit codes, returns BQ_ERR_UNSUPPORTED.

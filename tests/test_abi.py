@@ -72,7 +72,7 @@ def test_quant_matmul_rejects_before_launch(L):
     assert qmm(L, b=ALIGNED, g=64, bits=5) == 3               # bits in {2, 3, 4, 6, 8}
     assert qmm(L, b=ALIGNED, g=64, bits=7) == 3
     assert qmm(L, tr=2) == 3
-    assert qmm(L, b=ALIGNED, g=64, bits=3, path=1) == 3       # 2/3/6-bit: GEMV to M = 8, then the pair
+    assert qmm(L, b=ALIGNED, g=64, bits=3, M=33, path=1) == 3  # 2/3/6-bit: forced GEMV to M = 32 (passes of 8)
     assert qmm(L, b=ALIGNED, g=64, bits=6, M=64, path=2) == 3
     assert qmm(L, b=ALIGNED, g=64, bits=2, M=64, path=2) == 3
     assert qmm(L, b=ALIGNED, g=64, tr=0, path=1) == 3         # transpose=0: GEMV to M = 8, then the pair

@@ -362,6 +362,25 @@ def test_affine_any_width_gemv(bits, M, N, K):
     assert_within_tolerance(y, y_ref, a_ref, f"bits={bits} M={M} {N}x{K}")
 
 
+@pytest.mark.parametrize("bits", [2, 3, 6])
+@pytest.mark.parametrize("M", [9, 16, 17, 32])
+@pytest.mark.parametrize("N,K", [(17, 96), (250, 2048)])
+def test_affine_any_width_gemv_passes(bits, M, N, K):
+    """Forced beyond 8 tokens, the any-width GEMV runs in passes of 8 tokens (the
+    last one ragged); each is checked against the oracle, and 33 tokens are
+    rejected."""
+    p = Problem(f"affine{bits}_g32", N, K, seed=bits * 300 + M + N)
+    wq, s, b = p.device()
+    x = p.x(M)
+    y = bq.quant_matmul_ex(x.cuda(), wq, s, b, 32, bits, True, "gemv")
+    torch.cuda.synchronize()
+    y_ref, a_ref = reference(x, p.wb)
+    assert_within_tolerance(y, y_ref, a_ref, f"bits={bits} M={M} {N}x{K}")
+    assert bq.quant_matmul_gemv_kernel(M, N, K, 32, bits, "gemv") == 3
+    with pytest.raises(bq.BqError, match="UNSUPPORTED"):
+        bq.quant_matmul_ex(p.x(33).cuda(), wq, s, b, 32, bits, True, "gemv")
+
+
 # ---------------------------------------------------------------- transpose = 0
 def _transposed_problem(bits: int, G: int, N: int, K: int, seed: int):
     """Affine W stored [K][N] (codes and groups along N), quantized by the oracle."""
