@@ -459,16 +459,17 @@ def test_2_3_6_bit_and_transpose0_edges():
 @pytest.mark.parametrize("bits", [2, 4, 8])
 @pytest.mark.parametrize("G", [32, 64, 128])
 @pytest.mark.parametrize("M", [1, 2, 3, 5, 8])
-@pytest.mark.parametrize("K", [100, 300, 1000])
+@pytest.mark.parametrize("K", [100, 300, 1000, 4200])
 def test_transpose0_decode_gemv(bits, G, M, K):
     """transpose = 0 at decode sizes with 2-, 4- or 8-bit codes: the GEMV over
-    [K][N] (any K, split over a cluster of 3 CTAs at K = 100 and up to 8 at K = 300
-    and 1000, ragged per-CTA ranges; N a multiple of the group, ragged against the
-    256- and 512-column clusters) is the dispatcher's choice up to 4 tokens (auto
-    and forced give the same bits) and can be forced up to 8; quant_matmul_noalloc
-    takes quant_matmul's path."""
+    [K][N] (any K, split over a cluster of 3 CTAs at K = 100 and up to 8 at K = 300,
+    1000 and 4200, ragged per-CTA ranges; at K = 4200 each CTA's 525 rows take two
+    passes of x staging; N a multiple of the group, ragged against the 256- and
+    512-column clusters) is the dispatcher's choice up to 4 tokens (auto and forced
+    give the same bits) and can be forced up to 8; quant_matmul_noalloc takes
+    quant_matmul's path."""
     if K != 100 and M not in (1, 8):
-        pytest.skip("K = 300 and 1000 at one and eight tokens")
+        pytest.skip("K = 300, 1000 and 4200 at one and eight tokens")
     N = 6 * G + 32 if G == 32 else 3 * G
     (wq, s, b), w_ref, g = _transposed_problem(bits, G, N, K, seed=bits * 100 + G + M)
     x = inputs.activations_bf16(M, K, g).cuda()
