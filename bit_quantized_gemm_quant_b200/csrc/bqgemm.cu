@@ -996,7 +996,8 @@ bq_status launch_gemv_t(WFmt fmt, const uint16_t* x, const void* wq, const uint1
                         uint16_t* y, int64_t M, int64_t N, int64_t K, int group_size, const DeviceInfo& di,
                         cudaStream_t st)
 {
-    if (N > INT32_MAX || K > INT32_MAX || M > kGtMaxM) return BQ_ERR_SHAPE;
+    // the kernel indexes columns in int, up to one cluster's width past N
+    if (N > INT32_MAX - 1024 || K > INT32_MAX || M > kGtMaxM) return BQ_ERR_SHAPE;
     const uint32_t* w = reinterpret_cast<const uint32_t*>(wq);
     auto by_m = [&](auto bits_tag) {
         constexpr int B = decltype(bits_tag)::value;
