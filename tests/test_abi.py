@@ -270,5 +270,9 @@ def test_decode_kernel_query(L):
     assert q(1, 8192, 2048, 32, 4, 0) == 0                 # K < 4096
     assert q(3, 12288, 4096, 32, 4, 4) == -1               # forced beyond two tokens
     assert q(1, 12288, 4096, 64, 3, 0) == 3                # 3-bit: any-width GEMV
+    assert q(8, 12288, 4096, 64, 6, 0) == 3                # ... up to 8 tokens by the dispatcher
+    assert q(9, 12288, 4096, 64, 2, 0) == -1               # then the pair
+    assert q(32, 12288, 4096, 64, 2, 1) == 3               # forced: passes of 8 tokens to 32
+    assert q(33, 12288, 4096, 64, 2, 1) == -1
     assert q(64, 12288, 4096, 32, 4, 0) == -1              # prefill: not a decode path
     assert q(0, 12288, 4096, 32, 4, 0) == -1
