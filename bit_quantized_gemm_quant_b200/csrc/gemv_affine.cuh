@@ -121,11 +121,12 @@ gemv_affine_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ 
 // A cluster of KS CTAs (up to 8 along the grid's y) owns 32 CPL output columns
 // and splits K into KS contiguous ranges, one per CTA.  A warp takes every 8th
 // row of its CTA's range, and its lanes read one contiguous run of that row:
-// lane l owns columns CPL l .. CPL l + CPL - 1 (CPL = 8 or 16 columns: 16 to 64
-// bits of the bit stream, so 2-, 4- and 8-bit codes; they share one group since
-// groups are >= 32 columns).  U rows are loaded before any is used, to keep
-// loads in flight; x is staged in shared memory as fp32 [row][token], 512 rows
-// at a time.  Per row and token a lane adds (x s) q for its columns and x z
+// lane l owns columns CPL l .. CPL l + CPL - 1 (CPL = 8 or 16 columns: 16 to
+// 128 bits of the bit stream, so 2-, 4- and 8-bit codes; they share one group
+// since groups are >= 32 columns).  Rows come in batches of U, two batches in
+// registers: the next batch's loads are in flight while the current one is
+// computed.  x is staged in shared memory as fp32 [row][token], 512 rows at a
+// time.  Per row and token a lane adds (x s) q for its columns and x z
 // once.  The 8 warps are summed through shared memory, then the KS CTAs'
 // partial sums through distributed shared memory, each in a fixed order, so the
 // result depends only on the shape and the cluster size.  The product is over
